@@ -1,0 +1,320 @@
+/*
+ * CPU oracle for the hybrid W4A4 + outlier linear layer (QUIK / Atom).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or
+ * calls this file; only the tests, the package's smoke check and the
+ * benchmark's CPU-baseline leg do.  It shares no code, header, table or
+ * constant with the CUDA library: it is a second, independent statement of
+ * what the layer computes, written to be checked by eye against the pages.
+ *
+ * What it follows (page title, passage):
+ *  - "QUIK: Towards End-to-End 4-Bit Inference on Generative Large Language
+ *    Models", abstract: most weights and activations are cast to 4 bits while
+ *    a few outlier weights/activations stay in higher precision (FP16).
+ *  - "Atom: Low-bit Quantization for Efficient and Accurate LLM Serving",
+ *    Summary: dynamic per-input activation scales and fine-grained group
+ *    quantization; Key points: symmetric quantization (no zero points);
+ *    Interesting ideas I1: outlier channels are reordered to the end so the
+ *    high-precision part is one contiguous block; I3: outliers kept in INT8.
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *  - scale s = max|v| / 7 in fp32 over the INT4 positions only (the outlier
+ *    block is excluded); code q = clamp(rintf(v / s), -7, 7) with an IEEE
+ *    fp32 division and round-half-to-even; an all-zero row/group gives s = 0
+ *    and all codes 0.
+ *  - groups are 128 consecutive *reordered* INT4 positions.
+ *  - INT8 outliers: s = max|v| / 127, q = clamp(rintf(v / s), -127, 127),
+ *    one scale per row (per token for X, per output channel for W).
+ *  - packing: byte i of a row holds code 2i in the low nibble and code 2i+1
+ *    in the high nibble, both 4-bit two's complement.
+ *  - integer dot products in int64 (checked to fit int32); dequantisation,
+ *    outlier products and bias in fp64; the output is NOT rounded to fp16.
+ *
+ * Every function is plain, row-by-row C; OpenMP only splits independent rows.
+ * Return value: 0 on success, negative on a violated precondition.
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <math.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_EBADARG -1
+#define ORACLE_EOVERFLOW -2
+#define ORACLE_ENOMEM -3
+
+/* IEEE 754 binary16 -> binary64, from the format's definition:
+ * normal  : (-1)^s * (1024 + m) * 2^(e - 25)
+ * subnorm : (-1)^s * m * 2^-24                                        */
+static double half_to_double(uint16_t h)
+{
+    int s = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int m = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + m), e - 25);
+    return s ? -v : v;
+}
+
+static float half_to_float(uint16_t h) { return (float)half_to_double(h); }
+
+/* Symmetric quantiser of one value: q = clamp(rint(v / s), -qmax, qmax),
+ * fp32 division, current (round-to-nearest-even) rounding mode. */
+static int quantize_value(float v, float s, int qmax)
+{
+    if (s == 0.0f)
+        return 0;
+    float r = rintf(v / s);
+    if (r > (float)qmax) r = (float)qmax;
+    if (r < (float)-qmax) r = (float)-qmax;
+    return (int)r;
+}
+
+/* 4-bit two's complement nibble -> signed code. */
+static int nibble_to_code(unsigned nib) { return nib >= 8 ? (int)nib - 16 : (int)nib; }
+
+/*
+ * oracle_quantize_rows -- reorder, scale, quantise and pack R rows of a
+ * [R, K] fp16 matrix.  Used for activations X (one row per token) and for
+ * weights W (one row per output channel): the pages apply the same symmetric
+ * rule to both.
+ *
+ *  X      : [R, K] fp16 bit patterns, row-major
+ *  perm   : [K]; reordered column j is source column perm[j]; j >= K - k_o
+ *           are the outlier channels
+ *  group  : 0 (one scale per row) or the group width (e.g. 128)
+ *  outlier_int8 : 0 -> O is fp16 [R, k_o] (bit copy); 1 -> O is int8
+ *           [R, k_o] with o_scale [R]
+ *  Q      : [R, (K - k_o) / 2] packed codes
+ *  scale  : [R] (group == 0) or [R, (K - k_o) / group]
+ */
+int oracle_quantize_rows(int64_t R, int64_t K, int64_t k_o, int64_t group, int outlier_int8,
+                         const uint16_t *X, const int32_t *perm,
+                         uint8_t *Q, float *scale, void *O, float *o_scale)
+{
+    if (R < 0 || K < 0 || k_o < 0 || k_o > K) return ORACLE_EBADARG;
+    const int64_t Ki = K - k_o;
+    if (Ki % 2) return ORACLE_EBADARG;
+    if (group < 0 || (group > 0 && Ki % group)) return ORACLE_EBADARG;
+    const int64_t gs = group > 0 ? group : Ki;          /* positions per scale */
+    const int64_t G = group > 0 ? Ki / group : 1;      /* scales per row      */
+    for (int64_t j = 0; j < K; ++j)
+        if (perm[j] < 0 || perm[j] >= K) return ORACLE_EBADARG;
+
+    int err = ORACLE_OK;
+#pragma omp parallel
+    {
+        float *xr = (float *)malloc(sizeof(float) * (size_t)(K > 0 ? K : 1));
+        int *codes = (int *)malloc(sizeof(int) * (size_t)(Ki > 0 ? Ki : 1));
+        if (!xr || !codes) {
+#pragma omp atomic write
+            err = ORACLE_ENOMEM;
+        }
+        /* every thread reaches the work-sharing loop; one without buffers skips its rows */
+#pragma omp for schedule(static)
+            for (int64_t r = 0; r < R; ++r) {
+                if (!xr || !codes) continue;
+                /* step 1: reorder (Atom I1) */
+                for (int64_t j = 0; j < K; ++j)
+                    xr[j] = half_to_float(X[r * K + perm[j]]);
+
+                /* steps 2-3: per-row (or per-group) scale, then codes */
+                for (int64_t g = 0; g < G; ++g) {
+                    float amax = 0.0f;
+                    for (int64_t j = g * gs; j < (g + 1) * gs; ++j)
+                        if (fabsf(xr[j]) > amax) amax = fabsf(xr[j]);
+                    float s = amax / 7.0f;
+                    scale[r * G + g] = s;
+                    for (int64_t j = g * gs; j < (g + 1) * gs; ++j)
+                        codes[j] = quantize_value(xr[j], s, 7);
+                }
+
+                /* step 4: pack, low nibble = even position */
+                for (int64_t i = 0; i < Ki / 2; ++i)
+                    Q[r * (Ki / 2) + i] =
+                        (uint8_t)((codes[2 * i] & 0xF) | ((codes[2 * i + 1] & 0xF) << 4));
+
+                /* step 6: the outlier block (reordered positions Ki .. K-1) */
+                if (k_o > 0) {
+                    if (!outlier_int8) {
+                        uint16_t *o16 = (uint16_t *)O;
+                        for (int64_t i = 0; i < k_o; ++i)
+                            o16[r * k_o + i] = X[r * K + perm[Ki + i]];
+                    } else {
+                        int8_t *o8 = (int8_t *)O;
+                        float amax = 0.0f;
+                        for (int64_t i = 0; i < k_o; ++i)
+                            if (fabsf(xr[Ki + i]) > amax) amax = fabsf(xr[Ki + i]);
+                        float s = amax / 127.0f;
+                        o_scale[r] = s;
+                        for (int64_t i = 0; i < k_o; ++i)
+                            o8[r * k_o + i] = (int8_t)quantize_value(xr[Ki + i], s, 127);
+                    }
+                } else if (outlier_int8 && o_scale) {
+                    o_scale[r] = 0.0f;
+                }
+            }
+        free(xr);
+        free(codes);
+    }
+    return err;
+}
+
+/*
+ * oracle_int_gemm -- exact integer product of packed INT4 codes.
+ *  acc[m, n]           = sum_{j < Ki} qx[m, j] * qw[n, j]            (group == 0)
+ *  acc[g, m, n]        = sum_{j in group g} qx[m, j] * qw[n, j]      (group > 0)
+ * Sums are taken in int64 and must fit int32.
+ */
+int oracle_int_gemm(int64_t M, int64_t N, int64_t Ki, int64_t group,
+                    const uint8_t *Xq, const uint8_t *Wq, int32_t *acc)
+{
+    if (M < 0 || N < 0 || Ki < 0 || Ki % 2) return ORACLE_EBADARG;
+    if (group < 0 || (group > 0 && Ki % group)) return ORACLE_EBADARG;
+    const int64_t gs = group > 0 ? group : Ki;
+    const int64_t G = group > 0 ? Ki / group : 1;
+    const int64_t rb = Ki / 2;
+    int err = ORACLE_OK;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            for (int64_t g = 0; g < G; ++g) {
+                int64_t sum = 0;
+                for (int64_t j = g * gs; j < (g + 1) * gs; ++j) {
+                    unsigned bx = Xq[m * rb + j / 2], bw = Wq[n * rb + j / 2];
+                    int cx = nibble_to_code(j % 2 ? bx >> 4 : bx & 0xF);
+                    int cw = nibble_to_code(j % 2 ? bw >> 4 : bw & 0xF);
+                    sum += (int64_t)cx * (int64_t)cw;
+                }
+                if (sum > INT32_MAX || sum < INT32_MIN) {
+#pragma omp atomic write
+                    err = ORACLE_EOVERFLOW;
+                }
+                acc[(g * M + m) * N + n] = (int32_t)sum;
+            }
+        }
+    }
+    return err;
+}
+
+/* One output element of the layer, in fp64, from quantised operands.
+ * Y = sum_g A_g * sx[m,g] * sw[n,g]  +  O  +  bias[n]                  */
+static double linear_element(int64_t m, int64_t n, int64_t M, int64_t N, int64_t K, int64_t k_o,
+                             int64_t group, int outlier_int8,
+                             const uint8_t *Xq, const float *sx, const void *Xo, const float *sxo,
+                             const uint8_t *Wq, const float *sw, const void *Wo, const float *swo,
+                             const uint16_t *bias, int32_t *acc_out, int *overflow)
+{
+    (void)M; (void)N;
+    const int64_t Ki = K - k_o;
+    const int64_t gs = group > 0 ? group : Ki;
+    const int64_t G = group > 0 ? Ki / group : 1;
+    const int64_t rb = Ki / 2;
+    double y = 0.0;
+
+    /* steps 5 and 7: exact integer sums, dequantised in fp64 */
+    for (int64_t g = 0; g < G; ++g) {
+        int64_t sum = 0;
+        for (int64_t j = g * gs; j < (g + 1) * gs; ++j) {
+            unsigned bx = Xq[m * rb + j / 2], bw = Wq[n * rb + j / 2];
+            int cx = nibble_to_code(j % 2 ? bx >> 4 : bx & 0xF);
+            int cw = nibble_to_code(j % 2 ? bw >> 4 : bw & 0xF);
+            sum += (int64_t)cx * (int64_t)cw;
+        }
+        if (sum > INT32_MAX || sum < INT32_MIN) *overflow = 1;
+        if (acc_out) acc_out[g] = (int32_t)sum;
+        if (Ki > 0)
+            y += (double)sum * (double)sx[m * G + g] * (double)sw[n * G + g];
+    }
+
+    /* step 6: the outlier block */
+    if (k_o > 0) {
+        if (!outlier_int8) {
+            const uint16_t *xo = (const uint16_t *)Xo, *wo = (const uint16_t *)Wo;
+            double o = 0.0;
+            for (int64_t i = 0; i < k_o; ++i)
+                o += half_to_double(xo[m * k_o + i]) * half_to_double(wo[n * k_o + i]);
+            y += o;
+        } else {
+            const int8_t *xo = (const int8_t *)Xo, *wo = (const int8_t *)Wo;
+            int64_t sum = 0;
+            for (int64_t i = 0; i < k_o; ++i)
+                sum += (int64_t)xo[m * k_o + i] * (int64_t)wo[n * k_o + i];
+            y += (double)sum * (double)sxo[m] * (double)swo[n];
+        }
+    }
+    if (bias)
+        y += half_to_double(bias[n]);
+    return y;
+}
+
+/*
+ * oracle_linear -- the full fp64 output Y [M, N] from quantised operands.
+ * Xo/Wo are fp16 [*, k_o] (outlier_int8 == 0) or int8 [*, k_o] with
+ * sxo [M] / swo [N] (outlier_int8 == 1).  bias is fp16 [N] or NULL.
+ */
+int oracle_linear(int64_t M, int64_t N, int64_t K, int64_t k_o, int64_t group, int outlier_int8,
+                  const uint8_t *Xq, const float *sx, const void *Xo, const float *sxo,
+                  const uint8_t *Wq, const float *sw, const void *Wo, const float *swo,
+                  const uint16_t *bias, double *Y)
+{
+    if (M < 0 || N < 0 || K < 0 || k_o < 0 || k_o > K || (K - k_o) % 2) return ORACLE_EBADARG;
+    if (group < 0 || (group > 0 && (K - k_o) % group)) return ORACLE_EBADARG;
+    int overflow = 0;
+#pragma omp parallel for schedule(static) reduction(| : overflow)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n)
+            Y[m * N + n] = linear_element(m, n, M, N, K, k_o, group, outlier_int8, Xq, sx, Xo,
+                                          sxo, Wq, sw, Wo, swo, bias, NULL, &overflow);
+    return overflow ? ORACLE_EOVERFLOW : ORACLE_OK;
+}
+
+/*
+ * oracle_linear_sampled -- the same output at `count` chosen (ms[i], ns[i])
+ * positions only; for full-size layers where the whole product would take
+ * the CPU too long.  acc (optional) receives the G integer sums per sample
+ * ([count, G], G = 1 without groups).
+ */
+int oracle_linear_sampled(int64_t M, int64_t N, int64_t K, int64_t k_o, int64_t group,
+                          int outlier_int8,
+                          const uint8_t *Xq, const float *sx, const void *Xo, const float *sxo,
+                          const uint8_t *Wq, const float *sw, const void *Wo, const float *swo,
+                          const uint16_t *bias, int64_t count, const int64_t *ms,
+                          const int64_t *ns, double *Y, int32_t *acc)
+{
+    if (M < 0 || N < 0 || K < 0 || k_o < 0 || k_o > K || (K - k_o) % 2) return ORACLE_EBADARG;
+    if (group < 0 || (group > 0 && (K - k_o) % group)) return ORACLE_EBADARG;
+    const int64_t G = group > 0 ? (K - k_o) / group : 1;
+    for (int64_t i = 0; i < count; ++i)
+        if (ms[i] < 0 || ms[i] >= M || ns[i] < 0 || ns[i] >= N) return ORACLE_EBADARG;
+    int overflow = 0;
+#pragma omp parallel for schedule(static) reduction(| : overflow)
+    for (int64_t i = 0; i < count; ++i)
+        Y[i] = linear_element(ms[i], ns[i], M, N, K, k_o, group, outlier_int8, Xq, sx, Xo, sxo,
+                              Wq, sw, Wo, swo, bias, acc ? acc + i * G : NULL, &overflow);
+    return overflow ? ORACLE_EOVERFLOW : ORACLE_OK;
+}
+
+/* Number of OpenMP threads the oracle would use (for reporting). */
+int oracle_num_threads(void)
+{
+    int n = 1;
+#pragma omp parallel
+    {
+#pragma omp single
+        {
+#ifdef _OPENMP
+            n = omp_get_num_threads();
+#endif
+        }
+    }
+    return n;
+}

@@ -1,0 +1,25 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the CUDA library")
+
+
+def pytest_collection_modifyitems(config, items):
+    # Keep the GPU tests skippable in a plain CPU run only when explicitly deselected;
+    # a GPU test that runs without a GPU must fail loudly, not pass silently.
+    pass
+
+
+@pytest.fixture(scope="session")
+def oracle_mod():
+    import oracle
+    oracle.build()
+    return oracle
