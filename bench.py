@@ -1,0 +1,418 @@
+#!/usr/bin/env python3
+"""Benchmark of the hybrid W4A4 + outlier linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-cpu-baseline]
+
+One step = one pass of the hot path over one batch: quantise + reorder the
+activations (quik_quantize_reorder), then the INT4 x INT4 GEMM with the
+outlier sub-product and the dequantising epilogue (quik_gemm); the weights
+are packed once before timing (offline).  The default workload is the
+Llama-7B attention projection (M=2048 tokens, N=K=4096, 128 FP16 outliers).
+
+Timing: W untimed warm-up steps, then exactly K steps; before every step a
+256 MiB buffer is written (flushing the 126 MB L2, outside the step's
+events); each step is bracketed by CUDA events on the launching stream
+(quantise and GEMM separately); the K steps are bracketed by a barrier and
+torch.cuda.synchronize() on both sides; the reported time is the max over
+ranks.  With N > 1 every rank runs an independent replica on its own GPU
+(weak scaling; the layer has no exchange step), and `value` is the ops of all
+ranks divided by the slowest rank's time.
+
+Prints ONE JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A4+outlier linear TOPS & µs/call at Llama shapes; % of dense INT8 peak"
+UNIT = "TOPS"
+FLUSH_BYTES = 256 << 20
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "w4a4_gemm_llama7b_attn_2048x4096x4096.md")
+GEMM_SOURCES = [os.path.join(ROOT, "mixed_precision_quantized_quantize_b200", "csrc", f)
+                for f in ("gemm.cu", "sm100.cuh")]
+# nominal dense-rate ratio INT8 : BF16 on B200 (4.5 : 2.25 PFLOP/s)
+INT8_PER_BF16 = 2.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+# ----------------------------------------------------------------- peaks and profiles
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return {"bf16_tflops": FALLBACK_BF16_TFLOPS, "hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+def gemm_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in GEMM_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """dram bytes per launch from the committed ncu summary, if it matches this kernel."""
+    try:
+        with open(PROFILE_SUMMARY) as f:
+            text = f.read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if line.startswith("traffic_bytes_per_launch:"):
+            vals["t"] = line.split(":", 1)[1].strip()
+        if line.startswith("gemm_source_sha256_16:"):
+            vals["h"] = line.split(":", 1)[1].strip()
+    if vals.get("h") != gemm_source_hash() or "t" not in vals:
+        return None
+    try:
+        return float(vals["t"])
+    except ValueError:
+        return None
+
+
+# ----------------------------------------------------------------- clocks (NVML, read only)
+class ClockSampler:
+    """Samples SM clock, power and throttle reasons every ~5 ms in a thread."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int):
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self._ok = False
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self._ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for n, b in self.REASONS.items() if self.reasons & b]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------- CPU oracle legs
+def cpu_oracle_step(cfg, d, rows: int):
+    """One bounded CPU pass of the layer: quantise `rows` token rows, then their
+    full output rows (every column) from the pre-packed weights."""
+    import oracle
+    X = d["X"][:rows].numpy()
+    xq = oracle.quantize_rows(X, d["perm_np"], cfg.k_o, cfg.group, cfg.outlier_int8)
+    wq = d["w_oracle"]
+    oracle.linear(xq[0], xq[1], xq[2] if cfg.k_o else None, xq[3], wq[0], wq[1],
+                  wq[2] if cfg.k_o else None, wq[3], d["bias_np"], cfg.K, cfg.k_o, cfg.group)
+
+
+def prepare_cpu_inputs(cfg, d):
+    import oracle
+    d["perm_np"] = d["perm"].numpy()
+    d["bias_np"] = None if d["bias"] is None else d["bias"].numpy()
+    d["w_oracle"] = oracle.quantize_rows(d["W"].numpy(), d["perm_np"], cfg.k_o, cfg.group,
+                                         cfg.outlier_int8)
+
+
+def cpu_baseline(cfg, d, budget_s: float = 10.0):
+    """Time the oracle, as it stands, on a bounded sample of the workload."""
+    import oracle
+    prepare_cpu_inputs(cfg, d)
+    threads = oracle.num_threads()
+    rows = max(1, min(cfg.M, threads))
+    while True:
+        t0 = time.perf_counter()
+        cpu_oracle_step(cfg, d, rows)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or rows >= cfg.M:
+            break
+        rows = min(cfg.M, max(rows + 1, int(rows * min(8.0, 1.2 * budget_s / max(dt, 1e-3)))))
+    ops = 2.0 * rows * cfg.N * cfg.K
+    return {"value": ops / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{rows} of {cfg.M} token rows x all {cfg.N} columns "
+                      f"(quantise + fp64 layer output), {dt:.1f} s"}
+
+
+# ----------------------------------------------------------------- aggregation
+def aggregate(step_times_s, ops_per_rank: float, world: int, reduce_max):
+    """Whole-job throughput from this rank's per-step times (weak scaling:
+    every rank does ops_per_rank per step)."""
+    local = float(sum(step_times_s))
+    total = reduce_max(local)
+    steps = len(step_times_s)
+    value = world * ops_per_rank * steps / total / 1e12
+    return value, total / steps
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args, rank, local_rank, world):
+    import torch
+    import torch.distributed as dist
+
+    import mixed_precision_quantized_quantize_b200 as q
+    from mixed_precision_quantized_quantize_b200 import workloads as wl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def reduce_max(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+
+    name = args.workload or wl.BENCH_CONFIG
+    cfg = wl.CONFIGS[name]
+    d = wl.make_layer(cfg)
+    X = d["X"].to(dev)
+    perm = d["perm"].to(dev)
+    bias = d["bias"].to(dev) if d["bias"] is not None else None
+    layer = q.QuikLinear(d["W"].to(dev), perm, cfg.k_o, cfg.group, cfg.outlier_int8, bias)
+    shape = layer.shape(cfg.M)
+    Xq, sx, Xo, sxo = q._binding._quant_outputs(cfg.M, cfg.K, cfg.k_o, cfg.group,
+                                                cfg.outlier_int8, dev)
+    Y = torch.empty((cfg.M, cfg.N), dtype=torch.float16, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        q.quik_quantize_reorder(shape, X, perm, Xq, sx, Xo, sxo, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        q.quik_gemm(shape, Xq, sx, Xo, sxo, layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale,
+                    bias, Y, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert q.quik_sync_check(stream) == q.QUIK_OK
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(args.steps):
+            flush.zero_()
+            step(events[i])
+        torch.cuda.synchronize()
+    barrier()
+    status = q.quik_sync_check(stream)
+    if status != q.QUIK_OK:
+        raise RuntimeError(f"device error after timed region: {q.status_string(status)}")
+    step_s = [e[0].elapsed_time(e[2]) / 1e3 for e in events]
+    gemm_s = [e[1].elapsed_time(e[2]) / 1e3 for e in events]
+    quant_s = [e[0].elapsed_time(e[1]) / 1e3 for e in events]
+    value, t_step = aggregate(step_s, cfg.ops, world, reduce_max)
+    gemm_avg = reduce_max(float(np.mean(gemm_s)))
+    quant_avg = reduce_max(float(np.mean(quant_s)))
+
+    # ---- end to end through the public call with host buffers (pinned)
+    Xh = d["X"].pin_memory()
+    Yh = torch.empty((cfg.M, cfg.N), dtype=torch.float16).pin_memory()
+    Xd = torch.empty_like(X)
+    e2e_steps = max(10, args.steps // 4)
+
+    def e2e_step():
+        Xd.copy_(Xh, non_blocking=True)
+        layer(Xd, out=Y, stream=stream)
+        Yh.copy_(Y, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(e2e_steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(e2e_steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        e2e_step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_value, _ = aggregate([a.elapsed_time(b) / 1e3 for a, b in ev], cfg.ops, world, reduce_max)
+
+    peaks, peak_kind = measured_peaks()
+    int8_peak = float(peaks["bf16_tflops"]) * INT8_PER_BF16
+    gemm_tops = cfg.ops / gemm_avg / 1e12
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": round(t_step * 1e3, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int4",
+        "data": "synthetic",
+        "config": {
+            "workload": name, "M": cfg.M, "N": cfg.N, "K": cfg.K, "k_o": cfg.k_o,
+            "group_size": cfg.group, "outliers": "int8" if cfg.outlier_int8 else "fp16",
+            "bias": cfg.bias, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "flushed before every step (256 MiB write, outside the step's events)",
+            "step": "quik_quantize_reorder + quik_gemm (weights packed once, offline)",
+        },
+        "us_per_call": round(t_step * 1e6, 2),
+        "pct_int8_peak": round(100.0 * value / world / int8_peak, 2),
+        "breakdown_us": {"quantize_reorder": round(quant_avg * 1e6, 2),
+                         "w4a4_gemm": round(gemm_avg * 1e6, 2)},
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "w4a4_gemm (INT4 codes widened to INT8, tcgen05 kind::i8)",
+            "achieved": round(gemm_tops, 2),
+            "peak": round(int8_peak, 1),
+            "unit": "TFLOP/s",
+            "frac": round(gemm_tops / int8_peak, 4),
+            "traffic": profiled_traffic(),
+            "peak_source": (f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
+                            f"{INT8_PER_BF16} (nominal INT8:BF16 dense ratio); integer ops "
+                            f"counted 2 per multiply-add"),
+        },
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
+                "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2,
+                "call": "quik_linear via QuikLinear, pinned host X in, host Y out"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": sampler.summary(),
+    }
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, d)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- reference arm (the oracle)
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    from mixed_precision_quantized_quantize_b200 import workloads as wl
+    name = args.workload or wl.BENCH_CONFIG
+    cfg = wl.CONFIGS[name]
+    d = wl.make_layer(cfg)
+    prepare_cpu_inputs(cfg, d)
+    threads = oracle.num_threads()
+    rows = max(1, min(cfg.M, threads))  # one token row per OpenMP thread per step
+    for _ in range(max(3, args.warmup)):
+        cpu_oracle_step(cfg, d, rows)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        cpu_oracle_step(cfg, d, rows)
+        times.append(time.perf_counter() - t0)
+    ops = 2.0 * rows * cfg.N * cfg.K
+    t = float(np.mean(times))
+    value = ops / t / 1e12
+    sample = (f"each step: {rows} of {cfg.M} token rows x all {cfg.N} columns "
+              f"(quantise + fp64 layer output)")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4",
+        "data": "synthetic",
+        "config": {"workload": name, "M": cfg.M, "N": cfg.N, "K": cfg.K, "k_o": cfg.k_o,
+                   "group_size": cfg.group, "outliers": "int8" if cfg.outlier_int8 else "fp16",
+                   "parallelism": "host cores (OpenMP over rows)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse()
+    rank, local_rank, world = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, local_rank, world)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,180 @@
+/*
+ * quik.h -- C ABI of the B200 (sm_100a) hybrid W4A4 + outlier linear layer.
+ *
+ * The layer (QUIK abstract; Atom summary, key points and ideas I1-I3):
+ *   X  fp16 [M, K] activations, W fp16 [N, K] weights, perm int32 [K].
+ *   Reordered channel j is source channel perm[j]; the last k_o reordered
+ *   channels are the outliers, kept in FP16 (QUIK) or INT8 (Atom, idea I3),
+ *   the other K_i = K - k_o are quantised to symmetric INT4 (Atom key point
+ *   "symmetric quantization") with a dynamic scale per token (activations)
+ *   or per output channel (weights), or per group of 128 reordered channels
+ *   (Atom summary, "fine-grained group quantization").
+ *   Y fp16 [M, N] = sum_g A_g * sx[m,g] * sw[n,g] + O[m,n] + bias[n],
+ *   A_g = exact integer sum of INT4 code products over group g,
+ *   O = outlier-block product (FP16 inputs, fp32 sum; or INT8 -> INT32 times
+ *   the two INT8 scales).
+ *
+ * Quantiser (readings where the pages are silent):
+ *   s = max|v| / 7 in fp32 over the INT4 positions of the row (or group);
+ *   q = clamp(rint(v / s), -7, 7), IEEE fp32 division, round half to even;
+ *   a zero row/group has s = 0 and codes 0.  INT8 outliers use 127.
+ *
+ * Byte layout of packed INT4 (Xq, Wq): row-major [rows, K_i / 2]; byte i of a
+ * row holds code 2i in bits 0-3 and code 2i+1 in bits 4-7, two's complement.
+ * Scales: fp32, [rows] or [rows, G] (G = K_i / 128) row-major.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE memory owned by the caller; the library
+ *     never allocates device memory and keeps no pointer after returning.
+ *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream) and is asynchronous: nothing synchronises.
+ *   - Every function returns a quik_status; nothing throws across the ABI.
+ *   - Arguments are validated before any launch: non-NULL pointers that are
+ *     16-byte aligned, M, N >= 1, 0 <= k_o <= K, K_i % 32 == 0, k_o % 16 == 0,
+ *     K <= 32768, group_size 0 or 128 (then K_i % 128 == 0).  Any violation
+ *     returns QUIK_ERR_INVALID_ARG with nothing enqueued.  Pointers that are
+ *     unused for the shape (outlier buffers when k_o == 0, INT8 scales in FP16
+ *     mode, bias) may be NULL.
+ *   - perm must be a permutation of 0..K-1; this is the caller's promise and
+ *     is not checked.
+ *   - A launch failure returns QUIK_ERR_CUDA.  Every wait inside the GEMM
+ *     kernel is bounded; if one runs out the kernel records it in a device
+ *     error word and exits cleanly, and quik_sync_check reports
+ *     QUIK_ERR_TIMEOUT.
+ *   - Thread safety: entry points may be called concurrently from several
+ *     host threads (no mutable host state besides one-time initialisation).
+ */
+#ifndef QUIK_H_
+#define QUIK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QUIK_API __attribute__((visibility("default")))
+#else
+#define QUIK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QUIK_OK = 0,
+    QUIK_ERR_INVALID_ARG = 1,
+    QUIK_ERR_UNSUPPORTED = 2,
+    QUIK_ERR_CUDA = 3,
+    QUIK_ERR_TIMEOUT = 4
+} quik_status;
+
+typedef enum {
+    QUIK_OUTLIER_FP16 = 0, /* QUIK: outlier block stays FP16 */
+    QUIK_OUTLIER_INT8 = 1  /* Atom idea I3: outlier block in INT8, fp32 scale per row */
+} quik_outlier_t;
+
+typedef struct {
+    int32_t M;          /* tokens (rows of X and Y) */
+    int32_t N;          /* output channels (rows of W, columns of Y) */
+    int32_t K;          /* input channels */
+    int32_t k_o;        /* outlier channels (last k_o of the reordering) */
+    int32_t group_size; /* 0: per-token / per-channel scales; 128: per group */
+    int32_t outlier;    /* a quik_outlier_t */
+} quik_shape;
+
+/* Opaque cudaStream_t. */
+typedef void *quik_stream_t;
+
+/*
+ * quik_workspace_size -- bytes of device workspace quik_linear needs for the
+ * quantised activations (packed codes, scales, outlier block), each part
+ * 256-byte aligned.  Returns 0 for an invalid shape.
+ */
+QUIK_API size_t quik_workspace_size(const quik_shape *shape);
+
+/*
+ * quik_quantize_reorder -- step "dynamic quantisation + reordering" of the
+ * activations (Atom summary and idea I2; QUIK abstract).  One kernel reads X
+ * once, gathers the columns through perm, computes the per-token (or
+ * per-group) INT4 scales, packs the codes and copies (FP16) or quantises
+ * (INT8) the outlier block.
+ *   X_f16    [M, K] fp16, row-major
+ *   perm     [K] int32
+ *   Xq       out [M, K_i/2] packed INT4
+ *   x_scale  out fp32 [M] or [M, G]
+ *   Xo       out [M, k_o] fp16 or int8 (may be NULL when k_o == 0)
+ *   xo_scale out fp32 [M], INT8 outliers only (NULL otherwise)
+ */
+QUIK_API quik_status quik_quantize_reorder(const quik_shape *shape, const void *X_f16, const int32_t *perm,
+                                  void *Xq, float *x_scale, void *Xo, float *xo_scale,
+                                  quik_stream_t stream);
+
+/*
+ * quik_pack_weights -- offline weight preparation (QUIK sample names
+ * pack_to_i4 / two_compl; Atom idea I1): the same reorder + symmetric
+ * quantiser applied to the rows of W (one scale per output channel, or per
+ * channel and group), round-to-nearest codes.
+ *   W_f16 [N, K] fp16; Wq out [N, K_i/2]; w_scale out [N] or [N, G];
+ *   Wo out [N, k_o] fp16 or int8; wo_scale out [N] (INT8 outliers only).
+ */
+QUIK_API quik_status quik_pack_weights(const quik_shape *shape, const void *W_f16, const int32_t *perm,
+                              void *Wq, float *w_scale, void *Wo, float *wo_scale,
+                              quik_stream_t stream);
+
+/*
+ * quik_gemm -- INT4 x INT4 product with exact INT32 accumulation (tensor
+ * cores, Atom key points), the outlier sub-product, and the dequantising
+ * epilogue Y = A*sx*sw (+ per group) + O + bias, rounded to fp16.
+ *   Xq [M, K_i/2], x_scale, Xo [M, k_o], xo_scale : quantised activations
+ *   Wq [N, K_i/2], w_scale, Wo [N, k_o], wo_scale : packed weights
+ *   bias_f16 [N] or NULL;  Y_f16 out [M, N] fp16 row-major
+ */
+QUIK_API quik_status quik_gemm(const quik_shape *shape,
+                      const void *Xq, const float *x_scale, const void *Xo, const float *xo_scale,
+                      const void *Wq, const float *w_scale, const void *Wo, const float *wo_scale,
+                      const void *bias_f16, void *Y_f16, quik_stream_t stream);
+
+/*
+ * quik_linear -- the whole layer on fp16 activations: quik_quantize_reorder
+ * into `workspace` followed by quik_gemm, both on `stream`.
+ *   workspace : device buffer of at least quik_workspace_size(shape) bytes
+ *               (caller-owned; reused freely between calls on one stream).
+ */
+QUIK_API quik_status quik_linear(const quik_shape *shape, const void *X_f16, const int32_t *perm,
+                        const void *Wq, const float *w_scale, const void *Wo,
+                        const float *wo_scale, const void *bias_f16, void *Y_f16,
+                        void *workspace, size_t workspace_bytes, quik_stream_t stream);
+
+/*
+ * quik_gemm_i32_debug -- test entry: the exact integer sums of the INT4 part
+ * as computed by the tensor-core main loop, acc [M, N] int32 (or [G, M, N]
+ * with groups), and for INT8 outliers the outlier block's integer sums
+ * acc_outlier [M, N] (NULL otherwise).
+ */
+QUIK_API quik_status quik_gemm_i32_debug(const quik_shape *shape, const void *Xq, const void *Wq,
+                                const void *Xo, const void *Wo, int32_t *acc,
+                                int32_t *acc_outlier, quik_stream_t stream);
+
+/*
+ * quik_sync_check -- synchronise `stream`, then report (and clear) the
+ * device error word: QUIK_ERR_TIMEOUT if a bounded wait ran out in any
+ * kernel since the last check, QUIK_ERR_CUDA on a CUDA error, else QUIK_OK.
+ */
+QUIK_API quik_status quik_sync_check(quik_stream_t stream);
+
+/*
+ * quik_selftest_timeout -- test entry for the failure detector: launches one
+ * CTA that waits on a barrier nothing will complete, with a wait limit of
+ * `limit_us` microseconds (1 .. 1000000).  The wait runs out, the kernel
+ * records QUIK_ERR_TIMEOUT and returns; quik_sync_check then reports it.
+ */
+QUIK_API quik_status quik_selftest_timeout(uint32_t limit_us, quik_stream_t stream);
+
+/* Static string for a status code. */
+QUIK_API const char *quik_status_string(quik_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QUIK_H_ */

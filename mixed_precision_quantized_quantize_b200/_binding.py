@@ -1,0 +1,260 @@
+"""ctypes binding of libquik_b200.so (the C ABI in include/quik.h).
+
+Argument marshalling only: every function below checks dtypes / devices,
+turns torch tensors into device pointers and calls the C entry point of the
+same name on the current CUDA stream.  Convenience helpers allocate the
+output tensors with torch (device memory is PyTorch's job here); all
+arithmetic runs in the library's kernels.  There is no CPU fallback: if the
+library is missing, or a tensor is not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libquik_b200.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "quik.h")
+
+QUIK_OK, QUIK_ERR_INVALID_ARG, QUIK_ERR_UNSUPPORTED, QUIK_ERR_CUDA, QUIK_ERR_TIMEOUT = range(5)
+QUIK_OUTLIER_FP16, QUIK_OUTLIER_INT8 = 0, 1
+GROUP = 128
+
+
+class QuikError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+class quik_shape(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int32), ("N", ctypes.c_int32), ("K", ctypes.c_int32),
+                ("k_o", ctypes.c_int32), ("group_size", ctypes.c_int32),
+                ("outlier", ctypes.c_int32)]
+
+
+_P = ctypes.c_void_p
+_S = ctypes.POINTER(quik_shape)
+_SIGS = {
+    "quik_workspace_size": (ctypes.c_size_t, [_S]),
+    "quik_quantize_reorder": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P]),
+    "quik_pack_weights": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P]),
+    "quik_gemm": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "quik_linear": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "quik_gemm_i32_debug": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P]),
+    "quik_sync_check": (ctypes.c_int, [_P]),
+    "quik_selftest_timeout": (ctypes.c_int, [ctypes.c_uint32, _P]),
+    "quik_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+}
+_lib = None
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/quik.h declares."""
+    text = open(HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(quik_[a-z0-9_]+)\s*\(", text)))
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m mixed_precision_quantized_quantize_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype, f.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().quik_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != QUIK_OK:
+        raise QuikError(status, what)
+
+
+def make_shape(M: int, N: int, K: int, k_o: int, group_size: int = 0,
+               outlier: int = QUIK_OUTLIER_FP16) -> quik_shape:
+    return quik_shape(M, N, K, k_o, group_size, outlier)
+
+
+def _ptr(t, dtype=None, what="tensor"):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{what} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{what} must live on a CUDA device")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{what} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    return t.data_ptr() if t.numel() > 0 else None
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+# ------------------------------------------------------------------ raw entry points
+def quik_workspace_size(shape: quik_shape) -> int:
+    return int(lib().quik_workspace_size(ctypes.byref(shape)))
+
+
+def quik_quantize_reorder(shape, X, perm, Xq, x_scale, Xo, xo_scale, stream=None):
+    _check(lib().quik_quantize_reorder(
+        ctypes.byref(shape), _ptr(X, torch.float16, "X"), _ptr(perm, torch.int32, "perm"),
+        _ptr(Xq, torch.uint8, "Xq"), _ptr(x_scale, torch.float32, "x_scale"), _ptr(Xo, None, "Xo"),
+        _ptr(xo_scale, torch.float32, "xo_scale"), _stream(stream)), "quik_quantize_reorder")
+
+
+def quik_pack_weights(shape, W, perm, Wq, w_scale, Wo, wo_scale, stream=None):
+    _check(lib().quik_pack_weights(
+        ctypes.byref(shape), _ptr(W, torch.float16, "W"), _ptr(perm, torch.int32, "perm"),
+        _ptr(Wq, torch.uint8, "Wq"), _ptr(w_scale, torch.float32, "w_scale"), _ptr(Wo, None, "Wo"),
+        _ptr(wo_scale, torch.float32, "wo_scale"), _stream(stream)), "quik_pack_weights")
+
+
+def quik_gemm(shape, Xq, x_scale, Xo, xo_scale, Wq, w_scale, Wo, wo_scale, bias, Y, stream=None):
+    _check(lib().quik_gemm(
+        ctypes.byref(shape), _ptr(Xq, torch.uint8, "Xq"), _ptr(x_scale, torch.float32, "x_scale"),
+        _ptr(Xo, None, "Xo"), _ptr(xo_scale, torch.float32, "xo_scale"),
+        _ptr(Wq, torch.uint8, "Wq"), _ptr(w_scale, torch.float32, "w_scale"),
+        _ptr(Wo, None, "Wo"), _ptr(wo_scale, torch.float32, "wo_scale"),
+        _ptr(bias, torch.float16, "bias"), _ptr(Y, torch.float16, "Y"), _stream(stream)), "quik_gemm")
+
+
+def quik_linear(shape, X, perm, Wq, w_scale, Wo, wo_scale, bias, Y, workspace, stream=None):
+    _check(lib().quik_linear(
+        ctypes.byref(shape), _ptr(X, torch.float16, "X"), _ptr(perm, torch.int32, "perm"),
+        _ptr(Wq, torch.uint8, "Wq"), _ptr(w_scale, torch.float32, "w_scale"),
+        _ptr(Wo, None, "Wo"), _ptr(wo_scale, torch.float32, "wo_scale"),
+        _ptr(bias, torch.float16, "bias"), _ptr(Y, torch.float16, "Y"),
+        _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)), "quik_linear")
+
+
+def quik_gemm_i32_debug(shape, Xq, Wq, Xo, Wo, acc, acc_outlier, stream=None):
+    _check(lib().quik_gemm_i32_debug(
+        ctypes.byref(shape), _ptr(Xq, torch.uint8, "Xq"), _ptr(Wq, torch.uint8, "Wq"),
+        _ptr(Xo, None, "Xo"), _ptr(Wo, None, "Wo"), _ptr(acc, torch.int32, "acc"),
+        _ptr(acc_outlier, torch.int32, "acc_outlier"), _stream(stream)), "quik_gemm_i32_debug")
+
+
+def quik_sync_check(stream=None) -> int:
+    return int(lib().quik_sync_check(_stream(stream)))
+
+
+def quik_selftest_timeout(limit_us: int, stream=None):
+    _check(lib().quik_selftest_timeout(int(limit_us), _stream(stream)), "quik_selftest_timeout")
+
+
+def quik_status_string(status: int) -> str:
+    return status_string(status)
+
+
+# ------------------------------------------------------------------ allocating helpers
+def _outlier_kind(int8: bool) -> int:
+    return QUIK_OUTLIER_INT8 if int8 else QUIK_OUTLIER_FP16
+
+
+def _quant_outputs(rows: int, K: int, k_o: int, group: int, int8: bool, device):
+    Ki = K - k_o
+    G = Ki // group if group else 1
+    Q = torch.empty((rows, Ki // 2), dtype=torch.uint8, device=device)
+    scale = torch.empty((rows, G) if group else (rows,), dtype=torch.float32, device=device)
+    O = torch.empty((rows, k_o), dtype=torch.int8 if int8 else torch.float16, device=device)
+    o_scale = torch.empty((rows,), dtype=torch.float32, device=device) if int8 else None
+    return Q, scale, O, o_scale
+
+
+def quantize_reorder(X: torch.Tensor, perm: torch.Tensor, k_o: int, group: int = 0,
+                     outlier_int8: bool = False, stream=None):
+    """Activations -> (Xq, x_scale, Xo, xo_scale), allocated on X's device."""
+    M, K = X.shape
+    shape = make_shape(M, 1, K, k_o, group, _outlier_kind(outlier_int8))
+    out = _quant_outputs(M, K, k_o, group, outlier_int8, X.device)
+    quik_quantize_reorder(shape, X, perm, *out, stream=stream)
+    return out
+
+
+def pack_weights(W: torch.Tensor, perm: torch.Tensor, k_o: int, group: int = 0,
+                 outlier_int8: bool = False, stream=None):
+    """Weights -> (Wq, w_scale, Wo, wo_scale), allocated on W's device."""
+    N, K = W.shape
+    shape = make_shape(1, N, K, k_o, group, _outlier_kind(outlier_int8))
+    out = _quant_outputs(N, K, k_o, group, outlier_int8, W.device)
+    quik_pack_weights(shape, W, perm, *out, stream=stream)
+    return out
+
+
+def gemm(xq, wq, K: int, k_o: int, group: int = 0, bias=None, stream=None):
+    """Y fp16 [M, N] from quantised activations xq and packed weights wq (4-tuples)."""
+    Xq, sx, Xo, sxo = xq
+    Wq, sw, Wo, swo = wq
+    M, N = sx.shape[0], sw.shape[0]
+    int8 = Xo.dtype == torch.int8
+    shape = make_shape(M, N, K, k_o, group, _outlier_kind(int8))
+    Y = torch.empty((M, N), dtype=torch.float16, device=sx.device)
+    quik_gemm(shape, Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias, Y, stream=stream)
+    return Y
+
+
+def gemm_i32(Xq, Wq, K: int, k_o: int, group: int = 0, Xo=None, Wo=None, stream=None):
+    """Raw integer sums: acc [M, N] (or [G, M, N]) and, for INT8 outliers, acc_o [M, N]."""
+    M, N = Xq.shape[0], Wq.shape[0]
+    Ki = K - k_o
+    G = Ki // group if group else 1
+    int8 = Xo is not None and Xo.dtype == torch.int8
+    shape = make_shape(M, N, K, k_o, group, _outlier_kind(int8))
+    acc = torch.empty((G, M, N) if group else (M, N), dtype=torch.int32, device=Xq.device)
+    acc_o = torch.empty((M, N), dtype=torch.int32, device=Xq.device) if int8 and k_o else None
+    quik_gemm_i32_debug(shape, Xq, Wq, Xo if int8 else None, Wo if int8 else None, acc, acc_o,
+                        stream=stream)
+    return acc, acc_o
+
+
+class QuikLinear:
+    """A hybrid W4A4 + outlier linear layer with packed weights resident on the GPU.
+
+    ``QuikLinear(W, perm, k_o, group, outlier_int8, bias)`` packs W once
+    (quik_pack_weights); calling it on fp16 activations runs quik_linear into
+    a workspace it keeps.
+    """
+
+    def __init__(self, W: torch.Tensor, perm: torch.Tensor, k_o: int, group: int = 0,
+                 outlier_int8: bool = False, bias: torch.Tensor | None = None):
+        self.N, self.K = W.shape
+        self.k_o, self.group, self.outlier_int8 = k_o, group, outlier_int8
+        self.perm = perm
+        self.bias = bias
+        self.Wq, self.w_scale, self.Wo, self.wo_scale = pack_weights(W, perm, k_o, group, outlier_int8)
+        self._ws = None
+
+    def shape(self, M: int) -> quik_shape:
+        return make_shape(M, self.N, self.K, self.k_o, self.group, _outlier_kind(self.outlier_int8))
+
+    def workspace(self, M: int, device) -> torch.Tensor:
+        need = quik_workspace_size(self.shape(M))
+        if need == 0:
+            raise QuikError(QUIK_ERR_INVALID_ARG, "quik_workspace_size")
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty((need,), dtype=torch.uint8, device=device)
+        return self._ws
+
+    def __call__(self, X: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        M = X.shape[0]
+        Y = out if out is not None else torch.empty((M, self.N), dtype=torch.float16, device=X.device)
+        quik_linear(self.shape(M), X, self.perm, self.Wq, self.w_scale, self.Wo, self.wo_scale,
+                    self.bias, Y, self.workspace(M, X.device), stream=stream)
+        return Y

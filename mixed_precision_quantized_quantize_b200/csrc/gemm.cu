@@ -1,0 +1,637 @@
+// gemm.cu -- the hybrid W4A4 + outlier product on sm_100a tensor cores.
+//
+// Computes, for a BM x BN tile of Y (QUIK abstract; "Atom: Low-bit
+// Quantization for Efficient and Accurate LLM Serving", summary and ideas
+// I1 / I3):
+//   A[m,n]  = sum_{j < K_i} qx[m,j] qw[n,j]        exact, INT32 (tensor cores)
+//   O[m,n]  = sum_{i < k_o} Xo[m,i] Wo[n,i]         fp16 -> fp32, or int8 -> int32
+//   Y[m,n]  = A sx[m] sw[n] + O (x sxo[m] swo[n] for INT8) + bias[n]  -> fp16
+// or, with groups of 128 (Atom summary, fine-grained groups), one INT32 sum
+// A_g per group, each dequantised with sx[m,g] sw[n,g] and added in fp32.
+//
+// Blackwell has no INT4 MMA.  Each 4-bit code c is widened to the signed
+// byte 16*c, which needs no sign extension: for a packed word w the odd
+// codes are w & 0xF0F0F0F0 and the even codes (w << 4) & 0xF0F0F0F0.  The
+// tcgen05 kind::i8 MMA then accumulates 256 * A exactly in INT32 (|A| <=
+// 49*K_i, so 256*|A| < 2^31 for K_i < 171196) and the epilogue shifts right
+// by 8.  Both operands place the even codes of a 16-byte packed chunk in the
+// first 16 unpacked bytes and the odd codes in the next 16, the same
+// K-permutation on both sides, so every dot product is unchanged.
+//
+// Warp roles in one CTA (one output tile per CTA):
+//   warp 0      TMA producer: packed INT4 tiles of Xq / Wq into a staging
+//               ring; FP16 (or INT8) outlier tiles directly into the operand
+//               ring (128-byte swizzled K-major, the layout the MMA reads);
+//   warp 1      TMEM allocator and the single thread that issues tcgen05.mma;
+//   NT warps    unpack: staging ring -> operand ring (swizzled INT8);
+//   NE warps    epilogue: TMEM -> registers -> dequantise -> fp16 stores
+//               (grouped mode: drain each group's INT32 sum while the next
+//               group accumulates in the other TMEM buffer).
+// Every mbarrier wait is bounded (2 s); on expiry the CTA records the error
+// in g_error_word, stops issuing work, waits for its in-flight copies and
+// MMAs, frees TMEM and exits.
+#include <algorithm>
+#include <cstring>
+
+#include <cuda_fp16.h>
+
+#include "quik_internal.h"
+#include "sm100.cuh"
+
+namespace quik {
+
+__device__ unsigned int g_error_word;
+
+namespace {
+
+using namespace ptx;
+
+constexpr int BM = 128;       // tile rows (tokens); one TMEM lane per row
+constexpr int KB = 128;       // INT4 codes per k-block = one scale group
+constexpr int PK_ROW = 64;    // packed bytes per row per k-block
+constexpr int OP_ROW = 128;   // unpacked bytes per row per k-block (one swizzle row)
+
+template <int BN_, bool GROUPED_, bool OUT_INT8_, bool DEBUG_>
+struct Cfg {
+    static constexpr int BN = BN_;
+    static constexpr bool GROUPED = GROUPED_;
+    static constexpr bool OUT_INT8 = OUT_INT8_;
+    static constexpr bool DEBUG = DEBUG_;
+    static constexpr int NT = GROUPED ? 4 : 8;  // unpack warps
+    static constexpr int NE = GROUPED ? 8 : 4;  // epilogue warps (multiple of 4)
+    static constexpr int THREADS = (2 + NT + NE) * 32;
+    static constexpr int SP = GROUPED ? 4 : 3;  // packed staging stages
+    static constexpr int SU = GROUPED ? 4 : 3;  // operand stages
+    static constexpr int PK_STAGE = (BM + BN) * PK_ROW;
+    static constexpr int OP_STAGE = (BM + BN) * OP_ROW;
+    static constexpr int OP_OFF = 0;
+    static constexpr int PK_OFF = SU * OP_STAGE;
+    static constexpr int SMEM = PK_OFF + SP * PK_STAGE + 1024;  // + alignment slack
+    // TMEM columns: non-grouped: INT32 sum [0,BN) + outlier sum [BN,2BN);
+    // grouped: two alternating group buffers [0,BN) and [BN,2BN).
+    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int CHUNKS = (BM + BN) * (PK_ROW / 16);     // 16-byte packed chunks
+    static constexpr int CHUNKS_PER_THREAD = CHUNKS / (NT * 32);
+    static constexpr int EPI_COLS = BN / (NE / 4);                // columns per epilogue warp
+    static_assert(CHUNKS % (NT * 32) == 0, "unpack work must split evenly");
+    static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation is a power of two");
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+struct GemmParams {
+    int M, N, Ki, k_o, nkb_i, nkb_o, G;
+    const float *sx, *sw, *sxo, *swo;
+    const uint16_t *bias;
+    uint16_t *Y;
+    int32_t *acc_dbg, *acc_o_dbg;
+};
+
+__device__ __forceinline__ void set_abort(volatile int *abort_flag) {
+    *abort_flag = 1;
+    atomicOr(&g_error_word, 1u);
+}
+
+// Bounded wait that also gives up at once when another role has aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            set_abort(abort_flag);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// Exact int32 -> fp32 for |v| < 2^22: place v in the mantissa of 1.5 * 2^23.
+__device__ __forceinline__ float small_int_to_float(int32_t v) {
+    return __int_as_float(v + 0x4B400000) - 12582912.0f;
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tm_xq,
+                     const __grid_constant__ CUtensorMap tm_wq,
+                     const __grid_constant__ CUtensorMap tm_xo,
+                     const __grid_constant__ CUtensorMap tm_wo, const GemmParams p) {
+    constexpr int BN = C::BN, SP = C::SP, SU = C::SU, NT = C::NT, NE = C::NE;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t pk_full[SP], pk_empty[SP], op_full[SU], op_empty[SU];
+    __shared__ uint64_t acc_full[2], acc_empty[2], mma_done;
+    __shared__ uint32_t tmem_base_s;
+    __shared__ int abort_s;
+    __shared__ __align__(16) float epi_sw[NE][C::EPI_COLS];
+
+    // 1024-byte aligned base (the swizzle pattern repeats every 1024 bytes)
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+    const uint32_t smem_base = smem_u32(smem);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+    volatile int *abort_flag = &abort_s;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < SP; ++s) {
+            mbar_init(&pk_full[s], 1);
+            mbar_init(&pk_empty[s], NT);
+        }
+        for (int s = 0; s < SU; ++s) {
+            mbar_init(&op_full[s], NT);
+            mbar_init(&op_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], NE);
+        }
+        mbar_init(&mma_done, 1);
+        abort_s = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(&tmem_base_s, C::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_s;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            if (p.nkb_i > 0) {
+                tma_prefetch_desc(&tm_xq);
+                tma_prefetch_desc(&tm_wq);
+            }
+            if (p.nkb_o > 0) {
+                tma_prefetch_desc(&tm_xo);
+                tma_prefetch_desc(&tm_wo);
+            }
+            int last_pk[SP], last_op[SU];
+            for (int s = 0; s < SP; ++s) last_pk[s] = -1;
+            for (int s = 0; s < SU; ++s) last_op[s] = -1;
+            bool ok = true;
+            for (int kb = 0; kb < p.nkb_i && ok; ++kb) {
+                const int s = kb % SP;
+                if (!(ok = wait_bar(&pk_empty[s], ((kb / SP) & 1) ^ 1, abort_flag))) break;
+                uint8_t *dst = smem + C::PK_OFF + s * C::PK_STAGE;
+                mbar_arrive_expect_tx(&pk_full[s], C::PK_STAGE);
+                tma_load_2d(dst, &tm_xq, kb * PK_ROW, m0, &pk_full[s]);
+                tma_load_2d(dst + BM * PK_ROW, &tm_wq, kb * PK_ROW, n0, &pk_full[s]);
+                last_pk[s] = kb;
+            }
+            // outlier k-blocks: 64 fp16 (or 128 int8) channels = 128 bytes per row
+            for (int ko = 0; ko < p.nkb_o && ok; ++ko) {
+                const int kb = p.nkb_i + ko, s = kb % SU;
+                if (!(ok = wait_bar(&op_empty[s], ((kb / SU) & 1) ^ 1, abort_flag))) break;
+                uint8_t *dst = smem + C::OP_OFF + s * C::OP_STAGE;
+                const int x = C::OUT_INT8 ? ko * 128 : ko * 64;
+                mbar_arrive_expect_tx(&op_full[s], C::OP_STAGE);
+                for (int a = 1; a < NT; ++a) mbar_arrive(&op_full[s]);  // count NT per phase
+                tma_load_2d(dst, &tm_xo, x, m0, &op_full[s]);
+                tma_load_2d(dst + BM * OP_ROW, &tm_wo, x, n0, &op_full[s]);
+                last_op[s] = kb;
+            }
+            // never leave the CTA with a bulk copy still writing its shared memory
+            for (int s = 0; s < SP; ++s)
+                if (last_pk[s] >= 0) mbar_wait_bounded(&pk_full[s], (last_pk[s] / SP) & 1, kWaitLimitNs);
+            for (int s = 0; s < SU; ++s)
+                if (last_op[s] >= 0) mbar_wait_bounded(&op_full[s], (last_op[s] / SU) & 1, kWaitLimitNs);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_i8 = idesc_s8_s32(BM, BN);
+            const uint32_t id_f16 = idesc_f16_f32(BM, BN);
+            bool ok = true;
+            for (int kb = 0; kb < p.nkb_i && ok; ++kb) {
+                const int s = kb % SU;
+                uint32_t d = tmem;
+                if (C::GROUPED) {
+                    const int b = kb & 1;
+                    if (!(ok = wait_bar(&acc_empty[b], ((kb >> 1) & 1) ^ 1, abort_flag))) break;
+                    d = tmem + b * BN;
+                }
+                if (!(ok = wait_bar(&op_full[s], (kb / SU) & 1, abort_flag))) break;
+                tc_fence_after();
+                const uint32_t a_addr = smem_base + C::OP_OFF + s * C::OP_STAGE;
+                const uint32_t b_addr = a_addr + BM * OP_ROW;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t acc = C::GROUPED ? (k > 0) : (kb > 0 || k > 0);
+                    mma_i8(d, sw128_kmajor_desc(a_addr + 32 * k), sw128_kmajor_desc(b_addr + 32 * k),
+                           id_i8, acc);
+                }
+                mma_commit(&op_empty[s]);
+                if (C::GROUPED) mma_commit(&acc_full[kb & 1]);
+            }
+            if (p.nkb_o > 0 && ok) {
+                uint32_t d = tmem + BN;
+                int b = 0;
+                if (C::GROUPED) {
+                    b = p.nkb_i & 1;
+                    ok = wait_bar(&acc_empty[b], ((p.nkb_i >> 1) & 1) ^ 1, abort_flag);
+                    d = tmem + b * BN;
+                }
+                for (int ko = 0; ko < p.nkb_o && ok; ++ko) {
+                    const int kb = p.nkb_i + ko, s = kb % SU;
+                    if (!(ok = wait_bar(&op_full[s], (kb / SU) & 1, abort_flag))) break;
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_base + C::OP_OFF + s * C::OP_STAGE;
+                    const uint32_t b_addr = a_addr + BM * OP_ROW;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t acc = (ko > 0 || k > 0);
+                        const uint64_t ad = sw128_kmajor_desc(a_addr + 32 * k);
+                        const uint64_t bd = sw128_kmajor_desc(b_addr + 32 * k);
+                        if (C::OUT_INT8)
+                            mma_i8(d, ad, bd, id_i8, acc);
+                        else
+                            mma_f16(d, ad, bd, id_f16, acc);
+                    }
+                    mma_commit(&op_empty[s]);
+                }
+                if (C::GROUPED && ok) mma_commit(&acc_full[b]);
+            }
+            if (!C::GROUPED) mma_commit(&acc_full[0]);
+            // all MMAs issued by this thread have finished before TMEM is freed
+            mma_commit(&mma_done);
+            mbar_wait_bounded(&mma_done, 0, kWaitLimitNs);
+        }
+        __syncwarp();
+    } else if (warp < 2 + NT) {
+        // ------------------------------------------------------------ unpack INT4 -> INT8
+        const int t = threadIdx.x - 64;
+        for (int kb = 0; kb < p.nkb_i; ++kb) {
+            const int sp = kb % SP, su = kb % SU;
+            bool ok = wait_bar(&pk_full[sp], (kb / SP) & 1, abort_flag) &&
+                      wait_bar(&op_empty[su], ((kb / SU) & 1) ^ 1, abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const uint8_t *pk = smem + C::PK_OFF + sp * C::PK_STAGE;
+            uint8_t *op = smem + C::OP_OFF + su * C::OP_STAGE;
+#pragma unroll
+            for (int i = 0; i < C::CHUNKS_PER_THREAD; ++i) {
+                // A rows [0, BM) then B rows [BM, BM+BN): one matrix of BM+BN rows
+                const int c = t + i * NT * 32;
+                const int r = c >> 2, ch = c & 3;
+                const uint4 v = *reinterpret_cast<const uint4 *>(pk + r * PK_ROW + ch * 16);
+                uint4 lo, hi;
+                lo.x = (v.x << 4) & 0xF0F0F0F0u;  hi.x = v.x & 0xF0F0F0F0u;
+                lo.y = (v.y << 4) & 0xF0F0F0F0u;  hi.y = v.y & 0xF0F0F0F0u;
+                lo.z = (v.z << 4) & 0xF0F0F0F0u;  hi.z = v.z & 0xF0F0F0F0u;
+                lo.w = (v.w << 4) & 0xF0F0F0F0u;  hi.w = v.w & 0xF0F0F0F0u;
+                uint8_t *row = op + r * OP_ROW;
+                *reinterpret_cast<uint4 *>(row + (((2 * ch) ^ (r & 7)) << 4)) = lo;
+                *reinterpret_cast<uint4 *>(row + (((2 * ch + 1) ^ (r & 7)) << 4)) = hi;
+            }
+            fence_proxy_async_smem();  // generic-proxy writes -> visible to the MMA
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&pk_empty[sp]);
+                mbar_arrive(&op_full[su]);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - (2 + NT);
+        const int q = warp & 3;  // TMEM lanes [32q, 32q+32) are this warp's
+        const int col0 = (ew >> 2) * C::EPI_COLS;
+        const int row = m0 + q * 32 + lane;
+        const bool row_ok = row < p.M;
+        const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
+        float *ssw = epi_sw[ew];
+
+        if (!C::GROUPED) {
+            bool ok = wait_bar(&acc_full[0], 0, abort_flag);
+            if (__all_sync(0xffffffffu, ok)) {
+                tc_fence_after();
+                const float sxr = (row_ok && p.Ki > 0) ? p.sx[row] : 0.0f;
+                const float sxo = (row_ok && C::OUT_INT8 && p.nkb_o > 0) ? p.sxo[row] : 0.0f;
+                for (int cc = 0; cc < C::EPI_COLS; cc += 32) {
+                    const int nb = n0 + col0 + cc;
+                    uint32_t a[32], o[32];
+                    if (p.Ki > 0) tmem_ld_32x32b_x32(t_lane + col0 + cc, a);
+                    if (p.nkb_o > 0) tmem_ld_32x32b_x32(t_lane + BN + col0 + cc, o);
+                    tmem_ld_wait();
+                    if (C::DEBUG) {
+                        if (row_ok) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) {
+                                const int n = nb + j;
+                                if (n < p.N) {
+                                    if (p.Ki > 0)
+                                        p.acc_dbg[(size_t)row * p.N + n] = static_cast<int32_t>(a[j]) >> 8;
+                                    if (C::OUT_INT8 && p.nkb_o > 0 && p.acc_o_dbg)
+                                        p.acc_o_dbg[(size_t)row * p.N + n] = static_cast<int32_t>(o[j]);
+                                }
+                            }
+                        }
+                        continue;
+                    }
+                    // per-column factors, staged once per chunk in this warp's slot
+                    {
+                        const int n = nb + lane;
+                        float swv = 0.0f;
+                        if (n < p.N) {
+                            if (p.Ki > 0) swv = p.sw[n];
+                        }
+                        ssw[cc + lane] = swv;
+                    }
+                    __syncwarp();
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        float y[2];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int jj = j + h, n = nb + jj;
+                            float v = 0.0f;
+                            if (p.Ki > 0)
+                                v = static_cast<float>(static_cast<int32_t>(a[jj]) >> 8) * sxr * ssw[cc + jj];
+                            if (p.nkb_o > 0) {
+                                if (C::OUT_INT8) {
+                                    const float swo = n < p.N ? __ldg(p.swo + n) : 0.0f;
+                                    v += static_cast<float>(static_cast<int32_t>(o[jj])) * sxo * swo;
+                                } else {
+                                    v += __uint_as_float(o[jj]);
+                                }
+                            }
+                            if (p.bias != nullptr && n < p.N)
+                                v += __half2float(__ushort_as_half(__ldg(p.bias + n)));
+                            y[h] = v;
+                        }
+                        packed[j / 2] = pack_half2(y[0], y[1]);
+                    }
+                    if (row_ok) {
+                        uint16_t *yrow = p.Y + (size_t)row * p.N;
+                        if (nb + 32 <= p.N && (p.N & 7) == 0) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(yrow + nb);
+#pragma unroll
+                            for (int v4 = 0; v4 < 4; ++v4)
+                                dst[v4] = make_uint4(packed[4 * v4], packed[4 * v4 + 1],
+                                                     packed[4 * v4 + 2], packed[4 * v4 + 3]);
+                        } else {
+                            for (int j = 0; j < 32; ++j)
+                                if (nb + j < p.N)
+                                    yrow[nb + j] = static_cast<uint16_t>(packed[j / 2] >> (16 * (j & 1)));
+                        }
+                    }
+                    __syncwarp();
+                }
+                tc_fence_before();
+            }
+        } else {
+            // grouped: running fp32 sums of this warp's EPI_COLS columns, in registers
+            float ysum[C::EPI_COLS];
+#pragma unroll
+            for (int j = 0; j < C::EPI_COLS; ++j) ysum[j] = 0.0f;
+            bool ok = true;
+            for (int g = 0; g < p.nkb_i && ok; ++g) {
+                const int b = g & 1;
+                // stage this group's weight scales for the warp's columns
+#pragma unroll
+                for (int cc = 0; cc < C::EPI_COLS; cc += 32) {
+                    const int n = n0 + col0 + cc + lane;
+                    ssw[cc + lane] = n < p.N ? p.sw[(size_t)n * p.G + g] : 0.0f;
+                }
+                // fold the 16 x 16 operand scaling (2^-8) into the row factor
+                const float sxg = row_ok ? p.sx[(size_t)row * p.G + g] * (1.0f / 256.0f) : 0.0f;
+                __syncwarp();
+                ok = wait_bar(&acc_full[b], (g >> 1) & 1, abort_flag);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int cc = 0; cc < C::EPI_COLS; cc += 32) {
+                    uint32_t a[32];
+                    tmem_ld_32x32b_x32(t_lane + b * BN + col0 + cc, a);
+                    tmem_ld_wait();
+                    if (C::DEBUG) {
+                        if (row_ok)
+                            for (int j = 0; j < 32; ++j) {
+                                const int n = n0 + col0 + cc + j;
+                                if (n < p.N)
+                                    p.acc_dbg[((size_t)g * p.M + row) * p.N + n] =
+                                        static_cast<int32_t>(a[j]) >> 8;
+                            }
+                        continue;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float f = small_int_to_float(static_cast<int32_t>(a[j])) * ssw[cc + j];
+                        ysum[cc + j] = fmaf(f, sxg, ysum[cc + j]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[b]);
+            }
+            if (ok && p.nkb_o > 0) {
+                const int b = p.nkb_i & 1;
+                ok = wait_bar(&acc_full[b], (p.nkb_i >> 1) & 1, abort_flag);
+                if (__all_sync(0xffffffffu, ok)) {
+                    tc_fence_after();
+                    const float sxo = (row_ok && C::OUT_INT8) ? p.sxo[row] : 0.0f;
+#pragma unroll
+                    for (int cc = 0; cc < C::EPI_COLS; cc += 32) {
+                        uint32_t o[32];
+                        tmem_ld_32x32b_x32(t_lane + b * BN + col0 + cc, o);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int n = n0 + col0 + cc + j;
+                            if (C::DEBUG) {
+                                if (C::OUT_INT8 && row_ok && n < p.N && p.acc_o_dbg)
+                                    p.acc_o_dbg[(size_t)row * p.N + n] = static_cast<int32_t>(o[j]);
+                            } else if (C::OUT_INT8) {
+                                const float swo = n < p.N ? __ldg(p.swo + n) : 0.0f;
+                                ysum[cc + j] += static_cast<float>(static_cast<int32_t>(o[j])) * sxo * swo;
+                            } else {
+                                ysum[cc + j] += __uint_as_float(o[j]);
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                } else {
+                    ok = false;
+                }
+            }
+            if (ok && !C::DEBUG && row_ok) {
+                uint16_t *yrow = p.Y + (size_t)row * p.N;
+#pragma unroll
+                for (int cc = 0; cc < C::EPI_COLS; cc += 32) {
+                    const int nb = n0 + col0 + cc;
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        float y0 = ysum[cc + j], y1 = ysum[cc + j + 1];
+                        if (p.bias != nullptr) {
+                            if (nb + j < p.N) y0 += __half2float(__ushort_as_half(__ldg(p.bias + nb + j)));
+                            if (nb + j + 1 < p.N) y1 += __half2float(__ushort_as_half(__ldg(p.bias + nb + j + 1)));
+                        }
+                        packed[j / 2] = pack_half2(y0, y1);
+                    }
+                    if (nb + 32 <= p.N && (p.N & 7) == 0) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(yrow + nb);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            dst[v4] = make_uint4(packed[4 * v4], packed[4 * v4 + 1], packed[4 * v4 + 2],
+                                                 packed[4 * v4 + 3]);
+                    } else {
+                        for (int j = 0; j < 32; ++j)
+                            if (nb + j < p.N)
+                                yrow[nb + j] = static_cast<uint16_t>(packed[j / 2] >> (16 * (j & 1)));
+                    }
+                }
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ----------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(ptr);
+    }();
+    return fn;
+}
+
+// 2-D row-major map: `inner` elements per row (contiguous), `rows` rows,
+// `stride` bytes between rows; box of box_inner x box_rows.
+bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
+              uint64_t rows, uint64_t stride, uint32_t box_inner, uint32_t box_rows,
+              CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {stride};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <class C>
+quik_status run(const GemmArgs &a, cudaStream_t stream) {
+    static_assert(sizeof(C) > 0, "");
+    const int Ki = a.K - a.k_o;
+    CUtensorMap mxq, mwq, mxo, mwo;
+    std::memset(&mxq, 0, sizeof(mxq));
+    std::memset(&mwq, 0, sizeof(mwq));
+    std::memset(&mxo, 0, sizeof(mxo));
+    std::memset(&mwo, 0, sizeof(mwo));
+    if (Ki > 0) {
+        if (!make_map(&mxq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Xq, Ki / 2, a.M, Ki / 2, PK_ROW, BM,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !make_map(&mwq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wq, Ki / 2, a.N, Ki / 2, PK_ROW,
+                      C::BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return QUIK_ERR_CUDA;
+    }
+    const bool outliers = a.k_o > 0 && a.Xo != nullptr;  // debug entry may skip them
+    if (outliers) {
+        const bool i8 = C::OUT_INT8;
+        const CUtensorMapDataType dt =
+            i8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+        const uint64_t es = i8 ? 1 : 2;
+        const uint32_t bi = i8 ? 128 : 64;
+        if (!make_map(&mxo, dt, a.Xo, a.k_o, a.M, a.k_o * es, bi, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&mwo, dt, a.Wo, a.k_o, a.N, a.k_o * es, bi, C::BN,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+            return QUIK_ERR_CUDA;
+    }
+    GemmParams p{};
+    p.M = a.M;
+    p.N = a.N;
+    p.Ki = Ki;
+    p.k_o = a.k_o;
+    p.nkb_i = (Ki + KB - 1) / KB;
+    p.nkb_o = !outliers ? 0 : (C::OUT_INT8 ? (a.k_o + 127) / 128 : (a.k_o + 63) / 64);
+    p.G = a.group > 0 ? Ki / a.group : 1;
+    p.sx = a.sx;
+    p.sw = a.sw;
+    p.sxo = a.sxo;
+    p.swo = a.swo;
+    p.bias = a.bias;
+    p.Y = a.Y;
+    p.acc_dbg = a.acc_dbg;
+    p.acc_o_dbg = a.acc_o_dbg;
+
+    auto kern = w4a4_gemm_kernel<C>;
+    if (!attribute_set_once(reinterpret_cast<const void *>(kern), C::SMEM)) return QUIK_ERR_CUDA;
+    const dim3 grid((a.N + C::BN - 1) / C::BN, (a.M + BM - 1) / BM);
+    kern<<<grid, C::THREADS, C::SMEM, stream>>>(mxq, mwq, mxo, mwo, p);
+    return cudaGetLastError() == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
+}
+
+template <bool DEBUG>
+quik_status dispatch(const GemmArgs &a, cudaStream_t stream) {
+    if (a.group > 0)
+        return a.out_int8 ? run<Cfg<128, true, true, DEBUG>>(a, stream)
+                          : run<Cfg<128, true, false, DEBUG>>(a, stream);
+    return a.out_int8 ? run<Cfg<256, false, true, DEBUG>>(a, stream)
+                      : run<Cfg<256, false, false, DEBUG>>(a, stream);
+}
+
+// A CTA waiting on a barrier that nothing completes: exercises the bounded
+// wait and the error word without a fault.
+__global__ void timeout_selftest_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, limit_ns)) atomicOr(&g_error_word, 1u);
+    __syncthreads();
+}
+
+}  // namespace
+
+quik_status launch_gemm(const GemmArgs &a, cudaStream_t stream) {
+    return a.debug ? dispatch<true>(a, stream) : dispatch<false>(a, stream);
+}
+
+quik_status launch_timeout_selftest(uint32_t limit_us, cudaStream_t stream) {
+    timeout_selftest_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(limit_us) * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
+}
+
+quik_status sync_check(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return QUIK_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return QUIK_ERR_CUDA;
+    if (word != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+            return QUIK_ERR_CUDA;
+        return QUIK_ERR_TIMEOUT;
+    }
+    return QUIK_OK;
+}
+
+}  // namespace quik

@@ -1,0 +1,215 @@
+// quantize.cu -- reorder + dynamic symmetric INT4 quantisation + nibble packing
+// of the rows of an fp16 matrix, with the outlier block copied (FP16) or
+// quantised to INT8.  Serves activations (one row per token; "Atom: Low-bit
+// Quantization for Efficient and Accurate LLM Serving", summary: dynamic
+// per-input scales, reordering fused into one pass, idea I2) and the offline
+// weight pack (one row per output channel; QUIK sample names pack_to_i4 /
+// two_compl).
+//
+// One CTA owns one row at a time (grid-stride over rows, 256 threads):
+//   1. the CTA stages perm (as uint16) once, then per row loads the fp16 row
+//      into shared memory with coalesced 16-byte streaming loads;
+//   2. each thread gathers 8 reordered positions per 32-bit output word
+//      (up to MAXW words, kept in registers), takes their absmax;
+//   3. per-row scale: block reduction; per-group scale (128 positions =
+//      16 words = 16 adjacent lanes): 4-step xor shuffle;
+//   4. codes are packed 8 per word and stored coalesced (a warp writes 128
+//      contiguous bytes);
+//   5. outlier positions Ki..K-1 are gathered and copied, or quantised with
+//      their own absmax/127 scale.
+// The kernel is bound by HBM bandwidth (2 bytes read per element, 0.5 byte
+// written per INT4 element).
+#include <algorithm>
+
+#include <cuda_fp16.h>
+
+#include "quik_internal.h"
+
+namespace quik {
+namespace {
+
+constexpr int kQThreads = 256;
+
+struct QParams {
+    const uint16_t *X;
+    const int32_t *perm;
+    int rows, K, k_o;
+    uint8_t *Q;
+    float *scale;
+    void *O;
+    float *o_scale;
+};
+
+__device__ __forceinline__ float h2f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
+
+// q = clamp(rint(v / s), -qmax, qmax) with the quotient correctly rounded to
+// fp32 (IEEE division, round half to even), q = 0 when s == 0.
+// Fast path: t = v * fl(1/s).  With u = 2^-24, |t - fl(v/s)| <= 3u|v/s|(1+u),
+// so when t is farther than 5e-7*max(|t|,1) > 3u|t|(1+3u) from a half-integer
+// (the only places where rint changes value), fl(v/s) lies on the same side
+// and rounds to the same integer.  Otherwise the exact quotient decides.
+__device__ __forceinline__ int quant_code(float v, float s, float rs, int qmax) {
+    if (s == 0.0f) return 0;
+    float t = __fmul_rn(v, rs);
+    float r = rintf(t);
+    if (0.5f - fabsf(t - r) <= 5e-7f * fmaxf(fabsf(t), 1.0f)) r = rintf(__fdiv_rn(v, s));
+    const int q = static_cast<int>(r);
+    return max(-qmax, min(qmax, q));
+}
+
+__device__ __forceinline__ float warp_max(float m) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    return m;
+}
+
+template <bool GROUPED, bool OUT_INT8, int MAXW>
+__global__ void __launch_bounds__(kQThreads) quantize_rows_kernel(QParams p) {
+    extern __shared__ __align__(16) uint8_t qsmem[];
+    __shared__ float red_a[kQThreads / 32];
+    __shared__ float red_b[kQThreads / 32];
+    const int K = p.K, Ki = K - p.k_o;
+    const int Kp = (K + 7) & ~7;
+    uint16_t *perm_s = reinterpret_cast<uint16_t *>(qsmem);
+    uint16_t *row_s = perm_s + Kp;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nwords = Ki / 8;
+    const int G = GROUPED ? Ki / kGroup : 1;
+
+    for (int i = tid; i < K; i += kQThreads) perm_s[i] = static_cast<uint16_t>(p.perm[i]);
+
+    for (int row = blockIdx.x; row < p.rows; row += gridDim.x) {
+        // (1) stage the row; the barrier also publishes perm_s on the first pass
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.X + static_cast<size_t>(row) * K);
+        for (int i = tid; i < K / 8; i += kQThreads)
+            reinterpret_cast<uint4 *>(row_s)[i] = __ldcs(src + i);
+        __syncthreads();
+
+        // (2) gather 8 reordered values per word, absmax per word
+        uint32_t v[MAXW][4];
+        float wmax[MAXW];
+#pragma unroll
+        for (int i = 0; i < MAXW; ++i) {
+            const int w = tid + i * kQThreads;
+            wmax[i] = 0.0f;
+            if (w < nwords) {
+                const uint4 ix = *reinterpret_cast<const uint4 *>(perm_s + 8 * w);
+                const uint32_t idx[4] = {ix.x, ix.y, ix.z, ix.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint16_t a = row_s[idx[k] & 0xffffu], b = row_s[idx[k] >> 16];
+                    v[i][k] = static_cast<uint32_t>(a) | (static_cast<uint32_t>(b) << 16);
+                    wmax[i] = fmaxf(wmax[i], fmaxf(fabsf(h2f(a)), fabsf(h2f(b))));
+                }
+            }
+        }
+
+        // (3) scales
+        float s[MAXW];
+        if (GROUPED) {
+#pragma unroll
+            for (int i = 0; i < MAXW; ++i) {
+                float m = wmax[i];
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                s[i] = __fdiv_rn(m, 7.0f);
+                const int w = tid + i * kQThreads;
+                if (w < nwords && (lane & 15) == 0)
+                    p.scale[static_cast<size_t>(row) * G + w / 16] = s[i];
+            }
+        } else {
+            float m = 0.0f;
+#pragma unroll
+            for (int i = 0; i < MAXW; ++i) m = fmaxf(m, wmax[i]);
+            m = warp_max(m);
+            if (lane == 0) red_a[warp] = m;
+            __syncthreads();
+            m = red_a[0];
+#pragma unroll
+            for (int k = 1; k < kQThreads / 32; ++k) m = fmaxf(m, red_a[k]);
+            const float sr = __fdiv_rn(m, 7.0f);
+#pragma unroll
+            for (int i = 0; i < MAXW; ++i) s[i] = sr;
+            if (tid == 0) p.scale[row] = sr;
+        }
+
+        // (4) codes, 8 per word, code 2i in the low nibble of byte i
+        uint32_t *qrow = reinterpret_cast<uint32_t *>(p.Q + static_cast<size_t>(row) * (Ki / 2));
+#pragma unroll
+        for (int i = 0; i < MAXW; ++i) {
+            const int w = tid + i * kQThreads;
+            if (w < nwords) {
+                const float rs = s[i] != 0.0f ? __frcp_rn(s[i]) : 0.0f;
+                uint32_t word = 0;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int q0 = quant_code(h2f(static_cast<uint16_t>(v[i][k] & 0xffffu)), s[i], rs, 7);
+                    const int q1 = quant_code(h2f(static_cast<uint16_t>(v[i][k] >> 16)), s[i], rs, 7);
+                    word |= (static_cast<uint32_t>(q0) & 0xFu) << (8 * k);
+                    word |= (static_cast<uint32_t>(q1) & 0xFu) << (8 * k + 4);
+                }
+                qrow[w] = word;
+            }
+        }
+
+        // (5) the outlier block
+        if (p.k_o > 0) {
+            if (!OUT_INT8) {
+                uint16_t *o = static_cast<uint16_t *>(p.O) + static_cast<size_t>(row) * p.k_o;
+                for (int i = tid; i < p.k_o; i += kQThreads) o[i] = row_s[perm_s[Ki + i]];
+            } else {
+                float m = 0.0f;
+                for (int i = tid; i < p.k_o; i += kQThreads)
+                    m = fmaxf(m, fabsf(h2f(row_s[perm_s[Ki + i]])));
+                m = warp_max(m);
+                if (lane == 0) red_b[warp] = m;
+                __syncthreads();
+                m = red_b[0];
+#pragma unroll
+                for (int k = 1; k < kQThreads / 32; ++k) m = fmaxf(m, red_b[k]);
+                const float so = __fdiv_rn(m, 127.0f);
+                const float rso = so != 0.0f ? __frcp_rn(so) : 0.0f;
+                if (tid == 0) p.o_scale[row] = so;
+                int8_t *o = static_cast<int8_t *>(p.O) + static_cast<size_t>(row) * p.k_o;
+                for (int i = tid; i < p.k_o; i += kQThreads)
+                    o[i] = static_cast<int8_t>(quant_code(h2f(row_s[perm_s[Ki + i]]), so, rso, 127));
+            }
+        } else if (OUT_INT8 && p.o_scale != nullptr && tid == 0) {
+            p.o_scale[row] = 0.0f;
+        }
+        __syncthreads();  // row_s and the reduction slots are reused by the next row
+    }
+}
+
+template <bool GROUPED, bool OUT_INT8, int MAXW>
+cudaError_t launch_q(const QParams &p, cudaStream_t stream) {
+    auto kern = quantize_rows_kernel<GROUPED, OUT_INT8, MAXW>;
+    const int Kp = (p.K + 7) & ~7;
+    const size_t smem = static_cast<size_t>(Kp) * 2 * sizeof(uint16_t);
+    if (!attribute_set_once(reinterpret_cast<const void *>(kern), static_cast<int>(smem)))
+        return cudaErrorInvalidConfiguration;
+    // up to 8 resident 256-thread CTAs per SM; rows beyond that are grid-strided
+    const int grid = std::max(1, std::min(p.rows, sm_count() * 8));
+    kern<<<grid, kQThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <bool GROUPED, bool OUT_INT8>
+cudaError_t launch_q_w(const QParams &p, cudaStream_t stream) {
+    const int words_per_thread = ((p.K - p.k_o) / 8 + kQThreads - 1) / kQThreads;
+    if (words_per_thread <= 2) return launch_q<GROUPED, OUT_INT8, 2>(p, stream);
+    if (words_per_thread <= 4) return launch_q<GROUPED, OUT_INT8, 4>(p, stream);
+    if (words_per_thread <= 8) return launch_q<GROUPED, OUT_INT8, 8>(p, stream);
+    return launch_q<GROUPED, OUT_INT8, 16>(p, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_rows(const QuantizeArgs &a, cudaStream_t stream) {
+    QParams p{a.X, a.perm, a.rows, a.K, a.k_o, a.Q, a.scale, a.O, a.o_scale};
+    if (a.group > 0)
+        return a.out_int8 ? launch_q_w<true, true>(p, stream) : launch_q_w<true, false>(p, stream);
+    return a.out_int8 ? launch_q_w<false, true>(p, stream) : launch_q_w<false, false>(p, stream);
+}
+
+}  // namespace quik

@@ -1,0 +1,60 @@
+// quik_internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/quik.h"
+
+namespace quik {
+
+constexpr int kMaxK = 32768;       // largest K the quantiser stages in shared memory
+constexpr int kGroup = 128;        // the one supported group width
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s bound on every in-kernel wait
+
+// Reorder + quantise + pack `rows` rows of a [rows, K] fp16 matrix.
+struct QuantizeArgs {
+    const uint16_t *X;
+    const int32_t *perm;
+    int rows, K, k_o, group;
+    bool out_int8;
+    uint8_t *Q;
+    float *scale;
+    void *O;
+    float *o_scale;
+};
+cudaError_t launch_quantize_rows(const QuantizeArgs &a, cudaStream_t stream);
+
+// INT4 x INT4 (+ outlier) product with the dequantising epilogue, or the raw
+// integer sums when acc_dbg is set.
+struct GemmArgs {
+    int M, N, K, k_o, group;
+    bool out_int8;
+    const void *Xq;
+    const float *sx;
+    const void *Xo;
+    const float *sxo;
+    const void *Wq;
+    const float *sw;
+    const void *Wo;
+    const float *swo;
+    const uint16_t *bias;
+    uint16_t *Y;
+    bool debug;          // write the integer sums instead of Y
+    int32_t *acc_dbg;    // [M,N] or [G,M,N] integer sums of the INT4 part (debug only)
+    int32_t *acc_o_dbg;  // INT8 outliers' integer sums (debug only)
+};
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+// Raise `kernel`'s dynamic shared-memory limit on the current device to the
+// device maximum (once per kernel and device); false if dyn_smem_bytes
+// cannot fit or a CUDA call fails.
+bool attribute_set_once(const void *kernel, int dyn_smem_bytes);
+quik_status launch_gemm(const GemmArgs &a, cudaStream_t stream);
+
+quik_status sync_check(cudaStream_t stream);
+quik_status launch_timeout_selftest(uint32_t limit_us, cudaStream_t stream);
+
+}  // namespace quik

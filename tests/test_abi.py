@@ -1,0 +1,91 @@
+"""The C-ABI library without a GPU: it loads, exports every function that
+include/quik.h declares, and its host-side logic (status strings, workspace
+sizes, argument validation that returns before any CUDA call) behaves as the
+header documents."""
+import ctypes
+import subprocess
+
+import pytest
+
+import mixed_precision_quantized_quantize_b200 as q
+from mixed_precision_quantized_quantize_b200 import build as qbuild
+
+
+@pytest.fixture(scope="module")
+def L():
+    qbuild.build()
+    return q.lib()
+
+
+def test_exports_every_header_function(L):
+    names = q.header_functions()
+    assert "quik_linear" in names and "quik_pack_weights" in names
+    out = subprocess.run(["nm", "-D", "--defined-only", q.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for n in names:
+        assert n in exported, n
+        assert hasattr(L, n)
+    # nothing else of ours leaks out of the library
+    assert {e for e in exported if e.startswith("quik")} == set(names)
+
+
+def test_status_strings(L):
+    for s, name in [(q.QUIK_OK, "QUIK_OK"), (q.QUIK_ERR_INVALID_ARG, "QUIK_ERR_INVALID_ARG"),
+                    (q.QUIK_ERR_UNSUPPORTED, "QUIK_ERR_UNSUPPORTED"),
+                    (q.QUIK_ERR_CUDA, "QUIK_ERR_CUDA"), (q.QUIK_ERR_TIMEOUT, "QUIK_ERR_TIMEOUT")]:
+        assert q.status_string(s) == name
+
+
+def _ws(M, N, K, k_o, group=0, outlier=0):
+    return q.quik_workspace_size(q.make_shape(M, N, K, k_o, group, outlier))
+
+
+def test_workspace_size(L):
+    r = lambda b: (b + 255) // 256 * 256
+    # FP16 outliers: codes, per-token scales, fp16 outlier block
+    assert _ws(2048, 4096, 4096, 128) == r(2048 * 3968 // 2) + r(2048 * 4) + r(2048 * 128 * 2)
+    # grouped + INT8 outliers: G scales per token, int8 block, one INT8 scale per token
+    G = (8192 - 128) // 128
+    assert _ws(1024, 22016, 8192, 128, 128, 1) == (r(1024 * 8064 // 2) + r(1024 * G * 4)
+                                                   + r(1024 * 128) + r(1024 * 4))
+    assert _ws(16, 256, 256, 0) == r(16 * 128) + r(16 * 4)
+
+
+@pytest.mark.parametrize("shape", [
+    (0, 16, 256, 32, 0, 0),       # M < 1
+    (16, 0, 256, 32, 0, 0),       # N < 1
+    (16, 16, 256, 300, 0, 0),     # k_o > K
+    (16, 16, 256, -16, 0, 0),     # k_o < 0
+    (16, 16, 272, 32, 0, 0),      # K_i = 240 not a multiple of 32
+    (16, 16, 264, 8, 0, 0),       # k_o not a multiple of 16
+    (16, 16, 320, 32, 128, 0),    # grouped with K_i = 288, not a multiple of 128
+    (16, 16, 256, 0, -1, 0),      # negative group size
+    (16, 16, 256, 0, 0, 5),       # unknown outlier kind
+    (16, 16, 65536, 0, 0, 0),     # K above the supported maximum
+])
+def test_invalid_shapes_rejected(L, shape):
+    assert _ws(*shape) == 0
+    s = q.make_shape(*shape)
+    st = L.quik_quantize_reorder(ctypes.byref(s), None, None, None, None, None, None, None)
+    assert st == q.QUIK_ERR_INVALID_ARG
+
+
+def test_unsupported_group_size(L):
+    s = q.make_shape(16, 16, 256, 0, 64, 0)
+    assert L.quik_gemm(ctypes.byref(s), *([None] * 11)) == q.QUIK_ERR_UNSUPPORTED
+
+
+def test_null_and_misaligned_pointers_rejected(L):
+    s = q.make_shape(16, 16, 256, 32, 0, 0)
+    assert L.quik_quantize_reorder(ctypes.byref(s), None, None, None, None, None, None, None) \
+        == q.QUIK_ERR_INVALID_ARG
+    # misaligned (but otherwise fake, never dereferenced) addresses
+    bad = ctypes.c_void_p(0x1001)
+    good = ctypes.c_void_p(0x1000)
+    assert L.quik_quantize_reorder(ctypes.byref(s), bad, good, good, good, good, None, None) \
+        == q.QUIK_ERR_INVALID_ARG
+    assert L.quik_linear(ctypes.byref(s), good, good, good, good, good, None, None, good, good,
+                         1, None) == q.QUIK_ERR_INVALID_ARG  # workspace too small
+    assert L.quik_selftest_timeout(0, None) == q.QUIK_ERR_INVALID_ARG
+    assert L.quik_selftest_timeout(2000000, None) == q.QUIK_ERR_INVALID_ARG

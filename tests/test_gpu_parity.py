@@ -1,0 +1,233 @@
+"""Parity of the CUDA path with the CPU oracle, element by element.
+
+Codes, scales, outlier blocks and INT32 sums must be bit-exact; fp16 outputs
+must satisfy |y - ref| / max(|ref|, 1e-2) <= 2e-3 (ref in fp64).  Shapes span
+several tiles with ragged tails in M, N and K; degenerate cases (k_o = 0,
+k_o = K, zero rows, exact ties) are included.  All calls go through the C ABI.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import mixed_precision_quantized_quantize_b200 as q
+from mixed_precision_quantized_quantize_b200 import workloads as wl
+
+from helpers import (assert_quant_equal, assert_y_close, gpu_tuple_np, np16, oracle_quant)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    q.lib()
+    oracle.build()
+    yield
+    assert q.quik_sync_check() == q.QUIK_OK
+
+
+# (M, N, K, k_o, group, int8, bias)
+SHAPES = [
+    (16, 256, 256, 32, 0, False, True),      # the tiny layer
+    (200, 300, 640, 64, 0, False, True),     # ragged M, N; K_i = 576 = 4.5 k-blocks
+    (130, 520, 1056, 32, 0, False, False),   # 2 M tiles, 3 N tiles
+    (64, 100, 256, 0, 0, False, True),       # no outliers; N % 8 != 0
+    (64, 256, 256, 256, 0, False, True),     # everything is outlier (FP16 GEMM)
+    (70, 300, 544, 32, 0, True, True),       # INT8 outliers, partial INT8 k-block
+    (150, 260, 1152, 128, 128, True, True),  # groups + INT8 outliers
+    (100, 200, 640, 128, 128, False, False), # groups + FP16 outliers
+    (96, 136, 512, 0, 128, True, True),      # groups, no outliers
+    (48, 144, 128, 128, 128, True, False),   # groups, everything outlier (INT8)
+    (257, 513, 2080, 32, 0, False, True),    # 3 x 3 tiles, long K
+]
+
+
+def _case(M, N, K, k_o, group, int8, bias, seed):
+    cfg = wl.custom_config(M, N, K, k_o, group, int8, bias, outlier_mult=30.0,
+                           student_t=(seed % 2 == 1))
+    return cfg, wl.make_layer(cfg, seed_offset=seed)
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=[str(s) for s in SHAPES])
+def test_quantize_and_pack_bit_exact(shape):
+    M, N, K, k_o, group, int8, bias = shape
+    cfg, d = _case(*shape, seed=7)
+    perm_d = d["perm"].to(DEV)
+    gx = q.quantize_reorder(d["X"].to(DEV), perm_d, k_o, group, int8)
+    gw = q.pack_weights(d["W"].to(DEV), perm_d, k_o, group, int8)
+    torch.cuda.synchronize()
+    assert_quant_equal(gpu_tuple_np(gx), oracle_quant(d["X"], d["perm"], k_o, group, int8), "X")
+    assert_quant_equal(gpu_tuple_np(gw), oracle_quant(d["W"], d["perm"], k_o, group, int8), "W")
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=[str(s) for s in SHAPES])
+def test_int32_sums_bit_exact(shape):
+    M, N, K, k_o, group, int8, bias = shape
+    cfg, d = _case(*shape, seed=11)
+    perm_d = d["perm"].to(DEV)
+    gx = q.quantize_reorder(d["X"].to(DEV), perm_d, k_o, group, int8)
+    gw = q.pack_weights(d["W"].to(DEV), perm_d, k_o, group, int8)
+    acc, acc_o = q.gemm_i32(gx[0], gw[0], K, k_o, group, gx[2], gw[2])
+    torch.cuda.synchronize()
+    ox = oracle_quant(d["X"], d["perm"], k_o, group, int8)
+    ow = oracle_quant(d["W"], d["perm"], k_o, group, int8)
+    if K - k_o > 0:
+        ref = oracle.int_gemm(ox[0], ow[0], group)
+        np.testing.assert_array_equal(acc.cpu().numpy(), ref)
+    if int8 and k_o > 0:
+        ref_o = ox[2].astype(np.int64) @ ow[2].astype(np.int64).T
+        np.testing.assert_array_equal(acc_o.cpu().numpy(), ref_o)
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=[str(s) for s in SHAPES])
+def test_linear_output_within_tolerance(shape):
+    M, N, K, k_o, group, int8, bias = shape
+    cfg, d = _case(*shape, seed=13)
+    perm_d = d["perm"].to(DEV)
+    b = d["bias"].to(DEV) if d["bias"] is not None else None
+    layer = q.QuikLinear(d["W"].to(DEV), perm_d, k_o, group, int8, b)
+    Y = layer(d["X"].to(DEV))
+    # the same result through quantize + gemm as two calls
+    gx = q.quantize_reorder(d["X"].to(DEV), perm_d, k_o, group, int8)
+    Y2 = q.gemm(gx, (layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale), K, k_o, group, b)
+    torch.cuda.synchronize()
+    ref = oracle.layer(np16(d["X"]), np16(d["W"]), d["perm"].numpy(),
+                       None if d["bias"] is None else np16(d["bias"]), k_o, group, int8)["Y"]
+    y = Y.float().cpu().numpy()
+    assert_y_close(y, ref, f"linear {shape}")
+    np.testing.assert_array_equal(Y.cpu().numpy().view(np.uint16), Y2.cpu().numpy().view(np.uint16))
+
+
+def test_zero_rows_and_ties():
+    """All-zero rows give zero scales and codes; exact half-way values round to even."""
+    M, N, K, k_o = 40, 64, 256, 32
+    rng = np.random.default_rng(3)
+    X = rng.standard_normal((M, K)).astype(np.float16)
+    X[3] = 0
+    X[17] = 0
+    # ties: with max|x| = 7 (s = 1), x in {k + 0.5} lands exactly between codes
+    X[5] = np.resize(np.array([7, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.5], np.float16), K)
+    perm = np.arange(K, dtype=np.int32)
+    perm_t = torch.from_numpy(perm)
+    for group, int8 in [(0, False), (0, True), (128, True)]:
+        Kq = K if group == 0 else 128 + k_o  # grouped needs K_i % 128 == 0
+        Xk = np.ascontiguousarray(X[:, :Kq])
+        pk = torch.from_numpy(np.arange(Kq, dtype=np.int32))
+        g = q.quantize_reorder(torch.from_numpy(Xk).to(DEV), pk.to(DEV), k_o, group, int8)
+        torch.cuda.synchronize()
+        assert_quant_equal(gpu_tuple_np(g), oracle.quantize_rows(Xk, pk.numpy(), k_o, group, int8))
+        sc = g[1].cpu().numpy().reshape(M, -1)
+        assert (sc[3] == 0).all() and (sc[17] == 0).all()
+    del perm_t
+
+
+def test_canary_guards_untouched():
+    """Writes stay inside the output buffers: guard bytes around each are unchanged."""
+    M, N, K, k_o = 130, 300, 640, 64
+    cfg, d = _case(M, N, K, k_o, 0, False, True, seed=5)
+    G = 4096
+    pat = 0xA5
+
+    def guarded(nbytes):
+        buf = torch.full((G + nbytes + G,), pat, dtype=torch.uint8, device=DEV)
+        return buf, buf[G:G + nbytes]
+
+    Ki = K - k_o
+    bq, Xq = guarded(M * Ki // 2)
+    bs, sxb = guarded(M * 4)
+    bo, Xob = guarded(M * k_o * 2)
+    by, Yb = guarded(M * N * 2)
+    perm_d = d["perm"].to(DEV)
+    shape = q.make_shape(M, N, K, k_o)
+    q.quik_quantize_reorder(shape, d["X"].to(DEV), perm_d, Xq, sxb.view(torch.float32),
+                            Xob.view(torch.float16), None)
+    gw = q.pack_weights(d["W"].to(DEV), perm_d, k_o)
+    q.quik_gemm(shape, Xq, sxb.view(torch.float32), Xob.view(torch.float16), None, gw[0], gw[1],
+                gw[2], None, d["bias"].to(DEV), Yb.view(torch.float16))
+    torch.cuda.synchronize()
+    for buf in (bq, bs, bo, by):
+        h = buf.cpu().numpy()
+        assert (h[:G] == pat).all() and (h[-G:] == pat).all()
+
+
+def test_timeout_is_reported_without_fault():
+    assert q.quik_sync_check() == q.QUIK_OK
+    q.quik_selftest_timeout(2000)  # 2 ms limit on a barrier nothing completes
+    assert q.quik_sync_check() == q.QUIK_ERR_TIMEOUT
+    assert q.quik_sync_check() == q.QUIK_OK  # the word was cleared
+    # the context is still usable
+    x = torch.ones(4, device=DEV)
+    assert float(x.sum()) == 4.0
+
+
+def test_invalid_arguments_enqueue_nothing():
+    X = torch.zeros((16, 256), dtype=torch.float16, device=DEV)
+    perm = torch.arange(256, dtype=torch.int32, device=DEV)
+    with pytest.raises(q.QuikError) as e:
+        q.quantize_reorder(X, perm, 24)  # k_o not a multiple of 16
+    assert e.value.status == q.QUIK_ERR_INVALID_ARG
+    with pytest.raises(q.QuikError) as e:
+        q.quik_quantize_reorder(q.make_shape(16, 1, 256, 32, 64), X, perm, None, None, None, None)
+    assert e.value.status == q.QUIK_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------------------ full-size layers
+FULL = [
+    ("tiny_16x256x256", None),
+    ("llama7b_attn_2048x4096x4096", None),
+    ("llama7b_up_16x11008x4096", None),
+    ("llama7b_up_256x11008x4096", None),
+    ("llama7b_up_2048x11008x4096", None),
+    ("llama65b_mlp_grouped_1024x22016x8192", None),
+    ("llama7b_down_fused_4096x4096x11008", None),
+]
+
+
+def _samples(M, N, count, seed):
+    rng = np.random.default_rng(seed)
+    ms = rng.integers(0, M, count)
+    ns = rng.integers(0, N, count)
+    # always include the corners and the last row / column
+    extra_m = np.array([0, M - 1, 0, M - 1, M // 2])
+    extra_n = np.array([0, N - 1, N - 1, 0, N // 2])
+    return np.concatenate([ms, extra_m]), np.concatenate([ns, extra_n])
+
+
+@pytest.mark.parametrize("name", [f[0] for f in FULL])
+def test_full_size_layer(name):
+    cfg = wl.CONFIGS[name]
+    d = wl.make_layer(cfg)
+    perm_d = d["perm"].to(DEV)
+    b = d["bias"].to(DEV) if d["bias"] is not None else None
+    X = d["X"].to(DEV)
+    layer = q.QuikLinear(d["W"].to(DEV), perm_d, cfg.k_o, cfg.group, cfg.outlier_int8, b)
+    Y = layer(X)
+    gx = q.quantize_reorder(X, perm_d, cfg.k_o, cfg.group, cfg.outlier_int8)
+    torch.cuda.synchronize()
+    ox = oracle_quant(d["X"], d["perm"], cfg.k_o, cfg.group, cfg.outlier_int8)
+    ow = oracle_quant(d["W"], d["perm"], cfg.k_o, cfg.group, cfg.outlier_int8)
+    # every code, scale and outlier value, activations and weights
+    assert_quant_equal(gpu_tuple_np(gx), ox, f"{name} X")
+    assert_quant_equal(gpu_tuple_np((layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale)), ow,
+                       f"{name} W")
+    # outputs at sampled positions, each computed by the oracle one by one
+    ms, ns = _samples(cfg.M, cfg.N, 3000, seed=1)
+    bias_np = None if d["bias"] is None else np16(d["bias"])
+    ref, ref_acc = oracle.linear_sampled(ox[0], ox[1], ox[2] if cfg.k_o else None, ox[3],
+                                         ow[0], ow[1], ow[2] if cfg.k_o else None, ow[3], bias_np,
+                                         cfg.K, cfg.k_o, cfg.group, ms, ns)
+    y = Y.float().cpu().numpy()[ms, ns]
+    assert_y_close(y, ref, name)
+    # integer sums at sampled positions, from a row/column slice of the same kernel
+    if not cfg.group:
+        rows = np.unique(ms)[:256]
+        cols = np.unique(ns)[:512]
+        r_t = torch.from_numpy(rows).to(DEV)
+        c_t = torch.from_numpy(cols).to(DEV)
+        acc, _ = q.gemm_i32(gx[0][r_t].contiguous(), layer.Wq[c_t].contiguous(), cfg.K, cfg.k_o, 0)
+        acc = acc.cpu().numpy()
+        full = oracle.int_gemm(ox[0][rows], ow[0][cols], 0)
+        np.testing.assert_array_equal(acc, full)
