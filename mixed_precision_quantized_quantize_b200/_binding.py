@@ -16,7 +16,9 @@ import re
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libquik_b200.so")
+# QUIK_LIBRARY may name another build of the same library (e.g. the
+# self-checking variant libquik_b200_checked.so); default: the in-tree build.
+LIB_PATH = os.environ.get("QUIK_LIBRARY") or os.path.join(_HERE, "libquik_b200.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "quik.h")
 
 QUIK_OK, QUIK_ERR_INVALID_ARG, QUIK_ERR_UNSUPPORTED, QUIK_ERR_CUDA, QUIK_ERR_TIMEOUT = range(5)

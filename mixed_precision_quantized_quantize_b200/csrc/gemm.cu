@@ -19,17 +19,17 @@
 // K-permutation on both sides, so every dot product is unchanged.
 //
 // Warp roles in one CTA (one output tile per CTA):
-//   warp 0      TMA producer: packed INT4 tiles of Xq / Wq into a staging
-//               ring; FP16 (or INT8) outlier tiles directly into the operand
-//               ring (128-byte swizzled K-major, the layout the MMA reads);
+//   warp 0      TMA producer: packed INT4 tiles of Xq / Wq into a staging ring;
 //   warp 1      TMEM allocator and the single thread that issues tcgen05.mma;
-//   NT warps    unpack: staging ring -> operand ring (swizzled INT8);
+//   NT warps    fill the operand ring (128-byte swizzled K-major, the layout
+//               the MMA reads) in k-block order: unpacked INT4 k-blocks from
+//               the staging ring, then FP16 (or INT8) outlier tiles by TMA;
 //   NE warps    epilogue: TMEM -> registers -> dequantise -> fp16 stores
 //               (grouped mode: drain each group's INT32 sum while the next
 //               group accumulates in the other TMEM buffer).
-// Every mbarrier wait is bounded (2 s); on expiry the CTA records the error
-// in g_error_word, stops issuing work, waits for its in-flight copies and
-// MMAs, frees TMEM and exits.
+// Every mbarrier wait is bounded (2 s); on expiry the CTA counts the error in
+// g_error_word, stops issuing work, waits for its in-flight copies and MMAs,
+// frees TMEM and exits; other CTAs see the count change and give up too.
 #include <algorithm>
 #include <cstring>
 
@@ -41,6 +41,7 @@
 namespace quik {
 
 __device__ unsigned int g_error_word;
+QUIK_CHECK_DECL
 
 namespace {
 
@@ -86,20 +87,30 @@ struct GemmParams {
     int32_t *acc_dbg, *acc_o_dbg;
 };
 
-__device__ __forceinline__ void set_abort(volatile int *abort_flag) {
-    *abort_flag = 1;
-    atomicOr(&g_error_word, 1u);
+struct AbortState {
+    volatile int *flag;  // this CTA has given up (shared memory)
+    unsigned err0;       // the device error count when this CTA started
+};
+
+__device__ __forceinline__ void set_abort(const AbortState &ab) {
+    *ab.flag = 1;
+    atomicAdd(&g_error_word, 1u);
 }
 
-// Bounded wait that also gives up at once when another role has aborted.
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+// Bounded wait.  Gives up at once when another role of this CTA has given up
+// or when any CTA has recorded an error since this CTA started.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, const AbortState &ab) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
-    while (true) {
+    for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
+        if (*ab.flag) return false;
+        if ((it & 255u) == 255u && *reinterpret_cast<volatile unsigned *>(&g_error_word) != ab.err0) {
+            *ab.flag = 1;
+            return false;
+        }
         if (global_timer_ns() - t0 > kWaitLimitNs) {
-            set_abort(abort_flag);
+            set_abort(ab);
             return false;
         }
     }
@@ -127,6 +138,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __shared__ uint64_t acc_full[2], acc_empty[2], mma_done;
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
+    __shared__ unsigned err0_s;
     __shared__ __align__(16) float epi_sw[NE][C::EPI_COLS];
 
     // 1024-byte aligned base (the swizzle pattern repeats every 1024 bytes)
@@ -136,7 +148,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
-    volatile int *abort_flag = &abort_s;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < SP; ++s) {
@@ -153,6 +164,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         mbar_init(&mma_done, 1);
         abort_s = 0;
+        err0_s = *reinterpret_cast<volatile unsigned *>(&g_error_word);
         fence_barrier_init();
     }
     if (warp == 1) tmem_alloc(&tmem_base_s, C::TMEM_COLS);
@@ -160,6 +172,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_s;
+    const AbortState abort_flag{&abort_s, err0_s};
+    QUIK_CHECK((smem_base & 1023u) == 0 && smem_base + C::SMEM - 1024 <= 232448u, 12);
+    QUIK_CHECK((tmem & 0xFFFFu) + C::TMEM_COLS <= 512u && (tmem >> 16) == 0, 13);
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -168,13 +183,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 tma_prefetch_desc(&tm_xq);
                 tma_prefetch_desc(&tm_wq);
             }
-            if (p.nkb_o > 0) {
-                tma_prefetch_desc(&tm_xo);
-                tma_prefetch_desc(&tm_wo);
-            }
-            int last_pk[SP], last_op[SU];
+            int last_pk[SP];
             for (int s = 0; s < SP; ++s) last_pk[s] = -1;
-            for (int s = 0; s < SU; ++s) last_op[s] = -1;
             bool ok = true;
             for (int kb = 0; kb < p.nkb_i && ok; ++kb) {
                 const int s = kb % SP;
@@ -185,23 +195,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 tma_load_2d(dst + BM * PK_ROW, &tm_wq, kb * PK_ROW, n0, &pk_full[s]);
                 last_pk[s] = kb;
             }
-            // outlier k-blocks: 64 fp16 (or 128 int8) channels = 128 bytes per row
-            for (int ko = 0; ko < p.nkb_o && ok; ++ko) {
-                const int kb = p.nkb_i + ko, s = kb % SU;
-                if (!(ok = wait_bar(&op_empty[s], ((kb / SU) & 1) ^ 1, abort_flag))) break;
-                uint8_t *dst = smem + C::OP_OFF + s * C::OP_STAGE;
-                const int x = C::OUT_INT8 ? ko * 128 : ko * 64;
-                mbar_arrive_expect_tx(&op_full[s], C::OP_STAGE);
-                for (int a = 1; a < NT; ++a) mbar_arrive(&op_full[s]);  // count NT per phase
-                tma_load_2d(dst, &tm_xo, x, m0, &op_full[s]);
-                tma_load_2d(dst + BM * OP_ROW, &tm_wo, x, n0, &op_full[s]);
-                last_op[s] = kb;
-            }
             // never leave the CTA with a bulk copy still writing its shared memory
             for (int s = 0; s < SP; ++s)
                 if (last_pk[s] >= 0) mbar_wait_bounded(&pk_full[s], (last_pk[s] / SP) & 1, kWaitLimitNs);
-            for (int s = 0; s < SU; ++s)
-                if (last_op[s] >= 0) mbar_wait_bounded(&op_full[s], (last_op[s] / SU) & 1, kWaitLimitNs);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -267,9 +263,39 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         __syncwarp();
     } else if (warp < 2 + NT) {
         // ------------------------------------------------------------ unpack INT4 -> INT8
+        // These warps fill every operand stage in k-block order (unpacked INT4
+        // k-blocks, then the outlier k-blocks by TMA), so each of their waits
+        // is for the current or the previous phase of its barrier, the
+        // condition under which a parity wait is exact.
         const int t = threadIdx.x - 64;
-        for (int kb = 0; kb < p.nkb_i; ++kb) {
+        int last_op[SU];
+        for (int s = 0; s < SU; ++s) last_op[s] = -1;
+        if (t == 0 && p.nkb_o > 0) {
+            tma_prefetch_desc(&tm_xo);
+            tma_prefetch_desc(&tm_wo);
+        }
+        for (int kb = 0; kb < p.nkb_i + p.nkb_o; ++kb) {
             const int sp = kb % SP, su = kb % SU;
+            if (kb >= p.nkb_i) {
+                // outlier k-block: 64 fp16 (or 128 int8) channels = 128 bytes per row
+                const bool ok = wait_bar(&op_empty[su], ((kb / SU) & 1) ^ 1, abort_flag);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                if (lane == 0) {
+                    if (t == 0) {
+                        const int ko = kb - p.nkb_i;
+                        const int x = C::OUT_INT8 ? ko * 128 : ko * 64;
+                        uint8_t *dst = smem + C::OP_OFF + su * C::OP_STAGE;
+                        mbar_arrive_expect_tx(&op_full[su], C::OP_STAGE);
+                        tma_load_2d(dst, &tm_xo, x, m0, &op_full[su]);
+                        tma_load_2d(dst + BM * OP_ROW, &tm_wo, x, n0, &op_full[su]);
+                        last_op[su] = kb;
+                    } else {
+                        mbar_arrive(&op_full[su]);
+                    }
+                }
+                __syncwarp();
+                continue;
+            }
             bool ok = wait_bar(&pk_full[sp], (kb / SP) & 1, abort_flag) &&
                       wait_bar(&op_empty[su], ((kb / SU) & 1) ^ 1, abort_flag);
             if (!__all_sync(0xffffffffu, ok)) break;
@@ -280,6 +306,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 // A rows [0, BM) then B rows [BM, BM+BN): one matrix of BM+BN rows
                 const int c = t + i * NT * 32;
                 const int r = c >> 2, ch = c & 3;
+                if (!QUIK_CHECK(r < BM + C::BN && t >= 0 && t < NT * 32, 10)) continue;
                 const uint4 v = *reinterpret_cast<const uint4 *>(pk + r * PK_ROW + ch * 16);
                 uint4 lo, hi;
                 lo.x = (v.x << 4) & 0xF0F0F0F0u;  hi.x = v.x & 0xF0F0F0F0u;
@@ -297,6 +324,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 mbar_arrive(&op_full[su]);
             }
         }
+        // never leave the CTA with a bulk copy still writing its shared memory
+        if (t == 0)
+            for (int s = 0; s < SU; ++s)
+                if (last_op[s] >= 0) mbar_wait_bounded(&op_full[s], (last_op[s] / SU) & 1, kWaitLimitNs);
     } else {
         // ------------------------------------------------------------ epilogue
         const int ew = warp - (2 + NT);
@@ -311,7 +342,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             bool ok = wait_bar(&acc_full[0], 0, abort_flag);
             if (__all_sync(0xffffffffu, ok)) {
                 tc_fence_after();
-                const float sxr = (row_ok && p.Ki > 0) ? p.sx[row] : 0.0f;
+                const float sxr = (row_ok && p.Ki > 0 && QUIK_CHECK(row < p.M, 15)) ? p.sx[row] : 0.0f;
                 const float sxo = (row_ok && C::OUT_INT8 && p.nkb_o > 0) ? p.sxo[row] : 0.0f;
                 for (int cc = 0; cc < C::EPI_COLS; cc += 32) {
                     const int nb = n0 + col0 + cc;
@@ -338,7 +369,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     {
                         const int n = nb + lane;
                         float swv = 0.0f;
-                        if (n < p.N) {
+                        if (n < p.N && QUIK_CHECK(cc + lane < C::EPI_COLS, 16)) {
                             if (p.Ki > 0) swv = p.sw[n];
                         }
                         ssw[cc + lane] = swv;
@@ -398,10 +429,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
                 for (int cc = 0; cc < C::EPI_COLS; cc += 32) {
                     const int n = n0 + col0 + cc + lane;
-                    ssw[cc + lane] = n < p.N ? p.sw[(size_t)n * p.G + g] : 0.0f;
+                    ssw[cc + lane] = (n < p.N && QUIK_CHECK(g < p.G && cc + lane < C::EPI_COLS, 16))
+                                         ? p.sw[(size_t)n * p.G + g] : 0.0f;
                 }
                 // fold the 16 x 16 operand scaling (2^-8) into the row factor
-                const float sxg = row_ok ? p.sx[(size_t)row * p.G + g] * (1.0f / 256.0f) : 0.0f;
+                const float sxg = (row_ok && QUIK_CHECK(g < p.G, 15))
+                                      ? p.sx[(size_t)row * p.G + g] * (1.0f / 256.0f) : 0.0f;
                 __syncwarp();
                 ok = wait_bar(&acc_full[b], (g >> 1) & 1, abort_flag);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -409,6 +442,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
                 for (int cc = 0; cc < C::EPI_COLS; cc += 32) {
                     uint32_t a[32];
+                    QUIK_CHECK(b * BN + col0 + cc + 32 <= C::TMEM_COLS, 14);
                     tmem_ld_32x32b_x32(t_lane + b * BN + col0 + cc, a);
                     tmem_ld_wait();
                     if (C::DEBUG) {
@@ -606,7 +640,7 @@ __global__ void timeout_selftest_kernel(uint64_t limit_ns) {
         fence_barrier_init();
     }
     __syncthreads();
-    if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, limit_ns)) atomicOr(&g_error_word, 1u);
+    if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, limit_ns)) atomicAdd(&g_error_word, 1u);
     __syncthreads();
 }
 
@@ -620,6 +654,14 @@ quik_status launch_timeout_selftest(uint32_t limit_us, cudaStream_t stream) {
     timeout_selftest_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(limit_us) * 1000ull);
     return cudaGetLastError() == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
 }
+
+#ifdef QUIK_CHECKS
+extern "C" __attribute__((visibility("default"))) unsigned long long qchk_gemm_word() {
+    unsigned long long v = 0;
+    cudaMemcpyFromSymbol(&v, g_check_word, sizeof(v));
+    return v;
+}
+#endif
 
 quik_status sync_check(cudaStream_t stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return QUIK_ERR_CUDA;

@@ -26,6 +26,9 @@
 #include "quik_internal.h"
 
 namespace quik {
+
+QUIK_CHECK_DECL
+
 namespace {
 
 constexpr int kQThreads = 256;
@@ -92,11 +95,15 @@ __global__ void __launch_bounds__(kQThreads) quantize_rows_kernel(QParams p) {
         for (int i = 0; i < MAXW; ++i) {
             const int w = tid + i * kQThreads;
             wmax[i] = 0.0f;
-            if (w < nwords) {
+            if (w < nwords && QUIK_CHECK(8 * w + 8 <= Kp, 2)) {
                 const uint4 ix = *reinterpret_cast<const uint4 *>(perm_s + 8 * w);
                 const uint32_t idx[4] = {ix.x, ix.y, ix.z, ix.w};
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
+                    if (!QUIK_CHECK((idx[k] & 0xffffu) < (uint32_t)K && (idx[k] >> 16) < (uint32_t)K, 1)) {
+                        v[i][k] = 0;
+                        continue;
+                    }
                     const uint16_t a = row_s[idx[k] & 0xffffu], b = row_s[idx[k] >> 16];
                     v[i][k] = static_cast<uint32_t>(a) | (static_cast<uint32_t>(b) << 16);
                     wmax[i] = fmaxf(wmax[i], fmaxf(fabsf(h2f(a)), fabsf(h2f(b))));
@@ -114,7 +121,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_rows_kernel(QParams p) {
                 for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
                 s[i] = __fdiv_rn(m, 7.0f);
                 const int w = tid + i * kQThreads;
-                if (w < nwords && (lane & 15) == 0)
+                if (w < nwords && (lane & 15) == 0 && QUIK_CHECK(w / 16 < G, 3))
                     p.scale[static_cast<size_t>(row) * G + w / 16] = s[i];
             }
         } else {
@@ -138,7 +145,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_rows_kernel(QParams p) {
 #pragma unroll
         for (int i = 0; i < MAXW; ++i) {
             const int w = tid + i * kQThreads;
-            if (w < nwords) {
+            if (w < nwords && QUIK_CHECK(4 * w + 4 <= Ki / 2, 4)) {
                 const float rs = s[i] != 0.0f ? __frcp_rn(s[i]) : 0.0f;
                 uint32_t word = 0;
 #pragma unroll
@@ -156,7 +163,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_rows_kernel(QParams p) {
         if (p.k_o > 0) {
             if (!OUT_INT8) {
                 uint16_t *o = static_cast<uint16_t *>(p.O) + static_cast<size_t>(row) * p.k_o;
-                for (int i = tid; i < p.k_o; i += kQThreads) o[i] = row_s[perm_s[Ki + i]];
+                for (int i = tid; i < p.k_o; i += kQThreads)
+                    if (QUIK_CHECK(perm_s[Ki + i] < K, 5)) o[i] = row_s[perm_s[Ki + i]];
             } else {
                 float m = 0.0f;
                 for (int i = tid; i < p.k_o; i += kQThreads)
@@ -213,3 +221,11 @@ cudaError_t launch_quantize_rows(const QuantizeArgs &a, cudaStream_t stream) {
 }
 
 }  // namespace quik
+
+#ifdef QUIK_CHECKS
+extern "C" __attribute__((visibility("default"))) unsigned long long qchk_quantize_word() {
+    unsigned long long v = 0;
+    cudaMemcpyFromSymbol(&v, quik::g_check_word, sizeof(v));
+    return v;
+}
+#endif

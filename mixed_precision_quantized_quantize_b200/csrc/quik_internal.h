@@ -7,6 +7,22 @@
 
 #include "../../include/quik.h"
 
+// Optional self-checks (build with -DQUIK_CHECKS): bounds and alignment of
+// every computed index are verified before use; the first violation is
+// recorded as (tag << 32 | source line) in a per-file device word and the
+// access is skipped.  Off in normal builds (the macro folds to `true`).
+#ifdef QUIK_CHECKS
+#define QUIK_CHECK_DECL __device__ unsigned long long g_check_word;
+#define QUIK_CHECK(cond, tag)                                                                  \
+    ((cond) ? true                                                                             \
+            : (atomicCAS(&g_check_word, 0ull,                                                  \
+                         (static_cast<unsigned long long>(tag) << 32) | __LINE__),             \
+               false))
+#else
+#define QUIK_CHECK_DECL
+#define QUIK_CHECK(cond, tag) true
+#endif
+
 namespace quik {
 
 constexpr int kMaxK = 32768;       // largest K the quantiser stages in shared memory

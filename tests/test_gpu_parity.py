@@ -42,6 +42,10 @@ SHAPES = [
     (96, 136, 512, 0, 128, True, True),      # groups, no outliers
     (48, 144, 128, 128, 128, True, False),   # groups, everything outlier (INT8)
     (257, 513, 2080, 32, 0, False, True),    # 3 x 3 tiles, long K
+    # long K: the operand ring wraps many times before the outlier k-blocks
+    # (a producer running ahead must never alias a barrier phase)
+    (200, 300, 8320, 128, 128, True, True),  # 64 groups + INT8 outliers
+    (130, 260, 8256, 64, 0, False, True),    # 64 INT4 k-blocks + FP16 outliers
 ]
 
 
