@@ -146,6 +146,37 @@ QUIK_API quik_status quik_linear(const quik_shape *shape, const void *X_f16, con
                         void *workspace, size_t workspace_bytes, quik_stream_t stream);
 
 /*
+ * quik_linear_noalloc -- quik_linear for callers that cannot allocate device
+ * memory.  (No counterpart in the papers; an addition of this library.)
+ *
+ * Some callers have no way to provide quik_linear's workspace: a host
+ * framework that owns every device allocation through a fixed memory plan and
+ * hands its plugins no workspace, or a latency-critical path that must not
+ * call cudaMalloc, which may synchronise the whole device.  This entry point
+ * takes the same arguments as quik_linear minus the workspace and uses a
+ * workspace of QUIK_NOALLOC_SCRATCH_BYTES that the library keeps in its own
+ * device data segment: every GPU that loads the library holds it until the
+ * process exits.  No call allocates or frees anything.
+ *   - Shapes whose quik_workspace_size exceeds QUIK_NOALLOC_SCRATCH_BYTES
+ *     return QUIK_ERR_UNSUPPORTED (use quik_linear with your own workspace).
+ *   - All calls on a device share that one workspace: two calls whose work
+ *     overlaps on the GPU (different streams, no ordering between them) race
+ *     and may corrupt each other's results.  Order them on one stream.
+ *   - The workspace keeps the last call's contents; each call rewrites every
+ *     byte it reads, so no clearing is needed.
+ *   - The first call on each device looks up the workspace's device address
+ *     (with that device current) and caches it; make that first call before
+ *     any stream capture.
+ * Errors and argument rules are those of quik_linear.
+ */
+#define QUIK_NOALLOC_SCRATCH_BYTES (32u << 20)
+QUIK_API quik_status quik_linear_noalloc(const quik_shape *shape, const void *X_f16,
+                                         const int32_t *perm, const void *Wq,
+                                         const float *w_scale, const void *Wo,
+                                         const float *wo_scale, const void *bias_f16,
+                                         void *Y_f16, quik_stream_t stream);
+
+/*
  * quik_gemm_i32_debug -- test entry: the exact integer sums of the INT4 part
  * as computed by the tensor-core main loop, acc [M, N] int32 (or [G, M, N]
  * with groups), and for INT8 outliers the outlier block's integer sums

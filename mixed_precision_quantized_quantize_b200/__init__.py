@@ -27,6 +27,7 @@ from ._binding import (  # noqa: F401
     quik_gemm,
     quik_gemm_i32_debug,
     quik_linear,
+    quik_linear_noalloc,
     quik_pack_weights,
     quik_quantize_reorder,
     quik_selftest_timeout,

@@ -46,6 +46,7 @@ _SIGS = {
     "quik_pack_weights": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P]),
     "quik_gemm": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "quik_linear": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "quik_linear_noalloc": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "quik_gemm_i32_debug": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P]),
     "quik_sync_check": (ctypes.c_int, [_P]),
     "quik_selftest_timeout": (ctypes.c_int, [ctypes.c_uint32, _P]),
@@ -144,6 +145,17 @@ def quik_linear(shape, X, perm, Wq, w_scale, Wo, wo_scale, bias, Y, workspace, s
         _ptr(Wo, None, "Wo"), _ptr(wo_scale, torch.float32, "wo_scale"),
         _ptr(bias, torch.float16, "bias"), _ptr(Y, torch.float16, "Y"),
         _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)), "quik_linear")
+
+
+def quik_linear_noalloc(shape, X, perm, Wq, w_scale, Wo, wo_scale, bias, Y, stream=None):
+    """quik_linear on the library's own fixed workspace (for callers that cannot
+    allocate device memory); see include/quik.h."""
+    _check(lib().quik_linear_noalloc(
+        ctypes.byref(shape), _ptr(X, torch.float16, "X"), _ptr(perm, torch.int32, "perm"),
+        _ptr(Wq, torch.uint8, "Wq"), _ptr(w_scale, torch.float32, "w_scale"),
+        _ptr(Wo, None, "Wo"), _ptr(wo_scale, torch.float32, "wo_scale"),
+        _ptr(bias, torch.float16, "bias"), _ptr(Y, torch.float16, "Y"), _stream(stream)),
+        "quik_linear_noalloc")
 
 
 def quik_gemm_i32_debug(shape, Xq, Wq, Xo, Wo, acc, acc_outlier, stream=None):

@@ -52,17 +52,39 @@ constexpr int KB = 128;       // INT4 codes per k-block = one scale group
 constexpr int PK_ROW = 64;    // packed bytes per row per k-block
 constexpr int OP_ROW = 128;   // unpacked bytes per row per k-block (one swizzle row)
 
-template <int BN_, bool GROUPED_, bool OUT_INT8_, bool DEBUG_>
+// Pipeline shape of the per-channel-scale kernel (compile-time tuning knobs).
+#ifndef QUIK_NG_BN
+#define QUIK_NG_BN 256  // tile columns
+#endif
+#ifndef QUIK_NG_NT
+#define QUIK_NG_NT 8    // unpack warps
+#endif
+#ifndef QUIK_NG_NE
+#define QUIK_NG_NE 4    // epilogue warps
+#endif
+#ifndef QUIK_NG_SP
+#define QUIK_NG_SP 3    // packed staging stages
+#endif
+#ifndef QUIK_NG_SU
+#define QUIK_NG_SU 3    // operand stages
+#endif
+#ifndef QUIK_NG_MINB
+#define QUIK_NG_MINB 1  // CTAs resident per SM
+#endif
+
+template <int BN_, bool GROUPED_, bool OUT_INT8_, bool DEBUG_, int NT_, int NE_, int SP_, int SU_,
+          int MINB_>
 struct Cfg {
     static constexpr int BN = BN_;
     static constexpr bool GROUPED = GROUPED_;
     static constexpr bool OUT_INT8 = OUT_INT8_;
     static constexpr bool DEBUG = DEBUG_;
-    static constexpr int NT = GROUPED ? 4 : 8;  // unpack warps
-    static constexpr int NE = GROUPED ? 8 : 4;  // epilogue warps (multiple of 4)
+    static constexpr int NT = NT_;  // unpack warps
+    static constexpr int NE = NE_;  // epilogue warps (multiple of 4)
+    static constexpr int MINB = MINB_;
     static constexpr int THREADS = (2 + NT + NE) * 32;
-    static constexpr int SP = GROUPED ? 4 : 3;  // packed staging stages
-    static constexpr int SU = GROUPED ? 4 : 3;  // operand stages
+    static constexpr int SP = SP_;  // packed staging stages
+    static constexpr int SU = SU_;  // operand stages
     static constexpr int PK_STAGE = (BM + BN) * PK_ROW;
     static constexpr int OP_STAGE = (BM + BN) * OP_ROW;
     static constexpr int OP_OFF = 0;
@@ -75,9 +97,17 @@ struct Cfg {
     static constexpr int CHUNKS_PER_THREAD = CHUNKS / (NT * 32);
     static constexpr int EPI_COLS = BN / (NE / 4);                // columns per epilogue warp
     static_assert(CHUNKS % (NT * 32) == 0, "unpack work must split evenly");
+    static_assert(NE % 4 == 0, "epilogue warps cover the four TMEM lane quadrants");
+    static_assert(TMEM_COLS * MINB <= 512, "TMEM of all resident CTAs");
     static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation is a power of two");
     static_assert(SMEM <= 232448, "shared memory budget");
 };
+
+template <bool OUT_INT8, bool DEBUG>
+using CfgChannel = Cfg<QUIK_NG_BN, false, OUT_INT8, DEBUG, QUIK_NG_NT, QUIK_NG_NE, QUIK_NG_SP,
+                       QUIK_NG_SU, QUIK_NG_MINB>;
+template <bool OUT_INT8, bool DEBUG>
+using CfgGroup = Cfg<128, true, OUT_INT8, DEBUG, 4, 8, 4, 4, 1>;
 
 struct GemmParams {
     int M, N, Ki, k_o, nkb_i, nkb_o, G;
@@ -127,7 +157,7 @@ __device__ __forceinline__ float small_int_to_float(int32_t v) {
 }
 
 template <class C>
-__global__ void __launch_bounds__(C::THREADS, 1)
+__global__ void __launch_bounds__(C::THREADS, C::MINB)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tm_xq,
                      const __grid_constant__ CUtensorMap tm_wq,
                      const __grid_constant__ CUtensorMap tm_xo,
@@ -173,8 +203,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = tmem_base_s;
     const AbortState abort_flag{&abort_s, err0_s};
-    QUIK_CHECK((smem_base & 1023u) == 0 && smem_base + C::SMEM - 1024 <= 232448u, 12);
-    QUIK_CHECK((tmem & 0xFFFFu) + C::TMEM_COLS <= 512u && (tmem >> 16) == 0, 13);
+    (void)QUIK_CHECK((smem_base & 1023u) == 0 && smem_base + C::SMEM - 1024 <= 232448u, 12);
+    (void)QUIK_CHECK((tmem & 0xFFFFu) + C::TMEM_COLS <= 512u && (tmem >> 16) == 0, 13);
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -442,7 +472,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
                 for (int cc = 0; cc < C::EPI_COLS; cc += 32) {
                     uint32_t a[32];
-                    QUIK_CHECK(b * BN + col0 + cc + 32 <= C::TMEM_COLS, 14);
+                    (void)QUIK_CHECK(b * BN + col0 + cc + 32 <= C::TMEM_COLS, 14);
                     tmem_ld_32x32b_x32(t_lane + b * BN + col0 + cc, a);
                     tmem_ld_wait();
                     if (C::DEBUG) {
@@ -625,10 +655,10 @@ quik_status run(const GemmArgs &a, cudaStream_t stream) {
 template <bool DEBUG>
 quik_status dispatch(const GemmArgs &a, cudaStream_t stream) {
     if (a.group > 0)
-        return a.out_int8 ? run<Cfg<128, true, true, DEBUG>>(a, stream)
-                          : run<Cfg<128, true, false, DEBUG>>(a, stream);
-    return a.out_int8 ? run<Cfg<256, false, true, DEBUG>>(a, stream)
-                      : run<Cfg<256, false, false, DEBUG>>(a, stream);
+        return a.out_int8 ? run<CfgGroup<true, DEBUG>>(a, stream)
+                          : run<CfgGroup<false, DEBUG>>(a, stream);
+    return a.out_int8 ? run<CfgChannel<true, DEBUG>>(a, stream)
+                      : run<CfgChannel<false, DEBUG>>(a, stream);
 }
 
 // A CTA waiting on a barrier that nothing completes: exercises the bounded

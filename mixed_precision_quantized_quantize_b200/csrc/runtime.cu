@@ -3,8 +3,6 @@
 // library's only mutable host state; both are guarded for concurrent callers.
 #include <atomic>
 #include <mutex>
-#include <set>
-#include <utility>
 
 #include "quik_internal.h"
 
@@ -13,8 +11,13 @@ namespace quik {
 namespace {
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
+// (kernel, device) pairs already configured; a fixed table, so that launches
+// never allocate host memory either.
+constexpr int kMaxKernels = 64;
 std::mutex g_attr_mu;
-std::set<std::pair<const void *, int>> g_attr_done;  // (kernel, device)
+const void *g_attr_kernel[kMaxKernels];
+unsigned long long g_attr_devmask[kMaxKernels];
+int g_attr_n = 0;
 }  // namespace
 
 int sm_count() {
@@ -32,8 +35,18 @@ int sm_count() {
 bool attribute_set_once(const void *kernel, int dyn_smem_bytes) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (dev >= kMaxDevices) return false;
     std::lock_guard<std::mutex> lock(g_attr_mu);
-    if (g_attr_done.count({kernel, dev})) return true;
+    int slot = -1;
+    for (int i = 0; i < g_attr_n; ++i)
+        if (g_attr_kernel[i] == kernel) slot = i;
+    if (slot >= 0 && (g_attr_devmask[slot] >> dev) & 1ull) return true;
+    if (slot < 0) {
+        if (g_attr_n == kMaxKernels) return false;
+        slot = g_attr_n++;
+        g_attr_kernel[slot] = kernel;
+        g_attr_devmask[slot] = 0;
+    }
     // raise to the largest size any launch of this kernel uses
     int max_optin = 0;
     if (cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
@@ -46,7 +59,7 @@ bool attribute_set_once(const void *kernel, int dyn_smem_bytes) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, want) !=
         cudaSuccess)
         return false;
-    g_attr_done.insert({kernel, dev});
+    g_attr_devmask[slot] |= 1ull << dev;
     return true;
 }
 
