@@ -43,6 +43,25 @@ namespace quik {
 __device__ unsigned int g_error_word;
 QUIK_CHECK_DECL
 
+// Optional pipeline timeline (build with -DQUIK_TRACE): SM clock stamps of
+// each role's per-k-block events for the first two CTAs of a launch.
+#ifdef QUIK_TRACE
+constexpr int kTraceCtas = 2, kTraceEvents = 12, kTraceKb = 96;
+__device__ unsigned long long g_trace[kTraceCtas][kTraceEvents][kTraceKb];
+#define QUIK_TRACE_AT(ev, kb)                                                                   \
+    do {                                                                                        \
+        const int _c = blockIdx.x + blockIdx.y * gridDim.x;                                     \
+        if (_c < kTraceCtas && (kb) >= 0 && (kb) < kTraceKb) g_trace[_c][ev][kb] = clock64();   \
+    } while (0)
+#else
+#define QUIK_TRACE_AT(ev, kb) \
+    do {                      \
+    } while (0)
+#endif
+// events: 0 producer issued packed k-block (TMEM-A kernel: last B warp arrived),
+// 1 unpack start (after waits), 2 unpack done (TMEM-A kernel: last A warp), 3 MMA issued k-block, 4 epilogue saw accumulator,
+// 5 epilogue done, 6 CTA start, 7 CTA end
+
 namespace {
 
 using namespace ptx;
@@ -197,6 +216,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
         err0_s = *reinterpret_cast<volatile unsigned *>(&g_error_word);
         fence_barrier_init();
     }
+    if (threadIdx.x == 0) QUIK_TRACE_AT(6, 0);
     if (warp == 1) tmem_alloc(&tmem_base_s, C::TMEM_COLS);
     tc_fence_before();
     __syncthreads();
@@ -224,6 +244,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 tma_load_2d(dst, &tm_xq, kb * PK_ROW, m0, &pk_full[s]);
                 tma_load_2d(dst + BM * PK_ROW, &tm_wq, kb * PK_ROW, n0, &pk_full[s]);
                 last_pk[s] = kb;
+                QUIK_TRACE_AT(0, kb);
             }
             // never leave the CTA with a bulk copy still writing its shared memory
             for (int s = 0; s < SP; ++s)
@@ -246,6 +267,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 }
                 if (!(ok = wait_bar(&op_full[s], (kb / SU) & 1, abort_flag))) break;
                 tc_fence_after();
+                QUIK_TRACE_AT(3, kb);
                 const uint32_t a_addr = smem_base + C::OP_OFF + s * C::OP_STAGE;
                 const uint32_t b_addr = a_addr + BM * OP_ROW;
 #pragma unroll
@@ -329,6 +351,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
             bool ok = wait_bar(&pk_full[sp], (kb / SP) & 1, abort_flag) &&
                       wait_bar(&op_empty[su], ((kb / SU) & 1) ^ 1, abort_flag);
             if (!__all_sync(0xffffffffu, ok)) break;
+            if (t == 0) QUIK_TRACE_AT(1, kb);
             const uint8_t *pk = smem + C::PK_OFF + sp * C::PK_STAGE;
             uint8_t *op = smem + C::OP_OFF + su * C::OP_STAGE;
 #pragma unroll
@@ -353,6 +376,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 mbar_arrive(&pk_empty[sp]);
                 mbar_arrive(&op_full[su]);
             }
+            if (t == 0) QUIK_TRACE_AT(2, kb);
         }
         // never leave the CTA with a bulk copy still writing its shared memory
         if (t == 0)
@@ -369,9 +393,16 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
         float *ssw = epi_sw[ew];
 
         if (!C::GROUPED) {
+            // this warp's per-column weight scales, loaded before the accumulator is ready
+            for (int c = lane; c < C::EPI_COLS; c += 32) {
+                const int n = n0 + col0 + c;
+                ssw[c] = (n < p.N && p.Ki > 0) ? p.sw[n] : 0.0f;
+            }
+            __syncwarp();
             bool ok = wait_bar(&acc_full[0], 0, abort_flag);
             if (__all_sync(0xffffffffu, ok)) {
                 tc_fence_after();
+                if (ew == 0 && lane == 0) QUIK_TRACE_AT(4, 0);
                 const float sxr = (row_ok && p.Ki > 0 && QUIK_CHECK(row < p.M, 15)) ? p.sx[row] : 0.0f;
                 const float sxo = (row_ok && C::OUT_INT8 && p.nkb_o > 0) ? p.sxo[row] : 0.0f;
                 for (int cc = 0; cc < C::EPI_COLS; cc += 32) {
@@ -395,16 +426,6 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                         }
                         continue;
                     }
-                    // per-column factors, staged once per chunk in this warp's slot
-                    {
-                        const int n = nb + lane;
-                        float swv = 0.0f;
-                        if (n < p.N && QUIK_CHECK(cc + lane < C::EPI_COLS, 16)) {
-                            if (p.Ki > 0) swv = p.sw[n];
-                        }
-                        ssw[cc + lane] = swv;
-                    }
-                    __syncwarp();
                     uint32_t packed[16];
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
@@ -414,7 +435,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                             const int jj = j + h, n = nb + jj;
                             float v = 0.0f;
                             if (p.Ki > 0)
-                                v = static_cast<float>(static_cast<int32_t>(a[jj]) >> 8) * sxr * ssw[cc + jj];
+                                v = small_int_to_float(static_cast<int32_t>(a[jj]) >> 8) * sxr * ssw[cc + jj];
                             if (p.nkb_o > 0) {
                                 if (C::OUT_INT8) {
                                     const float swo = n < p.N ? __ldg(p.swo + n) : 0.0f;
@@ -446,6 +467,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                     __syncwarp();
                 }
                 tc_fence_before();
+                if (ew == 0 && lane == 0) QUIK_TRACE_AT(5, 0);
             }
         } else {
             // grouped: running fp32 sums of this warp's EPI_COLS columns, in registers
@@ -559,9 +581,400 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
     // ---------------------------------------------------------------- teardown
     tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0) QUIK_TRACE_AT(7, 0);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ============================================================================
+// Per-channel-scale kernel, activations (operand A) in tensor memory.
+//
+// Shared-memory bandwidth bounds the kernel above: per 128-code k-block of a
+// 128 x 256 tile it moves 24 KB of packed codes in by TMA, reads them back,
+// writes 48 KB of unpacked bytes and the MMA reads those 48 KB again
+// (144 KB per 4 Mi multiply-adds against ~128 B/clk).  Here the A rows never
+// touch shared memory: A threads load their row's packed codes from global
+// memory (several k-blocks ahead), unpack in registers and write tensor
+// memory with tcgen05.st; tcgen05.mma reads A from TMEM.  Only B goes through
+// shared memory (TMA staging 16 KB, read back 16 KB, unpacked 32 KB, MMA
+// reads 32 KB: 96 KB per k-block).  The B unpack warps keep no global loads
+// in flight, so the proxy fence that publishes their stores to the MMA only
+// waits for their own shared-memory stores.
+//
+//   warp 0        TMEM allocator; lane 0 issues the MMAs
+//   warp 1        TMA producer of the packed staging ring, in unit order:
+//                 one unit per INT4 k-block (the B tile, 256 rows x 64 B),
+//                 three per outlier k-block (two halves of the Wo tile, then
+//                 the Xo tile)
+//   warps 2-5     A: one thread per tile row (= its TMEM lane): load, unpack,
+//                 tcgen05.st 32 columns per k-block; then the epilogue
+//   warps 6-13    B: staging -> 128-byte swizzled K-major operand stage
+//                 (unpacked INT4 k-blocks; copied outlier tiles)
+// TMEM: INT32 sums in columns [0,256); A stages [256, 256+32 S) while the INT4
+// k-blocks run; after them (and a drain of the MMA pipe) the outlier sums in
+// [256, 512), with both outlier operands in shared memory.
+namespace ts {
+constexpr int BN = 256;
+constexpr int S = 3;                  // operand stages
+constexpr int SP = 4;                 // packed staging stages
+constexpr int NA = 4, NB = 8;         // A warps, B warps
+constexpr int THREADS = (2 + NA + NB) * 32;
+constexpr int B_BYTES = BN * OP_ROW;  // unpacked B k-block / outlier W tile
+constexpr int XO_BYTES = BM * OP_ROW; // outlier X tile
+constexpr int STAGE = B_BYTES + XO_BYTES;
+constexpr int PK_BYTES = BN * PK_ROW; // one staging unit (= BM * OP_ROW)
+constexpr int PK_OFF = S * STAGE;
+constexpr int SMEM = PK_OFF + SP * PK_BYTES + 1024;
+constexpr int ACC_COL = 0, A_COL = 256, O_COL = 256, TMEM_COLS = 512;
+constexpr int PF = 4;                 // k-blocks of A loads in flight per thread
+static_assert(PK_BYTES == XO_BYTES, "an Xo tile fills one staging unit");
+static_assert(A_COL + 32 * S <= TMEM_COLS, "A stages fit in tensor memory");
+static_assert(SMEM <= 232448, "shared memory budget");
+}  // namespace ts
+
+__device__ __forceinline__ void unpack16(const uint4 v, uint4 &lo, uint4 &hi) {
+    lo.x = (v.x << 4) & 0xF0F0F0F0u;  hi.x = v.x & 0xF0F0F0F0u;
+    lo.y = (v.y << 4) & 0xF0F0F0F0u;  hi.y = v.y & 0xF0F0F0F0u;
+    lo.z = (v.z << 4) & 0xF0F0F0F0u;  hi.z = v.z & 0xF0F0F0F0u;
+    lo.w = (v.w << 4) & 0xF0F0F0F0u;  hi.w = v.w & 0xF0F0F0F0u;
+}
+
+template <bool OUT_INT8, bool DEBUG>
+__global__ void __launch_bounds__(ts::THREADS, 1)
+    w4a4_gemm_ts_kernel(const __grid_constant__ CUtensorMap tm_wq,
+                        const __grid_constant__ CUtensorMap tm_wo,
+                        const __grid_constant__ CUtensorMap tm_xo,
+                        const uint8_t *__restrict__ Xq, const GemmParams p) {
+    using namespace ts;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t op_full[S], op_empty[S], pk_full[SP], pk_empty[SP];
+    __shared__ uint64_t acc_full, drain, mma_done;
+    __shared__ uint32_t tmem_base_s;
+    __shared__ int abort_s;
+    __shared__ unsigned err0_s;
+    // per-column epilogue factors of the tile, staged once by the A warps
+    __shared__ __align__(16) float col_sw[BN], col_swo[BN], col_bias[BN];
+
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+    const uint32_t smem_base = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+    const int nkb = p.nkb_i + p.nkb_o;
+    const int nunits = p.nkb_i + 3 * p.nkb_o;  // staging units
+    const int rb = p.Ki / 2;                   // packed bytes per row
+
+    if (threadIdx.x == 0) {
+        QUIK_TRACE_AT(6, 0);
+        for (int st = 0; st < S; ++st) {
+            mbar_init(&op_full[st], NA + NB);
+            mbar_init(&op_empty[st], 1);
+        }
+        for (int st = 0; st < SP; ++st) {
+            mbar_init(&pk_full[st], 1);
+            mbar_init(&pk_empty[st], NB);
+        }
+        mbar_init(&acc_full, 1);
+        mbar_init(&drain, 1);
+        mbar_init(&mma_done, 1);
+        abort_s = 0;
+        err0_s = *reinterpret_cast<volatile unsigned *>(&g_error_word);
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc(&tmem_base_s, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_s;
+    const AbortState ab{&abort_s, err0_s};
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_i8 = idesc_s8_s32(BM, BN);
+            const uint32_t id_f16 = idesc_f16_f32(BM, BN);
+            bool ok = true;
+            for (int kb = 0; kb < p.nkb_i && ok; ++kb) {
+                const int st = kb % S;
+                if (!(ok = wait_bar(&op_full[st], (kb / S) & 1, ab))) break;
+                tc_fence_after();
+                QUIK_TRACE_AT(3, kb);
+                const uint32_t b_addr = smem_base + st * STAGE;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_i8_ts(tmem + ACC_COL, tmem + A_COL + 32 * st + 8 * k,
+                              sw128_kmajor_desc(b_addr + 32 * k), id_i8, (kb > 0 || k > 0));
+                mma_commit(&op_empty[st]);
+            }
+            if (ok && p.nkb_o > 0) {
+                if (p.nkb_i > 0) {
+                    // the outlier sums overwrite the A-stage columns: every INT4
+                    // MMA finishes reading them first
+                    mma_commit(&drain);
+                    ok = wait_bar(&drain, 0, ab);
+                }
+                for (int kb = p.nkb_i; kb < nkb && ok; ++kb) {
+                    const int st = kb % S, ko = kb - p.nkb_i;
+                    if (!(ok = wait_bar(&op_full[st], (kb / S) & 1, ab))) break;
+                    tc_fence_after();
+                    const uint32_t b_addr = smem_base + st * STAGE;
+                    const uint32_t a_addr = b_addr + B_BYTES;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t ad = sw128_kmajor_desc(a_addr + 32 * k);
+                        const uint64_t bd = sw128_kmajor_desc(b_addr + 32 * k);
+                        if (OUT_INT8)
+                            mma_i8(tmem + O_COL, ad, bd, id_i8, (ko > 0 || k > 0));
+                        else
+                            mma_f16(tmem + O_COL, ad, bd, id_f16, (ko > 0 || k > 0));
+                    }
+                    mma_commit(&op_empty[st]);
+                }
+            }
+            mma_commit(&acc_full);
+            mma_commit(&mma_done);
+            mbar_wait_bounded(&mma_done, 0, kWaitLimitNs);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            if (p.nkb_i > 0) tma_prefetch_desc(&tm_wq);
+            if (p.nkb_o > 0) {
+                tma_prefetch_desc(&tm_wo);
+                tma_prefetch_desc(&tm_xo);
+            }
+            int last[SP];
+            for (int st = 0; st < SP; ++st) last[st] = -1;
+            for (int u = 0; u < nunits; ++u) {
+                const int st = u % SP;
+                if (!wait_bar(&pk_empty[st], ((u / SP) & 1) ^ 1, ab)) break;
+                uint8_t *dst = smem + PK_OFF + st * PK_BYTES;
+                mbar_arrive_expect_tx(&pk_full[st], PK_BYTES);
+                if (u < p.nkb_i) {
+                    tma_load_2d(dst, &tm_wq, u * PK_ROW, n0, &pk_full[st]);
+                } else {
+                    const int v = u - p.nkb_i, ko = v / 3, part = v % 3;
+                    if (part < 2)  // half of the Wo tile: 256 rows x 64 bytes
+                        tma_load_2d(dst, &tm_wo, ko * OP_ROW + part * 64, n0, &pk_full[st]);
+                    else           // the Xo tile: 128 rows x 128 bytes
+                        tma_load_2d(dst, &tm_xo, ko * OP_ROW, m0, &pk_full[st]);
+                }
+                last[st] = u;
+            }
+            // never leave the CTA with a bulk copy still writing its shared memory
+            for (int st = 0; st < SP; ++st)
+                if (last[st] >= 0) mbar_wait_bounded(&pk_full[st], (last[st] / SP) & 1, kWaitLimitNs);
+        }
+        __syncwarp();
+    } else if (warp < 2 + NA) {
+        // ------------------------------------------------------------ A rows -> TMEM
+        const int q = warp & 3;
+        const int r = q * 32 + lane;  // tile row = TMEM lane
+        const int grow = m0 + r;
+        const bool row_ok = grow < p.M;
+        const uint8_t *xrow = Xq + (size_t)grow * rb;
+        const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
+        uint4 buf[PF][4];
+        auto load = [&](int kb, uint4(&d)[4]) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int off = kb * PK_ROW + c * 16;
+                d[c] = (row_ok && off < rb) ? ldg_nc_v4(xrow + off) : make_uint4(0, 0, 0, 0);
+            }
+        };
+#pragma unroll
+        for (int j = 0; j < PF; ++j)
+            if (j < p.nkb_i) load(j, buf[j]);
+        bool ok = true;
+        for (int kb0 = 0; kb0 < p.nkb_i && ok; kb0 += PF) {
+#pragma unroll
+            for (int j = 0; j < PF; ++j) {
+                const int kb = kb0 + j;
+                if (kb >= p.nkb_i || !ok) break;
+                const int st = kb % S;
+                ok = wait_bar(&op_empty[st], ((kb / S) & 1) ^ 1, ab);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                uint32_t w[32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint4 lo, hi;
+                    unpack16(buf[j][c], lo, hi);
+                    w[8 * c + 0] = lo.x; w[8 * c + 1] = lo.y; w[8 * c + 2] = lo.z; w[8 * c + 3] = lo.w;
+                    w[8 * c + 4] = hi.x; w[8 * c + 5] = hi.y; w[8 * c + 6] = hi.z; w[8 * c + 7] = hi.w;
+                }
+                tmem_st_32x32b_x32(t_lane + A_COL + 32 * st, w);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&op_full[st]);
+#ifdef QUIK_TRACE
+                if (lane == 0 && blockIdx.x + blockIdx.y * gridDim.x < kTraceCtas && kb < kTraceKb)
+                    atomicMax(&g_trace[blockIdx.x + blockIdx.y * gridDim.x][2][kb], clock64());
+#endif
+                if (kb + PF < p.nkb_i) load(kb + PF, buf[j]);
+            }
+        }
+        // outlier k-blocks: both operands arrive through shared memory; these
+        // warps only keep the stage's arrival count
+        for (int kb = p.nkb_i; kb < nkb && ok; ++kb) {
+            const int st = kb % S;
+            ok = wait_bar(&op_empty[st], ((kb / S) & 1) ^ 1, ab);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            if (lane == 0) mbar_arrive(&op_full[st]);
+        }
+
+        // ------------------------------------------------------------ epilogue
+        // Stage the tile's per-column factors while the last MMAs run.
+        for (int c = threadIdx.x - 64; c < BN; c += 32 * NA) {
+            const int n = n0 + c;
+            const bool in = n < p.N;
+            col_sw[c] = (in && p.Ki > 0) ? p.sw[n] : 0.0f;
+            col_swo[c] = (in && OUT_INT8 && p.nkb_o > 0) ? p.swo[n] : 0.0f;
+            col_bias[c] = (in && p.bias != nullptr) ? __half2float(__ushort_as_half(p.bias[n])) : 0.0f;
+        }
+        named_barrier_sync(1, 32 * NA);
+        ok = ok && wait_bar(&acc_full, 0, ab);
+        if (__all_sync(0xffffffffu, ok)) {
+            tc_fence_after();
+            if (q == 1 && lane == 0) QUIK_TRACE_AT(4, 0);
+            const float sxr = (row_ok && p.Ki > 0) ? p.sx[grow] : 0.0f;
+            const float sxo = (row_ok && OUT_INT8 && p.nkb_o > 0) ? p.sxo[grow] : 0.0f;
+            uint16_t *yrow = p.Y + (size_t)grow * p.N;
+            for (int cc = 0; cc < BN; cc += 32) {
+                const int nb = n0 + cc;
+                uint32_t a[32], o[32];
+                if (p.Ki > 0) tmem_ld_32x32b_x32(t_lane + ACC_COL + cc, a);
+                if (p.nkb_o > 0) tmem_ld_32x32b_x32(t_lane + O_COL + cc, o);
+                tmem_ld_wait();
+                if (DEBUG) {
+                    if (row_ok) {
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) {
+                            const int n = nb + jj;
+                            if (n < p.N) {
+                                if (p.Ki > 0)
+                                    p.acc_dbg[(size_t)grow * p.N + n] = static_cast<int32_t>(a[jj]) >> 8;
+                                if (OUT_INT8 && p.nkb_o > 0 && p.acc_o_dbg)
+                                    p.acc_o_dbg[(size_t)grow * p.N + n] = static_cast<int32_t>(o[jj]);
+                            }
+                        }
+                    }
+                    continue;
+                }
+                uint32_t packed[16];
+#pragma unroll
+                for (int jj = 0; jj < 32; jj += 2) {
+                    float y[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int c = cc + jj + h;
+                        // exact: |A| <= 49 K_i < 2^22 after the shift by 8
+                        float v = small_int_to_float(static_cast<int32_t>(a[jj + h]) >> 8) * sxr * col_sw[c];
+                        if (p.Ki == 0) v = 0.0f;
+                        if (p.nkb_o > 0) {
+                            if (OUT_INT8)  // up to 127*127*k_o: plain conversion
+                                v += static_cast<float>(static_cast<int32_t>(o[jj + h])) * sxo * col_swo[c];
+                            else
+                                v += __uint_as_float(o[jj + h]);
+                        }
+                        y[h] = v + col_bias[c];
+                    }
+                    packed[jj / 2] = pack_half2(y[0], y[1]);
+                }
+                if (row_ok) {
+                    if (nb + 32 <= p.N && (p.N & 7) == 0) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(yrow + nb);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            dst[v4] = make_uint4(packed[4 * v4], packed[4 * v4 + 1],
+                                                 packed[4 * v4 + 2], packed[4 * v4 + 3]);
+                    } else {
+                        for (int jj = 0; jj < 32; ++jj)
+                            if (nb + jj < p.N)
+                                yrow[nb + jj] = static_cast<uint16_t>(packed[jj / 2] >> (16 * (jj & 1)));
+                    }
+                }
+            }
+            tc_fence_before();
+            if (q == 1 && lane == 0) QUIK_TRACE_AT(5, 0);
+        }
+    } else {
+        // ------------------------------------------------------------ B: staging -> operand stage
+        const int tb = threadIdx.x - 32 * (2 + NA);  // 0 .. 32*NB-1
+        bool ok = true;
+        int u = 0;  // staging unit
+        for (int kb = 0; kb < nkb && ok; ++kb) {
+            const int st = kb % S;
+            ok = wait_bar(&op_empty[st], ((kb / S) & 1) ^ 1, ab);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            if (tb == 0) QUIK_TRACE_AT(1, kb);
+            uint8_t *bst = smem + st * STAGE;
+            const int nparts = kb < p.nkb_i ? 1 : 3;
+            for (int part = 0; part < nparts && ok; ++part, ++u) {
+                const int ps = u % SP;
+                ok = wait_bar(&pk_full[ps], (u / SP) & 1, ab);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                if (tb == 0 && part == 0) QUIK_TRACE_AT(8, kb);
+                const uint8_t *pk = smem + PK_OFF + ps * PK_BYTES;
+                if (kb < p.nkb_i) {
+                    // 256 rows x 4 chunks: unpack each 16-byte chunk into two
+                    const int ch = tb & 3;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int row = tb / 4 + 64 * i;
+                        const uint4 v = *reinterpret_cast<const uint4 *>(pk + row * PK_ROW + ch * 16);
+                        uint4 lo, hi;
+                        unpack16(v, lo, hi);
+                        uint8_t *rp = bst + row * OP_ROW;
+                        *reinterpret_cast<uint4 *>(rp + (((2 * ch) ^ (row & 7)) << 4)) = lo;
+                        *reinterpret_cast<uint4 *>(rp + (((2 * ch + 1) ^ (row & 7)) << 4)) = hi;
+                    }
+                } else if (part < 2) {
+                    // half of the Wo tile: 256 rows x 4 chunks -> chunks 4 part + c
+                    const int c = tb & 3;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int row = tb / 4 + 64 * i;
+                        const uint4 v = *reinterpret_cast<const uint4 *>(pk + row * PK_ROW + c * 16);
+                        *reinterpret_cast<uint4 *>(bst + row * OP_ROW + (((4 * part + c) ^ (row & 7)) << 4)) = v;
+                    }
+                } else {
+                    // the Xo tile: 128 rows x 8 chunks
+                    const int c = tb & 7;
+                    uint8_t *xo = bst + B_BYTES;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int row = tb / 8 + 32 * i;
+                        const uint4 v = *reinterpret_cast<const uint4 *>(pk + row * OP_ROW + c * 16);
+                        *reinterpret_cast<uint4 *>(xo + row * OP_ROW + ((c ^ (row & 7)) << 4)) = v;
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&pk_empty[ps]);
+            }
+            if (!ok) break;
+            if (tb == 0) QUIK_TRACE_AT(9, kb);
+            fence_proxy_async_smem();  // generic-proxy stores -> visible to the MMA
+            if (tb == 0) QUIK_TRACE_AT(10, kb);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&op_full[st]);
+#ifdef QUIK_TRACE
+            if (lane == 0 && blockIdx.x + blockIdx.y * gridDim.x < kTraceCtas && kb < kTraceKb)
+                atomicMax(&g_trace[blockIdx.x + blockIdx.y * gridDim.x][0][kb], clock64());
+#endif
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) QUIK_TRACE_AT(7, 0);
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
@@ -652,8 +1065,55 @@ quik_status run(const GemmArgs &a, cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
 }
 
+template <bool OUT_INT8, bool DEBUG>
+quik_status run_ts(const GemmArgs &a, cudaStream_t stream) {
+    const int Ki = a.K - a.k_o;
+    const bool outliers = a.k_o > 0 && a.Xo != nullptr;  // debug entry may skip them
+    const uint64_t ob = static_cast<uint64_t>(a.k_o) * (OUT_INT8 ? 1 : 2);  // outlier bytes per row
+    CUtensorMap mwq, mwo, mxo;
+    std::memset(&mwq, 0, sizeof(mwq));
+    std::memset(&mwo, 0, sizeof(mwo));
+    std::memset(&mxo, 0, sizeof(mxo));
+    if (Ki > 0 && !make_map(&mwq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wq, Ki / 2, a.N, Ki / 2, PK_ROW,
+                            ts::BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return QUIK_ERR_CUDA;
+    // outlier blocks as plain bytes: Wo in 64-byte halves of 256 rows, Xo in 128-byte rows
+    if (outliers &&
+        (!make_map(&mwo, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wo, ob, a.N, ob, 64, ts::BN,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
+         !make_map(&mxo, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Xo, ob, a.M, ob, OP_ROW, BM,
+                   CU_TENSOR_MAP_SWIZZLE_NONE)))
+        return QUIK_ERR_CUDA;
+    GemmParams p{};
+    p.M = a.M;
+    p.N = a.N;
+    p.Ki = Ki;
+    p.k_o = a.k_o;
+    p.nkb_i = (Ki + KB - 1) / KB;
+    p.nkb_o = !outliers ? 0 : (OUT_INT8 ? (a.k_o + 127) / 128 : (a.k_o + 63) / 64);
+    p.G = 1;
+    p.sx = a.sx;
+    p.sw = a.sw;
+    p.sxo = a.sxo;
+    p.swo = a.swo;
+    p.bias = a.bias;
+    p.Y = a.Y;
+    p.acc_dbg = a.acc_dbg;
+    p.acc_o_dbg = a.acc_o_dbg;
+    auto kern = w4a4_gemm_ts_kernel<OUT_INT8, DEBUG>;
+    if (!attribute_set_once(reinterpret_cast<const void *>(kern), ts::SMEM)) return QUIK_ERR_CUDA;
+    const dim3 grid((a.N + ts::BN - 1) / ts::BN, (a.M + BM - 1) / BM);
+    kern<<<grid, ts::THREADS, ts::SMEM, stream>>>(mwq, mwo, mxo, static_cast<const uint8_t *>(a.Xq),
+                                                  p);
+    return cudaGetLastError() == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
+}
+
 template <bool DEBUG>
 quik_status dispatch(const GemmArgs &a, cudaStream_t stream) {
+#ifndef QUIK_NG_LEGACY
+    if (a.group == 0)
+        return a.out_int8 ? run_ts<true, DEBUG>(a, stream) : run_ts<false, DEBUG>(a, stream);
+#endif
     if (a.group > 0)
         return a.out_int8 ? run<CfgGroup<true, DEBUG>>(a, stream)
                           : run<CfgGroup<false, DEBUG>>(a, stream);
@@ -684,6 +1144,16 @@ quik_status launch_timeout_selftest(uint32_t limit_us, cudaStream_t stream) {
     timeout_selftest_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(limit_us) * 1000ull);
     return cudaGetLastError() == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
 }
+
+#ifdef QUIK_TRACE
+extern "C" __attribute__((visibility("default"))) int qtrace_read(unsigned long long *dst) {
+    return cudaMemcpyFromSymbol(dst, g_trace, sizeof(g_trace)) == cudaSuccess ? 0 : -1;
+}
+extern "C" __attribute__((visibility("default"))) int qtrace_clear() {
+    static unsigned long long zero[sizeof(g_trace) / sizeof(unsigned long long)];
+    return cudaMemcpyToSymbol(g_trace, zero, sizeof(g_trace)) == cudaSuccess ? 0 : -1;
+}
+#endif
 
 #ifdef QUIK_CHECKS
 extern "C" __attribute__((visibility("default"))) unsigned long long qchk_gemm_word() {

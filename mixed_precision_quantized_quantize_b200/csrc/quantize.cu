@@ -45,25 +45,76 @@ struct QParams {
 
 __device__ __forceinline__ float h2f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
 
-// q = clamp(rint(v / s), -qmax, qmax) with the quotient correctly rounded to
-// fp32 (IEEE division, round half to even), q = 0 when s == 0.
-// Fast path: t = v * fl(1/s).  With u = 2^-24, |t - fl(v/s)| <= 3u|v/s|(1+u),
-// so when t is farther than 5e-7*max(|t|,1) > 3u|t|(1+3u) from a half-integer
-// (the only places where rint changes value), fl(v/s) lies on the same side
-// and rounds to the same integer.  Otherwise the exact quotient decides.
-__device__ __forceinline__ int quant_code(float v, float s, float rs, int qmax) {
+// Rounding by the addition of 1.5 * 2^23: for |t| < 2^22 the fp32 sum
+// t + 1.5*2^23 is rounded (to nearest, ties to even) to an integer, so its bit
+// pattern is 0x4B400000 + rint(t) and (sum - 1.5*2^23) == rint(t) exactly.
+constexpr float kRound = 12582912.0f;
+constexpr uint32_t kRoundBits = 0x4B400000u;
+// Packing 8 codes q_k into nibbles: word = 0x88888888 + sum_k q_k * 16^k
+// holds the offset digits q_k + 8 in [1, 15] without carries; xor 0x88888888
+// turns them into 4-bit two's complement.  With the rounding bit patterns
+// b_k = 0x4B400000 + q_k the constant term is folded in advance (mod 2^32).
+constexpr uint32_t kPackBias = 0x88888888u - kRoundBits * 0x11111111u;
+
+// Exact code of one value (the rare near-tie path): rint of the correctly
+// rounded fp32 quotient, clamped, 0 when s == 0.
+__device__ __forceinline__ int exact_code(float v, float s, int qmax) {
     if (s == 0.0f) return 0;
-    float t = __fmul_rn(v, rs);
-    float r = rintf(t);
-    if (0.5f - fabsf(t - r) <= 5e-7f * fmaxf(fabsf(t), 1.0f)) r = rintf(__fdiv_rn(v, s));
-    const int q = static_cast<int>(r);
+    const int q = __float2int_rn(__fdiv_rn(v, s));
     return max(-qmax, min(qmax, q));
+}
+
+// Eight codes of one 32-bit output word from four half2 values.
+//   Fast path: t = v * fl(1/s).  With u = 2^-24, |t - fl(v/s)| <= 3u|v/s|(1+u)
+//   <= 1.3e-6 for |v/s| <= 7 (|v| <= max|v|, so |v/s| <= 7(1+u)^2), hence
+//   unless t lies within 2e-6 of a half-integer (the only points where rint
+//   changes value) fl(v/s) rounds to the same integer.  |t - rint(t)| is
+//   computed exactly (Sterbenz), and a word with any near-tie is redone with
+//   IEEE divisions.  No clamp is needed: |rint(t)| <= 7.
+__device__ __forceinline__ uint32_t pack_codes8(const uint32_t (&h)[4], float s, float rs) {
+    uint32_t word = kPackBias;
+    float dmax = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[k]));
+        // explicit roundings: the product must not be contracted into the add
+        const float t0 = __fmul_rn(f.x, rs), t1 = __fmul_rn(f.y, rs);
+        const float m0 = __fadd_rn(t0, kRound), m1 = __fadd_rn(t1, kRound);
+        dmax = fmaxf(dmax, fmaxf(fabsf(__fsub_rn(t0, __fsub_rn(m0, kRound))),
+                                 fabsf(__fsub_rn(t1, __fsub_rn(m1, kRound)))));
+        word += __float_as_uint(m0) << (8 * k);
+        word += __float_as_uint(m1) << (8 * k + 4);
+    }
+    if (dmax > 0.5f - 2e-6f) {  // near a tie somewhere in this word: exact divisions
+        word = 0x88888888u;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int q0 = exact_code(h2f(static_cast<uint16_t>(h[k] & 0xffffu)), s, 7);
+            const int q1 = exact_code(h2f(static_cast<uint16_t>(h[k] >> 16)), s, 7);
+            word += static_cast<uint32_t>(q0) << (8 * k);
+            word += static_cast<uint32_t>(q1) << (8 * k + 4);
+        }
+    }
+    return word ^ 0x88888888u;
+}
+
+// INT8 outlier code (same fast path; |v/s| <= 127 widens the tie margin).
+__device__ __forceinline__ int code8(float v, float s, float rs) {
+    const float t = __fmul_rn(v, rs);
+    const float m = __fadd_rn(t, kRound);
+    if (fabsf(__fsub_rn(t, __fsub_rn(m, kRound))) > 0.5f - 4e-5f) return exact_code(v, s, 127);
+    return static_cast<int>(__float_as_uint(m) - kRoundBits);
 }
 
 __device__ __forceinline__ float warp_max(float m) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     return m;
+}
+
+__device__ __forceinline__ float half2_absmax(uint32_t m2) {
+    const __half2 a = __habs2(*reinterpret_cast<const __half2 *>(&m2));
+    return fmaxf(__low2float(a), __high2float(a));
 }
 
 template <bool GROUPED, bool OUT_INT8, int MAXW>
@@ -88,7 +139,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_rows_kernel(QParams p) {
             reinterpret_cast<uint4 *>(row_s)[i] = __ldcs(src + i);
         __syncthreads();
 
-        // (2) gather 8 reordered values per word, absmax per word
+        // (2) gather 8 reordered values per word (as 4 half2), absmax per word
         uint32_t v[MAXW][4];
         float wmax[MAXW];
 #pragma unroll
@@ -98,16 +149,18 @@ __global__ void __launch_bounds__(kQThreads) quantize_rows_kernel(QParams p) {
             if (w < nwords && QUIK_CHECK(8 * w + 8 <= Kp, 2)) {
                 const uint4 ix = *reinterpret_cast<const uint4 *>(perm_s + 8 * w);
                 const uint32_t idx[4] = {ix.x, ix.y, ix.z, ix.w};
+                __half2 m2 = __float2half2_rn(0.0f);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     if (!QUIK_CHECK((idx[k] & 0xffffu) < (uint32_t)K && (idx[k] >> 16) < (uint32_t)K, 1)) {
                         v[i][k] = 0;
                         continue;
                     }
-                    const uint16_t a = row_s[idx[k] & 0xffffu], b = row_s[idx[k] >> 16];
-                    v[i][k] = static_cast<uint32_t>(a) | (static_cast<uint32_t>(b) << 16);
-                    wmax[i] = fmaxf(wmax[i], fmaxf(fabsf(h2f(a)), fabsf(h2f(b))));
+                    const uint32_t a = row_s[idx[k] & 0xffffu], b = row_s[idx[k] >> 16];
+                    v[i][k] = a | (b << 16);
+                    m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __half2 *>(&v[i][k])));
                 }
+                wmax[i] = half2_absmax(*reinterpret_cast<const uint32_t *>(&m2));
             }
         }
 
@@ -147,15 +200,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_rows_kernel(QParams p) {
             const int w = tid + i * kQThreads;
             if (w < nwords && QUIK_CHECK(4 * w + 4 <= Ki / 2, 4)) {
                 const float rs = s[i] != 0.0f ? __frcp_rn(s[i]) : 0.0f;
-                uint32_t word = 0;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int q0 = quant_code(h2f(static_cast<uint16_t>(v[i][k] & 0xffffu)), s[i], rs, 7);
-                    const int q1 = quant_code(h2f(static_cast<uint16_t>(v[i][k] >> 16)), s[i], rs, 7);
-                    word |= (static_cast<uint32_t>(q0) & 0xFu) << (8 * k);
-                    word |= (static_cast<uint32_t>(q1) & 0xFu) << (8 * k + 4);
-                }
-                qrow[w] = word;
+                qrow[w] = pack_codes8(v[i], s[i], rs);
             }
         }
 
@@ -180,7 +225,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_rows_kernel(QParams p) {
                 if (tid == 0) p.o_scale[row] = so;
                 int8_t *o = static_cast<int8_t *>(p.O) + static_cast<size_t>(row) * p.k_o;
                 for (int i = tid; i < p.k_o; i += kQThreads)
-                    o[i] = static_cast<int8_t>(quant_code(h2f(row_s[perm_s[Ki + i]]), so, rso, 127));
+                    o[i] = static_cast<int8_t>(code8(h2f(row_s[perm_s[Ki + i]]), so, rso));
             }
         } else if (OUT_INT8 && p.o_scale != nullptr && tid == 0) {
             p.o_scale[row] = 0.0f;
