@@ -1167,6 +1167,8 @@ quik_status sync_check(cudaStream_t stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return QUIK_ERR_CUDA;
     unsigned int word = 0;
     if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return QUIK_ERR_CUDA;
+    const unsigned int qword = take_quantize_errors();
+    if (qword != 0 && word == 0) return QUIK_ERR_TIMEOUT;
     if (word != 0) {
         const unsigned int zero = 0;
         if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess)

@@ -7,8 +7,9 @@
 // two_compl).
 //
 // One CTA owns one row at a time (grid-stride over rows, 256 threads):
-//   1. the CTA stages perm (as uint16) once, then per row loads the fp16 row
-//      into shared memory with coalesced 16-byte streaming loads;
+//   1. the CTA stages perm (as uint16) once; the rows arrive in a ring of up
+//      to three shared-memory buffers, each filled by one TMA bulk copy issued
+//      as soon as the buffer is free, so several rows per CTA are in flight;
 //   2. each thread gathers 8 reordered positions per 32-bit output word
 //      (up to MAXW words, kept in registers), takes their absmax;
 //   3. per-row scale: block reduction; per-group scale (128 positions =
@@ -20,14 +21,20 @@
 // The kernel is bound by HBM bandwidth (2 bytes read per element, 0.5 byte
 // written per INT4 element).
 #include <algorithm>
+#include <atomic>
 
 #include <cuda_fp16.h>
 
 #include "quik_internal.h"
+#include "sm100.cuh"
 
 namespace quik {
 
 QUIK_CHECK_DECL
+
+// Count of bounded waits that ran out in this file's kernels (read and
+// cleared by quik_sync_check through take_quantize_errors).
+__device__ unsigned int g_quant_error;
 
 namespace {
 
@@ -37,6 +44,7 @@ struct QParams {
     const uint16_t *X;
     const int32_t *perm;
     int rows, K, k_o;
+    int nring;  // row buffers per CTA (1..3)
     uint8_t *Q;
     float *scale;
     void *O;
@@ -122,22 +130,44 @@ __global__ void __launch_bounds__(kQThreads) quantize_rows_kernel(QParams p) {
     extern __shared__ __align__(16) uint8_t qsmem[];
     __shared__ float red_a[kQThreads / 32];
     __shared__ float red_b[kQThreads / 32];
+    __shared__ uint64_t row_full[3];
+    __shared__ int give_up;
     const int K = p.K, Ki = K - p.k_o;
     const int Kp = (K + 7) & ~7;
     uint16_t *perm_s = reinterpret_cast<uint16_t *>(qsmem);
-    uint16_t *row_s = perm_s + Kp;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nwords = Ki / 8;
     const int G = GROUPED ? Ki / kGroup : 1;
+    const uint32_t row_bytes = static_cast<uint32_t>(K) * 2;
 
+    auto ring = [&](int j) { return perm_s + Kp * (1 + j % p.nring); };
+    auto issue = [&](int j) {  // thread 0: bulk-copy this CTA's j-th row into its buffer
+        const int row = blockIdx.x + j * gridDim.x;
+        if (row < p.rows) {
+            ptx::mbar_arrive_expect_tx(&row_full[j % p.nring], row_bytes);
+            ptx::bulk_load(ring(j), p.X + static_cast<size_t>(row) * K, row_bytes, &row_full[j % p.nring]);
+        }
+    };
+    if (tid == 0) {
+        for (int s = 0; s < p.nring; ++s) ptx::mbar_init(&row_full[s], 1);
+        give_up = 0;
+        ptx::fence_barrier_init();
+        for (int j = 0; j < p.nring; ++j) issue(j);
+    }
     for (int i = tid; i < K; i += kQThreads) perm_s[i] = static_cast<uint16_t>(p.perm[i]);
+    __syncthreads();
 
-    for (int row = blockIdx.x; row < p.rows; row += gridDim.x) {
-        // (1) stage the row; the barrier also publishes perm_s on the first pass
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.X + static_cast<size_t>(row) * K);
-        for (int i = tid; i < K / 8; i += kQThreads)
-            reinterpret_cast<uint4 *>(row_s)[i] = __ldcs(src + i);
+    for (int j = 0;; ++j) {
+        const int row = blockIdx.x + j * gridDim.x;
+        if (row >= p.rows) break;
+        // (1) wait for this row's buffer (bounded; on expiry the row is skipped)
+        if (tid == 0 && !ptx::mbar_wait_bounded(&row_full[j % p.nring], (j / p.nring) & 1, kWaitLimitNs)) {
+            give_up = 1;
+            atomicAdd(&g_quant_error, 1u);
+        }
         __syncthreads();
+        if (give_up) break;
+        const uint16_t *row_s = ring(j);
 
         // (2) gather 8 reordered values per word (as 4 half2), absmax per word
         uint32_t v[MAXW][4];
@@ -230,19 +260,43 @@ __global__ void __launch_bounds__(kQThreads) quantize_rows_kernel(QParams p) {
         } else if (OUT_INT8 && p.o_scale != nullptr && tid == 0) {
             p.o_scale[row] = 0.0f;
         }
-        __syncthreads();  // row_s and the reduction slots are reused by the next row
+        __syncthreads();  // buffer and reduction slots are free again
+        if (tid == 0) issue(j + p.nring);
     }
+    // never leave the CTA with a bulk copy still writing its shared memory
+    if (tid == 0)
+        for (int s = 0; s < p.nring; ++s) {
+            // the last row issued into slot s, if any
+            int last = -1;
+            for (int j = s; blockIdx.x + j * gridDim.x < p.rows; j += p.nring) last = j;
+            if (last >= 0) ptx::mbar_wait_bounded(&row_full[s], (last / p.nring) & 1, kWaitLimitNs);
+        }
 }
 
 template <bool GROUPED, bool OUT_INT8, int MAXW>
-cudaError_t launch_q(const QParams &p, cudaStream_t stream) {
+cudaError_t launch_q(QParams p, cudaStream_t stream) {
     auto kern = quantize_rows_kernel<GROUPED, OUT_INT8, MAXW>;
     const int Kp = (p.K + 7) & ~7;
-    const size_t smem = static_cast<size_t>(Kp) * 2 * sizeof(uint16_t);
+    const size_t row_bytes = static_cast<size_t>(Kp) * sizeof(uint16_t);
+    // perm (uint16) plus up to three row buffers within ~200 KB of shared memory
+    p.nring = static_cast<int>(std::min<size_t>(3, (200u << 10) / row_bytes - 1));
+    if (p.nring < 1) return cudaErrorInvalidConfiguration;
+    const size_t smem = row_bytes * (1 + p.nring);
     if (!attribute_set_once(reinterpret_cast<const void *>(kern), static_cast<int>(smem)))
         return cudaErrorInvalidConfiguration;
-    // up to 8 resident 256-thread CTAs per SM; rows beyond that are grid-strided
-    const int grid = std::max(1, std::min(p.rows, sm_count() * 8));
+    // grid: every CTA that fits at once, rows grid-strided; the occupancy of
+    // the last shared-memory size seen is cached (one query per new K)
+    static std::atomic<long long> occ_cache{-1};  // (smem << 8) | CTAs per SM
+    long long c = occ_cache.load(std::memory_order_relaxed);
+    int per_sm = 0;
+    if (c >= 0 && (c >> 8) == static_cast<long long>(smem)) {
+        per_sm = static_cast<int>(c & 0xff);
+    } else {
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kQThreads, smem);
+        if (e != cudaSuccess) return e;
+        occ_cache.store((static_cast<long long>(smem) << 8) | (per_sm & 0xff), std::memory_order_relaxed);
+    }
+    const int grid = std::max(1, std::min(p.rows, sm_count() * std::max(per_sm, 1)));
     kern<<<grid, kQThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
@@ -259,10 +313,20 @@ cudaError_t launch_q_w(const QParams &p, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_quantize_rows(const QuantizeArgs &a, cudaStream_t stream) {
-    QParams p{a.X, a.perm, a.rows, a.K, a.k_o, a.Q, a.scale, a.O, a.o_scale};
+    QParams p{a.X, a.perm, a.rows, a.K, a.k_o, 1, a.Q, a.scale, a.O, a.o_scale};
     if (a.group > 0)
         return a.out_int8 ? launch_q_w<true, true>(p, stream) : launch_q_w<true, false>(p, stream);
     return a.out_int8 ? launch_q_w<false, true>(p, stream) : launch_q_w<false, false>(p, stream);
+}
+
+unsigned int take_quantize_errors() {
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_quant_error, sizeof(word)) != cudaSuccess) return 0;
+    if (word != 0) {
+        const unsigned int zero = 0;
+        cudaMemcpyToSymbol(g_quant_error, &zero, sizeof(zero));
+    }
+    return word;
 }
 
 }  // namespace quik
