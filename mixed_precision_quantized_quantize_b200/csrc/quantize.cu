@@ -148,14 +148,34 @@ __global__ void __launch_bounds__(kQThreads) quantize_rows_kernel(QParams p) {
             ptx::bulk_load(ring(j), p.X + static_cast<size_t>(row) * K, row_bytes, &row_full[j % p.nring]);
         }
     };
+    // Stage perm as uint16: one bulk copy of the int32 vector into the (still
+    // unused) row buffers, then an in-shared-memory narrowing.  A strided loop
+    // of global loads here would cost one memory latency per iteration.
+    __shared__ uint64_t perm_full;
+    int32_t *perm32 = reinterpret_cast<int32_t *>(perm_s + Kp);  // needs 4K <= 2 Kp nring bytes
     if (tid == 0) {
         for (int s = 0; s < p.nring; ++s) ptx::mbar_init(&row_full[s], 1);
+        ptx::mbar_init(&perm_full, 1);
         give_up = 0;
         ptx::fence_barrier_init();
-        for (int j = 0; j < p.nring; ++j) issue(j);
+        ptx::mbar_arrive_expect_tx(&perm_full, static_cast<uint32_t>(K) * 4);
+        ptx::bulk_load(perm32, p.perm, static_cast<uint32_t>(K) * 4, &perm_full);
+        if (!ptx::mbar_wait_bounded(&perm_full, 0, kWaitLimitNs)) {
+            give_up = 1;
+            atomicAdd(&g_quant_error, 1u);
+        }
     }
-    for (int i = tid; i < K; i += kQThreads) perm_s[i] = static_cast<uint16_t>(p.perm[i]);
     __syncthreads();
+    for (int i = tid; i < K / 4; i += kQThreads) {  // K % 4 == 0
+        const int4 v = reinterpret_cast<const int4 *>(perm32)[i];
+        reinterpret_cast<uint2 *>(perm_s)[i] =
+            make_uint2(static_cast<uint32_t>(v.x) | (static_cast<uint32_t>(v.y) << 16),
+                       static_cast<uint32_t>(v.z) | (static_cast<uint32_t>(v.w) << 16));
+    }
+    __syncthreads();  // perm_s ready; the row buffers may now be overwritten
+    if (give_up) return;
+    if (tid == 0)
+        for (int j = 0; j < p.nring; ++j) issue(j);
 
     for (int j = 0;; ++j) {
         const int row = blockIdx.x + j * gridDim.x;
@@ -280,7 +300,7 @@ cudaError_t launch_q(QParams p, cudaStream_t stream) {
     const size_t row_bytes = static_cast<size_t>(Kp) * sizeof(uint16_t);
     // perm (uint16) plus up to three row buffers within ~200 KB of shared memory
     p.nring = static_cast<int>(std::min<size_t>(3, (200u << 10) / row_bytes - 1));
-    if (p.nring < 1) return cudaErrorInvalidConfiguration;
+    if (p.nring < 2) return cudaErrorInvalidConfiguration;  // the ring also stages perm (int32)
     const size_t smem = row_bytes * (1 + p.nring);
     if (!attribute_set_once(reinterpret_cast<const void *>(kern), static_cast<int>(smem)))
         return cudaErrorInvalidConfiguration;
