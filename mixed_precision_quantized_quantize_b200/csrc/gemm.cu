@@ -18,15 +18,16 @@
 // first 16 unpacked bytes and the odd codes in the next 16, the same
 // K-permutation on both sides, so every dot product is unchanged.
 //
-// Warp roles in one CTA (one output tile per CTA):
-//   warp 0      TMA producer: packed INT4 tiles of Xq / Wq into a staging ring;
-//   warp 1      TMEM allocator and the single thread that issues tcgen05.mma;
-//   NT warps    fill the operand ring (128-byte swizzled K-major, the layout
-//               the MMA reads) in k-block order: unpacked INT4 k-blocks from
-//               the staging ring, then FP16 (or INT8) outlier tiles by TMA;
-//   NE warps    epilogue: TMEM -> registers -> dequantise -> fp16 stores
-//               (grouped mode: drain each group's INT32 sum while the next
-//               group accumulates in the other TMEM buffer).
+// Two kernels:
+//   * per-channel scales: a CTA pair per 256 x 256 tile (cta_group::2),
+//     activations in tensor memory, B through shared memory (described
+//     above w4a4_gemm_pair_kernel);
+//   * per-group scales: one CTA per 128 x 128 tile, both operands in shared
+//     memory.  Warp 0 is the TMA producer of a packed staging ring, warp 1
+//     allocates TMEM and issues tcgen05.mma, NT warps unpack into the
+//     128-byte swizzled K-major operand ring (then copy the outlier tiles),
+//     NE warps drain each group's INT32 sum while the next group accumulates
+//     in the other TMEM buffer.
 // Every mbarrier wait is bounded (2 s); on expiry the CTA counts the error in
 // g_error_word, stops issuing work, waits for its in-flight copies and MMAs,
 // frees TMEM and exits; other CTAs see the count change and give up too.
@@ -71,26 +72,6 @@ constexpr int KB = 128;       // INT4 codes per k-block = one scale group
 constexpr int PK_ROW = 64;    // packed bytes per row per k-block
 constexpr int OP_ROW = 128;   // unpacked bytes per row per k-block (one swizzle row)
 
-// Pipeline shape of the per-channel-scale kernel (compile-time tuning knobs).
-#ifndef QUIK_NG_BN
-#define QUIK_NG_BN 256  // tile columns
-#endif
-#ifndef QUIK_NG_NT
-#define QUIK_NG_NT 8    // unpack warps
-#endif
-#ifndef QUIK_NG_NE
-#define QUIK_NG_NE 4    // epilogue warps
-#endif
-#ifndef QUIK_NG_SP
-#define QUIK_NG_SP 3    // packed staging stages
-#endif
-#ifndef QUIK_NG_SU
-#define QUIK_NG_SU 3    // operand stages
-#endif
-#ifndef QUIK_NG_MINB
-#define QUIK_NG_MINB 1  // CTAs resident per SM
-#endif
-
 template <int BN_, bool GROUPED_, bool OUT_INT8_, bool DEBUG_, int NT_, int NE_, int SP_, int SU_,
           int MINB_>
 struct Cfg {
@@ -122,9 +103,6 @@ struct Cfg {
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-template <bool OUT_INT8, bool DEBUG>
-using CfgChannel = Cfg<QUIK_NG_BN, false, OUT_INT8, DEBUG, QUIK_NG_NT, QUIK_NG_NE, QUIK_NG_SP,
-                       QUIK_NG_SU, QUIK_NG_MINB>;
 template <bool OUT_INT8, bool DEBUG>
 using CfgGroup = Cfg<128, true, OUT_INT8, DEBUG, 4, 8, 4, 4, 1>;
 
@@ -588,52 +566,6 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
     }
 }
 
-// ============================================================================
-// Per-channel-scale kernel, activations (operand A) in tensor memory.
-//
-// Shared-memory bandwidth bounds the kernel above: per 128-code k-block of a
-// 128 x 256 tile it moves 24 KB of packed codes in by TMA, reads them back,
-// writes 48 KB of unpacked bytes and the MMA reads those 48 KB again
-// (144 KB per 4 Mi multiply-adds against ~128 B/clk).  Here the A rows never
-// touch shared memory: A threads load their row's packed codes from global
-// memory (several k-blocks ahead), unpack in registers and write tensor
-// memory with tcgen05.st; tcgen05.mma reads A from TMEM.  Only B goes through
-// shared memory (TMA staging 16 KB, read back 16 KB, unpacked 32 KB, MMA
-// reads 32 KB: 96 KB per k-block).  The B unpack warps keep no global loads
-// in flight, so the proxy fence that publishes their stores to the MMA only
-// waits for their own shared-memory stores.
-//
-//   warp 0        TMEM allocator; lane 0 issues the MMAs
-//   warp 1        TMA producer of the packed staging ring, in unit order:
-//                 one unit per INT4 k-block (the B tile, 256 rows x 64 B),
-//                 three per outlier k-block (two halves of the Wo tile, then
-//                 the Xo tile)
-//   warps 2-5     A: one thread per tile row (= its TMEM lane): load, unpack,
-//                 tcgen05.st 32 columns per k-block; then the epilogue
-//   warps 6-13    B: staging -> 128-byte swizzled K-major operand stage
-//                 (unpacked INT4 k-blocks; copied outlier tiles)
-// TMEM: INT32 sums in columns [0,256); A stages [256, 256+32 S) while the INT4
-// k-blocks run; after them (and a drain of the MMA pipe) the outlier sums in
-// [256, 512), with both outlier operands in shared memory.
-namespace ts {
-constexpr int BN = 256;
-constexpr int S = 3;                  // operand stages
-constexpr int SP = 4;                 // packed staging stages
-constexpr int NA = 4, NB = 8;         // A warps, B warps
-constexpr int THREADS = (2 + NA + NB) * 32;
-constexpr int B_BYTES = BN * OP_ROW;  // unpacked B k-block / outlier W tile
-constexpr int XO_BYTES = BM * OP_ROW; // outlier X tile
-constexpr int STAGE = B_BYTES + XO_BYTES;
-constexpr int PK_BYTES = BN * PK_ROW; // one staging unit (= BM * OP_ROW)
-constexpr int PK_OFF = S * STAGE;
-constexpr int SMEM = PK_OFF + SP * PK_BYTES + 1024;
-constexpr int ACC_COL = 0, A_COL = 256, O_COL = 256, TMEM_COLS = 512;
-constexpr int PF = 4;                 // k-blocks of A loads in flight per thread
-static_assert(PK_BYTES == XO_BYTES, "an Xo tile fills one staging unit");
-static_assert(A_COL + 32 * S <= TMEM_COLS, "A stages fit in tensor memory");
-static_assert(SMEM <= 232448, "shared memory budget");
-}  // namespace ts
-
 __device__ __forceinline__ void unpack16(const uint4 v, uint4 &lo, uint4 &hi) {
     lo.x = (v.x << 4) & 0xF0F0F0F0u;  hi.x = v.x & 0xF0F0F0F0u;
     lo.y = (v.y << 4) & 0xF0F0F0F0u;  hi.y = v.y & 0xF0F0F0F0u;
@@ -641,35 +573,90 @@ __device__ __forceinline__ void unpack16(const uint4 v, uint4 &lo, uint4 &hi) {
     lo.w = (v.w << 4) & 0xF0F0F0F0u;  hi.w = v.w & 0xF0F0F0F0u;
 }
 
+// ============================================================================
+// Per-channel-scale kernel on a CTA pair (cta_group::2), activations in
+// tensor memory.
+//
+// Two CTAs of a cluster share one 256 x 256 output tile.  Each holds 128 rows
+// of A and of the output, and half of B (128 of the 256 columns) in its
+// shared memory; the leader issues tcgen05.mma.cta_group::2 with M = 256,
+// which reads both halves.  The A rows never touch shared memory: A threads
+// load their row's packed codes from global memory (several k-blocks ahead),
+// unpack in registers and write tensor memory with tcgen05.st; the MMA reads
+// A from TMEM.  Only B goes through shared memory: per k-block and SM, TMA
+// staging 8 KB, read back 8 KB, unpacked 16 KB, MMA read 16 KB.  (With one
+// CTA per 128 x 256 tile that is 96 KB per k-block, which bounds the kernel
+// by shared-memory bandwidth.)  The B unpack warps keep no global loads in
+// flight, so the proxy fence that publishes their stores to the MMA only
+// waits for their own shared-memory stores.
+//
+// Peer warps signal the leader's "operand full" barriers with remote mbarrier
+// arrivals on cluster addresses (the instruction's default semantics, as in
+// CUTLASS's two-SM pipelines; an explicit release at cluster scope measured
+// 1.6x slower end to end); MMA completion reaches both CTAs through a
+// multicast commit.
+//
+//   warp 0        TMEM allocator (both CTAs); the leader's lane 0 issues the MMAs
+//   warp 1        TMA producer of the packed staging ring, in unit order:
+//                 one unit per INT4 k-block (this CTA's 128 rows of the B
+//                 tile), two per outlier k-block (Wo rows, then Xo rows)
+//   warps 2-5     A: one thread per tile row (= its TMEM lane): load, unpack,
+//                 tcgen05.st 32 columns per k-block; then the epilogue
+//   warps 6-13    B: staging -> 128-byte swizzled K-major operand stage
+//                 (unpacked INT4 k-blocks; copied outlier tiles)
+// TMEM (each CTA): INT32 sums in columns [0,256); A stages [256, 256+32 S)
+// while the INT4 k-blocks run; after them (and a drain of the MMA pipe) the
+// outlier sums in [256, 512), with both outlier operands in shared memory.
+namespace pair {
+constexpr int BN = 256;                   // pair tile columns (each CTA holds BN/2 of B)
+constexpr int BNH = BN / 2;
+constexpr int S = 4;                      // operand stages
+constexpr int SP = 4;                     // packed staging stages
+constexpr int NA = 4, NB = 8;  // A warps, B warps (per CTA)
+constexpr int THREADS = (2 + NA + NB) * 32;
+constexpr int B_BYTES = BNH * OP_ROW;     // this CTA's unpacked half of B / outlier W rows
+constexpr int XO_BYTES = BM * OP_ROW;     // outlier X tile (this CTA's 128 rows)
+constexpr int STAGE = B_BYTES + XO_BYTES;
+constexpr int UNIT = BM * OP_ROW;         // staging unit: 16 KB
+constexpr int PK_OFF = S * STAGE;
+constexpr int SMEM = PK_OFF + SP * UNIT + 1024;
+constexpr int ACC_COL = 0, A_COL = 256, O_COL = 256, TMEM_COLS = 512;
+constexpr int PF = 4;                     // k-blocks of A loads in flight per thread
+static_assert(A_COL + 32 * S <= TMEM_COLS, "A stages fit in tensor memory");
+static_assert(SMEM <= 232448, "shared memory budget");
+}  // namespace pair
+
 template <bool OUT_INT8, bool DEBUG>
-__global__ void __launch_bounds__(ts::THREADS, 1)
-    w4a4_gemm_ts_kernel(const __grid_constant__ CUtensorMap tm_wq,
-                        const __grid_constant__ CUtensorMap tm_wo,
-                        const __grid_constant__ CUtensorMap tm_xo,
-                        const uint8_t *__restrict__ Xq, const GemmParams p) {
-    using namespace ts;
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
+    w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_wq,
+                          const __grid_constant__ CUtensorMap tm_wo,
+                          const __grid_constant__ CUtensorMap tm_xo,
+                          const uint8_t *__restrict__ Xq, const GemmParams p) {
+    using namespace pair;
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t op_full[S], op_empty[S], pk_full[SP], pk_empty[SP];
     __shared__ uint64_t acc_full, drain, mma_done;
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     __shared__ unsigned err0_s;
-    // per-column epilogue factors of the tile, staged once by the A warps
     __shared__ __align__(16) float col_sw[BN], col_swo[BN], col_bias[BN];
 
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
     const uint32_t smem_base = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+    const uint32_t rank = cluster_ctarank();     // 0 = leader
+    const int m0 = blockIdx.y * 2 * BM + rank * BM;  // this CTA's A / output rows
+    const int n0 = (blockIdx.x >> 1) * BN;           // the pair's output columns
+    const int nb0 = n0 + rank * BNH;                 // this CTA's rows of W (half of B)
     const int nkb = p.nkb_i + p.nkb_o;
-    const int nunits = p.nkb_i + 3 * p.nkb_o;  // staging units
-    const int rb = p.Ki / 2;                   // packed bytes per row
+    const int nunits = p.nkb_i + 2 * p.nkb_o;        // staging units
+    const int rb = p.Ki / 2;
 
     if (threadIdx.x == 0) {
         QUIK_TRACE_AT(6, 0);
         for (int st = 0; st < S; ++st) {
-            mbar_init(&op_full[st], NA + NB);
+            mbar_init(&op_full[st], 2 * (NA + NB));  // used in the leader only
             mbar_init(&op_empty[st], 1);
         }
         for (int st = 0; st < SP; ++st) {
@@ -683,18 +670,20 @@ __global__ void __launch_bounds__(ts::THREADS, 1)
         err0_s = *reinterpret_cast<volatile unsigned *>(&g_error_word);
         fence_barrier_init();
     }
-    if (warp == 0) tmem_alloc(&tmem_base_s, TMEM_COLS);
+    if (warp == 0) tmem_alloc_pair(&tmem_base_s, TMEM_COLS);
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // barrier initialisation and TMEM allocation visible to both CTAs
     tc_fence_after();
     const uint32_t tmem = tmem_base_s;
     const AbortState ab{&abort_s, err0_s};
+    // the leader's "operand full" barriers, as cluster addresses
+    auto leader_full = [&](int st) { return mapa_shared(smem_u32(&op_full[st]), 0); };
 
     if (warp == 0) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t id_i8 = idesc_s8_s32(BM, BN);
-            const uint32_t id_f16 = idesc_f16_f32(BM, BN);
+        // ------------------------------------------------------------ MMA issuer (leader)
+        if (rank == 0 && lane == 0) {
+            const uint32_t id_i8 = idesc_s8_s32(2 * BM, BN);
+            const uint32_t id_f16 = idesc_f16_f32(2 * BM, BN);
             bool ok = true;
             for (int kb = 0; kb < p.nkb_i && ok; ++kb) {
                 const int st = kb % S;
@@ -704,15 +693,15 @@ __global__ void __launch_bounds__(ts::THREADS, 1)
                 const uint32_t b_addr = smem_base + st * STAGE;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_i8_ts(tmem + ACC_COL, tmem + A_COL + 32 * st + 8 * k,
-                              sw128_kmajor_desc(b_addr + 32 * k), id_i8, (kb > 0 || k > 0));
-                mma_commit(&op_empty[st]);
+                    mma2_i8_ts(tmem + ACC_COL, tmem + A_COL + 32 * st + 8 * k,
+                               sw128_kmajor_desc(b_addr + 32 * k), id_i8, (kb > 0 || k > 0));
+                mma2_commit_both(&op_empty[st]);
             }
             if (ok && p.nkb_o > 0) {
                 if (p.nkb_i > 0) {
                     // the outlier sums overwrite the A-stage columns: every INT4
                     // MMA finishes reading them first
-                    mma_commit(&drain);
+                    mma2_commit_local(&drain);
                     ok = wait_bar(&drain, 0, ab);
                 }
                 for (int kb = p.nkb_i; kb < nkb && ok; ++kb) {
@@ -726,20 +715,20 @@ __global__ void __launch_bounds__(ts::THREADS, 1)
                         const uint64_t ad = sw128_kmajor_desc(a_addr + 32 * k);
                         const uint64_t bd = sw128_kmajor_desc(b_addr + 32 * k);
                         if (OUT_INT8)
-                            mma_i8(tmem + O_COL, ad, bd, id_i8, (ko > 0 || k > 0));
+                            mma2_i8(tmem + O_COL, ad, bd, id_i8, (ko > 0 || k > 0));
                         else
-                            mma_f16(tmem + O_COL, ad, bd, id_f16, (ko > 0 || k > 0));
+                            mma2_f16(tmem + O_COL, ad, bd, id_f16, (ko > 0 || k > 0));
                     }
-                    mma_commit(&op_empty[st]);
+                    mma2_commit_both(&op_empty[st]);
                 }
             }
-            mma_commit(&acc_full);
-            mma_commit(&mma_done);
+            mma2_commit_both(&acc_full);
+            mma2_commit_local(&mma_done);
             mbar_wait_bounded(&mma_done, 0, kWaitLimitNs);
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ------------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------ TMA producer (each CTA)
         if (lane == 0) {
             if (p.nkb_i > 0) tma_prefetch_desc(&tm_wq);
             if (p.nkb_o > 0) {
@@ -751,15 +740,17 @@ __global__ void __launch_bounds__(ts::THREADS, 1)
             for (int u = 0; u < nunits; ++u) {
                 const int st = u % SP;
                 if (!wait_bar(&pk_empty[st], ((u / SP) & 1) ^ 1, ab)) break;
-                uint8_t *dst = smem + PK_OFF + st * PK_BYTES;
-                mbar_arrive_expect_tx(&pk_full[st], PK_BYTES);
-                if (u < p.nkb_i) {
-                    tma_load_2d(dst, &tm_wq, u * PK_ROW, n0, &pk_full[st]);
+                uint8_t *dst = smem + PK_OFF + st * UNIT;
+                QUIK_TRACE_AT(11, u);
+                if (u < p.nkb_i) {  // this CTA's 128 rows of the packed B tile
+                    mbar_arrive_expect_tx(&pk_full[st], BNH * PK_ROW);
+                    tma_load_2d(dst, &tm_wq, u * PK_ROW, nb0, &pk_full[st]);
                 } else {
-                    const int v = u - p.nkb_i, ko = v / 3, part = v % 3;
-                    if (part < 2)  // half of the Wo tile: 256 rows x 64 bytes
-                        tma_load_2d(dst, &tm_wo, ko * OP_ROW + part * 64, n0, &pk_full[st]);
-                    else           // the Xo tile: 128 rows x 128 bytes
+                    const int v = u - p.nkb_i, ko = v / 2;
+                    mbar_arrive_expect_tx(&pk_full[st], UNIT);
+                    if (v % 2 == 0)  // this CTA's 128 rows of Wo, 128 bytes each
+                        tma_load_2d(dst, &tm_wo, ko * OP_ROW, nb0, &pk_full[st]);
+                    else             // this CTA's 128 rows of Xo
                         tma_load_2d(dst, &tm_xo, ko * OP_ROW, m0, &pk_full[st]);
                 }
                 last[st] = u;
@@ -770,7 +761,7 @@ __global__ void __launch_bounds__(ts::THREADS, 1)
         }
         __syncwarp();
     } else if (warp < 2 + NA) {
-        // ------------------------------------------------------------ A rows -> TMEM
+        // ------------------------------------------------------------ A rows -> TMEM (each CTA)
         const int q = warp & 3;
         const int r = q * 32 + lane;  // tile row = TMEM lane
         const int grow = m0 + r;
@@ -809,7 +800,7 @@ __global__ void __launch_bounds__(ts::THREADS, 1)
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&op_full[st]);
+                if (lane == 0) mbar_arrive_remote(leader_full(st));
 #ifdef QUIK_TRACE
                 if (lane == 0 && blockIdx.x + blockIdx.y * gridDim.x < kTraceCtas && kb < kTraceKb)
                     atomicMax(&g_trace[blockIdx.x + blockIdx.y * gridDim.x][2][kb], clock64());
@@ -817,17 +808,15 @@ __global__ void __launch_bounds__(ts::THREADS, 1)
                 if (kb + PF < p.nkb_i) load(kb + PF, buf[j]);
             }
         }
-        // outlier k-blocks: both operands arrive through shared memory; these
-        // warps only keep the stage's arrival count
+        // outlier k-blocks: both operands arrive through shared memory
         for (int kb = p.nkb_i; kb < nkb && ok; ++kb) {
             const int st = kb % S;
             ok = wait_bar(&op_empty[st], ((kb / S) & 1) ^ 1, ab);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            if (lane == 0) mbar_arrive(&op_full[st]);
+            if (lane == 0) mbar_arrive_remote(leader_full(st));
         }
 
-        // ------------------------------------------------------------ epilogue
-        // Stage the tile's per-column factors while the last MMAs run.
+        // ------------------------------------------------------------ epilogue (each CTA)
         for (int c = threadIdx.x - 64; c < BN; c += 32 * NA) {
             const int n = n0 + c;
             const bool in = n < p.N;
@@ -871,11 +860,10 @@ __global__ void __launch_bounds__(ts::THREADS, 1)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int c = cc + jj + h;
-                        // exact: |A| <= 49 K_i < 2^22 after the shift by 8
                         float v = small_int_to_float(static_cast<int32_t>(a[jj + h]) >> 8) * sxr * col_sw[c];
                         if (p.Ki == 0) v = 0.0f;
                         if (p.nkb_o > 0) {
-                            if (OUT_INT8)  // up to 127*127*k_o: plain conversion
+                            if (OUT_INT8)
                                 v += static_cast<float>(static_cast<int32_t>(o[jj + h])) * sxo * col_swo[c];
                             else
                                 v += __uint_as_float(o[jj + h]);
@@ -902,29 +890,29 @@ __global__ void __launch_bounds__(ts::THREADS, 1)
             if (q == 1 && lane == 0) QUIK_TRACE_AT(5, 0);
         }
     } else {
-        // ------------------------------------------------------------ B: staging -> operand stage
+        // ------------------------------------------------------------ B half: staging -> operand stage
         const int tb = threadIdx.x - 32 * (2 + NA);  // 0 .. 32*NB-1
         bool ok = true;
-        int u = 0;  // staging unit
+        int u = 0;
         for (int kb = 0; kb < nkb && ok; ++kb) {
             const int st = kb % S;
             ok = wait_bar(&op_empty[st], ((kb / S) & 1) ^ 1, ab);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            if (tb == 0) QUIK_TRACE_AT(1, kb);
             uint8_t *bst = smem + st * STAGE;
-            const int nparts = kb < p.nkb_i ? 1 : 3;
+            if (tb == 0) QUIK_TRACE_AT(1, kb);
+            const int nparts = kb < p.nkb_i ? 1 : 2;
             for (int part = 0; part < nparts && ok; ++part, ++u) {
                 const int ps = u % SP;
                 ok = wait_bar(&pk_full[ps], (u / SP) & 1, ab);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 if (tb == 0 && part == 0) QUIK_TRACE_AT(8, kb);
-                const uint8_t *pk = smem + PK_OFF + ps * PK_BYTES;
+                const uint8_t *pk = smem + PK_OFF + ps * UNIT;
                 if (kb < p.nkb_i) {
-                    // 256 rows x 4 chunks: unpack each 16-byte chunk into two
+                    // 128 rows x 4 chunks: unpack each 16-byte chunk into two
                     const int ch = tb & 3;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int row = tb / 4 + 64 * i;
+                    for (int i = 0; i < 128 / (8 * NB); ++i) {
+                        const int row = tb / 4 + 8 * NB * i;
                         const uint4 v = *reinterpret_cast<const uint4 *>(pk + row * PK_ROW + ch * 16);
                         uint4 lo, hi;
                         unpack16(v, lo, hi);
@@ -932,24 +920,16 @@ __global__ void __launch_bounds__(ts::THREADS, 1)
                         *reinterpret_cast<uint4 *>(rp + (((2 * ch) ^ (row & 7)) << 4)) = lo;
                         *reinterpret_cast<uint4 *>(rp + (((2 * ch + 1) ^ (row & 7)) << 4)) = hi;
                     }
-                } else if (part < 2) {
-                    // half of the Wo tile: 256 rows x 4 chunks -> chunks 4 part + c
-                    const int c = tb & 3;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int row = tb / 4 + 64 * i;
-                        const uint4 v = *reinterpret_cast<const uint4 *>(pk + row * PK_ROW + c * 16);
-                        *reinterpret_cast<uint4 *>(bst + row * OP_ROW + (((4 * part + c) ^ (row & 7)) << 4)) = v;
-                    }
                 } else {
-                    // the Xo tile: 128 rows x 8 chunks
+                    // Wo rows (part 0) into the B area, Xo rows (part 1) into the A area:
+                    // 128 rows x 8 chunks each
                     const int c = tb & 7;
-                    uint8_t *xo = bst + B_BYTES;
+                    uint8_t *dst = part == 0 ? bst : bst + B_BYTES;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int row = tb / 8 + 32 * i;
+                    for (int i = 0; i < 32 / NB; ++i) {
+                        const int row = tb / 8 + 4 * NB * i;
                         const uint4 v = *reinterpret_cast<const uint4 *>(pk + row * OP_ROW + c * 16);
-                        *reinterpret_cast<uint4 *>(xo + row * OP_ROW + ((c ^ (row & 7)) << 4)) = v;
+                        *reinterpret_cast<uint4 *>(dst + row * OP_ROW + ((c ^ (row & 7)) << 4)) = v;
                     }
                 }
                 __syncwarp();
@@ -957,10 +937,10 @@ __global__ void __launch_bounds__(ts::THREADS, 1)
             }
             if (!ok) break;
             if (tb == 0) QUIK_TRACE_AT(9, kb);
-            fence_proxy_async_smem();  // generic-proxy stores -> visible to the MMA
+            fence_proxy_async_smem();  // generic-proxy stores -> visible to the pair's MMA
             if (tb == 0) QUIK_TRACE_AT(10, kb);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&op_full[st]);
+            if (lane == 0) mbar_arrive_remote(leader_full(st));
 #ifdef QUIK_TRACE
             if (lane == 0 && blockIdx.x + blockIdx.y * gridDim.x < kTraceCtas && kb < kTraceKb)
                 atomicMax(&g_trace[blockIdx.x + blockIdx.y * gridDim.x][0][kb], clock64());
@@ -971,10 +951,11 @@ __global__ void __launch_bounds__(ts::THREADS, 1)
     // ---------------------------------------------------------------- teardown
     tc_fence_before();
     __syncthreads();
+    cluster_sync();  // neither CTA leaves while the pair's MMAs or remote arrivals may touch it
     if (threadIdx.x == 0) QUIK_TRACE_AT(7, 0);
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        tmem_dealloc_pair(tmem, TMEM_COLS);
     }
 }
 
@@ -1066,7 +1047,7 @@ quik_status run(const GemmArgs &a, cudaStream_t stream) {
 }
 
 template <bool OUT_INT8, bool DEBUG>
-quik_status run_ts(const GemmArgs &a, cudaStream_t stream) {
+quik_status run_pair(const GemmArgs &a, cudaStream_t stream) {
     const int Ki = a.K - a.k_o;
     const bool outliers = a.k_o > 0 && a.Xo != nullptr;  // debug entry may skip them
     const uint64_t ob = static_cast<uint64_t>(a.k_o) * (OUT_INT8 ? 1 : 2);  // outlier bytes per row
@@ -1075,11 +1056,11 @@ quik_status run_ts(const GemmArgs &a, cudaStream_t stream) {
     std::memset(&mwo, 0, sizeof(mwo));
     std::memset(&mxo, 0, sizeof(mxo));
     if (Ki > 0 && !make_map(&mwq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wq, Ki / 2, a.N, Ki / 2, PK_ROW,
-                            ts::BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+                            pair::BNH, CU_TENSOR_MAP_SWIZZLE_NONE))
         return QUIK_ERR_CUDA;
-    // outlier blocks as plain bytes: Wo in 64-byte halves of 256 rows, Xo in 128-byte rows
+    // outlier blocks as plain bytes, 128 rows x 128 bytes per unit
     if (outliers &&
-        (!make_map(&mwo, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wo, ob, a.N, ob, 64, ts::BN,
+        (!make_map(&mwo, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wo, ob, a.N, ob, OP_ROW, pair::BNH,
                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
          !make_map(&mxo, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Xo, ob, a.M, ob, OP_ROW, BM,
                    CU_TENSOR_MAP_SWIZZLE_NONE)))
@@ -1100,25 +1081,22 @@ quik_status run_ts(const GemmArgs &a, cudaStream_t stream) {
     p.Y = a.Y;
     p.acc_dbg = a.acc_dbg;
     p.acc_o_dbg = a.acc_o_dbg;
-    auto kern = w4a4_gemm_ts_kernel<OUT_INT8, DEBUG>;
-    if (!attribute_set_once(reinterpret_cast<const void *>(kern), ts::SMEM)) return QUIK_ERR_CUDA;
-    const dim3 grid((a.N + ts::BN - 1) / ts::BN, (a.M + BM - 1) / BM);
-    kern<<<grid, ts::THREADS, ts::SMEM, stream>>>(mwq, mwo, mxo, static_cast<const uint8_t *>(a.Xq),
-                                                  p);
+    auto kern = w4a4_gemm_pair_kernel<OUT_INT8, DEBUG>;
+    if (!attribute_set_once(reinterpret_cast<const void *>(kern), pair::SMEM)) return QUIK_ERR_CUDA;
+    const dim3 grid(2 * ((a.N + pair::BN - 1) / pair::BN), (a.M + 2 * BM - 1) / (2 * BM));
+    kern<<<grid, pair::THREADS, pair::SMEM, stream>>>(mwq, mwo, mxo,
+                                                      static_cast<const uint8_t *>(a.Xq), p);
     return cudaGetLastError() == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
 }
 
+// Per-channel scales: the CTA-pair kernel (faster than a single-CTA kernel
+// with 128-row tiles at every M measured, 16 to 4096); per-group scales: the
+// shared-memory-operand kernel.
 template <bool DEBUG>
 quik_status dispatch(const GemmArgs &a, cudaStream_t stream) {
-#ifndef QUIK_NG_LEGACY
     if (a.group == 0)
-        return a.out_int8 ? run_ts<true, DEBUG>(a, stream) : run_ts<false, DEBUG>(a, stream);
-#endif
-    if (a.group > 0)
-        return a.out_int8 ? run<CfgGroup<true, DEBUG>>(a, stream)
-                          : run<CfgGroup<false, DEBUG>>(a, stream);
-    return a.out_int8 ? run<CfgChannel<true, DEBUG>>(a, stream)
-                      : run<CfgChannel<false, DEBUG>>(a, stream);
+        return a.out_int8 ? run_pair<true, DEBUG>(a, stream) : run_pair<false, DEBUG>(a, stream);
+    return a.out_int8 ? run<CfgGroup<true, DEBUG>>(a, stream) : run<CfgGroup<false, DEBUG>>(a, stream);
 }
 
 // A CTA waiting on a barrier that nothing completes: exercises the bounded
