@@ -35,8 +35,10 @@
  *     returns QUIK_ERR_INVALID_ARG with nothing enqueued.  Pointers that are
  *     unused for the shape (outlier buffers when k_o == 0, INT8 scales in FP16
  *     mode, bias) may be NULL.
- *   - perm must be a permutation of 0..K-1; this is the caller's promise and
- *     is not checked.
+ *   - perm must be a permutation of 0..K-1.  Entries outside [0, K) are
+ *     never used as addresses: they read channel 0, are counted, and
+ *     quik_sync_check reports QUIK_ERR_INVALID_ARG.  Repeated entries are not
+ *     detected.
  *   - A launch failure returns QUIK_ERR_CUDA.  Every wait inside the GEMM
  *     kernel is bounded; if one runs out the kernel records it in a device
  *     error word and exits cleanly, and quik_sync_check reports
@@ -188,8 +190,9 @@ QUIK_API quik_status quik_gemm_i32_debug(const quik_shape *shape, const void *Xq
 
 /*
  * quik_sync_check -- synchronise `stream`, then report (and clear) the
- * device error word: QUIK_ERR_TIMEOUT if a bounded wait ran out in any
- * kernel since the last check, QUIK_ERR_CUDA on a CUDA error, else QUIK_OK.
+ * device error words: QUIK_ERR_TIMEOUT if a bounded wait ran out in any
+ * kernel since the last check, else QUIK_ERR_INVALID_ARG if a quantiser met
+ * a perm entry outside [0, K), QUIK_ERR_CUDA on a CUDA error, else QUIK_OK.
  */
 QUIK_API quik_status quik_sync_check(quik_stream_t stream);
 

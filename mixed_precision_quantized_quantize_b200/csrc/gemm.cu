@@ -1143,16 +1143,16 @@ extern "C" __attribute__((visibility("default"))) unsigned long long qchk_gemm_w
 
 quik_status sync_check(cudaStream_t stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return QUIK_ERR_CUDA;
-    unsigned int word = 0;
+    unsigned int word = 0, bad_perm = 0;
     if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return QUIK_ERR_CUDA;
-    const unsigned int qword = take_quantize_errors();
-    if (qword != 0 && word == 0) return QUIK_ERR_TIMEOUT;
+    const unsigned int qword = take_quantize_errors(&bad_perm);
     if (word != 0) {
         const unsigned int zero = 0;
         if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess)
             return QUIK_ERR_CUDA;
-        return QUIK_ERR_TIMEOUT;
     }
+    if (word != 0 || qword != 0) return QUIK_ERR_TIMEOUT;
+    if (bad_perm != 0) return QUIK_ERR_INVALID_ARG;
     return QUIK_OK;
 }
 

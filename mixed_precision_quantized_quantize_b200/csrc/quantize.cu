@@ -6,20 +6,32 @@
 // weight pack (one row per output channel; QUIK sample names pack_to_i4 /
 // two_compl).
 //
-// One CTA owns one row at a time (grid-stride over rows, 256 threads):
-//   1. the CTA stages perm (as uint16) once; the rows arrive in a ring of up
-//      to three shared-memory buffers, each filled by one TMA bulk copy issued
-//      as soon as the buffer is free, so several rows per CTA are in flight;
-//   2. each thread gathers 8 reordered positions per 32-bit output word
-//      (up to MAXW words, kept in registers), takes their absmax;
-//   3. per-row scale: block reduction; per-group scale (128 positions =
-//      16 words = 16 adjacent lanes): 4-step xor shuffle;
-//   4. codes are packed 8 per word and stored coalesced (a warp writes 128
-//      contiguous bytes);
+// Work split.  A team of TT = 32 * ceil(words / (32 W)) threads (a word = 8
+// codes; W words per thread) owns one row at a time; a CTA holds up to four
+// teams, which share one table of perm and otherwise run independently (their
+// own named barrier, their own ring of 2-4 row slots); CTAs are persistent and
+// rows are strided over all teams of the grid.  Per CTA:
+//   0. thread 0 starts one bulk copy of perm (int32) and those of every
+//      team's first rows (one per slot); all threads then turn perm in place into the
+//      table of byte offsets into a row (uint32; for K > 16384 uint16 element
+//      indices, built from 16-byte global loads).  An entry outside [0, K)
+//      becomes 0 and is reported (never used as an address).
+// Per row, in one team:
+//   1. the team leader waits for the row; a named barrier (OR-reducing a
+//      timeout flag) hands it to the team and frees the slot of the previous
+//      row, which the leader refills with the row a ring ahead;
+//   2. each thread gathers 8 reordered positions per word (as 4 half2), W
+//      words in registers, and takes their absmax;
+//   3. per-row scale: warp shuffles and a second team barrier; per-group
+//      scale (128 positions = 16 words = 16 adjacent lanes): 4-step xor
+//      shuffle.  s = fl(m / 7) is computed exactly in integer arithmetic
+//      (m is an fp16 value: at most 11 significant bits);
+//   4. codes are packed 8 per word (paired fp32 arithmetic) and stored
+//      coalesced (a warp writes 128 contiguous bytes);
 //   5. outlier positions Ki..K-1 are gathered and copied, or quantised with
-//      their own absmax/127 scale.
-// The kernel is bound by HBM bandwidth (2 bytes read per element, 0.5 byte
-// written per INT4 element).
+//      their own scale fl(absmax / 127).
+// The kernel is meant to be bound by HBM bandwidth (2 bytes read per
+// element, 0.5 byte written per INT4 code).
 #include <algorithm>
 #include <atomic>
 
@@ -32,19 +44,25 @@ namespace quik {
 
 QUIK_CHECK_DECL
 
-// Count of bounded waits that ran out in this file's kernels (read and
-// cleared by quik_sync_check through take_quantize_errors).
+// Count of bounded waits that ran out in this file's kernels, and of perm
+// entries outside [0, K) (both read and cleared by quik_sync_check through
+// take_quantize_errors).
 __device__ unsigned int g_quant_error;
+__device__ unsigned int g_quant_bad_perm;
 
 namespace {
 
-constexpr int kQThreads = 256;
+constexpr int kQMaxThreads = 512;  // 16 warps: up to 2048 words (W = 4) or 4096 (W = 8)
+constexpr int kQMaxTeams = 4;
+constexpr int kQMaxRing = 4;
 
 struct QParams {
     const uint16_t *X;
     const int32_t *perm;
     int rows, K, k_o;
-    int nring;  // row buffers per CTA (1..3)
+    int team_threads;  // TT, a multiple of 32
+    int teams;         // teams per CTA (1 .. 4)
+    int ring;          // row slots per team (2 .. 4)
     uint8_t *Q;
     float *scale;
     void *O;
@@ -64,6 +82,88 @@ constexpr uint32_t kRoundBits = 0x4B400000u;
 // b_k = 0x4B400000 + q_k the constant term is folded in advance (mod 2^32).
 constexpr uint32_t kPackBias = 0x88888888u - kRoundBits * 0x11111111u;
 
+// fl(m / D) for an odd divisor 2^(L-1) < D < 2^L and m >= 0 an fp16 value
+// widened to fp32 (so m == 0 or m is a normal fp32 with at most 11
+// significant bits).  With m = S 2^(E-150), S the 24-bit significand, the
+// quotient's 24-bit significand is the integer nearest to S 2^sh / D for the
+// shift sh in {L-1, L} that puts it in [2^23, 2^24]; the rounding is exact
+// integer arithmetic and never meets a tie (2 * remainder is even, D odd).
+template <uint32_t D, int L>
+__device__ __forceinline__ float div_exact(float m) {
+    static_assert((D & 1u) && D > (1u << (L - 1)) && D < (1u << L), "odd D in (2^(L-1), 2^L)");
+    const uint32_t b = __float_as_uint(m);
+    if (b == 0u) return 0.0f;
+    const uint32_t E = b >> 23;
+    const uint32_t S = (b & 0x7FFFFFu) | 0x800000u;
+    const int sh = (static_cast<uint64_t>(S) << L) < (static_cast<uint64_t>(D) << 24) ? L : L - 1;
+    const uint32_t num = S << sh;  // < 2^31
+    uint32_t q = num / D;
+    const uint32_t rem = num - q * D;
+    q += (2u * rem > D) ? 1u : 0u;
+    uint32_t e = E - static_cast<uint32_t>(sh);
+    if (q == (1u << 24)) {  // rounded up to the next binade
+        q = 1u << 23;
+        e += 1u;
+    }
+    return __uint_as_float((e << 23) | (q & 0x7FFFFFu));
+}
+
+// Hardware reciprocal (relative error at most 2^-23 for normal s; 0 for s == 0).
+__device__ __forceinline__ float rcp_approx(float s) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+    return s != 0.0f ? r : 0.0f;
+}
+
+// Paired fp32 arithmetic (sm_100 f32x2): two lanes per instruction, each
+// rounded to nearest like its scalar form.
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t r, float &a, float &b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+// The half2 (lo of a, lo of b) from two 16-bit loads.
+__device__ __forceinline__ uint32_t pair16(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+// Per lane, the operand of larger magnitude (its sign is not used): an
+// absmax that needs no separate |.|.
+__device__ __forceinline__ uint32_t absmax2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // Exact code of one value (the rare near-tie path): rint of the correctly
 // rounded fp32 quotient, clamped, 0 when s == 0.
 __device__ __forceinline__ int exact_code(float v, float s, int qmax) {
@@ -73,23 +173,31 @@ __device__ __forceinline__ int exact_code(float v, float s, int qmax) {
 }
 
 // Eight codes of one 32-bit output word from four half2 values.
-//   Fast path: t = v * fl(1/s).  With u = 2^-24, |t - fl(v/s)| <= 3u|v/s|(1+u)
-//   <= 1.3e-6 for |v/s| <= 7 (|v| <= max|v|, so |v/s| <= 7(1+u)^2), hence
-//   unless t lies within 2e-6 of a half-integer (the only points where rint
-//   changes value) fl(v/s) rounds to the same integer.  |t - rint(t)| is
-//   computed exactly (Sterbenz), and a word with any near-tie is redone with
-//   IEEE divisions.  No clamp is needed: |rint(t)| <= 7.
+//   Fast path: r = rint(v * rs) of the exact product (one fused
+//   multiply-add with 1.5 * 2^23), rs the hardware reciprocal of s (relative
+//   error <= 2u, u = 2^-24).  |v rs - fl(v/s)| <= |v/s| 3u <= 1.3e-6 for
+//   |v/s| <= 7(1+u) (|v| <= max|v|), so unless v rs lies within 2e-6 of a
+//   half-integer (the only points where rint changes value) fl(v/s) rounds
+//   to r as well.  The residual v rs - r comes from a second fused
+//   multiply-add (relative error u), and a word with any near-tie is redone
+//   with IEEE divisions.  No clamp is needed: |r| <= 7.
 __device__ __forceinline__ uint32_t pack_codes8(const uint32_t (&h)[4], float s, float rs) {
     uint32_t word = kPackBias;
     float dmax = 0.0f;
+    const uint64_t rs2 = f2(rs, rs), kr2 = f2(kRound, kRound);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[k]));
-        // explicit roundings: the product must not be contracted into the add
-        const float t0 = __fmul_rn(f.x, rs), t1 = __fmul_rn(f.y, rs);
-        const float m0 = __fadd_rn(t0, kRound), m1 = __fadd_rn(t1, kRound);
-        dmax = fmaxf(dmax, fmaxf(fabsf(__fsub_rn(t0, __fsub_rn(m0, kRound))),
-                                 fabsf(__fsub_rn(t1, __fsub_rn(m1, kRound)))));
+        const uint64_t v2 = f2(f.x, f.y);
+        const uint64_t m = f2_fma(v2, rs2, kr2);           // 1.5*2^23 + rint(v rs)
+        const uint64_t r = f2_sub(m, kr2);                 // rint(v rs), exact
+        float r0, r1;
+        f2_split(r, r0, r1);
+        const uint64_t d = f2_fma(v2, rs2, f2(-r0, -r1));  // v rs - rint(v rs)
+        float m0, m1, d0, d1;
+        f2_split(m, m0, m1);
+        f2_split(d, d0, d1);
+        dmax = max3(dmax, fabsf(d0), fabsf(d1));
         word += __float_as_uint(m0) << (8 * k);
         word += __float_as_uint(m1) << (8 * k + 4);
     }
@@ -106,11 +214,12 @@ __device__ __forceinline__ uint32_t pack_codes8(const uint32_t (&h)[4], float s,
     return word ^ 0x88888888u;
 }
 
-// INT8 outlier code (same fast path; |v/s| <= 127 widens the tie margin).
+// INT8 outlier code (same fast path; |v/s| <= 127(1+u) gives an error bound
+// of 2.3e-5 inside the 4e-5 tie margin).
 __device__ __forceinline__ int code8(float v, float s, float rs) {
-    const float t = __fmul_rn(v, rs);
-    const float m = __fadd_rn(t, kRound);
-    if (fabsf(__fsub_rn(t, __fsub_rn(m, kRound))) > 0.5f - 4e-5f) return exact_code(v, s, 127);
+    const float m = __fmaf_rn(v, rs, kRound);
+    const float r = __fsub_rn(m, kRound);
+    if (fabsf(__fmaf_rn(v, rs, -r)) > 0.5f - 4e-5f) return exact_code(v, s, 127);
     return static_cast<int>(__float_as_uint(m) - kRoundBits);
 }
 
@@ -125,227 +234,365 @@ __device__ __forceinline__ float half2_absmax(uint32_t m2) {
     return fmaxf(__low2float(a), __high2float(a));
 }
 
-template <bool GROUPED, bool OUT_INT8, int MAXW>
-__global__ void __launch_bounds__(kQThreads) quantize_rows_kernel(QParams p) {
+// Named barrier over one team (ids 1..4; id 0 is __syncthreads), returning
+// the OR of `pred` over the team's threads.
+__device__ __forceinline__ bool team_sync_or(int id, int nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void team_sync(int id, int nthreads) {
+    asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// P32: the perm table holds byte offsets (uint32); else element indices (uint16).
+template <bool GROUPED, bool OUT_INT8, int W, bool P32>
+__global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : GROUPED ? 64 : 56)
+    quantize_rows_kernel(QParams p) {
     extern __shared__ __align__(16) uint8_t qsmem[];
-    __shared__ float red_a[kQThreads / 32];
-    __shared__ float red_b[kQThreads / 32];
-    __shared__ uint64_t row_full[3];
-    __shared__ int give_up;
-    const int K = p.K, Ki = K - p.k_o;
-    const int Kp = (K + 7) & ~7;
-    uint16_t *perm_s = reinterpret_cast<uint16_t *>(qsmem);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ float red[kQMaxTeams][2][kQMaxThreads / 32];  // warp maxima, two slots per team
+    __shared__ uint64_t row_full[kQMaxTeams][kQMaxRing];
+    const int K = p.K, Ki = K - p.k_o;  // K % 16 == 0
+    const int TT = p.team_threads;
+    const int team = threadIdx.x / TT, tl = threadIdx.x - team * TT;  // team-local thread
+    const int lane = threadIdx.x & 31, twarp = tl >> 5;
+    const int bar_id = 1 + team;
     const int nwords = Ki / 8;
     const int G = GROUPED ? Ki / kGroup : 1;
     const uint32_t row_bytes = static_cast<uint32_t>(K) * 2;
-
-    auto ring = [&](int j) { return perm_s + Kp * (1 + j % p.nring); };
-    auto issue = [&](int j) {  // thread 0: bulk-copy this CTA's j-th row into its buffer
-        const int row = blockIdx.x + j * gridDim.x;
+    const uint32_t perm_bytes = P32 ? row_bytes * 2 : row_bytes;
+    const int stride = gridDim.x * p.teams;  // rows between a team's consecutive rows
+    const int first = blockIdx.x * p.teams + team;
+    const int NR = p.ring;
+    auto slot_off = [&](int t, int j) { return perm_bytes + (t * NR + j % NR) * row_bytes; };
+    auto issue = [&](int t, int j) {  // bulk-copy team t's j-th row into its slot j % NR
+        const int row = blockIdx.x * p.teams + t + j * stride;
         if (row < p.rows) {
-            ptx::mbar_arrive_expect_tx(&row_full[j % p.nring], row_bytes);
-            ptx::bulk_load(ring(j), p.X + static_cast<size_t>(row) * K, row_bytes, &row_full[j % p.nring]);
+            ptx::mbar_arrive_expect_tx(&row_full[t][j % NR], row_bytes);
+            ptx::bulk_load(qsmem + slot_off(t, j), p.X + static_cast<size_t>(row) * K, row_bytes,
+                           &row_full[t][j % NR]);
         }
     };
-    // Stage perm as uint16: one bulk copy of the int32 vector into the (still
-    // unused) row buffers, then an in-shared-memory narrowing.  A strided loop
-    // of global loads here would cost one memory latency per iteration.
     __shared__ uint64_t perm_full;
-    int32_t *perm32 = reinterpret_cast<int32_t *>(perm_s + Kp);  // needs 4K <= 2 Kp nring bytes
-    if (tid == 0) {
-        for (int s = 0; s < p.nring; ++s) ptx::mbar_init(&row_full[s], 1);
+    if (threadIdx.x == 0) {
+        for (int t = 0; t < p.teams; ++t)
+            for (int r = 0; r < NR; ++r) ptx::mbar_init(&row_full[t][r], 1);
         ptx::mbar_init(&perm_full, 1);
-        give_up = 0;
         ptx::fence_barrier_init();
-        ptx::mbar_arrive_expect_tx(&perm_full, static_cast<uint32_t>(K) * 4);
-        ptx::bulk_load(perm32, p.perm, static_cast<uint32_t>(K) * 4, &perm_full);
-        if (!ptx::mbar_wait_bounded(&perm_full, 0, kWaitLimitNs)) {
-            give_up = 1;
-            atomicAdd(&g_quant_error, 1u);
+        if (P32) {  // the int32 perm lands in the table area and is converted in place
+            ptx::mbar_arrive_expect_tx(&perm_full, perm_bytes);
+            ptx::bulk_load(qsmem, p.perm, perm_bytes, &perm_full);
         }
+        for (int t = 0; t < p.teams; ++t)
+            for (int r = 0; r < NR; ++r) issue(t, r);
     }
-    __syncthreads();
-    for (int i = tid; i < K / 4; i += kQThreads) {  // K % 4 == 0
-        const int4 v = reinterpret_cast<const int4 *>(perm32)[i];
-        reinterpret_cast<uint2 *>(perm_s)[i] =
-            make_uint2(static_cast<uint32_t>(v.x) | (static_cast<uint32_t>(v.y) << 16),
-                       static_cast<uint32_t>(v.z) | (static_cast<uint32_t>(v.w) << 16));
+    // (0) the perm table, while the first rows are in flight
+    bool perm_lost = false;  // the perm copy did not arrive in time
+    {
+        const unsigned uk = static_cast<unsigned>(K);
+        bool bad = false;
+        if (P32) {
+            __syncthreads();  // perm_full initialised
+            perm_lost = !ptx::mbar_wait_bounded_sleep(&perm_full, 0, kWaitLimitNs);
+        }
+        for (int i = threadIdx.x; i < K / 4; i += blockDim.x) {
+            uint4 v;
+            if (P32) {
+                v = reinterpret_cast<const uint4 *>(qsmem)[i];
+            } else {
+                const int4 g = __ldg(reinterpret_cast<const int4 *>(p.perm) + i);
+                v = make_uint4(static_cast<uint32_t>(g.x), static_cast<uint32_t>(g.y),
+                               static_cast<uint32_t>(g.z), static_cast<uint32_t>(g.w));
+            }
+            uint32_t e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                bad |= e[c] >= uk;
+                e[c] = e[c] < uk ? e[c] : 0u;
+            }
+            if (P32)
+                reinterpret_cast<uint4 *>(qsmem)[i] = make_uint4(2 * e[0], 2 * e[1], 2 * e[2], 2 * e[3]);
+            else
+                reinterpret_cast<uint2 *>(qsmem)[i] = make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16));
+        }
+        if (bad && blockIdx.x == 0) atomicAdd(&g_quant_bad_perm, 1u);
     }
-    __syncthreads();  // perm_s ready; the row buffers may now be overwritten
-    if (give_up) return;
-    if (tid == 0)
-        for (int j = 0; j < p.nring; ++j) issue(j);
+    // perm table and row barriers visible to all; if the perm copy was lost no
+    // row is processed (a late copy could still overwrite the table)
+    perm_lost = __syncthreads_or(perm_lost);
+    if (perm_lost && threadIdx.x == 0) {
+        atomicAdd(&g_quant_error, 1u);
+        ptx::mbar_wait_bounded(&perm_full, 0, kWaitLimitNs);
+    }
+    if (team >= p.teams) return;
 
-    for (int j = 0;; ++j) {
-        const int row = blockIdx.x + j * gridDim.x;
+    int issued = 0;  // leader: this team's rows 0 .. issued-1 have been requested
+    while (issued < NR && first + issued * stride < p.rows) ++issued;
+    for (int j = 0; !perm_lost; ++j) {
+        const int row = first + j * stride;
         if (row >= p.rows) break;
-        // (1) wait for this row's buffer (bounded; on expiry the row is skipped)
-        if (tid == 0 && !ptx::mbar_wait_bounded(&row_full[j % p.nring], (j / p.nring) & 1, kWaitLimitNs)) {
-            give_up = 1;
-            atomicAdd(&g_quant_error, 1u);
+        // (1) the leader waits for this row (bounded); the barrier hands it to
+        // the team and ends every thread's use of the previous slot
+        bool ok = true;
+        if (tl == 0) ok = ptx::mbar_wait_bounded_sleep(&row_full[team][j % NR], (j / NR) & 1, kWaitLimitNs);
+        if (team_sync_or(bar_id, TT, !ok)) {
+            if (tl == 0) atomicAdd(&g_quant_error, 1u);
+            break;
         }
-        __syncthreads();
-        if (give_up) break;
-        const uint16_t *row_s = ring(j);
+        if (tl == 0 && j > 0) {  // the slot of row j-1 takes row j-1+NR
+            issue(team, j - 1 + NR);
+            if (first + (j - 1 + NR) * stride < p.rows) issued = j + NR;
+        }
+        const uint8_t *row_s = qsmem + slot_off(team, j);
+        auto at = [&](uint32_t off) -> uint32_t { return *reinterpret_cast<const uint16_t *>(row_s + off); };
+        auto element = [&](uint32_t k) -> uint32_t {  // byte offset of reordered position k
+            if (P32) return reinterpret_cast<const uint32_t *>(qsmem)[k];
+            return 2u * reinterpret_cast<const uint16_t *>(qsmem)[k];
+        };
 
         // (2) gather 8 reordered values per word (as 4 half2), absmax per word
-        uint32_t v[MAXW][4];
-        float wmax[MAXW];
+        uint32_t v[W][4];
+        float wmax[W];
 #pragma unroll
-        for (int i = 0; i < MAXW; ++i) {
-            const int w = tid + i * kQThreads;
+        for (int i = 0; i < W; ++i) {
+            const int w = tl + i * TT;
             wmax[i] = 0.0f;
-            if (w < nwords && QUIK_CHECK(8 * w + 8 <= Kp, 2)) {
-                const uint4 ix = *reinterpret_cast<const uint4 *>(perm_s + 8 * w);
-                const uint32_t idx[4] = {ix.x, ix.y, ix.z, ix.w};
-                __half2 m2 = __float2half2_rn(0.0f);
+            if (w < nwords) {
+                uint32_t off[8];
+                if (P32) {
+                    const uint4 a = reinterpret_cast<const uint4 *>(qsmem)[2 * w];
+                    const uint4 b = reinterpret_cast<const uint4 *>(qsmem)[2 * w + 1];
+                    off[0] = a.x; off[1] = a.y; off[2] = a.z; off[3] = a.w;
+                    off[4] = b.x; off[5] = b.y; off[6] = b.z; off[7] = b.w;
+                } else {
+                    const uint4 a = reinterpret_cast<const uint4 *>(qsmem)[w];
+                    const uint32_t x[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    if (!QUIK_CHECK((idx[k] & 0xffffu) < (uint32_t)K && (idx[k] >> 16) < (uint32_t)K, 1)) {
-                        v[i][k] = 0;
-                        continue;
+                    for (int c = 0; c < 4; ++c) {
+                        off[2 * c] = 2u * (x[c] & 0xffffu);
+                        off[2 * c + 1] = 2u * (x[c] >> 16);
                     }
-                    const uint32_t a = row_s[idx[k] & 0xffffu], b = row_s[idx[k] >> 16];
-                    v[i][k] = a | (b << 16);
-                    m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __half2 *>(&v[i][k])));
                 }
-                wmax[i] = half2_absmax(*reinterpret_cast<const uint32_t *>(&m2));
+#pragma unroll
+                for (int k = 0; k < 4; ++k) v[i][k] = pair16(at(off[2 * k]), at(off[2 * k + 1]));
+                wmax[i] = half2_absmax(absmax2(absmax2(v[i][0], v[i][1]), absmax2(v[i][2], v[i][3])));
             }
         }
 
         // (3) scales
-        float s[MAXW];
+        float s[W], r[W];
         if (GROUPED) {
 #pragma unroll
-            for (int i = 0; i < MAXW; ++i) {
+            for (int i = 0; i < W; ++i) {
                 float m = wmax[i];
 #pragma unroll
                 for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                s[i] = __fdiv_rn(m, 7.0f);
-                const int w = tid + i * kQThreads;
+                s[i] = div_exact<7, 3>(m);
+                r[i] = rcp_approx(s[i]);
+                const int w = tl + i * TT;
                 if (w < nwords && (lane & 15) == 0 && QUIK_CHECK(w / 16 < G, 3))
                     p.scale[static_cast<size_t>(row) * G + w / 16] = s[i];
             }
         } else {
             float m = 0.0f;
 #pragma unroll
-            for (int i = 0; i < MAXW; ++i) m = fmaxf(m, wmax[i]);
+            for (int i = 0; i < W; ++i) m = fmaxf(m, wmax[i]);
             m = warp_max(m);
-            if (lane == 0) red_a[warp] = m;
-            __syncthreads();
-            m = red_a[0];
+            if (lane == 0) red[team][j & 1][twarp] = m;
+            team_sync(bar_id, TT);
+            m = 0.0f;
+            for (int k = 0; k < (TT >> 5); ++k) m = fmaxf(m, red[team][j & 1][k]);
+            const float sr = div_exact<7, 3>(m), rr = rcp_approx(sr);
 #pragma unroll
-            for (int k = 1; k < kQThreads / 32; ++k) m = fmaxf(m, red_a[k]);
-            const float sr = __fdiv_rn(m, 7.0f);
-#pragma unroll
-            for (int i = 0; i < MAXW; ++i) s[i] = sr;
-            if (tid == 0) p.scale[row] = sr;
+            for (int i = 0; i < W; ++i) {
+                s[i] = sr;
+                r[i] = rr;
+            }
+            if (tl == 0) p.scale[row] = sr;
         }
 
         // (4) codes, 8 per word, code 2i in the low nibble of byte i
         uint32_t *qrow = reinterpret_cast<uint32_t *>(p.Q + static_cast<size_t>(row) * (Ki / 2));
 #pragma unroll
-        for (int i = 0; i < MAXW; ++i) {
-            const int w = tid + i * kQThreads;
-            if (w < nwords && QUIK_CHECK(4 * w + 4 <= Ki / 2, 4)) {
-                const float rs = s[i] != 0.0f ? __frcp_rn(s[i]) : 0.0f;
-                qrow[w] = pack_codes8(v[i], s[i], rs);
-            }
+        for (int i = 0; i < W; ++i) {
+            const int w = tl + i * TT;
+            if (w < nwords && QUIK_CHECK(4 * w + 4 <= Ki / 2, 4)) qrow[w] = pack_codes8(v[i], s[i], r[i]);
         }
 
         // (5) the outlier block
         if (p.k_o > 0) {
             if (!OUT_INT8) {
                 uint16_t *o = static_cast<uint16_t *>(p.O) + static_cast<size_t>(row) * p.k_o;
-                for (int i = tid; i < p.k_o; i += kQThreads)
-                    if (QUIK_CHECK(perm_s[Ki + i] < K, 5)) o[i] = row_s[perm_s[Ki + i]];
+                for (int i = tl; i < p.k_o; i += TT)
+                    o[i] = static_cast<uint16_t>(at(element(Ki + i)));
             } else {
                 float m = 0.0f;
-                for (int i = tid; i < p.k_o; i += kQThreads)
-                    m = fmaxf(m, fabsf(h2f(row_s[perm_s[Ki + i]])));
+                for (int i = tl; i < p.k_o; i += TT)
+                    m = fmaxf(m, fabsf(h2f(static_cast<uint16_t>(at(element(Ki + i))))));
                 m = warp_max(m);
-                if (lane == 0) red_b[warp] = m;
-                __syncthreads();
-                m = red_b[0];
-#pragma unroll
-                for (int k = 1; k < kQThreads / 32; ++k) m = fmaxf(m, red_b[k]);
-                const float so = __fdiv_rn(m, 127.0f);
-                const float rso = so != 0.0f ? __frcp_rn(so) : 0.0f;
-                if (tid == 0) p.o_scale[row] = so;
+                // the other reduction slot: this row's slot is read above and
+                // is not written again before the next row's opening barrier
+                if (lane == 0) red[team][(j & 1) ^ 1][twarp] = m;
+                team_sync(bar_id, TT);
+                m = 0.0f;
+                for (int k = 0; k < (TT >> 5); ++k) m = fmaxf(m, red[team][(j & 1) ^ 1][k]);
+                const float so = div_exact<127, 7>(m), rso = rcp_approx(so);
+                if (tl == 0) p.o_scale[row] = so;
                 int8_t *o = static_cast<int8_t *>(p.O) + static_cast<size_t>(row) * p.k_o;
-                for (int i = tid; i < p.k_o; i += kQThreads)
-                    o[i] = static_cast<int8_t>(code8(h2f(row_s[perm_s[Ki + i]]), so, rso));
+                for (int i = tl; i < p.k_o; i += TT)
+                    o[i] = static_cast<int8_t>(
+                        code8(h2f(static_cast<uint16_t>(at(element(Ki + i)))), so, rso));
             }
-        } else if (OUT_INT8 && p.o_scale != nullptr && tid == 0) {
+        } else if (OUT_INT8 && p.o_scale != nullptr && tl == 0) {
             p.o_scale[row] = 0.0f;
         }
-        __syncthreads();  // buffer and reduction slots are free again
-        if (tid == 0) issue(j + p.nring);
     }
-    // never leave the CTA with a bulk copy still writing its shared memory
-    if (tid == 0)
-        for (int s = 0; s < p.nring; ++s) {
-            // the last row issued into slot s, if any
-            int last = -1;
-            for (int j = s; blockIdx.x + j * gridDim.x < p.rows; j += p.nring) last = j;
-            if (last >= 0) ptx::mbar_wait_bounded(&row_full[s], (last / p.nring) & 1, kWaitLimitNs);
-        }
+    // never leave the CTA with a bulk copy still writing its shared memory:
+    // wait for the last row requested into each of the team's slots
+    if (tl == 0)
+        for (int j = issued > NR ? issued - NR : 0; j < issued; ++j)
+            ptx::mbar_wait_bounded(&row_full[team][j % NR], (j / NR) & 1, kWaitLimitNs);
 }
 
-template <bool GROUPED, bool OUT_INT8, int MAXW>
-cudaError_t launch_q(QParams p, cudaStream_t stream) {
-    auto kern = quantize_rows_kernel<GROUPED, OUT_INT8, MAXW>;
-    const int Kp = (p.K + 7) & ~7;
-    const size_t row_bytes = static_cast<size_t>(Kp) * sizeof(uint16_t);
-    // perm (uint16) plus up to three row buffers within ~200 KB of shared memory
-    p.nring = static_cast<int>(std::min<size_t>(3, (200u << 10) / row_bytes - 1));
-    if (p.nring < 2) return cudaErrorInvalidConfiguration;  // the ring also stages perm (int32)
-    const size_t smem = row_bytes * (1 + p.nring);
-    if (!attribute_set_once(reinterpret_cast<const void *>(kern), static_cast<int>(smem)))
-        return cudaErrorInvalidConfiguration;
-    // grid: every CTA that fits at once, rows grid-strided; the occupancy of
-    // the last shared-memory size seen is cached (one query per new K)
-    static std::atomic<long long> occ_cache{-1};  // (smem << 8) | CTAs per SM
-    long long c = occ_cache.load(std::memory_order_relaxed);
-    int per_sm = 0;
-    if (c >= 0 && (c >> 8) == static_cast<long long>(smem)) {
-        per_sm = static_cast<int>(c & 0xff);
-    } else {
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kQThreads, smem);
-        if (e != cudaSuccess) return e;
-        occ_cache.store((static_cast<long long>(smem) << 8) | (per_sm & 0xff), std::memory_order_relaxed);
+struct QShape {
+    int W, TT, teams, ring;
+    bool p32;
+    size_t smem;
+};
+
+// Registers per thread of one kernel instance (queried once).
+template <bool GROUPED, bool OUT_INT8, int W, bool P32>
+int q_regs() {
+    static std::atomic<int> regs{0};
+    int r = regs.load(std::memory_order_relaxed);
+    if (r == 0) {
+        cudaFuncAttributes fa{};
+        if (cudaFuncGetAttributes(&fa, quantize_rows_kernel<GROUPED, OUT_INT8, W, P32>) != cudaSuccess)
+            return 0;
+        r = fa.numRegs;
+        regs.store(r, std::memory_order_relaxed);
     }
-    const int grid = std::max(1, std::min(p.rows, sm_count() * std::max(per_sm, 1)));
-    kern<<<grid, kQThreads, smem, stream>>>(p);
+    return r;
+}
+
+// CTAs of `threads` threads, `regs` registers each and `smem` bytes of
+// dynamic shared memory that fit on one SM (sm_100: 64 K registers allocated
+// per warp in units of 256, 2048 threads, 228 KB of shared memory with 1 KB
+// reserved per CTA).
+int ctas_per_sm(int threads, int regs, size_t smem) {
+    if (regs <= 0) return 0;
+    const int warps = (threads + 31) / 32;
+    const int regs_per_warp = ((regs * 32 + 255) / 256) * 256;
+    const int by_regs = 65536 / (regs_per_warp * warps);
+    const int by_threads = 2048 / (warps * 32);
+    const int by_smem = static_cast<int>((228u << 10) / (smem + 1024 + 1024));  // + static shared memory
+    return std::max(0, std::min(std::min(by_regs, by_threads), std::min(by_smem, 32)));
+}
+
+// W (words per thread): with few rows per SM (at most two), the fewest that
+// fit one row in 16 warps, for the shortest row latency; otherwise the fewest
+// that keep a team at 4 warps, up to 16 warps at W = 4 (K_i <= 16384), then
+// W = 8 (K_i <= 32768).  Then teams per CTA (at most 4 and 512 threads), row
+// slots per team (2 .. 4) and the perm table's width (uint32 byte offsets, or
+// uint16 indices with an extraction per element) are chosen for the most
+// teams per SM; ties go to the uint32 table, then to more slots.
+template <bool GROUPED, bool OUT_INT8>
+QShape q_shape(int rows, int K, int k_o) {
+    const int nwords = (K - k_o) / 8;
+    int W;
+    if (rows <= 2 * sm_count())
+        W = nwords <= 512 ? 1 : nwords <= 1024 ? 2 : nwords <= 2048 ? 4 : 8;
+    else
+        W = nwords <= 128 ? 1 : nwords <= 256 ? 2 : nwords <= 2048 ? 4 : 8;
+    const int TT = std::max(32, 32 * ((nwords + 32 * W - 1) / (32 * W)));
+    const size_t row = static_cast<size_t>(K) * 2;
+    QShape best{W, TT, 0, 0, true, 0};
+    int best_score = -1;
+    for (int p32 = 1; p32 >= 0; --p32) {
+        int regs = 0;
+        switch (W) {
+            case 1: regs = p32 ? q_regs<GROUPED, OUT_INT8, 1, true>() : q_regs<GROUPED, OUT_INT8, 1, false>(); break;
+            case 2: regs = p32 ? q_regs<GROUPED, OUT_INT8, 2, true>() : q_regs<GROUPED, OUT_INT8, 2, false>(); break;
+            case 4: regs = p32 ? q_regs<GROUPED, OUT_INT8, 4, true>() : q_regs<GROUPED, OUT_INT8, 4, false>(); break;
+            default: regs = p32 ? q_regs<GROUPED, OUT_INT8, 8, true>() : q_regs<GROUPED, OUT_INT8, 8, false>(); break;
+        }
+        const size_t table = p32 ? 2 * row : row;
+        for (int teams = std::min(kQMaxTeams, kQMaxThreads / TT); teams >= 1; --teams)
+            for (int ring = kQMaxRing; ring >= 2; --ring) {
+                const size_t smem = table + static_cast<size_t>(teams) * ring * row;
+                if (smem > (227u << 10) - 1024) continue;
+                const int per_sm = ctas_per_sm(TT * teams, regs, smem);
+                if (per_sm == 0) continue;
+                // teams per SM first; then the wider table; then deeper rings
+                const int score = (per_sm * teams) * 16 + p32 * 8 + ring;
+                if (score > best_score) {
+                    best_score = score;
+                    best = QShape{W, TT, teams, ring, p32 != 0, smem};
+                }
+            }
+    }
+    return best;
+}
+
+template <bool GROUPED, bool OUT_INT8, int W, bool P32>
+cudaError_t launch_q(QParams p, const QShape &qs, cudaStream_t stream) {
+    auto kern = quantize_rows_kernel<GROUPED, OUT_INT8, W, P32>;
+    p.team_threads = qs.TT;
+    p.teams = qs.teams;
+    p.ring = qs.ring;
+    const int threads = qs.TT * qs.teams;
+    if (qs.teams < 1 || qs.ring < 2 || qs.ring > kQMaxRing || threads > kQMaxThreads ||
+        qs.smem > (227u << 10))
+        return cudaErrorInvalidConfiguration;
+    if (!attribute_set_once(reinterpret_cast<const void *>(kern), static_cast<int>(qs.smem)))
+        return cudaErrorInvalidConfiguration;
+    const int per_sm = ctas_per_sm(threads, q_regs<GROUPED, OUT_INT8, W, P32>(), qs.smem);
+    // grid: every CTA that fits at once (persistent), or fewer when the rows run out
+    const int need = (p.rows + qs.teams - 1) / qs.teams;
+    const int grid = std::max(1, std::min(need, sm_count() * std::max(per_sm, 1)));
+    kern<<<grid, threads, qs.smem, stream>>>(p);
     return cudaGetLastError();
 }
 
 template <bool GROUPED, bool OUT_INT8>
 cudaError_t launch_q_w(const QParams &p, cudaStream_t stream) {
-    const int words_per_thread = ((p.K - p.k_o) / 8 + kQThreads - 1) / kQThreads;
-    if (words_per_thread <= 2) return launch_q<GROUPED, OUT_INT8, 2>(p, stream);
-    if (words_per_thread <= 4) return launch_q<GROUPED, OUT_INT8, 4>(p, stream);
-    if (words_per_thread <= 8) return launch_q<GROUPED, OUT_INT8, 8>(p, stream);
-    return launch_q<GROUPED, OUT_INT8, 16>(p, stream);
+    const QShape qs = q_shape<GROUPED, OUT_INT8>(p.rows, p.K, p.k_o);
+    switch (qs.W * 2 + (qs.p32 ? 1 : 0)) {
+        case 3: return launch_q<GROUPED, OUT_INT8, 1, true>(p, qs, stream);
+        case 2: return launch_q<GROUPED, OUT_INT8, 1, false>(p, qs, stream);
+        case 5: return launch_q<GROUPED, OUT_INT8, 2, true>(p, qs, stream);
+        case 4: return launch_q<GROUPED, OUT_INT8, 2, false>(p, qs, stream);
+        case 9: return launch_q<GROUPED, OUT_INT8, 4, true>(p, qs, stream);
+        case 8: return launch_q<GROUPED, OUT_INT8, 4, false>(p, qs, stream);
+        case 17: return launch_q<GROUPED, OUT_INT8, 8, true>(p, qs, stream);
+        default: return launch_q<GROUPED, OUT_INT8, 8, false>(p, qs, stream);
+    }
 }
 
 }  // namespace
 
 cudaError_t launch_quantize_rows(const QuantizeArgs &a, cudaStream_t stream) {
-    QParams p{a.X, a.perm, a.rows, a.K, a.k_o, 1, a.Q, a.scale, a.O, a.o_scale};
+    QParams p{a.X, a.perm, a.rows, a.K, a.k_o, 0, 0, 0, a.Q, a.scale, a.O, a.o_scale};
     if (a.group > 0)
         return a.out_int8 ? launch_q_w<true, true>(p, stream) : launch_q_w<true, false>(p, stream);
     return a.out_int8 ? launch_q_w<false, true>(p, stream) : launch_q_w<false, false>(p, stream);
 }
 
-unsigned int take_quantize_errors() {
-    unsigned int word = 0;
+unsigned int take_quantize_errors(unsigned int *bad_perm) {
+    unsigned int word = 0, bad = 0;
     if (cudaMemcpyFromSymbol(&word, g_quant_error, sizeof(word)) != cudaSuccess) return 0;
-    if (word != 0) {
-        const unsigned int zero = 0;
-        cudaMemcpyToSymbol(g_quant_error, &zero, sizeof(zero));
-    }
+    if (cudaMemcpyFromSymbol(&bad, g_quant_bad_perm, sizeof(bad)) != cudaSuccess) return 0;
+    const unsigned int zero = 0;
+    if (word != 0) cudaMemcpyToSymbol(g_quant_error, &zero, sizeof(zero));
+    if (bad != 0) cudaMemcpyToSymbol(g_quant_bad_perm, &zero, sizeof(zero));
+    if (bad_perm != nullptr) *bad_perm = bad;
     return word;
 }
 

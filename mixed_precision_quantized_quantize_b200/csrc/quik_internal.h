@@ -41,8 +41,9 @@ struct QuantizeArgs {
     float *o_scale;
 };
 cudaError_t launch_quantize_rows(const QuantizeArgs &a, cudaStream_t stream);
-// Read and clear the quantise kernels' count of expired waits (synchronous).
-unsigned int take_quantize_errors();
+// Read and clear the quantise kernels' count of expired waits (returned) and
+// of perm entries outside [0, K) (stored in *bad_perm when given); synchronous.
+unsigned int take_quantize_errors(unsigned int *bad_perm);
 
 // INT4 x INT4 (+ outlier) product with the dequantising epilogue, or the raw
 // integer sums when acc_dbg is set.

@@ -46,6 +46,8 @@ SHAPES = [
     # (a producer running ahead must never alias a barrier phase)
     (200, 300, 8320, 128, 128, True, True),  # 64 groups + INT8 outliers
     (130, 260, 8256, 64, 0, False, True),    # 64 INT4 k-blocks + FP16 outliers
+    # K_i = 20480: the quantiser's widest rows (8 words per thread, 10 warps)
+    (33, 72, 20544, 64, 0, True, True),
 ]
 
 
@@ -126,6 +128,54 @@ def test_zero_rows_and_ties():
         sc = g[1].cpu().numpy().reshape(M, -1)
         assert (sc[3] == 0).all() and (sc[17] == 0).all()
     del perm_t
+
+
+@pytest.mark.parametrize("group,int8", [(0, False), (0, True), (128, True)])
+def test_quantize_many_rows_per_cta(group, int8):
+    """8192 rows: every quantiser CTA walks several rows through its two-slot ring."""
+    M, K, k_o = 8192, 1024 + 64, 64
+    cfg, d = _case(M, 16, K, k_o, group, int8, False, seed=11)
+    g = q.quantize_reorder(d["X"].to(DEV), d["perm"].to(DEV), k_o, group, int8)
+    torch.cuda.synchronize()
+    assert_quant_equal(gpu_tuple_np(g), oracle_quant(d["X"], d["perm"], k_o, group, int8))
+
+
+@pytest.mark.parametrize("int8", [False, True])
+def test_scales_for_every_fp16_absmax(int8):
+    """Row r's absmax runs over every finite non-negative fp16 value: the scales are the
+    IEEE fp32 quotients fl(m / 7) and fl(m / 127), and codes match the oracle bit for bit."""
+    vals = np.arange(0, 0x7C00, dtype=np.uint16).view(np.float16)  # +0 .. 65504
+    M, Ki, k_o = len(vals), 32, 16
+    K = Ki + k_o
+    X = np.zeros((M, K), np.float16)
+    X[:, 0] = vals
+    X[:, 1] = -vals
+    X[:, 5] = (vals.astype(np.float32) * np.float32(0.3)).astype(np.float16)
+    X[:, 9] = (vals.astype(np.float32) * np.float32(-0.77)).astype(np.float16)
+    X[:, Ki] = vals
+    X[:, Ki + 3] = (vals.astype(np.float32) * np.float32(0.51)).astype(np.float16)
+    perm = torch.arange(K, dtype=torch.int32)
+    g = q.quantize_reorder(torch.from_numpy(X).to(DEV), perm.to(DEV), k_o, 0, int8)
+    torch.cuda.synchronize()
+    got = gpu_tuple_np(g)
+    m32 = vals.astype(np.float32)
+    np.testing.assert_array_equal(got[1].reshape(-1).view(np.uint32), (m32 / np.float32(7)).view(np.uint32))
+    if int8:
+        np.testing.assert_array_equal(got[3].reshape(-1).view(np.uint32), (m32 / np.float32(127)).view(np.uint32))
+    assert_quant_equal(got, oracle.quantize_rows(X, perm.numpy(), k_o, 0, int8))
+
+
+def test_out_of_range_perm_is_reported():
+    """perm entries outside [0, K) are never read out of bounds; sync_check reports them."""
+    M, K, k_o = 8, 256, 32
+    X = torch.randn((M, K), dtype=torch.float16, device=DEV)
+    perm = torch.arange(K, dtype=torch.int32)
+    perm[5] = K + 3
+    perm[9] = -1
+    assert q.quik_sync_check() == q.QUIK_OK
+    q.quantize_reorder(X, perm.to(DEV), k_o)
+    assert q.quik_sync_check() == q.QUIK_ERR_INVALID_ARG
+    assert q.quik_sync_check() == q.QUIK_OK  # the count was cleared
 
 
 def test_canary_guards_untouched():
