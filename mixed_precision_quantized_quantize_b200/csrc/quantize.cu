@@ -52,6 +52,11 @@ __device__ unsigned int g_quant_bad_perm;
 
 namespace {
 
+using ptx::f2;
+using ptx::f2_fma;
+using ptx::f2_split;
+using ptx::f2_sub;
+
 constexpr int kQMaxThreads = 512;  // 16 warps: up to 2048 words (W = 4) or 4096 (W = 8)
 constexpr int kQMaxTeams = 4;
 constexpr int kQMaxRing = 4;
@@ -115,36 +120,6 @@ __device__ __forceinline__ float rcp_approx(float s) {
     return s != 0.0f ? r : 0.0f;
 }
 
-// Paired fp32 arithmetic (sm_100 f32x2): two lanes per instruction, each
-// rounded to nearest like its scalar form.
-__device__ __forceinline__ uint64_t f2(float a, float b) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-__device__ __forceinline__ void f2_split(uint64_t r, float &a, float &b) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
-}
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
 // The half2 (lo of a, lo of b) from two 16-bit loads.
 __device__ __forceinline__ uint32_t pair16(uint32_t a, uint32_t b) {
     uint32_t r;
