@@ -106,6 +106,38 @@ def profiled_traffic():
         return None
 
 
+def library_context(cfg, X, W, flush, steps: int = 20):
+    """Same-shape library GEMMs for context (never this library's arithmetic): the fp16
+    product the method replaces (torch.matmul -> cuBLAS) and cuBLASLt INT8
+    (torch._int_mm, where its shape rules allow), each with the L2 flushed."""
+    import torch
+
+    def timed(fn):
+        for _ in range(3):
+            flush.zero_()
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for a, b in ev:
+            flush.zero_()
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        return float(np.median([a.elapsed_time(b) for a, b in ev])) * 1e3
+
+    Wt = W.t()
+    out = {"fp16_matmul_us": round(timed(lambda: torch.matmul(X, Wt)), 2)}
+    try:
+        g = torch.Generator(device=X.device).manual_seed(5)
+        Xi = torch.randint(-7, 8, (cfg.M, cfg.K), dtype=torch.int8, device=X.device, generator=g)
+        Wi = torch.randint(-7, 8, (cfg.K, cfg.N), dtype=torch.int8, device=X.device, generator=g)
+        out["int8_int_mm_us"] = round(timed(lambda: torch._int_mm(Xi, Wi)), 2)
+    except (RuntimeError, TypeError):
+        out["int8_int_mm_us"] = None
+    return out
+
+
 # ----------------------------------------------------------------- clocks (NVML, read only)
 class ClockSampler:
     """Samples SM clock, power and throttle reasons every ~5 ms in a thread."""
@@ -312,6 +344,19 @@ def run_ours(args, rank, local_rank, world):
     barrier()
     e2e_value, _ = aggregate([a.elapsed_time(b) / 1e3 for a, b in ev], cfg.ops, world, reduce_max)
 
+    # ---- the same step with a warm L2 (no flush between steps)
+    wev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(20)]
+    torch.cuda.synchronize()
+    for i in range(20):
+        wev[i][0].record(stream)
+        step()
+        wev[i][1].record(stream)
+    torch.cuda.synchronize()
+    warm_us = float(np.median([a.elapsed_time(b) for a, b in wev])) * 1e3
+    context = library_context(cfg, X, d["W"].to(dev), flush)
+    context["warm_l2_us_per_call"] = round(warm_us, 2)
+    context["layer_speedup_vs_fp16_matmul"] = round(context["fp16_matmul_us"] / (t_step * 1e6), 3)
+
     peaks, peak_kind = measured_peaks()
     int8_peak = float(peaks["bf16_tflops"]) * INT8_PER_BF16
     gemm_tops = cfg.ops / gemm_avg / 1e12
@@ -356,6 +401,7 @@ def run_ours(args, rank, local_rank, world):
                 "call": "quik_linear via QuikLinear, pinned host X in, host Y out"},
         "gpu_launches": 2 * args.steps,
         "clocks": sampler.summary(),
+        "context": context,
     }
     if world > 1:
         dist.barrier(device_ids=[local_rank])
