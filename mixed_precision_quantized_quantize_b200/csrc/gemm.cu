@@ -108,6 +108,7 @@ using CfgGroup = Cfg<128, true, OUT_INT8, DEBUG, 4, 8, 4, 4, 1>;
 
 struct GemmParams {
     int M, N, Ki, k_o, nkb_i, nkb_o, G;
+    int tma_y;  // pair kernel: Y leaves through shared memory and TMA stores
     const float *sx, *sw, *sxo, *swo;
     const uint16_t *bias;
     uint16_t *Y;
@@ -622,6 +623,9 @@ constexpr int PK_OFF = S * STAGE;
 constexpr int SMEM = PK_OFF + SP * UNIT + 1024;
 constexpr int ACC_COL = 0, A_COL = 256, O_COL = 256, TMEM_COLS = 512;
 constexpr int PF = 4;                     // k-blocks of A loads in flight per thread
+static_assert(NA == 4 && NB == 8, "the epilogue splits each lane quadrant's 8 column chunks 3 / 3 / 2");
+static_assert(STAGE % 1024 == 0 && B_BYTES % 1024 == 0, "128-byte-swizzled staging blocks");
+static_assert(XO_BYTES == 128 * 128 && S * 64 >= BN, "the output tile stages in the stages' outlier-X areas");
 static_assert(A_COL + 32 * S <= TMEM_COLS, "A stages fit in tensor memory");
 static_assert(SMEM <= 232448, "shared memory budget");
 }  // namespace pair
@@ -631,6 +635,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
     w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_wq,
                           const __grid_constant__ CUtensorMap tm_wo,
                           const __grid_constant__ CUtensorMap tm_xo,
+                          const __grid_constant__ CUtensorMap tm_y,
                           const uint8_t *__restrict__ Xq, const GemmParams p) {
     using namespace pair;
     extern __shared__ uint8_t smem_raw[];
@@ -760,80 +765,154 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
                 if (last[st] >= 0) mbar_wait_bounded(&pk_full[st], (last[st] / SP) & 1, kWaitLimitNs);
         }
         __syncwarp();
-    } else if (warp < 2 + NA) {
-        // ------------------------------------------------------------ A rows -> TMEM (each CTA)
-        const int q = warp & 3;
-        const int r = q * 32 + lane;  // tile row = TMEM lane
-        const int grow = m0 + r;
-        const bool row_ok = grow < p.M;
-        const uint8_t *xrow = Xq + (size_t)grow * rb;
-        const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
-        uint4 buf[PF][4];
-        auto load = [&](int kb, uint4(&d)[4]) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int off = kb * PK_ROW + c * 16;
-                d[c] = (row_ok && off < rb) ? ldg_nc_v4(xrow + off) : make_uint4(0, 0, 0, 0);
-            }
-        };
-#pragma unroll
-        for (int j = 0; j < PF; ++j)
-            if (j < p.nkb_i) load(j, buf[j]);
+    } else {
+        // A warps (TMEM operand) and B warps (shared-memory operand) feed the
+        // MMA, then all 12 run the epilogue
         bool ok = true;
-        for (int kb0 = 0; kb0 < p.nkb_i && ok; kb0 += PF) {
+        if (warp < 2 + NA) {
+            // ------------------------------------------------------------ A rows -> TMEM (each CTA)
+            const int q = warp & 3;
+            const int r = q * 32 + lane;  // tile row = TMEM lane
+            const int grow = m0 + r;
+            const bool row_ok = grow < p.M;
+            const uint8_t *xrow = Xq + (size_t)grow * rb;
+            const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
+            uint4 buf[PF][4];
+            auto load = [&](int kb, uint4(&d)[4]) {
 #pragma unroll
-            for (int j = 0; j < PF; ++j) {
-                const int kb = kb0 + j;
-                if (kb >= p.nkb_i || !ok) break;
+                for (int c = 0; c < 4; ++c) {
+                    const int off = kb * PK_ROW + c * 16;
+                    d[c] = (row_ok && off < rb) ? ldg_nc_v4(xrow + off) : make_uint4(0, 0, 0, 0);
+                }
+            };
+#pragma unroll
+            for (int j = 0; j < PF; ++j)
+                if (j < p.nkb_i) load(j, buf[j]);
+            for (int kb0 = 0; kb0 < p.nkb_i && ok; kb0 += PF) {
+#pragma unroll
+                for (int j = 0; j < PF; ++j) {
+                    const int kb = kb0 + j;
+                    if (kb >= p.nkb_i || !ok) break;
+                    const int st = kb % S;
+                    ok = wait_bar(&op_empty[st], ((kb / S) & 1) ^ 1, ab);
+                    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                    uint32_t w[32];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint4 lo, hi;
+                        unpack16(buf[j][c], lo, hi);
+                        w[8 * c + 0] = lo.x; w[8 * c + 1] = lo.y; w[8 * c + 2] = lo.z; w[8 * c + 3] = lo.w;
+                        w[8 * c + 4] = hi.x; w[8 * c + 5] = hi.y; w[8 * c + 6] = hi.z; w[8 * c + 7] = hi.w;
+                    }
+                    tmem_st_32x32b_x32(t_lane + A_COL + 32 * st, w);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(leader_full(st));
+    #ifdef QUIK_TRACE
+                    if (lane == 0 && blockIdx.x + blockIdx.y * gridDim.x < kTraceCtas && kb < kTraceKb)
+                        atomicMax(&g_trace[blockIdx.x + blockIdx.y * gridDim.x][2][kb], clock64());
+    #endif
+                    if (kb + PF < p.nkb_i) load(kb + PF, buf[j]);
+                }
+            }
+            // outlier k-blocks: both operands arrive through shared memory
+            for (int kb = p.nkb_i; kb < nkb && ok; ++kb) {
                 const int st = kb % S;
                 ok = wait_bar(&op_empty[st], ((kb / S) & 1) ^ 1, ab);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-                uint32_t w[32];
+                if (lane == 0) mbar_arrive_remote(leader_full(st));
+            }
+
+        } else {
+            // ------------------------------------------------------------ B half: staging -> operand stage
+            const int tb = threadIdx.x - 32 * (2 + NA);  // 0 .. 32*NB-1
+            int u = 0;
+            for (int kb = 0; kb < nkb && ok; ++kb) {
+                const int st = kb % S;
+                ok = wait_bar(&op_empty[st], ((kb / S) & 1) ^ 1, ab);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                uint8_t *bst = smem + st * STAGE;
+                if (tb == 0) QUIK_TRACE_AT(1, kb);
+                const int nparts = kb < p.nkb_i ? 1 : 2;
+                for (int part = 0; part < nparts && ok; ++part, ++u) {
+                    const int ps = u % SP;
+                    ok = wait_bar(&pk_full[ps], (u / SP) & 1, ab);
+                    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                    if (tb == 0 && part == 0) QUIK_TRACE_AT(8, kb);
+                    const uint8_t *pk = smem + PK_OFF + ps * UNIT;
+                    if (kb < p.nkb_i) {
+                        // 128 rows x 4 chunks: unpack each 16-byte chunk into two
+                        const int ch = tb & 3;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint4 lo, hi;
-                    unpack16(buf[j][c], lo, hi);
-                    w[8 * c + 0] = lo.x; w[8 * c + 1] = lo.y; w[8 * c + 2] = lo.z; w[8 * c + 3] = lo.w;
-                    w[8 * c + 4] = hi.x; w[8 * c + 5] = hi.y; w[8 * c + 6] = hi.z; w[8 * c + 7] = hi.w;
+                        for (int i = 0; i < 128 / (8 * NB); ++i) {
+                            const int row = tb / 4 + 8 * NB * i;
+                            const uint4 v = *reinterpret_cast<const uint4 *>(pk + row * PK_ROW + ch * 16);
+                            uint4 lo, hi;
+                            unpack16(v, lo, hi);
+                            uint8_t *rp = bst + row * OP_ROW;
+                            *reinterpret_cast<uint4 *>(rp + (((2 * ch) ^ (row & 7)) << 4)) = lo;
+                            *reinterpret_cast<uint4 *>(rp + (((2 * ch + 1) ^ (row & 7)) << 4)) = hi;
+                        }
+                    } else {
+                        // Wo rows (part 0) into the B area, Xo rows (part 1) into the A area:
+                        // 128 rows x 8 chunks each
+                        const int c = tb & 7;
+                        uint8_t *dst = part == 0 ? bst : bst + B_BYTES;
+#pragma unroll
+                        for (int i = 0; i < 32 / NB; ++i) {
+                            const int row = tb / 8 + 4 * NB * i;
+                            const uint4 v = *reinterpret_cast<const uint4 *>(pk + row * OP_ROW + c * 16);
+                            *reinterpret_cast<uint4 *>(dst + row * OP_ROW + ((c ^ (row & 7)) << 4)) = v;
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pk_empty[ps]);
                 }
-                tmem_st_32x32b_x32(t_lane + A_COL + 32 * st, w);
-                tmem_st_wait();
-                tc_fence_before();
+                if (!ok) break;
+                if (tb == 0) QUIK_TRACE_AT(9, kb);
+                fence_proxy_async_smem();  // generic-proxy stores -> visible to the pair's MMA
+                if (tb == 0) QUIK_TRACE_AT(10, kb);
                 __syncwarp();
                 if (lane == 0) mbar_arrive_remote(leader_full(st));
-#ifdef QUIK_TRACE
+    #ifdef QUIK_TRACE
                 if (lane == 0 && blockIdx.x + blockIdx.y * gridDim.x < kTraceCtas && kb < kTraceKb)
-                    atomicMax(&g_trace[blockIdx.x + blockIdx.y * gridDim.x][2][kb], clock64());
-#endif
-                if (kb + PF < p.nkb_i) load(kb + PF, buf[j]);
+                    atomicMax(&g_trace[blockIdx.x + blockIdx.y * gridDim.x][0][kb], clock64());
+    #endif
             }
-        }
-        // outlier k-blocks: both operands arrive through shared memory
-        for (int kb = p.nkb_i; kb < nkb && ok; ++kb) {
-            const int st = kb % S;
-            ok = wait_bar(&op_empty[st], ((kb / S) & 1) ^ 1, ab);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            if (lane == 0) mbar_arrive_remote(leader_full(st));
         }
 
         // ------------------------------------------------------------ epilogue (each CTA)
-        for (int c = threadIdx.x - 64; c < BN; c += 32 * NA) {
+        // The 12 A and B warps: each on its TMEM lane quadrant (warp % 4) and a
+        // third of the 256 columns (32-column chunks 0-2 / 3-5 / 6-7).  With
+        // tma_y the fp16 tile is staged, 128-byte swizzled, in the four stages'
+        // outlier-X areas (64 columns each; every MMA has finished reading them)
+        // and leaves by TMA stores; else each thread stores its row directly.
+        const int ep = threadIdx.x - 64;  // 0 .. 32 * (NA + NB) - 1
+        for (int c = ep; c < BN; c += 32 * (NA + NB)) {
             const int n = n0 + c;
             const bool in = n < p.N;
             col_sw[c] = (in && p.Ki > 0) ? p.sw[n] : 0.0f;
             col_swo[c] = (in && OUT_INT8 && p.nkb_o > 0) ? p.swo[n] : 0.0f;
             col_bias[c] = (in && p.bias != nullptr) ? __half2float(__ushort_as_half(p.bias[n])) : 0.0f;
         }
-        named_barrier_sync(1, 32 * NA);
+        named_barrier_sync(1, 32 * (NA + NB));
         ok = ok && wait_bar(&acc_full, 0, ab);
         if (__all_sync(0xffffffffu, ok)) {
             tc_fence_after();
-            if (q == 1 && lane == 0) QUIK_TRACE_AT(4, 0);
+            if (warp == 3 && lane == 0) QUIK_TRACE_AT(4, 0);
+            const int q = warp & 3;
+            const int wq = warp < 2 + NA ? 0 : warp < 6 + NA ? 1 : 2;  // A, first or second B warp
+            const int ch_lo = wq == 0 ? 0 : wq == 1 ? 3 : 6, ch_hi = wq == 0 ? 3 : wq == 1 ? 6 : 8;
+            const int r = q * 32 + lane;  // tile row = TMEM lane
+            const int grow = m0 + r;
+            const bool row_ok = grow < p.M;
+            const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
             const float sxr = (row_ok && p.Ki > 0) ? p.sx[grow] : 0.0f;
             const float sxo = (row_ok && OUT_INT8 && p.nkb_o > 0) ? p.sxo[grow] : 0.0f;
             uint16_t *yrow = p.Y + (size_t)grow * p.N;
-            for (int cc = 0; cc < BN; cc += 32) {
-                const int nb = n0 + cc;
+            for (int ch = ch_lo; ch < ch_hi; ++ch) {
+                const int cc = ch * 32, nb = n0 + cc;
                 uint32_t a[32], o[32];
                 if (p.Ki > 0) tmem_ld_32x32b_x32(t_lane + ACC_COL + cc, a);
                 if (p.nkb_o > 0) tmem_ld_32x32b_x32(t_lane + O_COL + cc, o);
@@ -872,7 +951,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
                     }
                     packed[jj / 2] = pack_half2(y[0], y[1]);
                 }
-                if (row_ok) {
+                if (p.tma_y) {
+                    // 64-column block ch/2 lives in stage (ch/2)'s outlier-X area
+                    uint8_t *blk = smem + (ch >> 1) * STAGE + B_BYTES + r * 128;
+                    const int c16 = (ch & 1) * 4;
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4)
+                        *reinterpret_cast<uint4 *>(blk + (((c16 + v4) ^ (r & 7)) << 4)) =
+                            make_uint4(packed[4 * v4], packed[4 * v4 + 1], packed[4 * v4 + 2], packed[4 * v4 + 3]);
+                } else if (row_ok) {
                     if (nb + 32 <= p.N && (p.N & 7) == 0) {
                         uint4 *dst = reinterpret_cast<uint4 *>(yrow + nb);
 #pragma unroll
@@ -887,64 +974,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
                 }
             }
             tc_fence_before();
-            if (q == 1 && lane == 0) QUIK_TRACE_AT(5, 0);
+            if (p.tma_y) fence_proxy_async_smem();  // staged tile -> visible to the TMA stores
+            if (warp == 3 && lane == 0) QUIK_TRACE_AT(5, 0);
         }
-    } else {
-        // ------------------------------------------------------------ B half: staging -> operand stage
-        const int tb = threadIdx.x - 32 * (2 + NA);  // 0 .. 32*NB-1
-        bool ok = true;
-        int u = 0;
-        for (int kb = 0; kb < nkb && ok; ++kb) {
-            const int st = kb % S;
-            ok = wait_bar(&op_empty[st], ((kb / S) & 1) ^ 1, ab);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            uint8_t *bst = smem + st * STAGE;
-            if (tb == 0) QUIK_TRACE_AT(1, kb);
-            const int nparts = kb < p.nkb_i ? 1 : 2;
-            for (int part = 0; part < nparts && ok; ++part, ++u) {
-                const int ps = u % SP;
-                ok = wait_bar(&pk_full[ps], (u / SP) & 1, ab);
-                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-                if (tb == 0 && part == 0) QUIK_TRACE_AT(8, kb);
-                const uint8_t *pk = smem + PK_OFF + ps * UNIT;
-                if (kb < p.nkb_i) {
-                    // 128 rows x 4 chunks: unpack each 16-byte chunk into two
-                    const int ch = tb & 3;
-#pragma unroll
-                    for (int i = 0; i < 128 / (8 * NB); ++i) {
-                        const int row = tb / 4 + 8 * NB * i;
-                        const uint4 v = *reinterpret_cast<const uint4 *>(pk + row * PK_ROW + ch * 16);
-                        uint4 lo, hi;
-                        unpack16(v, lo, hi);
-                        uint8_t *rp = bst + row * OP_ROW;
-                        *reinterpret_cast<uint4 *>(rp + (((2 * ch) ^ (row & 7)) << 4)) = lo;
-                        *reinterpret_cast<uint4 *>(rp + (((2 * ch + 1) ^ (row & 7)) << 4)) = hi;
-                    }
-                } else {
-                    // Wo rows (part 0) into the B area, Xo rows (part 1) into the A area:
-                    // 128 rows x 8 chunks each
-                    const int c = tb & 7;
-                    uint8_t *dst = part == 0 ? bst : bst + B_BYTES;
-#pragma unroll
-                    for (int i = 0; i < 32 / NB; ++i) {
-                        const int row = tb / 8 + 4 * NB * i;
-                        const uint4 v = *reinterpret_cast<const uint4 *>(pk + row * OP_ROW + c * 16);
-                        *reinterpret_cast<uint4 *>(dst + row * OP_ROW + ((c ^ (row & 7)) << 4)) = v;
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&pk_empty[ps]);
-            }
-            if (!ok) break;
-            if (tb == 0) QUIK_TRACE_AT(9, kb);
-            fence_proxy_async_smem();  // generic-proxy stores -> visible to the pair's MMA
-            if (tb == 0) QUIK_TRACE_AT(10, kb);
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote(leader_full(st));
-#ifdef QUIK_TRACE
-            if (lane == 0 && blockIdx.x + blockIdx.y * gridDim.x < kTraceCtas && kb < kTraceKb)
-                atomicMax(&g_trace[blockIdx.x + blockIdx.y * gridDim.x][0][kb], clock64());
-#endif
+        named_barrier_sync(1, 32 * (NA + NB));  // tile staged
+        if (threadIdx.x == 32 * (2 + NA) && p.tma_y && ok && m0 < p.M) {
+            for (int b = 0; b < BN / 64; ++b)
+                if (n0 + 64 * b < p.N) tma_store_2d(&tm_y, smem + b * STAGE + B_BYTES, n0 + 64 * b, m0);
+            bulk_commit_group();
+            bulk_wait_group0();  // the stores complete before the CTA leaves
         }
     }
 
@@ -1081,10 +1119,17 @@ quik_status run_pair(const GemmArgs &a, cudaStream_t stream) {
     p.Y = a.Y;
     p.acc_dbg = a.acc_dbg;
     p.acc_o_dbg = a.acc_o_dbg;
+    // Y by TMA stores of 128-row x 64-column blocks (128-byte swizzle) when its
+    // rows are 16-byte multiples; else per-thread stores
+    CUtensorMap my;
+    std::memset(&my, 0, sizeof(my));
+    p.tma_y = !DEBUG && (a.N % 8 == 0) &&
+              make_map(&my, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.Y, a.N, a.M, static_cast<uint64_t>(a.N) * 2,
+                       64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
     auto kern = w4a4_gemm_pair_kernel<OUT_INT8, DEBUG>;
     if (!attribute_set_once(reinterpret_cast<const void *>(kern), pair::SMEM)) return QUIK_ERR_CUDA;
     const dim3 grid(2 * ((a.N + pair::BN - 1) / pair::BN), (a.M + 2 * BM - 1) / (2 * BM));
-    kern<<<grid, pair::THREADS, pair::SMEM, stream>>>(mwq, mwo, mxo,
+    kern<<<grid, pair::THREADS, pair::SMEM, stream>>>(mwq, mwo, mxo, my,
                                                       static_cast<const uint8_t *>(a.Xq), p);
     return cudaGetLastError() == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
 }
