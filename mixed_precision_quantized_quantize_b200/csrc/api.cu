@@ -117,7 +117,7 @@ static quik_status gemm_impl(const quik_shape *shape, const void *Xq, const floa
                              const void *Xo, const float *xo_scale, const void *Wq,
                              const float *w_scale, const void *Wo, const float *wo_scale,
                              const void *bias, void *Y, bool debug, int32_t *acc,
-                             int32_t *acc_o, cudaStream_t stream) {
+                             int32_t *acc_o, cudaStream_t stream, bool after_quantize = false) {
     quik::GemmArgs a;
     a.M = shape->M;
     a.N = shape->N;
@@ -136,6 +136,7 @@ static quik_status gemm_impl(const quik_shape *shape, const void *Xq, const floa
     a.bias = static_cast<const uint16_t *>(bias);
     a.Y = static_cast<uint16_t *>(Y);
     a.debug = debug;
+    a.after_quantize = after_quantize;
     a.acc_dbg = acc;
     a.acc_o_dbg = acc_o;
     return quik::launch_gemm(a, stream);
@@ -172,8 +173,10 @@ quik_status quik_linear(const quik_shape *shape, const void *X_f16, const int32_
     float *sxo = int8_out(shape) ? reinterpret_cast<float *>(ws + w.sxo) : nullptr;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if ((st = quantize(shape, shape->M, X_f16, perm, Xq, sx, Xo, sxo, s)) != QUIK_OK) return st;
+    // the GEMM follows this quantiser on the same stream: its set-up and weight
+    // loads may overlap the quantiser's tail
     return gemm_impl(shape, Xq, sx, Xo, sxo, Wq, w_scale, Wo, wo_scale, bias_f16, Y_f16, false,
-                     nullptr, nullptr, s);
+                     nullptr, nullptr, s, true);
 }
 
 quik_status quik_gemm_i32_debug(const quik_shape *shape, const void *Xq, const void *Wq,

@@ -752,6 +752,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
                     tma_load_2d(dst, &tm_wq, u * PK_ROW, nb0, &pk_full[st]);
                 } else {
                     const int v = u - p.nkb_i, ko = v / 2;
+                    if (v == 0) grid_dependency_wait();  // Xo comes from the previous kernel
                     mbar_arrive_expect_tx(&pk_full[st], UNIT);
                     if (v % 2 == 0)  // this CTA's 128 rows of Wo, 128 bytes each
                         tma_load_2d(dst, &tm_wo, ko * OP_ROW, nb0, &pk_full[st]);
@@ -778,6 +779,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
             const uint8_t *xrow = Xq + (size_t)grow * rb;
             const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
             uint4 buf[PF][4];
+            grid_dependency_wait();  // Xq (and later sx) come from the previous kernel
             auto load = [&](int kb, uint4(&d)[4]) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -888,6 +890,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
         // tma_y the fp16 tile is staged, 128-byte swizzled, in the four stages'
         // outlier-X areas (64 columns each; every MMA has finished reading them)
         // and leaves by TMA stores; else each thread stores its row directly.
+        grid_dependency_wait();           // sx and sxo come from the previous kernel
         const int ep = threadIdx.x - 64;  // 0 .. 32 * (NA + NB) - 1
         for (int c = ep; c < BN; c += 32 * (NA + NB)) {
             const int n = n0 + c;
@@ -1129,9 +1132,26 @@ quik_status run_pair(const GemmArgs &a, cudaStream_t stream) {
     auto kern = w4a4_gemm_pair_kernel<OUT_INT8, DEBUG>;
     if (!attribute_set_once(reinterpret_cast<const void *>(kern), pair::SMEM)) return QUIK_ERR_CUDA;
     const dim3 grid(2 * ((a.N + pair::BN - 1) / pair::BN), (a.M + 2 * BM - 1) / (2 * BM));
-    kern<<<grid, pair::THREADS, pair::SMEM, stream>>>(mwq, mwo, mxo, my,
-                                                      static_cast<const uint8_t *>(a.Xq), p);
-    return cudaGetLastError() == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
+    if (!a.after_quantize) {
+        kern<<<grid, pair::THREADS, pair::SMEM, stream>>>(mwq, mwo, mxo, my,
+                                                          static_cast<const uint8_t *>(a.Xq), p);
+        return cudaGetLastError() == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
+    }
+    // programmatic dependent launch: the CTAs may start while the quantiser
+    // finishes; every read of its outputs waits on the grid dependency first
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(pair::THREADS);
+    cfg.dynamicSmemBytes = pair::SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const uint8_t *xq = static_cast<const uint8_t *>(a.Xq);
+    return cudaLaunchKernelEx(&cfg, kern, mwq, mwo, mxo, my, xq, p) == cudaSuccess ? QUIK_OK
+                                                                                  : QUIK_ERR_CUDA;
 }
 
 // Per-channel scales: the CTA-pair kernel (faster than a single-CTA kernel

@@ -53,6 +53,7 @@ __device__ unsigned int g_quant_bad_perm;
 namespace {
 
 using ptx::f2;
+using ptx::grid_launch_dependents;
 using ptx::f2_fma;
 using ptx::f2_split;
 using ptx::f2_sub;
@@ -256,6 +257,9 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : GROUPE
         }
     };
     __shared__ uint64_t perm_full;
+    // a GEMM launched after this kernel with a programmatic dependency may be
+    // scheduled now (it waits for this grid before it reads Xq and the scales)
+    grid_launch_dependents();
     if (threadIdx.x == 0) {
         for (int t = 0; t < p.teams; ++t)
             for (int r = 0; r < NR; ++r) ptx::mbar_init(&row_full[t][r], 1);

@@ -61,6 +61,8 @@ struct GemmArgs {
     const uint16_t *bias;
     uint16_t *Y;
     bool debug;          // write the integer sums instead of Y
+    bool after_quantize; // the previous kernel on the stream is this library's quantiser of Xq
+                         // (the GEMM may then start early: programmatic dependent launch)
     int32_t *acc_dbg;    // [M,N] or [G,M,N] integer sums of the INT4 part (debug only)
     int32_t *acc_o_dbg;  // INT8 outliers' integer sums (debug only)
 };

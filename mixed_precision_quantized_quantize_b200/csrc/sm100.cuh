@@ -101,6 +101,19 @@ __device__ __forceinline__ bool mbar_wait_bounded_sleep(uint64_t *bar, uint32_t 
     }
 }
 
+// ----------------------------------------------------------------- grid dependencies
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before the previous kernel of its stream ends;
+// grid_dependency_wait() blocks until that kernel has completed and its
+// memory is visible (a no-op without such a dependency).
+// grid_launch_dependents() lets the next such kernel start early.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------------- fences / barriers
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
