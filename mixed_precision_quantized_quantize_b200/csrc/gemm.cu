@@ -1000,6 +1000,316 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
     }
 }
 
+// ============================================================================
+// Decode-shaped product: M <= 32 tokens, per-channel scales, k_o <= 256.
+//
+// With a few tokens the layer is bound by reading W (N x K_i / 2 bytes), and a
+// 128-row token tile would leave most MMA rows empty.  Here the operands swap:
+// the MMA computes D[n, m] = sum_k W'[n,k] X'[m,k] with W as its 128-row A
+// operand and the tokens as its N (16 or 32), so no MMA row is idle.  One CTA
+// owns 128 rows of W:
+//   warp 0       TMEM allocator; lane 0 issues the MMAs: first the outlier
+//                block (kind::f16, or kind::i8 for INT8 outliers; both
+//                operands by TMA in the 128-byte-swizzled layout), then the
+//                INT4 k-blocks (kind::i8, A from tensor memory)
+//   warp 1       TMA producer: the outlier tiles once; then per k-block one
+//                unit of the packed W tile (128 rows x 64 bytes, 64-byte
+//                swizzle) and the packed token rows (32 x 64 bytes), in a
+//                10-deep ring
+//   warps 2-17   W, four groups of four warps taking k-blocks in turn (group
+//                g owns operand stage g, so four k-blocks are in flight; one
+//                group alone spends ~750 dependent cycles per k-block): row r
+//                = TMEM lane r reads its 64 packed bytes (the swizzle keeps
+//                the reads conflict-free), unpacks them and writes tensor
+//                memory; the group also unpacks the k-block's token rows into
+//                the 128-byte-swizzled X stage.  They keep no global loads in
+//                flight, so the proxy fence that publishes the X stage waits
+//                only for their own shared-memory stores.  Group 0 runs the
+//                epilogue, which writes Y[m, n] for fixed m across the lanes
+//                (coalesced).
+namespace gemv {
+constexpr int BW = 128;                      // W rows per CTA = TMEM lanes
+constexpr int MT = 32;                       // most tokens (the MMA's N: 16 or 32)
+constexpr int S = 4;                         // operand stages (A in TMEM, X in shared memory)
+constexpr int SPW = 10;                      // staging units
+constexpr int WUNIT = BW * PK_ROW;           // 8 KB of packed W
+constexpr int XUNIT = MT * PK_ROW;           // 2 KB of packed token rows
+constexpr int XSTAGE = MT * OP_ROW;          // 4 KB
+constexpr int KO_MAX = 256;                  // outlier channels handled here
+constexpr int OKB = 4;                       // outlier k-blocks of 128 bytes (k_o <= 256 fp16)
+constexpr int WO_TILE = BW * OP_ROW;         // 16 KB: 128 rows x 128 bytes
+constexpr int XO_TILE = MT * OP_ROW;         // 4 KB
+constexpr int NG = 4;                        // W warp groups (4 warps each), one per stage
+constexpr int NW = 4 * NG;                   // W warps
+constexpr int THREADS = (2 + NW) * 32;       // 576
+constexpr int XU_OFF = SPW * WUNIT;          // W staging first, then the token-row staging
+constexpr int X_OFF = XU_OFF + SPW * XUNIT;
+constexpr int WO_OFF = X_OFF + S * XSTAGE;
+constexpr int XO_OFF = WO_OFF + OKB * WO_TILE;
+constexpr int SMEM = XO_OFF + OKB * XO_TILE + 1024;  // + alignment
+constexpr int ACC_COL = 0, O_COL = 32, A_COL = 64, TMEM_COLS = 256;
+static_assert(A_COL + 32 * S <= TMEM_COLS, "A stages fit in tensor memory");
+static_assert(NG == S, "group g owns operand stage g");
+static_assert(X_OFF % 1024 == 0 && WO_OFF % 1024 == 0 && XO_OFF % 1024 == 0, "128-byte-swizzled tiles");
+static_assert(SMEM <= 232448, "shared memory budget");
+}  // namespace gemv
+
+template <bool OUT_INT8, bool DEBUG>
+__global__ void __launch_bounds__(gemv::THREADS, 1)
+    w4a4_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                     const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_xo,
+                     const GemmParams p) {
+    using namespace gemv;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t w_full[SPW], w_empty[SPW], op_full[S], op_empty[S], o_full, acc_full, mma_done;
+    __shared__ uint32_t tmem_base_s;
+    __shared__ int abort_s;
+    __shared__ unsigned err0_s;
+
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+    const uint32_t smem_base = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BW;
+    const int MP = p.M <= 16 ? 16 : 32;  // the MMA's N
+    const int nkb = p.nkb_i;
+    // outlier k-blocks of 128 bytes: 64 fp16 or 128 int8 channels each
+    const int oke = OUT_INT8 ? 128 : 64;
+    const int nko = (p.k_o + oke - 1) / oke;
+
+    const int early = nkb < SPW ? nkb : SPW;  // W units loaded before the CTA barrier
+    if (threadIdx.x == 0) QUIK_TRACE_AT(6, 0);
+    if (warp == 1 && lane == 0) {
+        // The producer's barriers, and the first ring of W tiles at once: W
+        // is not the previous kernel's output, and the first tiles' DRAM
+        // latency then overlaps the rest of the set-up.  Their token rows
+        // (and the tokens' outlier tile) follow after the grid dependency.
+        for (int i = 0; i < SPW; ++i) {
+            mbar_init(&w_full[i], 1);
+            mbar_init(&w_empty[i], 4);  // the four warps of the k-block's group
+        }
+        mbar_init(&o_full, 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+        if (nkb > 0) {
+            tma_prefetch_desc(&tm_w);
+            tma_prefetch_desc(&tm_x);
+        }
+        for (int u = 0; u < early; ++u) {
+            mbar_arrive_expect_tx(&w_full[u], WUNIT + XUNIT);
+            tma_load_2d(smem + u * WUNIT, &tm_w, u * PK_ROW, n0, &w_full[u]);
+            QUIK_TRACE_AT(11, u);
+        }
+        if (nko > 0) {
+            tma_prefetch_desc(&tm_wo);
+            tma_prefetch_desc(&tm_xo);
+            mbar_arrive_expect_tx(&o_full, nko * (WO_TILE + XO_TILE));
+            for (int kb = 0; kb < nko; ++kb)
+                tma_load_2d(smem + WO_OFF + kb * WO_TILE, &tm_wo, kb * oke, n0, &o_full);
+        }
+    }
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&op_full[i], 4);
+            mbar_init(&op_empty[i], 1);
+        }
+        mbar_init(&acc_full, 1);
+        mbar_init(&mma_done, 1);
+        abort_s = 0;
+        err0_s = *reinterpret_cast<volatile unsigned *>(&g_error_word);
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc(&tmem_base_s, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_s;
+    const AbortState ab{&abort_s, err0_s};
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            bool ok = true;
+            if (nko > 0) {  // the outlier block: both operands in shared memory
+                ok = wait_bar(&o_full, 0, ab);
+                QUIK_TRACE_AT(2, 0);
+                if (ok) {
+                    tc_fence_after();
+                    const uint32_t id_o = OUT_INT8 ? idesc_s8_s32(BW, MP) : idesc_f16_f32(BW, MP);
+                    for (int kb = 0; kb < nko; ++kb) {
+                        const uint32_t wo = smem_base + WO_OFF + kb * WO_TILE;
+                        const uint32_t xo = smem_base + XO_OFF + kb * XO_TILE;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint64_t ad = sw128_kmajor_desc(wo + 32 * k);
+                            const uint64_t bd = sw128_kmajor_desc(xo + 32 * k);
+                            if (OUT_INT8)
+                                mma_i8(tmem + O_COL, ad, bd, id_o, (kb > 0 || k > 0));
+                            else
+                                mma_f16(tmem + O_COL, ad, bd, id_o, (kb > 0 || k > 0));
+                        }
+                    }
+                }
+            }
+            const uint32_t idesc = idesc_s8_s32(BW, MP);
+            for (int kb = 0; kb < nkb && ok; ++kb) {
+                const int st = kb % S;
+                if (!(ok = wait_bar(&op_full[st], (kb / S) & 1, ab))) break;
+                QUIK_TRACE_AT(3, kb);
+                tc_fence_after();
+                const uint32_t xb = smem_base + X_OFF + st * XSTAGE;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_i8_ts(tmem + ACC_COL, tmem + A_COL + 32 * st + 8 * k, sw128_kmajor_desc(xb + 32 * k),
+                              idesc, (kb > 0 || k > 0));
+                mma_commit(&op_empty[st]);
+            }
+            if (ok) mma_commit(&acc_full);
+            mma_commit(&mma_done);
+            mbar_wait_bounded(&mma_done, 0, kWaitLimitNs);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            grid_dependency_wait();  // Xq and Xo come from the previous kernel
+            for (int kb = 0; kb < nko; ++kb)
+                tma_load_2d(smem + XO_OFF + kb * XO_TILE, &tm_xo, kb * oke, 0, &o_full);
+            for (int u = 0; u < early; ++u)
+                tma_load_2d(smem + XU_OFF + u * XUNIT, &tm_x, u * PK_ROW, 0, &w_full[u]);
+            int filled = early;  // units issued
+            for (int u = early; u < nkb; ++u, ++filled) {
+                const int st = u % SPW;
+                if (!wait_bar(&w_empty[st], ((u / SPW) & 1) ^ 1, ab)) break;
+                mbar_arrive_expect_tx(&w_full[st], WUNIT + XUNIT);
+                tma_load_2d(smem + st * WUNIT, &tm_w, u * PK_ROW, n0, &w_full[st]);
+                tma_load_2d(smem + XU_OFF + st * XUNIT, &tm_x, u * PK_ROW, 0, &w_full[st]);
+                QUIK_TRACE_AT(11, u);
+            }
+            // never leave the CTA with a bulk copy still writing its shared
+            // memory: slot i last held unit i + SPW * ((filled - 1 - i) / SPW)
+            for (int i = 0; i < early; ++i)
+                mbar_wait_bounded(&w_full[i], ((filled - 1 - i) / SPW) & 1, kWaitLimitNs);
+            if (nko > 0) mbar_wait_bounded(&o_full, 0, kWaitLimitNs);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ W rows -> TMEM, token rows -> X stage
+        const int q = warp & 3;           // TMEM lane quadrant
+        const int r = q * 32 + lane;      // W row in the tile = TMEM lane
+        const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
+        const int grp = (warp - 2) >> 2;  // this warp's group: k-blocks grp, grp + NG, ...
+        // this lane's share of the token rows: MP rows x 4 16-byte chunks over
+        // the group's 4 warps (one chunk per lane; lanes >= MP idle for MP = 16)
+        const int xw = (warp - 2) & 3;
+        const int x_row = xw * (MP / 4) + (lane >> 2), x_ch = lane & 3;
+        const bool x_on = lane < MP;
+        // epilogue operands of group 0, loaded now so that the epilogue waits
+        // on no global load: the row's weight scales and bias (not the
+        // previous kernel's output) before the grid dependency, the token
+        // scales (lane m holds token m's) after it
+        const int n = n0 + r;
+        const bool n_ok = n < p.N;
+        float swn = 0.0f, swon = 0.0f, bn = 0.0f, sxm = 0.0f, sxom = 0.0f;
+        if (grp == 0 && !DEBUG) {
+            if (n_ok && p.Ki > 0) swn = p.sw[n];
+            if (n_ok && OUT_INT8 && nko > 0) swon = p.swo[n];
+            if (n_ok && p.bias != nullptr) bn = __half2float(__ushort_as_half(p.bias[n]));
+        }
+        grid_dependency_wait();  // sx (and sxo) come from the previous kernel
+        if (grp == 0 && !DEBUG && lane < p.M) {
+            if (p.Ki > 0) sxm = p.sx[lane];
+            if (OUT_INT8 && nko > 0) sxom = p.sxo[lane];
+        }
+        bool ok = true;
+        for (int kb = grp; kb < nkb && ok; kb += NG) {
+            const int st = kb % S, ps = kb % SPW;
+            ok = wait_bar(&op_empty[st], ((kb / S) & 1) ^ 1, ab);
+            if (xw == 0 && lane == 0) QUIK_TRACE_AT(1, kb);
+            ok = ok && wait_bar(&w_full[ps], (kb / SPW) & 1, ab);
+            if (xw == 0 && lane == 0) QUIK_TRACE_AT(8, kb);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            if (x_on) {  // token row x_row, chunk x_ch -> two 16-byte unpacked chunks
+                const uint4 v = *reinterpret_cast<const uint4 *>(smem + XU_OFF + ps * XUNIT +
+                                                                 x_row * PK_ROW + x_ch * 16);
+                uint4 lo, hi;
+                unpack16(v, lo, hi);
+                uint8_t *xr = smem + X_OFF + st * XSTAGE + x_row * OP_ROW;
+                *reinterpret_cast<uint4 *>(xr + (((2 * x_ch) ^ (x_row & 7)) << 4)) = lo;
+                *reinterpret_cast<uint4 *>(xr + (((2 * x_ch + 1) ^ (x_row & 7)) << 4)) = hi;
+            }
+            // W row r: 4 chunks of 16 packed bytes, 64-byte swizzle
+            const uint8_t *wr = smem + ps * WUNIT + r * PK_ROW;
+            uint32_t w[32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(wr + ((c ^ ((r >> 1) & 3)) << 4));
+                uint4 lo, hi;
+                unpack16(v, lo, hi);
+                w[8 * c + 0] = lo.x; w[8 * c + 1] = lo.y; w[8 * c + 2] = lo.z; w[8 * c + 3] = lo.w;
+                w[8 * c + 4] = hi.x; w[8 * c + 5] = hi.y; w[8 * c + 6] = hi.z; w[8 * c + 7] = hi.w;
+            }
+            if (xw == 0 && lane == 0) QUIK_TRACE_AT(9, kb);
+            tmem_st_32x32b_x32(t_lane + A_COL + 32 * st, w);
+            tmem_st_wait();
+            fence_proxy_async_smem();  // the X stage's stores -> visible to the MMA
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&w_empty[ps]);
+                mbar_arrive(&op_full[st]);
+                if (xw == 0) QUIK_TRACE_AT(0, kb);
+            }
+        }
+        // ------------------------------------------------------------ epilogue (group 0)
+        if (grp == 0) {
+            ok = ok && wait_bar(&acc_full, 0, ab);
+            if (xw == 0 && lane == 0) QUIK_TRACE_AT(4, 0);
+            if (__all_sync(0xffffffffu, ok)) {
+                tc_fence_after();
+                // two halves of 16 tokens (the second only when M > 16)
+                for (int h = 0; h < 32 && h < p.M; h += 16) {
+                    uint32_t a[16], o[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) a[j] = o[j] = 0;
+                    if (nkb > 0) tmem_ld_32x32b_x16(t_lane + ACC_COL + h, a);
+                    if (nko > 0) tmem_ld_32x32b_x16(t_lane + O_COL + h, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int m = h + j;
+                        const float sx_m = __shfl_sync(0xffffffffu, sxm, m);
+                        const float sxo_m = __shfl_sync(0xffffffffu, sxom, m);
+                        if (m >= p.M || !n_ok) continue;
+                        const size_t at = (size_t)m * p.N + n;
+                        if (DEBUG) {
+                            if (p.Ki > 0) p.acc_dbg[at] = static_cast<int32_t>(a[j]) >> 8;
+                            if (OUT_INT8 && nko > 0 && p.acc_o_dbg) p.acc_o_dbg[at] = static_cast<int32_t>(o[j]);
+                            continue;
+                        }
+                        float y = p.Ki > 0 ? small_int_to_float(static_cast<int32_t>(a[j]) >> 8) * sx_m * swn : 0.0f;
+                        if (nko > 0)
+                            y += OUT_INT8 ? static_cast<float>(static_cast<int32_t>(o[j])) * sxo_m * swon
+                                          : __uint_as_float(o[j]);
+                        p.Y[at] = __half_as_ushort(__float2half_rn(y + bn));
+                    }
+                }
+                if (xw == 0 && lane == 0) QUIK_TRACE_AT(5, 0);
+                tc_fence_before();
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+    if (threadIdx.x == 0) QUIK_TRACE_AT(7, 0);
+}
+
 // ----------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -1154,11 +1464,78 @@ quik_status run_pair(const GemmArgs &a, cudaStream_t stream) {
                                                                                   : QUIK_ERR_CUDA;
 }
 
+// Decode-shaped launches: one CTA per 128 rows of W.
+template <bool OUT_INT8, bool DEBUG>
+quik_status run_gemv(const GemmArgs &a, cudaStream_t stream) {
+    const int Ki = a.K - a.k_o;
+    const bool outliers = a.k_o > 0 && a.Xo != nullptr;  // the debug entry may skip them
+    CUtensorMap mw, mx, mwo, mxo;
+    std::memset(&mw, 0, sizeof(mw));
+    std::memset(&mx, 0, sizeof(mx));
+    std::memset(&mwo, 0, sizeof(mwo));
+    std::memset(&mxo, 0, sizeof(mxo));
+    if (Ki > 0) {
+        // packed W rows: 64 bytes (one k-block) x 128 rows per box, 64-byte swizzle;
+        // packed token rows: 64 bytes x 32 rows per box (rows past M read as 0)
+        if (!make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wq, Ki / 2, a.N, Ki / 2, PK_ROW, gemv::BW,
+                      CU_TENSOR_MAP_SWIZZLE_64B) ||
+            !make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Xq, Ki / 2, a.M, Ki / 2, PK_ROW, gemv::MT,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+            return QUIK_ERR_CUDA;
+    }
+    if (outliers) {
+        // outlier blocks: 128-byte rows (64 fp16 or 128 int8 channels), the
+        // swizzled K-major layout the MMA reads
+        const CUtensorMapDataType dt = OUT_INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
+        const uint32_t oke = OUT_INT8 ? 128 : 64;
+        const uint64_t pitch = static_cast<uint64_t>(a.k_o) * (OUT_INT8 ? 1 : 2);
+        if (!make_map(&mwo, dt, a.Wo, a.k_o, a.N, pitch, oke, gemv::BW, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&mxo, dt, a.Xo, a.k_o, a.M, pitch, oke, gemv::MT, CU_TENSOR_MAP_SWIZZLE_128B))
+            return QUIK_ERR_CUDA;
+    }
+    GemmParams p{};
+    p.M = a.M;
+    p.N = a.N;
+    p.Ki = Ki;
+    p.k_o = outliers ? a.k_o : 0;
+    p.nkb_i = (Ki + KB - 1) / KB;
+    p.nkb_o = 0;
+    p.G = 1;
+    p.sx = a.sx;
+    p.sw = a.sw;
+    p.sxo = a.sxo;
+    p.swo = a.swo;
+    p.bias = a.bias;
+    p.Y = a.Y;
+    p.acc_dbg = a.acc_dbg;
+    p.acc_o_dbg = a.acc_o_dbg;
+    auto kern = w4a4_gemv_kernel<OUT_INT8, DEBUG>;
+    if (!attribute_set_once(reinterpret_cast<const void *>(kern), gemv::SMEM)) return QUIK_ERR_CUDA;
+    const dim3 grid((a.N + gemv::BW - 1) / gemv::BW);
+    if (!a.after_quantize) {
+        kern<<<grid, gemv::THREADS, gemv::SMEM, stream>>>(mw, mx, mwo, mxo, p);
+        return cudaGetLastError() == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(gemv::THREADS);
+    cfg.dynamicSmemBytes = gemv::SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, mw, mx, mwo, mxo, p) == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
+}
+
 // Per-channel scales: the CTA-pair kernel (faster than a single-CTA kernel
 // with 128-row tiles at every M measured, 16 to 4096); per-group scales: the
 // shared-memory-operand kernel.
 template <bool DEBUG>
 quik_status dispatch(const GemmArgs &a, cudaStream_t stream) {
+    if (a.group == 0 && a.M <= gemv::MT && a.k_o <= gemv::KO_MAX)
+        return a.out_int8 ? run_gemv<true, DEBUG>(a, stream) : run_gemv<false, DEBUG>(a, stream);
     if (a.group == 0)
         return a.out_int8 ? run_pair<true, DEBUG>(a, stream) : run_pair<false, DEBUG>(a, stream);
     return a.out_int8 ? run<CfgGroup<true, DEBUG>>(a, stream) : run<CfgGroup<false, DEBUG>>(a, stream);

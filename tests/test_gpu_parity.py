@@ -48,6 +48,13 @@ SHAPES = [
     (130, 260, 8256, 64, 0, False, True),    # 64 INT4 k-blocks + FP16 outliers
     # K_i = 20480: the quantiser's widest rows (8 words per thread, 10 warps)
     (33, 72, 20544, 64, 0, True, True),
+    # decode-shaped products (M <= 32, per-channel scales): W as the MMA's rows
+    (1, 128, 256, 32, 0, False, True),       # one token
+    (5, 300, 640, 64, 0, True, True),        # 5 tokens, ragged N, INT8 outliers
+    (17, 520, 1056, 32, 0, False, False),    # 17 tokens: the MMA's N = 32
+    (32, 136, 4160, 256, 0, False, True),    # 32 tokens, k_o = 256
+    (24, 264, 8320, 128, 0, True, False),    # long K (the W ring wraps 4 times), INT8 outliers
+    (16, 130, 160, 0, 0, False, True),       # no outliers, partial k-block, ragged N
 ]
 
 
