@@ -1030,26 +1030,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
 namespace gemv {
 constexpr int BW = 128;                      // W rows per CTA = TMEM lanes
 constexpr int MT = 32;                       // most tokens (the MMA's N: 16 or 32)
-constexpr int S = 4;                         // operand stages (A in TMEM, X in shared memory)
-constexpr int SPW = 10;                      // staging units
+#ifndef QUIK_GEMV_S
+#define QUIK_GEMV_S 8
+#endif
+#ifndef QUIK_GEMV_NI
+#define QUIK_GEMV_NI 2
+#endif
+constexpr int S = QUIK_GEMV_S;               // operand stages (A in TMEM, X in shared memory)
+#ifndef QUIK_GEMV_SPW
+#define QUIK_GEMV_SPW 10
+#endif
+constexpr int SPW = QUIK_GEMV_SPW;           // staging units
 constexpr int WUNIT = BW * PK_ROW;           // 8 KB of packed W
-constexpr int XUNIT = MT * PK_ROW;           // 2 KB of packed token rows
+constexpr int XUNIT = MT * PK_ROW;           // 2 KB of packed token rows (MP rows are loaded)
 constexpr int XSTAGE = MT * OP_ROW;          // 4 KB
-constexpr int KO_MAX = 256;                  // outlier channels handled here
-constexpr int OKB = 4;                       // outlier k-blocks of 128 bytes (k_o <= 256 fp16)
+constexpr int OKB = 2;                       // outlier k-blocks of 128-byte rows:
+constexpr int KO_MAX_F16 = 64 * OKB;         //   k_o <= 128 fp16 channels
+constexpr int KO_MAX_I8 = 128 * OKB;         //   or 256 int8 channels
 constexpr int WO_TILE = BW * OP_ROW;         // 16 KB: 128 rows x 128 bytes
 constexpr int XO_TILE = MT * OP_ROW;         // 4 KB
-constexpr int NG = 4;                        // W warp groups (4 warps each), one per stage
+constexpr int NG = 4;                        // W warp groups (4 warps each)
 constexpr int NW = 4 * NG;                   // W warps
-constexpr int THREADS = (2 + NW) * 32;       // 576
+constexpr int NI = QUIK_GEMV_NI;             // MMA issuers, each with its own accumulator
+constexpr int THREADS = (1 + NW + NI) * 32;
 constexpr int XU_OFF = SPW * WUNIT;          // W staging first, then the token-row staging
 constexpr int X_OFF = XU_OFF + SPW * XUNIT;
 constexpr int WO_OFF = X_OFF + S * XSTAGE;
 constexpr int XO_OFF = WO_OFF + OKB * WO_TILE;
 constexpr int SMEM = XO_OFF + OKB * XO_TILE + 1024;  // + alignment
-constexpr int ACC_COL = 0, O_COL = 32, A_COL = 64, TMEM_COLS = 256;
+constexpr int ACC_COL = 0, O_COL = 32 * NI, A_COL = O_COL + 32;  // one accumulator per issuer
+constexpr int TMEM_COLS = A_COL + 32 * S <= 256 ? 256 : 512;
 static_assert(A_COL + 32 * S <= TMEM_COLS, "A stages fit in tensor memory");
-static_assert(NG == S, "group g owns operand stage g");
+static_assert(S % NG == 0, "group g owns operand stages g, g + NG, ...");
+static_assert(S % NI == 0, "each stage belongs to one issuer");
 static_assert(X_OFF % 1024 == 0 && WO_OFF % 1024 == 0 && XO_OFF % 1024 == 0, "128-byte-swizzled tiles");
 static_assert(SMEM <= 232448, "shared memory budget");
 }  // namespace gemv
@@ -1061,7 +1074,7 @@ __global__ void __launch_bounds__(gemv::THREADS, 1)
                      const GemmParams p) {
     using namespace gemv;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ uint64_t w_full[SPW], w_empty[SPW], op_full[S], op_empty[S], o_full, acc_full, mma_done;
+    __shared__ uint64_t w_full[SPW], w_empty[SPW], op_full[S], op_empty[S], o_full, acc_full, mma_done[NI];
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     __shared__ unsigned err0_s;
@@ -1096,14 +1109,14 @@ __global__ void __launch_bounds__(gemv::THREADS, 1)
             tma_prefetch_desc(&tm_x);
         }
         for (int u = 0; u < early; ++u) {
-            mbar_arrive_expect_tx(&w_full[u], WUNIT + XUNIT);
+            mbar_arrive_expect_tx(&w_full[u], WUNIT + MP * PK_ROW);
             tma_load_2d(smem + u * WUNIT, &tm_w, u * PK_ROW, n0, &w_full[u]);
             QUIK_TRACE_AT(11, u);
         }
         if (nko > 0) {
             tma_prefetch_desc(&tm_wo);
             tma_prefetch_desc(&tm_xo);
-            mbar_arrive_expect_tx(&o_full, nko * (WO_TILE + XO_TILE));
+            mbar_arrive_expect_tx(&o_full, nko * (WO_TILE + MP * OP_ROW));
             for (int kb = 0; kb < nko; ++kb)
                 tma_load_2d(smem + WO_OFF + kb * WO_TILE, &tm_wo, kb * oke, n0, &o_full);
         }
@@ -1113,8 +1126,8 @@ __global__ void __launch_bounds__(gemv::THREADS, 1)
             mbar_init(&op_full[i], 4);
             mbar_init(&op_empty[i], 1);
         }
-        mbar_init(&acc_full, 1);
-        mbar_init(&mma_done, 1);
+        mbar_init(&acc_full, NI);
+        for (int i = 0; i < NI; ++i) mbar_init(&mma_done[i], 1);
         abort_s = 0;
         err0_s = *reinterpret_cast<volatile unsigned *>(&g_error_word);
         fence_barrier_init();
@@ -1126,11 +1139,15 @@ __global__ void __launch_bounds__(gemv::THREADS, 1)
     const uint32_t tmem = tmem_base_s;
     const AbortState ab{&abort_s, err0_s};
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ MMA issuer
+    const int issuer = warp == 0 ? 0 : warp >= 2 + NW ? warp - 1 - NW : -1;
+    if (issuer >= 0) {
+        // ------------------------------------------------------------ MMA issuers
+        // Issuer i takes k-blocks i, i + NI, ... into its own accumulator
+        // (TMEM columns 32 i ..), so NI MMA streams are in flight; issuer 0
+        // also does the outlier block.  The epilogue adds the accumulators.
         if (lane == 0) {
             bool ok = true;
-            if (nko > 0) {  // the outlier block: both operands in shared memory
+            if (issuer == 0 && nko > 0) {  // the outlier block: both operands in shared memory
                 ok = wait_bar(&o_full, 0, ab);
                 QUIK_TRACE_AT(2, 0);
                 if (ok) {
@@ -1152,7 +1169,8 @@ __global__ void __launch_bounds__(gemv::THREADS, 1)
                 }
             }
             const uint32_t idesc = idesc_s8_s32(BW, MP);
-            for (int kb = 0; kb < nkb && ok; ++kb) {
+            const uint32_t acc = tmem + ACC_COL + 32 * issuer;
+            for (int kb = issuer; kb < nkb && ok; kb += NI) {
                 const int st = kb % S;
                 if (!(ok = wait_bar(&op_full[st], (kb / S) & 1, ab))) break;
                 QUIK_TRACE_AT(3, kb);
@@ -1160,13 +1178,13 @@ __global__ void __launch_bounds__(gemv::THREADS, 1)
                 const uint32_t xb = smem_base + X_OFF + st * XSTAGE;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_i8_ts(tmem + ACC_COL, tmem + A_COL + 32 * st + 8 * k, sw128_kmajor_desc(xb + 32 * k),
-                              idesc, (kb > 0 || k > 0));
+                    mma_i8_ts(acc, tmem + A_COL + 32 * st + 8 * k, sw128_kmajor_desc(xb + 32 * k), idesc,
+                              (kb > issuer || k > 0));
                 mma_commit(&op_empty[st]);
             }
             if (ok) mma_commit(&acc_full);
-            mma_commit(&mma_done);
-            mbar_wait_bounded(&mma_done, 0, kWaitLimitNs);
+            mma_commit(&mma_done[issuer]);
+            mbar_wait_bounded(&mma_done[issuer], 0, kWaitLimitNs);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -1181,7 +1199,7 @@ __global__ void __launch_bounds__(gemv::THREADS, 1)
             for (int u = early; u < nkb; ++u, ++filled) {
                 const int st = u % SPW;
                 if (!wait_bar(&w_empty[st], ((u / SPW) & 1) ^ 1, ab)) break;
-                mbar_arrive_expect_tx(&w_full[st], WUNIT + XUNIT);
+                mbar_arrive_expect_tx(&w_full[st], WUNIT + MP * PK_ROW);
                 tma_load_2d(smem + st * WUNIT, &tm_w, u * PK_ROW, n0, &w_full[st]);
                 tma_load_2d(smem + XU_OFF + st * XUNIT, &tm_x, u * PK_ROW, 0, &w_full[st]);
                 QUIK_TRACE_AT(11, u);
@@ -1229,23 +1247,29 @@ __global__ void __launch_bounds__(gemv::THREADS, 1)
             ok = ok && wait_bar(&w_full[ps], (kb / SPW) & 1, ab);
             if (xw == 0 && lane == 0) QUIK_TRACE_AT(8, kb);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            if (x_on) {  // token row x_row, chunk x_ch -> two 16-byte unpacked chunks
-                const uint4 v = *reinterpret_cast<const uint4 *>(smem + XU_OFF + ps * XUNIT +
-                                                                 x_row * PK_ROW + x_ch * 16);
+            // the packed bytes into registers, then the staging slot goes
+            // back to the producer before the unpack: token row x_row, chunk
+            // x_ch; W row r, 4 chunks of 16 bytes (64-byte swizzle)
+            uint4 xv = make_uint4(0, 0, 0, 0), wv[4];
+            if (x_on)
+                xv = *reinterpret_cast<const uint4 *>(smem + XU_OFF + ps * XUNIT + x_row * PK_ROW + x_ch * 16);
+            const uint8_t *wr = smem + ps * WUNIT + r * PK_ROW;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) wv[c] = *reinterpret_cast<const uint4 *>(wr + ((c ^ ((r >> 1) & 3)) << 4));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&w_empty[ps]);
+            if (x_on) {  // two 16-byte unpacked chunks into the 128-byte-swizzled X stage
                 uint4 lo, hi;
-                unpack16(v, lo, hi);
+                unpack16(xv, lo, hi);
                 uint8_t *xr = smem + X_OFF + st * XSTAGE + x_row * OP_ROW;
                 *reinterpret_cast<uint4 *>(xr + (((2 * x_ch) ^ (x_row & 7)) << 4)) = lo;
                 *reinterpret_cast<uint4 *>(xr + (((2 * x_ch + 1) ^ (x_row & 7)) << 4)) = hi;
             }
-            // W row r: 4 chunks of 16 packed bytes, 64-byte swizzle
-            const uint8_t *wr = smem + ps * WUNIT + r * PK_ROW;
             uint32_t w[32];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(wr + ((c ^ ((r >> 1) & 3)) << 4));
                 uint4 lo, hi;
-                unpack16(v, lo, hi);
+                unpack16(wv[c], lo, hi);
                 w[8 * c + 0] = lo.x; w[8 * c + 1] = lo.y; w[8 * c + 2] = lo.z; w[8 * c + 3] = lo.w;
                 w[8 * c + 4] = hi.x; w[8 * c + 5] = hi.y; w[8 * c + 6] = hi.z; w[8 * c + 7] = hi.w;
             }
@@ -1256,7 +1280,6 @@ __global__ void __launch_bounds__(gemv::THREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&w_empty[ps]);
                 mbar_arrive(&op_full[st]);
                 if (xw == 0) QUIK_TRACE_AT(0, kb);
             }
@@ -1275,6 +1298,15 @@ __global__ void __launch_bounds__(gemv::THREADS, 1)
                     if (nkb > 0) tmem_ld_32x32b_x16(t_lane + ACC_COL + h, a);
                     if (nko > 0) tmem_ld_32x32b_x16(t_lane + O_COL + h, o);
                     tmem_ld_wait();
+                    // the other issuers' accumulators (those that took a k-block);
+                    // all are multiples of 256, so the sum is exact
+                    for (int i = 1; i < NI && i < nkb; ++i) {
+                        uint32_t t[16];
+                        tmem_ld_32x32b_x16(t_lane + ACC_COL + 32 * i + h, t);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) a[j] += t[j];
+                    }
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int m = h + j;
@@ -1476,10 +1508,12 @@ quik_status run_gemv(const GemmArgs &a, cudaStream_t stream) {
     std::memset(&mxo, 0, sizeof(mxo));
     if (Ki > 0) {
         // packed W rows: 64 bytes (one k-block) x 128 rows per box, 64-byte swizzle;
-        // packed token rows: 64 bytes x 32 rows per box (rows past M read as 0)
+        // packed token rows: 64 bytes x 16 or 32 rows per box, the MMA's N (rows
+        // past M read as 0)
+        const uint32_t mp = a.M <= 16 ? 16 : 32;
         if (!make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wq, Ki / 2, a.N, Ki / 2, PK_ROW, gemv::BW,
                       CU_TENSOR_MAP_SWIZZLE_64B) ||
-            !make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Xq, Ki / 2, a.M, Ki / 2, PK_ROW, gemv::MT,
+            !make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Xq, Ki / 2, a.M, Ki / 2, PK_ROW, mp,
                       CU_TENSOR_MAP_SWIZZLE_NONE))
             return QUIK_ERR_CUDA;
     }
@@ -1490,7 +1524,7 @@ quik_status run_gemv(const GemmArgs &a, cudaStream_t stream) {
         const uint32_t oke = OUT_INT8 ? 128 : 64;
         const uint64_t pitch = static_cast<uint64_t>(a.k_o) * (OUT_INT8 ? 1 : 2);
         if (!make_map(&mwo, dt, a.Wo, a.k_o, a.N, pitch, oke, gemv::BW, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map(&mxo, dt, a.Xo, a.k_o, a.M, pitch, oke, gemv::MT, CU_TENSOR_MAP_SWIZZLE_128B))
+            !make_map(&mxo, dt, a.Xo, a.k_o, a.M, pitch, oke, a.M <= 16 ? 16 : 32, CU_TENSOR_MAP_SWIZZLE_128B))
             return QUIK_ERR_CUDA;
     }
     GemmParams p{};
@@ -1534,7 +1568,7 @@ quik_status run_gemv(const GemmArgs &a, cudaStream_t stream) {
 // shared-memory-operand kernel.
 template <bool DEBUG>
 quik_status dispatch(const GemmArgs &a, cudaStream_t stream) {
-    if (a.group == 0 && a.M <= gemv::MT && a.k_o <= gemv::KO_MAX)
+    if (a.group == 0 && a.M <= gemv::MT && a.k_o <= (a.out_int8 ? gemv::KO_MAX_I8 : gemv::KO_MAX_F16))
         return a.out_int8 ? run_gemv<true, DEBUG>(a, stream) : run_gemv<false, DEBUG>(a, stream);
     if (a.group == 0)
         return a.out_int8 ? run_pair<true, DEBUG>(a, stream) : run_pair<false, DEBUG>(a, stream);

@@ -52,7 +52,10 @@ SHAPES = [
     (1, 128, 256, 32, 0, False, True),       # one token
     (5, 300, 640, 64, 0, True, True),        # 5 tokens, ragged N, INT8 outliers
     (17, 520, 1056, 32, 0, False, False),    # 17 tokens: the MMA's N = 32
-    (32, 136, 4160, 256, 0, False, True),    # 32 tokens, k_o = 256
+    (32, 136, 4224, 128, 0, False, True),    # 32 tokens, the largest FP16 outlier block (k_o = 128)
+    (32, 136, 4160, 256, 0, False, True),    # FP16 k_o = 256: past that block, the pair kernel
+    (8, 384, 4352, 256, 0, True, True),      # the largest INT8 outlier block (k_o = 256)
+    (4, 128, 128, 128, 0, False, True),      # everything is outlier
     (24, 264, 8320, 128, 0, True, False),    # long K (the W ring wraps 4 times), INT8 outliers
     (16, 130, 160, 0, 0, False, True),       # no outliers, partial k-block, ragged N
 ]
