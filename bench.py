@@ -41,7 +41,7 @@ sys.path.insert(0, ROOT)
 METRIC = "W4A4+outlier linear TOPS & µs/call at Llama shapes; % of dense INT8 peak"
 UNIT = "TOPS"
 FLUSH_BYTES = 256 << 20
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "w4a4_gemm_llama7b_attn_2048x4096x4096.md")
+PROFILE_DIR = os.path.join(ROOT, "profiles")
 GEMM_SOURCES = [os.path.join(ROOT, "mixed_precision_quantized_quantize_b200", "csrc", f)
                 for f in ("gemm.cu", "sm100.cuh")]
 # nominal dense-rate ratio INT8 : BF16 on B200 (4.5 : 2.25 PFLOP/s)
@@ -85,10 +85,23 @@ def gemm_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
+def gemm_kernel(cfg):
+    """The GEMM kernel the library dispatches for this layer, and its profile file."""
+    fits = cfg.k_o <= (256 if cfg.outlier_int8 else 128)
+    if cfg.group == 0 and cfg.M <= 32 and fits:
+        return ("w4a4_gemv (decode shapes: W rows as the MMA's M, tokens as N; INT4 codes "
+                "widened to INT8, tcgen05 kind::i8)", f"w4a4_gemv_{cfg.name}.md")
+    if cfg.group == 0:
+        return ("w4a4_gemm_pair (INT4 codes widened to INT8, tcgen05 kind::i8 on CTA pairs)",
+                f"w4a4_gemm_{cfg.name}.md")
+    return ("w4a4_gemm (grouped scales; INT4 codes widened to INT8, tcgen05 kind::i8)",
+            f"w4a4_gemm_grouped_{cfg.name}.md")
+
+
+def profiled_traffic(profile_file):
     """dram bytes per launch from the committed ncu summary, if it matches this kernel."""
     try:
-        with open(PROFILE_SUMMARY) as f:
+        with open(os.path.join(PROFILE_DIR, profile_file)) as f:
             text = f.read()
     except OSError:
         return None
@@ -375,6 +388,29 @@ def run_ours(args, rank, local_rank, world):
     peaks, peak_kind = measured_peaks()
     int8_peak = float(peaks["bf16_tflops"]) * INT8_PER_BF16
     gemm_tops = cfg.ops / gemm_avg / 1e12
+    kernel_name, profile_file = gemm_kernel(cfg)
+    hbm_peak = float(peaks["hbm_gbs"])
+    # the path's bound: the slower of the tensor work and the bytes it must move
+    if cfg.gemm_bytes / (hbm_peak * 1e9) > cfg.ops / (int8_peak * 1e12):
+        roofline = {
+            "bound": "hbm", "kernel": kernel_name,
+            "achieved": round(cfg.gemm_bytes / gemm_avg / 1e9, 1), "peak": hbm_peak,
+            "unit": "GB/s", "frac": round(cfg.gemm_bytes / gemm_avg / 1e9 / hbm_peak, 4),
+            "traffic": profiled_traffic(profile_file),
+            "algorithmic_bytes_per_launch": cfg.gemm_bytes,
+            "peak_source": f"{peak_kind} HBM copy bandwidth",
+        }
+    else:
+        roofline = {
+            "bound": "tensor", "kernel": kernel_name,
+            "achieved": round(gemm_tops, 2), "peak": round(int8_peak, 1), "unit": "TFLOP/s",
+            "frac": round(gemm_tops / int8_peak, 4),
+            "traffic": profiled_traffic(profile_file),
+            "algorithmic_bytes_per_launch": cfg.gemm_bytes,
+            "peak_source": (f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
+                            f"{INT8_PER_BF16} (nominal INT8:BF16 dense ratio); integer ops "
+                            f"counted 2 per multiply-add"),
+        }
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -400,18 +436,7 @@ def run_ours(args, rank, local_rank, world):
         "breakdown_us": {"quantize_reorder": round(quant_avg * 1e6, 2),
                          "w4a4_gemm": round(gemm_avg * 1e6, 2),
                          "two_calls_with_event_between": round(split_avg * 1e6, 2)},
-        "roofline": {
-            "bound": "tensor",
-            "kernel": "w4a4_gemm (INT4 codes widened to INT8, tcgen05 kind::i8)",
-            "achieved": round(gemm_tops, 2),
-            "peak": round(int8_peak, 1),
-            "unit": "TFLOP/s",
-            "frac": round(gemm_tops / int8_peak, 4),
-            "traffic": profiled_traffic(),
-            "peak_source": (f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
-                            f"{INT8_PER_BF16} (nominal INT8:BF16 dense ratio); integer ops "
-                            f"counted 2 per multiply-add"),
-        },
+        "roofline": roofline,
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
                 "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2,
                 "call": "quik_linear via QuikLinear, pinned host X in, host Y out"},

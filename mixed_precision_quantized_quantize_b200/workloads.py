@@ -52,6 +52,22 @@ class LayerConfig:
         """Multiply-adds x 2 over the full K (INT4 part and outliers)."""
         return 2 * self.M * self.N * self.K
 
+    @property
+    def gemm_bytes(self) -> int:
+        """Bytes the GEMM must move at least once: packed codes (half a byte
+        each), the outlier blocks, the fp32 scales, the fp16 output and bias."""
+        groups = self.K_i // 128 if self.group else 1
+        ob = 1 if self.outlier_int8 else 2
+        b = (self.M + self.N) * self.K_i // 2            # Xq, Wq
+        b += (self.M + self.N) * self.k_o * ob           # Xo, Wo
+        b += (self.M + self.N) * groups * 4              # sx, sw
+        if self.outlier_int8 and self.k_o:
+            b += (self.M + self.N) * 4                   # sxo, swo
+        b += self.M * self.N * 2                         # Y
+        if self.bias:
+            b += self.N * 2
+        return b
+
 
 # The five layer workloads (the third has three token counts).
 CONFIGS = {
