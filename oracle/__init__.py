@@ -39,11 +39,12 @@ def _load():
     global _lib
     if _lib is None:
         lib = ctypes.CDLL(build())
-        lib.oracle_quantize_rows.argtypes = [_I, _I, _I, _I, ctypes.c_int, _P, _P, _P, _P, _P, _P]
-        lib.oracle_int_gemm.argtypes = [_I, _I, _I, _I, _P, _P, _P]
-        lib.oracle_linear.argtypes = [_I, _I, _I, _I, _I, ctypes.c_int,
+        _C = ctypes.c_int
+        lib.oracle_quantize_rows.argtypes = [_I, _I, _I, _I, _C, _C, _P, _P, _P, _P, _P, _P]
+        lib.oracle_int_gemm.argtypes = [_I, _I, _I, _I, _C, _P, _P, _P]
+        lib.oracle_linear.argtypes = [_I, _I, _I, _I, _I, _C, _C,
                                       _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
-        lib.oracle_linear_sampled.argtypes = [_I, _I, _I, _I, _I, ctypes.c_int,
+        lib.oracle_linear_sampled.argtypes = [_I, _I, _I, _I, _I, _C, _C,
                                               _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                               _I, _P, _P, _P, _P]
         lib.oracle_num_threads.argtypes = []
@@ -68,44 +69,52 @@ def num_threads() -> int:
 
 
 def quantize_rows(X_f16: np.ndarray, perm: np.ndarray, k_o: int, group: int = 0,
-                  outlier_int8: bool = False):
-    """Reorder + quantise + pack the rows of ``X_f16`` ([R, K] float16).
+                  outlier_int8: bool = False, bits: int = 4):
+    """Reorder + quantise (+ pack) the rows of ``X_f16`` ([R, K] float16).
 
-    Returns (Q uint8 [R,(K-k_o)/2], scale float32 [R] or [R,G],
-             O float16 or int8 [R,k_o], o_scale float32 [R] or None).
+    Returns (Q, scale float32 [R] or [R,G], O float16 or int8 [R,k_o],
+             o_scale float32 [R] or None); Q is uint8 [R,(K-k_o)/2] packed INT4
+    (bits 4) or int8 [R,K-k_o] (bits 8).
     """
     X = np.ascontiguousarray(X_f16, dtype=np.float16)
     R, K = X.shape
     Ki = K - k_o
     G = Ki // group if group else 1
     perm = np.ascontiguousarray(perm, dtype=np.int32)
-    Q = np.zeros((R, Ki // 2), np.uint8)
+    Q = np.zeros((R, Ki), np.int8) if bits == 8 else np.zeros((R, Ki // 2), np.uint8)
     scale = np.zeros((R, G) if group else (R,), np.float32)
     O = np.zeros((R, k_o), np.int8 if outlier_int8 else np.float16)
     o_scale = np.zeros((R,), np.float32) if outlier_int8 else None
-    rc = _load().oracle_quantize_rows(R, K, k_o, group, int(outlier_int8),
+    rc = _load().oracle_quantize_rows(R, K, k_o, group, int(outlier_int8), int(bits),
                                       _ptr(X.view(np.uint16)), _ptr(perm), _ptr(Q),
                                       _ptr(scale), _ptr(O), _ptr(o_scale))
     _check(rc, "quantize_rows")
     return Q, scale, O, o_scale
 
 
+def _x_bits(Xq) -> int:
+    """8 for one signed byte per code (int8 array), 4 for packed nibbles."""
+    return 8 if Xq.dtype == np.int8 else 4
+
+
 def int_gemm(Xq: np.ndarray, Wq: np.ndarray, group: int = 0) -> np.ndarray:
-    """Exact INT32 sums of the packed codes: [M,N], or [G,M,N] with groups."""
-    Xq = np.ascontiguousarray(Xq, np.uint8)
+    """Exact INT32 sums of the codes (Xq packed INT4 uint8, or int8 codes;
+    Wq packed INT4): [M,N], or [G,M,N] with groups."""
+    xb = _x_bits(Xq)
+    Xq = np.ascontiguousarray(Xq.view(np.uint8))
     Wq = np.ascontiguousarray(Wq, np.uint8)
-    M, rb = Xq.shape
+    M = Xq.shape[0]
     N = Wq.shape[0]
-    Ki = 2 * rb
+    Ki = 2 * Wq.shape[1]
     G = Ki // group if group else 1
     acc = np.zeros((G, M, N), np.int32)
-    _check(_load().oracle_int_gemm(M, N, Ki, group, _ptr(Xq), _ptr(Wq), _ptr(acc)), "int_gemm")
+    _check(_load().oracle_int_gemm(M, N, Ki, group, xb, _ptr(Xq), _ptr(Wq), _ptr(acc)), "int_gemm")
     return acc if group else acc[0]
 
 
 def _linear_args(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias):
     c = np.ascontiguousarray
-    Xq, Wq = c(Xq, np.uint8), c(Wq, np.uint8)
+    Xq, Wq = c(Xq.view(np.uint8)), c(Wq, np.uint8)
     sx, sw = c(sx, np.float32), c(sw, np.float32)
     int8 = Xo is not None and Xo.dtype == np.int8
     if Xo is not None:
@@ -119,10 +128,11 @@ def _linear_args(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias):
 
 def linear(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias, K: int, k_o: int, group: int = 0):
     """fp64 Y [M,N] of the layer from quantised operands (no fp16 rounding)."""
+    xb = _x_bits(Xq)
     Xq, sx, Xo, sxo, Wq, sw, Wo, swo, b, int8 = _linear_args(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias)
     M, N = Xq.shape[0], Wq.shape[0]
     Y = np.zeros((M, N), np.float64)
-    rc = _load().oracle_linear(M, N, K, k_o, group, int(int8), _ptr(Xq), _ptr(sx), _ptr(Xo),
+    rc = _load().oracle_linear(M, N, K, k_o, group, int(int8), xb, _ptr(Xq), _ptr(sx), _ptr(Xo),
                                _ptr(sxo), _ptr(Wq), _ptr(sw), _ptr(Wo), _ptr(swo), _ptr(b), _ptr(Y))
     _check(rc, "linear")
     return Y
@@ -131,6 +141,7 @@ def linear(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias, K: int, k_o: int, group: int 
 def linear_sampled(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias, K: int, k_o: int, group: int,
                    ms: np.ndarray, ns: np.ndarray):
     """fp64 Y at the (ms[i], ns[i]) positions plus their integer sums [count, G]."""
+    xb = _x_bits(Xq)
     Xq, sx, Xo, sxo, Wq, sw, Wo, swo, b, int8 = _linear_args(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias)
     M, N = Xq.shape[0], Wq.shape[0]
     ms = np.ascontiguousarray(ms, np.int64)
@@ -138,7 +149,7 @@ def linear_sampled(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias, K: int, k_o: int, gro
     G = (K - k_o) // group if group else 1
     Y = np.zeros(len(ms), np.float64)
     acc = np.zeros((len(ms), max(G, 1)), np.int32)
-    rc = _load().oracle_linear_sampled(M, N, K, k_o, group, int(int8), _ptr(Xq), _ptr(sx),
+    rc = _load().oracle_linear_sampled(M, N, K, k_o, group, int(int8), xb, _ptr(Xq), _ptr(sx),
                                        _ptr(Xo), _ptr(sxo), _ptr(Wq), _ptr(sw), _ptr(Wo),
                                        _ptr(swo), _ptr(b), len(ms), _ptr(ms), _ptr(ns),
                                        _ptr(Y), _ptr(acc))
@@ -146,13 +157,15 @@ def linear_sampled(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias, K: int, k_o: int, gro
     return Y, acc
 
 
-def layer(X_f16, W_f16, perm, bias, k_o: int, group: int = 0, outlier_int8: bool = False):
-    """The whole layer from fp16 inputs: quantise X and W, then the fp64 output.
+def layer(X_f16, W_f16, perm, bias, k_o: int, group: int = 0, outlier_int8: bool = False,
+          act_bits: int = 4):
+    """The whole layer from fp16 inputs: quantise X (INT4, or INT8 when
+    act_bits == 8) and W (INT4), then the fp64 output.
 
     Returns a dict with every intermediate (codes, scales, outlier blocks, Y).
     """
     K = X_f16.shape[1]
-    Xq, sx, Xo, sxo = quantize_rows(X_f16, perm, k_o, group, outlier_int8)
+    Xq, sx, Xo, sxo = quantize_rows(X_f16, perm, k_o, group, outlier_int8, act_bits)
     Wq, sw, Wo, swo = quantize_rows(W_f16, perm, k_o, group, outlier_int8)
     Y = linear(Xq, sx, Xo if k_o else None, sxo, Wq, sw, Wo if k_o else None, swo, bias,
                K, k_o, group)

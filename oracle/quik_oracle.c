@@ -25,6 +25,12 @@
  *  - groups are 128 consecutive *reordered* INT4 positions.
  *  - INT8 outliers: s = max|v| / 127, q = clamp(rintf(v / s), -127, 127),
  *    one scale per row (per token for X, per output channel for W).
+ *  - 8-bit activations (W4A8): "QQQ: ... Quattuor-bit Quantization", the
+ *    abstract on the aggregated "smoothquant" abstracts page, pairs 4-bit
+ *    weights with 8-bit activations in per-channel (and per-group) GEMMs but
+ *    fixes no quantiser.  Reading: the INT8 rule above (divisor and clamp
+ *    127) applied per token to the non-outlier positions, one byte per code
+ *    in reordered order.
  *  - packing: byte i of a row holds code 2i in the low nibble and code 2i+1
  *    in the high nibble, both 4-bit two's complement.
  *  - integer dot products in int64 (checked to fit int32); dequantisation,
@@ -81,6 +87,17 @@ static int quantize_value(float v, float s, int qmax)
 /* 4-bit two's complement nibble -> signed code. */
 static int nibble_to_code(unsigned nib) { return nib >= 8 ? (int)nib - 16 : (int)nib; }
 
+/* Code j of row r of a quantised [*, Ki] operand: packed nibbles (bits 4,
+ * Ki / 2 bytes per row, code 2i in the low nibble of byte i) or one signed
+ * byte per code (bits 8, Ki bytes per row). */
+static int code_at(const uint8_t *Q, int64_t r, int64_t j, int64_t Ki, int bits)
+{
+    if (bits == 8)
+        return (int)(int8_t)Q[r * Ki + j];
+    unsigned b = Q[r * (Ki / 2) + j / 2];
+    return nibble_to_code(j % 2 ? b >> 4 : b & 0xF);
+}
+
 /*
  * oracle_quantize_rows -- reorder, scale, quantise and pack R rows of a
  * [R, K] fp16 matrix.  Used for activations X (one row per token) and for
@@ -93,14 +110,16 @@ static int nibble_to_code(unsigned nib) { return nib >= 8 ? (int)nib - 16 : (int
  *  group  : 0 (one scale per row) or the group width (e.g. 128)
  *  outlier_int8 : 0 -> O is fp16 [R, k_o] (bit copy); 1 -> O is int8
  *           [R, k_o] with o_scale [R]
- *  Q      : [R, (K - k_o) / 2] packed codes
+ *  bits   : 4 -> Q is [R, (K - k_o) / 2] packed codes, divisor and clamp 7;
+ *           8 -> Q is [R, K - k_o] signed bytes, divisor and clamp 127
  *  scale  : [R] (group == 0) or [R, (K - k_o) / group]
  */
 int oracle_quantize_rows(int64_t R, int64_t K, int64_t k_o, int64_t group, int outlier_int8,
-                         const uint16_t *X, const int32_t *perm,
+                         int bits, const uint16_t *X, const int32_t *perm,
                          uint8_t *Q, float *scale, void *O, float *o_scale)
 {
-    if (R < 0 || K < 0 || k_o < 0 || k_o > K) return ORACLE_EBADARG;
+    if (R < 0 || K < 0 || k_o < 0 || k_o > K || (bits != 4 && bits != 8)) return ORACLE_EBADARG;
+    const int qmax = bits == 8 ? 127 : 7;
     const int64_t Ki = K - k_o;
     if (Ki % 2) return ORACLE_EBADARG;
     if (group < 0 || (group > 0 && Ki % group)) return ORACLE_EBADARG;
@@ -131,16 +150,21 @@ int oracle_quantize_rows(int64_t R, int64_t K, int64_t k_o, int64_t group, int o
                     float amax = 0.0f;
                     for (int64_t j = g * gs; j < (g + 1) * gs; ++j)
                         if (fabsf(xr[j]) > amax) amax = fabsf(xr[j]);
-                    float s = amax / 7.0f;
+                    float s = amax / (float)qmax;
                     scale[r * G + g] = s;
                     for (int64_t j = g * gs; j < (g + 1) * gs; ++j)
-                        codes[j] = quantize_value(xr[j], s, 7);
+                        codes[j] = quantize_value(xr[j], s, qmax);
                 }
 
-                /* step 4: pack, low nibble = even position */
-                for (int64_t i = 0; i < Ki / 2; ++i)
-                    Q[r * (Ki / 2) + i] =
-                        (uint8_t)((codes[2 * i] & 0xF) | ((codes[2 * i + 1] & 0xF) << 4));
+                /* step 4: pack, low nibble = even position (or one byte per code) */
+                if (bits == 8) {
+                    for (int64_t j = 0; j < Ki; ++j)
+                        Q[r * Ki + j] = (uint8_t)(int8_t)codes[j];
+                } else {
+                    for (int64_t i = 0; i < Ki / 2; ++i)
+                        Q[r * (Ki / 2) + i] =
+                            (uint8_t)((codes[2 * i] & 0xF) | ((codes[2 * i + 1] & 0xF) << 4));
+                }
 
                 /* step 6: the outlier block (reordered positions Ki .. K-1) */
                 if (k_o > 0) {
@@ -169,31 +193,27 @@ int oracle_quantize_rows(int64_t R, int64_t K, int64_t k_o, int64_t group, int o
 }
 
 /*
- * oracle_int_gemm -- exact integer product of packed INT4 codes.
+ * oracle_int_gemm -- exact integer product of the quantised codes (W packed
+ * INT4; X packed INT4, or one byte per code when x_bits == 8).
  *  acc[m, n]           = sum_{j < Ki} qx[m, j] * qw[n, j]            (group == 0)
  *  acc[g, m, n]        = sum_{j in group g} qx[m, j] * qw[n, j]      (group > 0)
  * Sums are taken in int64 and must fit int32.
  */
-int oracle_int_gemm(int64_t M, int64_t N, int64_t Ki, int64_t group,
+int oracle_int_gemm(int64_t M, int64_t N, int64_t Ki, int64_t group, int x_bits,
                     const uint8_t *Xq, const uint8_t *Wq, int32_t *acc)
 {
-    if (M < 0 || N < 0 || Ki < 0 || Ki % 2) return ORACLE_EBADARG;
+    if (M < 0 || N < 0 || Ki < 0 || Ki % 2 || (x_bits != 4 && x_bits != 8)) return ORACLE_EBADARG;
     if (group < 0 || (group > 0 && Ki % group)) return ORACLE_EBADARG;
     const int64_t gs = group > 0 ? group : Ki;
     const int64_t G = group > 0 ? Ki / group : 1;
-    const int64_t rb = Ki / 2;
     int err = ORACLE_OK;
 #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m) {
         for (int64_t n = 0; n < N; ++n) {
             for (int64_t g = 0; g < G; ++g) {
                 int64_t sum = 0;
-                for (int64_t j = g * gs; j < (g + 1) * gs; ++j) {
-                    unsigned bx = Xq[m * rb + j / 2], bw = Wq[n * rb + j / 2];
-                    int cx = nibble_to_code(j % 2 ? bx >> 4 : bx & 0xF);
-                    int cw = nibble_to_code(j % 2 ? bw >> 4 : bw & 0xF);
-                    sum += (int64_t)cx * (int64_t)cw;
-                }
+                for (int64_t j = g * gs; j < (g + 1) * gs; ++j)
+                    sum += (int64_t)code_at(Xq, m, j, Ki, x_bits) * (int64_t)code_at(Wq, n, j, Ki, 4);
                 if (sum > INT32_MAX || sum < INT32_MIN) {
 #pragma omp atomic write
                     err = ORACLE_EOVERFLOW;
@@ -208,7 +228,7 @@ int oracle_int_gemm(int64_t M, int64_t N, int64_t Ki, int64_t group,
 /* One output element of the layer, in fp64, from quantised operands.
  * Y = sum_g A_g * sx[m,g] * sw[n,g]  +  O  +  bias[n]                  */
 static double linear_element(int64_t m, int64_t n, int64_t M, int64_t N, int64_t K, int64_t k_o,
-                             int64_t group, int outlier_int8,
+                             int64_t group, int outlier_int8, int x_bits,
                              const uint8_t *Xq, const float *sx, const void *Xo, const float *sxo,
                              const uint8_t *Wq, const float *sw, const void *Wo, const float *swo,
                              const uint16_t *bias, int32_t *acc_out, int *overflow)
@@ -217,18 +237,13 @@ static double linear_element(int64_t m, int64_t n, int64_t M, int64_t N, int64_t
     const int64_t Ki = K - k_o;
     const int64_t gs = group > 0 ? group : Ki;
     const int64_t G = group > 0 ? Ki / group : 1;
-    const int64_t rb = Ki / 2;
     double y = 0.0;
 
     /* steps 5 and 7: exact integer sums, dequantised in fp64 */
     for (int64_t g = 0; g < G; ++g) {
         int64_t sum = 0;
-        for (int64_t j = g * gs; j < (g + 1) * gs; ++j) {
-            unsigned bx = Xq[m * rb + j / 2], bw = Wq[n * rb + j / 2];
-            int cx = nibble_to_code(j % 2 ? bx >> 4 : bx & 0xF);
-            int cw = nibble_to_code(j % 2 ? bw >> 4 : bw & 0xF);
-            sum += (int64_t)cx * (int64_t)cw;
-        }
+        for (int64_t j = g * gs; j < (g + 1) * gs; ++j)
+            sum += (int64_t)code_at(Xq, m, j, Ki, x_bits) * (int64_t)code_at(Wq, n, j, Ki, 4);
         if (sum > INT32_MAX || sum < INT32_MIN) *overflow = 1;
         if (acc_out) acc_out[g] = (int32_t)sum;
         if (Ki > 0)
@@ -258,21 +273,24 @@ static double linear_element(int64_t m, int64_t n, int64_t M, int64_t N, int64_t
 
 /*
  * oracle_linear -- the full fp64 output Y [M, N] from quantised operands.
- * Xo/Wo are fp16 [*, k_o] (outlier_int8 == 0) or int8 [*, k_o] with
+ * Xq holds packed INT4 (x_bits 4) or one byte per code (x_bits 8); Wq packed
+ * INT4.  Xo/Wo are fp16 [*, k_o] (outlier_int8 == 0) or int8 [*, k_o] with
  * sxo [M] / swo [N] (outlier_int8 == 1).  bias is fp16 [N] or NULL.
  */
 int oracle_linear(int64_t M, int64_t N, int64_t K, int64_t k_o, int64_t group, int outlier_int8,
+                  int x_bits,
                   const uint8_t *Xq, const float *sx, const void *Xo, const float *sxo,
                   const uint8_t *Wq, const float *sw, const void *Wo, const float *swo,
                   const uint16_t *bias, double *Y)
 {
     if (M < 0 || N < 0 || K < 0 || k_o < 0 || k_o > K || (K - k_o) % 2) return ORACLE_EBADARG;
     if (group < 0 || (group > 0 && (K - k_o) % group)) return ORACLE_EBADARG;
+    if (x_bits != 4 && x_bits != 8) return ORACLE_EBADARG;
     int overflow = 0;
 #pragma omp parallel for schedule(static) reduction(| : overflow)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n)
-            Y[m * N + n] = linear_element(m, n, M, N, K, k_o, group, outlier_int8, Xq, sx, Xo,
+            Y[m * N + n] = linear_element(m, n, M, N, K, k_o, group, outlier_int8, x_bits, Xq, sx, Xo,
                                           sxo, Wq, sw, Wo, swo, bias, NULL, &overflow);
     return overflow ? ORACLE_EOVERFLOW : ORACLE_OK;
 }
@@ -284,7 +302,7 @@ int oracle_linear(int64_t M, int64_t N, int64_t K, int64_t k_o, int64_t group, i
  * ([count, G], G = 1 without groups).
  */
 int oracle_linear_sampled(int64_t M, int64_t N, int64_t K, int64_t k_o, int64_t group,
-                          int outlier_int8,
+                          int outlier_int8, int x_bits,
                           const uint8_t *Xq, const float *sx, const void *Xo, const float *sxo,
                           const uint8_t *Wq, const float *sw, const void *Wo, const float *swo,
                           const uint16_t *bias, int64_t count, const int64_t *ms,
@@ -292,13 +310,14 @@ int oracle_linear_sampled(int64_t M, int64_t N, int64_t K, int64_t k_o, int64_t 
 {
     if (M < 0 || N < 0 || K < 0 || k_o < 0 || k_o > K || (K - k_o) % 2) return ORACLE_EBADARG;
     if (group < 0 || (group > 0 && (K - k_o) % group)) return ORACLE_EBADARG;
+    if (x_bits != 4 && x_bits != 8) return ORACLE_EBADARG;
     const int64_t G = group > 0 ? (K - k_o) / group : 1;
     for (int64_t i = 0; i < count; ++i)
         if (ms[i] < 0 || ms[i] >= M || ns[i] < 0 || ns[i] >= N) return ORACLE_EBADARG;
     int overflow = 0;
 #pragma omp parallel for schedule(static) reduction(| : overflow)
     for (int64_t i = 0; i < count; ++i)
-        Y[i] = linear_element(ms[i], ns[i], M, N, K, k_o, group, outlier_int8, Xq, sx, Xo, sxo,
+        Y[i] = linear_element(ms[i], ns[i], M, N, K, k_o, group, outlier_int8, x_bits, Xq, sx, Xo, sxo,
                               Wq, sw, Wo, swo, bias, acc ? acc + i * G : NULL, &overflow);
     return overflow ? ORACLE_EOVERFLOW : ORACLE_OK;
 }

@@ -344,3 +344,90 @@ def test_sampled_agrees_with_full(oracle_mod):
     np.testing.assert_array_equal(Y, r["Y"][ms, ns])
     full = oracle_mod.int_gemm(r["Xq"], r["Wq"], group)
     np.testing.assert_array_equal(acc, full[:, ms, ns].T)
+
+
+# ----------------------------------------------------------------- 8-bit activations (W4A8)
+# The W4A8 reading: the INT8 rule of the outlier block (divisor and clamp 127)
+# applied per token to the non-outlier positions, one signed byte per code.
+def lossless_rows8(rng, R, n, exp_lo=-6, exp_hi=3):
+    """Rows of values code * 2^e, codes in [-127, 127] with a +-127 in every row."""
+    codes = rng.integers(-127, 128, size=(R, n))
+    scales = np.zeros((R, 1))
+    for r in range(R):
+        codes[r, rng.integers(0, n)] = rng.choice([-127, 127])
+        scales[r, 0] = 2.0 ** rng.integers(exp_lo, exp_hi)
+    return codes, scales, codes * scales
+
+
+def test_a8_codes_are_nearest_brute_force(oracle_mod):
+    rng = np.random.default_rng(21)
+    R, K, k_o = 5, 80, 16
+    X = (rng.standard_normal((R, K)) * rng.uniform(0.01, 10, size=(R, 1))).astype(np.float16)
+    perm = rng.permutation(K).astype(np.int32)
+    Q, s, _, _ = oracle_mod.quantize_rows(X, perm, k_o, 0, False, bits=8)
+    assert Q.dtype == np.int8 and Q.shape == (R, K - k_o)
+    Xr = X[:, perm[:K - k_o]].astype(np.float32)
+    for r in range(R):
+        amax = np.abs(Xr[r]).max()
+        # divisor 127 over the non-outlier positions only
+        assert abs(np.float64(s[r]) * 127 - amax) <= np.spacing(np.float32(amax))
+        for j in range(K - k_o):
+            assert int(Q[r, j]) == nearest_code(Xr[r, j], s[r], 127), (r, j)
+
+
+def test_a8_zero_row(oracle_mod):
+    X = np.zeros((2, 48), np.float16)
+    X[1, 7] = -2.0
+    Q, s, _, _ = oracle_mod.quantize_rows(X, np.arange(48, dtype=np.int32), 16, 0, False, bits=8)
+    assert s[0] == 0.0 and (Q[0] == 0).all()
+    assert Q[1, 7] == -127 and np.count_nonzero(Q[1]) == 1
+
+
+@pytest.mark.parametrize("M,N,K,k_o,int8", [
+    (6, 5, 96, 32, False),
+    (4, 7, 160, 32, True),
+    (5, 3, 64, 0, False),
+])
+def test_a8_lossless_equals_fp64_matmul(oracle_mod, M, N, K, k_o, int8):
+    rng = np.random.default_rng(M * 31 + K)
+    Ki = K - k_o
+    perm = rng.permutation(K).astype(np.int32)
+    cx, sx_true, vx = lossless_rows8(rng, M, Ki)
+    cw, sw_true, vw = lossless_rows(rng, N, Ki)
+    X = np.zeros((M, K)); W = np.zeros((N, K))
+    X[:, perm[:Ki]] = vx
+    W[:, perm[:Ki]] = vw
+    if int8:
+        ox, sxo, vxo = lossless_rows8(rng, M, k_o)
+        ow, swo, vwo = lossless_rows8(rng, N, k_o)
+    else:
+        vxo = rng.standard_normal((M, k_o)) * 40
+        vwo = rng.standard_normal((N, k_o)) * 0.05
+    X[:, perm[Ki:]] = vxo
+    W[:, perm[Ki:]] = vwo
+    X16, W16 = X.astype(np.float16), W.astype(np.float16)
+    assert (X16.astype(np.float64)[:, perm[:Ki]] == vx).all()
+    bias = (rng.standard_normal(N) * 0.01).astype(np.float16)
+    r = oracle_mod.layer(X16, W16, perm, bias, k_o, 0, int8, act_bits=8)
+    np.testing.assert_array_equal(r["Xq"].astype(np.int64), cx)
+    np.testing.assert_array_equal(decode(r["Wq"]), cw)
+    np.testing.assert_array_equal(r["sx"], sx_true[:, 0].astype(np.float32))
+    ref = _fp64_ref(X16, W16, bias)
+    np.testing.assert_allclose(r["Y"], ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_a8_int_gemm_equals_int64_matmul(oracle_mod):
+    rng = np.random.default_rng(22)
+    M, N, Ki = 8, 6, 192
+    Xq = rng.integers(-127, 128, size=(M, Ki)).astype(np.int8)
+    Wq = rng.integers(0, 256, size=(N, Ki // 2), dtype=np.uint8)
+    acc = oracle_mod.int_gemm(Xq, Wq, 0)
+    np.testing.assert_array_equal(acc, Xq.astype(np.int64) @ decode(Wq).T)
+    # the sampled path reads the same codes
+    sx = rng.uniform(0.1, 1, M).astype(np.float32)
+    sw = rng.uniform(0.1, 1, N).astype(np.float32)
+    ms, ns = rng.integers(0, M, 10), rng.integers(0, N, 10)
+    Y, a = oracle_mod.linear_sampled(Xq, sx, None, None, Wq, sw, None, None, None, Ki, 0, 0, ms, ns)
+    np.testing.assert_array_equal(a[:, 0], acc[ms, ns])
+    np.testing.assert_allclose(Y, acc[ms, ns] * sx[ms].astype(np.float64) * sw[ns].astype(np.float64),
+                               rtol=1e-15, atol=0)
