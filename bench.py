@@ -88,6 +88,9 @@ def gemm_source_hash() -> str:
 def gemm_kernel(cfg):
     """The GEMM kernel the library dispatches for this layer, and its profile file."""
     fits = cfg.k_o <= (256 if cfg.outlier_int8 else 128)
+    if cfg.act_bits == 8:
+        return ("w4a4_gemm_pair with INT8 activations (W4A8; weights widened from INT4, "
+                "tcgen05 kind::i8 on CTA pairs)", f"w4a4_gemm_{cfg.name}.md")
     if cfg.group == 0 and cfg.M <= 32 and fits:
         return ("w4a4_gemv (decode shapes: W rows as the MMA's M, tokens as N; INT4 codes "
                 "widened to INT8, tcgen05 kind::i8)", f"w4a4_gemv_{cfg.name}.md")
@@ -211,7 +214,7 @@ def cpu_oracle_step(cfg, d, rows: int):
     full output rows (every column) from the pre-packed weights."""
     import oracle
     X = d["X"][:rows].numpy()
-    xq = oracle.quantize_rows(X, d["perm_np"], cfg.k_o, cfg.group, cfg.outlier_int8)
+    xq = oracle.quantize_rows(X, d["perm_np"], cfg.k_o, cfg.group, cfg.outlier_int8, cfg.act_bits)
     wq = d["w_oracle"]
     oracle.linear(xq[0], xq[1], xq[2] if cfg.k_o else None, xq[3], wq[0], wq[1],
                   wq[2] if cfg.k_o else None, wq[3], d["bias_np"], cfg.K, cfg.k_o, cfg.group)
@@ -286,10 +289,11 @@ def run_ours(args, rank, local_rank, world):
     X = d["X"].to(dev)
     perm = d["perm"].to(dev)
     bias = d["bias"].to(dev) if d["bias"] is not None else None
-    layer = q.QuikLinear(d["W"].to(dev), perm, cfg.k_o, cfg.group, cfg.outlier_int8, bias)
+    layer = q.QuikLinear(d["W"].to(dev), perm, cfg.k_o, cfg.group, cfg.outlier_int8, bias,
+                         act_bits=cfg.act_bits)
     shape = layer.shape(cfg.M)
     Xq, sx, Xo, sxo = q._binding._quant_outputs(cfg.M, cfg.K, cfg.k_o, cfg.group,
-                                                cfg.outlier_int8, dev)
+                                                cfg.outlier_int8, dev, cfg.act_bits)
     Y = torch.empty((cfg.M, cfg.N), dtype=torch.float16, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -422,7 +426,7 @@ def run_ours(args, rank, local_rank, world):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "int4",
+        "dtype": "int4" if cfg.act_bits == 4 else "int4 weights x int8 activations",
         "data": "synthetic",
         "config": {
             "workload": name, "M": cfg.M, "N": cfg.N, "K": cfg.K, "k_o": cfg.k_o,

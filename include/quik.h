@@ -23,6 +23,14 @@
  * row holds code 2i in bits 0-3 and code 2i+1 in bits 4-7, two's complement.
  * Scales: fp32, [rows] or [rows, G] (G = K_i / 128) row-major.
  *
+ * 8-bit activations (W4A8; QQQ abstract: 4-bit weights with 8-bit
+ * activations, per-channel GEMM), selected by quik_shape.act_bits == 8: the
+ * activations' non-outlier positions use the INT8 rule of the outlier block,
+ * s = max|v| / 127 per token and q = clamp(rint(v / s), -127, 127); Xq is then
+ * int8 [M, K_i] row-major, one byte per code in reordered order.  Weights stay
+ * packed INT4.  Per-token scales only (group_size 0).
+
+ *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE memory owned by the caller; the library
  *     never allocates device memory and keeps no pointer after returning.
@@ -31,8 +39,9 @@
  *   - Every function returns a quik_status; nothing throws across the ABI.
  *   - Arguments are validated before any launch: non-NULL pointers that are
  *     16-byte aligned, M, N >= 1, 0 <= k_o <= K, K_i % 32 == 0, k_o % 16 == 0,
- *     K <= 32768, group_size 0 or 128 (then K_i % 128 == 0).  Any violation
- *     returns QUIK_ERR_INVALID_ARG with nothing enqueued.  Pointers that are
+ *     K <= 32768, group_size 0 or 128 (then K_i % 128 == 0), act_bits 0, 4 or
+ *     8.  Any violation returns QUIK_ERR_INVALID_ARG with nothing enqueued;
+ *     act_bits 8 with group_size 128 returns QUIK_ERR_UNSUPPORTED.  Pointers that are
  *     unused for the shape (outlier buffers when k_o == 0, INT8 scales in FP16
  *     mode, bias) may be NULL.
  *   - perm must be a permutation of 0..K-1.  Entries outside [0, K) are
@@ -82,6 +91,7 @@ typedef struct {
     int32_t k_o;        /* outlier channels (last k_o of the reordering) */
     int32_t group_size; /* 0: per-token / per-channel scales; 128: per group */
     int32_t outlier;    /* a quik_outlier_t */
+    int32_t act_bits;   /* activation codes: 0 or 4 -> INT4 (W4A4); 8 -> INT8 (W4A8) */
 } quik_shape;
 
 /* Opaque cudaStream_t. */
@@ -102,7 +112,7 @@ QUIK_API size_t quik_workspace_size(const quik_shape *shape);
  * (INT8) the outlier block.
  *   X_f16    [M, K] fp16, row-major
  *   perm     [K] int32
- *   Xq       out [M, K_i/2] packed INT4
+ *   Xq       out [M, K_i/2] packed INT4 (act_bits 8: int8 [M, K_i])
  *   x_scale  out fp32 [M] or [M, G]
  *   Xo       out [M, k_o] fp16 or int8 (may be NULL when k_o == 0)
  *   xo_scale out fp32 [M], INT8 outliers only (NULL otherwise)
@@ -115,7 +125,8 @@ QUIK_API quik_status quik_quantize_reorder(const quik_shape *shape, const void *
  * quik_pack_weights -- offline weight preparation (QUIK sample names
  * pack_to_i4 / two_compl; Atom idea I1): the same reorder + symmetric
  * quantiser applied to the rows of W (one scale per output channel, or per
- * channel and group), round-to-nearest codes.
+ * channel and group), round-to-nearest codes.  Always INT4, whatever
+ * act_bits.
  *   W_f16 [N, K] fp16; Wq out [N, K_i/2]; w_scale out [N] or [N, G];
  *   Wo out [N, k_o] fp16 or int8; wo_scale out [N] (INT8 outliers only).
  */
@@ -127,7 +138,8 @@ QUIK_API quik_status quik_pack_weights(const quik_shape *shape, const void *W_f1
  * quik_gemm -- INT4 x INT4 product with exact INT32 accumulation (tensor
  * cores, Atom key points), the outlier sub-product, and the dequantising
  * epilogue Y = A*sx*sw (+ per group) + O + bias, rounded to fp16.
- *   Xq [M, K_i/2], x_scale, Xo [M, k_o], xo_scale : quantised activations
+ *   Xq [M, K_i/2] (act_bits 8: int8 [M, K_i]), x_scale, Xo [M, k_o], xo_scale :
+ *                                                   quantised activations
  *   Wq [N, K_i/2], w_scale, Wo [N, k_o], wo_scale : packed weights
  *   bias_f16 [N] or NULL;  Y_f16 out [M, N] fp16 row-major
  */

@@ -35,7 +35,7 @@ class QuikError(RuntimeError):
 class quik_shape(ctypes.Structure):
     _fields_ = [("M", ctypes.c_int32), ("N", ctypes.c_int32), ("K", ctypes.c_int32),
                 ("k_o", ctypes.c_int32), ("group_size", ctypes.c_int32),
-                ("outlier", ctypes.c_int32)]
+                ("outlier", ctypes.c_int32), ("act_bits", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p
@@ -87,8 +87,8 @@ def _check(status: int, what: str):
 
 
 def make_shape(M: int, N: int, K: int, k_o: int, group_size: int = 0,
-               outlier: int = QUIK_OUTLIER_FP16) -> quik_shape:
-    return quik_shape(M, N, K, k_o, group_size, outlier)
+               outlier: int = QUIK_OUTLIER_FP16, act_bits: int = 4) -> quik_shape:
+    return quik_shape(M, N, K, k_o, group_size, outlier, act_bits)
 
 
 def _ptr(t, dtype=None, what="tensor"):
@@ -105,6 +105,11 @@ def _ptr(t, dtype=None, what="tensor"):
     return t.data_ptr() if t.numel() > 0 else None
 
 
+def _xq_dtype(shape: quik_shape):
+    """Quantised activations: packed INT4 bytes, or INT8 codes when act_bits == 8."""
+    return torch.int8 if shape.act_bits == 8 else torch.uint8
+
+
 def _stream(stream=None) -> int:
     s = stream if stream is not None else torch.cuda.current_stream()
     return s.cuda_stream
@@ -118,7 +123,7 @@ def quik_workspace_size(shape: quik_shape) -> int:
 def quik_quantize_reorder(shape, X, perm, Xq, x_scale, Xo, xo_scale, stream=None):
     _check(lib().quik_quantize_reorder(
         ctypes.byref(shape), _ptr(X, torch.float16, "X"), _ptr(perm, torch.int32, "perm"),
-        _ptr(Xq, torch.uint8, "Xq"), _ptr(x_scale, torch.float32, "x_scale"), _ptr(Xo, None, "Xo"),
+        _ptr(Xq, _xq_dtype(shape), "Xq"), _ptr(x_scale, torch.float32, "x_scale"), _ptr(Xo, None, "Xo"),
         _ptr(xo_scale, torch.float32, "xo_scale"), _stream(stream)), "quik_quantize_reorder")
 
 
@@ -131,7 +136,7 @@ def quik_pack_weights(shape, W, perm, Wq, w_scale, Wo, wo_scale, stream=None):
 
 def quik_gemm(shape, Xq, x_scale, Xo, xo_scale, Wq, w_scale, Wo, wo_scale, bias, Y, stream=None):
     _check(lib().quik_gemm(
-        ctypes.byref(shape), _ptr(Xq, torch.uint8, "Xq"), _ptr(x_scale, torch.float32, "x_scale"),
+        ctypes.byref(shape), _ptr(Xq, _xq_dtype(shape), "Xq"), _ptr(x_scale, torch.float32, "x_scale"),
         _ptr(Xo, None, "Xo"), _ptr(xo_scale, torch.float32, "xo_scale"),
         _ptr(Wq, torch.uint8, "Wq"), _ptr(w_scale, torch.float32, "w_scale"),
         _ptr(Wo, None, "Wo"), _ptr(wo_scale, torch.float32, "wo_scale"),
@@ -160,7 +165,7 @@ def quik_linear_noalloc(shape, X, perm, Wq, w_scale, Wo, wo_scale, bias, Y, stre
 
 def quik_gemm_i32_debug(shape, Xq, Wq, Xo, Wo, acc, acc_outlier, stream=None):
     _check(lib().quik_gemm_i32_debug(
-        ctypes.byref(shape), _ptr(Xq, torch.uint8, "Xq"), _ptr(Wq, torch.uint8, "Wq"),
+        ctypes.byref(shape), _ptr(Xq, _xq_dtype(shape), "Xq"), _ptr(Wq, torch.uint8, "Wq"),
         _ptr(Xo, None, "Xo"), _ptr(Wo, None, "Wo"), _ptr(acc, torch.int32, "acc"),
         _ptr(acc_outlier, torch.int32, "acc_outlier"), _stream(stream)), "quik_gemm_i32_debug")
 
@@ -182,10 +187,11 @@ def _outlier_kind(int8: bool) -> int:
     return QUIK_OUTLIER_INT8 if int8 else QUIK_OUTLIER_FP16
 
 
-def _quant_outputs(rows: int, K: int, k_o: int, group: int, int8: bool, device):
+def _quant_outputs(rows: int, K: int, k_o: int, group: int, int8: bool, device, bits: int = 4):
     Ki = K - k_o
     G = Ki // group if group else 1
-    Q = torch.empty((rows, Ki // 2), dtype=torch.uint8, device=device)
+    Q = (torch.empty((rows, Ki), dtype=torch.int8, device=device) if bits == 8 else
+         torch.empty((rows, Ki // 2), dtype=torch.uint8, device=device))
     scale = torch.empty((rows, G) if group else (rows,), dtype=torch.float32, device=device)
     O = torch.empty((rows, k_o), dtype=torch.int8 if int8 else torch.float16, device=device)
     o_scale = torch.empty((rows,), dtype=torch.float32, device=device) if int8 else None
@@ -193,11 +199,12 @@ def _quant_outputs(rows: int, K: int, k_o: int, group: int, int8: bool, device):
 
 
 def quantize_reorder(X: torch.Tensor, perm: torch.Tensor, k_o: int, group: int = 0,
-                     outlier_int8: bool = False, stream=None):
-    """Activations -> (Xq, x_scale, Xo, xo_scale), allocated on X's device."""
+                     outlier_int8: bool = False, stream=None, act_bits: int = 4):
+    """Activations -> (Xq, x_scale, Xo, xo_scale), allocated on X's device.
+    Xq is packed INT4 (uint8 [M, K_i/2]), or int8 [M, K_i] when act_bits == 8."""
     M, K = X.shape
-    shape = make_shape(M, 1, K, k_o, group, _outlier_kind(outlier_int8))
-    out = _quant_outputs(M, K, k_o, group, outlier_int8, X.device)
+    shape = make_shape(M, 1, K, k_o, group, _outlier_kind(outlier_int8), act_bits)
+    out = _quant_outputs(M, K, k_o, group, outlier_int8, X.device, act_bits)
     quik_quantize_reorder(shape, X, perm, *out, stream=stream)
     return out
 
@@ -218,7 +225,7 @@ def gemm(xq, wq, K: int, k_o: int, group: int = 0, bias=None, stream=None):
     Wq, sw, Wo, swo = wq
     M, N = sx.shape[0], sw.shape[0]
     int8 = Xo.dtype == torch.int8
-    shape = make_shape(M, N, K, k_o, group, _outlier_kind(int8))
+    shape = make_shape(M, N, K, k_o, group, _outlier_kind(int8), 8 if Xq.dtype == torch.int8 else 4)
     Y = torch.empty((M, N), dtype=torch.float16, device=sx.device)
     quik_gemm(shape, Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias, Y, stream=stream)
     return Y
@@ -230,7 +237,7 @@ def gemm_i32(Xq, Wq, K: int, k_o: int, group: int = 0, Xo=None, Wo=None, stream=
     Ki = K - k_o
     G = Ki // group if group else 1
     int8 = Xo is not None and Xo.dtype == torch.int8
-    shape = make_shape(M, N, K, k_o, group, _outlier_kind(int8))
+    shape = make_shape(M, N, K, k_o, group, _outlier_kind(int8), 8 if Xq.dtype == torch.int8 else 4)
     acc = torch.empty((G, M, N) if group else (M, N), dtype=torch.int32, device=Xq.device)
     acc_o = torch.empty((M, N), dtype=torch.int32, device=Xq.device) if int8 and k_o else None
     quik_gemm_i32_debug(shape, Xq, Wq, Xo if int8 else None, Wo if int8 else None, acc, acc_o,
@@ -239,24 +246,26 @@ def gemm_i32(Xq, Wq, K: int, k_o: int, group: int = 0, Xo=None, Wo=None, stream=
 
 
 class QuikLinear:
-    """A hybrid W4A4 + outlier linear layer with packed weights resident on the GPU.
+    """A hybrid W4A4 (or W4A8) + outlier linear layer with packed weights resident on the GPU.
 
-    ``QuikLinear(W, perm, k_o, group, outlier_int8, bias)`` packs W once
-    (quik_pack_weights); calling it on fp16 activations runs quik_linear into
-    a workspace it keeps.
+    ``QuikLinear(W, perm, k_o, group, outlier_int8, bias, act_bits)`` packs W
+    once (quik_pack_weights); calling it on fp16 activations runs quik_linear
+    into a workspace it keeps.  act_bits 8 quantises the activations to INT8.
     """
 
     def __init__(self, W: torch.Tensor, perm: torch.Tensor, k_o: int, group: int = 0,
-                 outlier_int8: bool = False, bias: torch.Tensor | None = None):
+                 outlier_int8: bool = False, bias: torch.Tensor | None = None, act_bits: int = 4):
         self.N, self.K = W.shape
         self.k_o, self.group, self.outlier_int8 = k_o, group, outlier_int8
+        self.act_bits = act_bits
         self.perm = perm
         self.bias = bias
         self.Wq, self.w_scale, self.Wo, self.wo_scale = pack_weights(W, perm, k_o, group, outlier_int8)
         self._ws = None
 
     def shape(self, M: int) -> quik_shape:
-        return make_shape(M, self.N, self.K, self.k_o, self.group, _outlier_kind(self.outlier_int8))
+        return make_shape(M, self.N, self.K, self.k_o, self.group, _outlier_kind(self.outlier_int8),
+                          self.act_bits)
 
     def workspace(self, M: int, device) -> torch.Tensor:
         need = quik_workspace_size(self.shape(M))

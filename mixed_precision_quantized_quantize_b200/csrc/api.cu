@@ -26,6 +26,8 @@ quik_status check_shape(const quik_shape *s) {
     if (s->group_size == kGroup && Ki % kGroup != 0) return QUIK_ERR_INVALID_ARG;
     if (s->outlier != QUIK_OUTLIER_FP16 && s->outlier != QUIK_OUTLIER_INT8)
         return QUIK_ERR_INVALID_ARG;
+    if (s->act_bits != 0 && s->act_bits != 4 && s->act_bits != 8) return QUIK_ERR_INVALID_ARG;
+    if (s->act_bits == 8 && s->group_size != 0) return QUIK_ERR_UNSUPPORTED;
     return QUIK_OK;
 }
 
@@ -35,6 +37,7 @@ inline int groups_of(const quik_shape *s) {
 }
 inline bool needs_scale(const quik_shape *s) { return groups_of(s) > 0; }
 inline bool int8_out(const quik_shape *s) { return s->outlier == QUIK_OUTLIER_INT8; }
+inline bool act8(const quik_shape *s) { return s->act_bits == 8; }
 
 // Rows of one operand: packed codes, scales, outlier block (+ INT8 scales).
 quik_status check_quant_ptrs(const quik_shape *s, const void *Q, const float *scale,
@@ -48,8 +51,9 @@ quik_status check_quant_ptrs(const quik_shape *s, const void *Q, const float *sc
     return QUIK_OK;
 }
 
-quik_status quantize(const quik_shape *s, int rows, const void *X, const int32_t *perm, void *Q,
-                     float *scale, void *O, float *o_scale, cudaStream_t stream) {
+// bits8: INT8 codes (activations of a W4A8 shape); weights are always INT4.
+quik_status quantize(const quik_shape *s, int rows, bool bits8, const void *X, const int32_t *perm,
+                     void *Q, float *scale, void *O, float *o_scale, cudaStream_t stream) {
     quik::QuantizeArgs a;
     a.X = static_cast<const uint16_t *>(X);
     a.perm = perm;
@@ -58,6 +62,7 @@ quik_status quantize(const quik_shape *s, int rows, const void *X, const int32_t
     a.k_o = s->k_o;
     a.group = s->group_size;
     a.out_int8 = int8_out(s);
+    a.bits8 = bits8;
     a.Q = static_cast<uint8_t *>(Q);
     a.scale = scale;
     a.O = O;
@@ -75,7 +80,7 @@ Workspace layout(const quik_shape *s) {
     const size_t G = static_cast<size_t>(groups_of(s));
     Workspace w;
     w.xq = 0;
-    w.sx = w.xq + round256(M * Ki / 2);
+    w.sx = w.xq + round256(act8(s) ? M * Ki : M * Ki / 2);
     w.xo = w.sx + round256(M * G * sizeof(float));
     w.sxo = w.xo + round256(M * s->k_o * (int8_out(s) ? 1 : 2));
     w.total = w.sxo + round256(int8_out(s) ? M * sizeof(float) : 0);
@@ -98,7 +103,7 @@ quik_status quik_quantize_reorder(const quik_shape *shape, const void *X_f16, co
     if (st != QUIK_OK) return st;
     if (!ok_ptr(X_f16) || !ok_ptr(perm)) return QUIK_ERR_INVALID_ARG;
     if ((st = check_quant_ptrs(shape, Xq, x_scale, Xo, xo_scale)) != QUIK_OK) return st;
-    return quantize(shape, shape->M, X_f16, perm, Xq, x_scale, Xo, xo_scale,
+    return quantize(shape, shape->M, act8(shape), X_f16, perm, Xq, x_scale, Xo, xo_scale,
                     static_cast<cudaStream_t>(stream));
 }
 
@@ -109,7 +114,7 @@ quik_status quik_pack_weights(const quik_shape *shape, const void *W_f16, const 
     if (st != QUIK_OK) return st;
     if (!ok_ptr(W_f16) || !ok_ptr(perm)) return QUIK_ERR_INVALID_ARG;
     if ((st = check_quant_ptrs(shape, Wq, w_scale, Wo, wo_scale)) != QUIK_OK) return st;
-    return quantize(shape, shape->N, W_f16, perm, Wq, w_scale, Wo, wo_scale,
+    return quantize(shape, shape->N, false, W_f16, perm, Wq, w_scale, Wo, wo_scale,
                     static_cast<cudaStream_t>(stream));
 }
 
@@ -125,6 +130,7 @@ static quik_status gemm_impl(const quik_shape *shape, const void *Xq, const floa
     a.k_o = shape->k_o;
     a.group = shape->group_size;
     a.out_int8 = int8_out(shape);
+    a.a8 = act8(shape);
     a.Xq = Xq;
     a.sx = x_scale;
     a.Xo = Xo;
@@ -172,7 +178,8 @@ quik_status quik_linear(const quik_shape *shape, const void *X_f16, const int32_
     void *Xo = ws + w.xo;
     float *sxo = int8_out(shape) ? reinterpret_cast<float *>(ws + w.sxo) : nullptr;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if ((st = quantize(shape, shape->M, X_f16, perm, Xq, sx, Xo, sxo, s)) != QUIK_OK) return st;
+    if ((st = quantize(shape, shape->M, act8(shape), X_f16, perm, Xq, sx, Xo, sxo, s)) != QUIK_OK)
+        return st;
     // the GEMM follows this quantiser on the same stream: its set-up and weight
     // loads may overlap the quantiser's tail
     return gemm_impl(shape, Xq, sx, Xo, sxo, Wq, w_scale, Wo, wo_scale, bias_f16, Y_f16, false,

@@ -154,6 +154,30 @@ __device__ __forceinline__ float small_int_to_float(int32_t v) {
     return __int_as_float(v + 0x4B400000) - 12582912.0f;
 }
 
+// The INT4-part sum from the tensor-core accumulator.  INT4 activations: both
+// operands carry a factor 16 (sum 256 A, |A| <= 49 K_i < 2^22: exact by the
+// magic-number add).  INT8 activations (W4A8): only the weights do (sum 16 A,
+// |A| <= 889 K_i, which can pass 2^22: a rounding conversion, exact below 2^24).
+template <bool A8>
+__device__ __forceinline__ int32_t acc_int(uint32_t raw) {
+    return static_cast<int32_t>(raw) >> (A8 ? 4 : 8);
+}
+template <bool A8>
+__device__ __forceinline__ float acc_float(uint32_t raw) {
+    return A8 ? __int2float_rn(acc_int<A8>(raw)) : small_int_to_float(acc_int<A8>(raw));
+}
+
+// W4A8: 32 INT8 codes (two 16-byte chunks, codes in order) in the order the
+// INT4 unpack gives the weights' codes: even positions of the 32, then odd.
+__device__ __forceinline__ void order_i8_chunk(const uint4 a, const uint4 b, uint32_t *w) {
+    const uint32_t x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        asm("prmt.b32 %0, %1, %2, 0x6420;" : "=r"(w[i]) : "r"(x[2 * i]), "r"(x[2 * i + 1]));
+        asm("prmt.b32 %0, %1, %2, 0x7531;" : "=r"(w[4 + i]) : "r"(x[2 * i]), "r"(x[2 * i + 1]));
+    }
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, C::MINB)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tm_xq,
@@ -630,7 +654,7 @@ static_assert(A_COL + 32 * S <= TMEM_COLS, "A stages fit in tensor memory");
 static_assert(SMEM <= 232448, "shared memory budget");
 }  // namespace pair
 
-template <bool OUT_INT8, bool DEBUG>
+template <bool OUT_INT8, bool DEBUG, bool A8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
     w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_wq,
                           const __grid_constant__ CUtensorMap tm_wo,
@@ -656,7 +680,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
     const int nb0 = n0 + rank * BNH;                 // this CTA's rows of W (half of B)
     const int nkb = p.nkb_i + p.nkb_o;
     const int nunits = p.nkb_i + 2 * p.nkb_o;        // staging units
-    const int rb = p.Ki / 2;
+    const int rb = A8 ? p.Ki : p.Ki / 2;             // bytes of an Xq row
 
     if (threadIdx.x == 0) {
         QUIK_TRACE_AT(6, 0);
@@ -778,33 +802,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
             const bool row_ok = grow < p.M;
             const uint8_t *xrow = Xq + (size_t)grow * rb;
             const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
-            uint4 buf[PF][4];
+            // a k-block of a row: 4 chunks of 16 packed bytes, or 8 of INT8 codes
+            constexpr int CH = A8 ? 8 : 4, KB_BYTES = A8 ? OP_ROW : PK_ROW, PFA = A8 ? PF / 2 : PF;
+            uint4 buf[PFA][CH];
             grid_dependency_wait();  // Xq (and later sx) come from the previous kernel
-            auto load = [&](int kb, uint4(&d)[4]) {
+            auto load = [&](int kb, uint4(&d)[CH]) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int off = kb * PK_ROW + c * 16;
+                for (int c = 0; c < CH; ++c) {
+                    const int off = kb * KB_BYTES + c * 16;
                     d[c] = (row_ok && off < rb) ? ldg_nc_v4(xrow + off) : make_uint4(0, 0, 0, 0);
                 }
             };
 #pragma unroll
-            for (int j = 0; j < PF; ++j)
+            for (int j = 0; j < PFA; ++j)
                 if (j < p.nkb_i) load(j, buf[j]);
-            for (int kb0 = 0; kb0 < p.nkb_i && ok; kb0 += PF) {
+            for (int kb0 = 0; kb0 < p.nkb_i && ok; kb0 += PFA) {
 #pragma unroll
-                for (int j = 0; j < PF; ++j) {
+                for (int j = 0; j < PFA; ++j) {
                     const int kb = kb0 + j;
                     if (kb >= p.nkb_i || !ok) break;
                     const int st = kb % S;
                     ok = wait_bar(&op_empty[st], ((kb / S) & 1) ^ 1, ab);
                     if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                     uint32_t w[32];
+                    if constexpr (A8) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint4 lo, hi;
-                        unpack16(buf[j][c], lo, hi);
-                        w[8 * c + 0] = lo.x; w[8 * c + 1] = lo.y; w[8 * c + 2] = lo.z; w[8 * c + 3] = lo.w;
-                        w[8 * c + 4] = hi.x; w[8 * c + 5] = hi.y; w[8 * c + 6] = hi.z; w[8 * c + 7] = hi.w;
+                        for (int c = 0; c < 4; ++c) order_i8_chunk(buf[j][2 * c], buf[j][2 * c + 1], w + 8 * c);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            uint4 lo, hi;
+                            unpack16(buf[j][c], lo, hi);
+                            w[8 * c + 0] = lo.x; w[8 * c + 1] = lo.y; w[8 * c + 2] = lo.z; w[8 * c + 3] = lo.w;
+                            w[8 * c + 4] = hi.x; w[8 * c + 5] = hi.y; w[8 * c + 6] = hi.z; w[8 * c + 7] = hi.w;
+                        }
                     }
                     tmem_st_32x32b_x32(t_lane + A_COL + 32 * st, w);
                     tmem_st_wait();
@@ -815,7 +846,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
                     if (lane == 0 && blockIdx.x + blockIdx.y * gridDim.x < kTraceCtas && kb < kTraceKb)
                         atomicMax(&g_trace[blockIdx.x + blockIdx.y * gridDim.x][2][kb], clock64());
     #endif
-                    if (kb + PF < p.nkb_i) load(kb + PF, buf[j]);
+                    if (kb + PFA < p.nkb_i) load(kb + PFA, buf[j]);
                 }
             }
             // outlier k-blocks: both operands arrive through shared memory
@@ -927,7 +958,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
                             const int n = nb + jj;
                             if (n < p.N) {
                                 if (p.Ki > 0)
-                                    p.acc_dbg[(size_t)grow * p.N + n] = static_cast<int32_t>(a[jj]) >> 8;
+                                    p.acc_dbg[(size_t)grow * p.N + n] = acc_int<A8>(a[jj]);
                                 if (OUT_INT8 && p.nkb_o > 0 && p.acc_o_dbg)
                                     p.acc_o_dbg[(size_t)grow * p.N + n] = static_cast<int32_t>(o[jj]);
                             }
@@ -942,7 +973,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int c = cc + jj + h;
-                        float v = small_int_to_float(static_cast<int32_t>(a[jj + h]) >> 8) * sxr * col_sw[c];
+                        float v = acc_float<A8>(a[jj + h]) * sxr * col_sw[c];
                         if (p.Ki == 0) v = 0.0f;
                         if (p.nkb_o > 0) {
                             if (OUT_INT8)
@@ -1429,7 +1460,7 @@ quik_status run(const GemmArgs &a, cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
 }
 
-template <bool OUT_INT8, bool DEBUG>
+template <bool OUT_INT8, bool DEBUG, bool A8>
 quik_status run_pair(const GemmArgs &a, cudaStream_t stream) {
     const int Ki = a.K - a.k_o;
     const bool outliers = a.k_o > 0 && a.Xo != nullptr;  // debug entry may skip them
@@ -1471,7 +1502,7 @@ quik_status run_pair(const GemmArgs &a, cudaStream_t stream) {
     p.tma_y = !DEBUG && (a.N % 8 == 0) &&
               make_map(&my, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.Y, a.N, a.M, static_cast<uint64_t>(a.N) * 2,
                        64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
-    auto kern = w4a4_gemm_pair_kernel<OUT_INT8, DEBUG>;
+    auto kern = w4a4_gemm_pair_kernel<OUT_INT8, DEBUG, A8>;
     if (!attribute_set_once(reinterpret_cast<const void *>(kern), pair::SMEM)) return QUIK_ERR_CUDA;
     const dim3 grid(2 * ((a.N + pair::BN - 1) / pair::BN), (a.M + 2 * BM - 1) / (2 * BM));
     if (!a.after_quantize) {
@@ -1568,10 +1599,14 @@ quik_status run_gemv(const GemmArgs &a, cudaStream_t stream) {
 // shared-memory-operand kernel.
 template <bool DEBUG>
 quik_status dispatch(const GemmArgs &a, cudaStream_t stream) {
+    if (a.a8) {  // INT8 activations (W4A8): per-token scales, the pair kernel
+        if (a.group != 0) return QUIK_ERR_UNSUPPORTED;
+        return a.out_int8 ? run_pair<true, DEBUG, true>(a, stream) : run_pair<false, DEBUG, true>(a, stream);
+    }
     if (a.group == 0 && a.M <= gemv::MT && a.k_o <= (a.out_int8 ? gemv::KO_MAX_I8 : gemv::KO_MAX_F16))
         return a.out_int8 ? run_gemv<true, DEBUG>(a, stream) : run_gemv<false, DEBUG>(a, stream);
     if (a.group == 0)
-        return a.out_int8 ? run_pair<true, DEBUG>(a, stream) : run_pair<false, DEBUG>(a, stream);
+        return a.out_int8 ? run_pair<true, DEBUG, false>(a, stream) : run_pair<false, DEBUG, false>(a, stream);
     return a.out_int8 ? run<CfgGroup<true, DEBUG>>(a, stream) : run<CfgGroup<false, DEBUG>>(a, stream);
 }
 

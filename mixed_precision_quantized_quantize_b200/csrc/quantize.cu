@@ -73,6 +73,7 @@ struct QParams {
     float *scale;
     void *O;
     float *o_scale;
+    int bits8;  // per-token rows only: INT8 codes (one byte each, divisor 127)
 };
 
 __device__ __forceinline__ float h2f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
@@ -188,6 +189,47 @@ __device__ __forceinline__ uint32_t pack_codes8(const uint32_t (&h)[4], float s,
         }
     }
     return word ^ 0x88888888u;
+}
+
+// Eight INT8 codes, one byte each in position order, from four half2 values
+// (W4A8 activations): the fast path below for every value, and IEEE
+// divisions for a word with any near-tie.
+__device__ __forceinline__ uint2 pack_codes8_i8(const uint32_t (&h)[4], float s, float rs) {
+    uint32_t q[8];
+    float dmax = 0.0f;
+    const uint64_t rs2 = f2(rs, rs), kr2 = f2(kRound, kRound);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[k]));
+        const uint64_t v2 = f2(f.x, f.y);
+        const uint64_t m = f2_fma(v2, rs2, kr2);           // 1.5*2^23 + rint(v rs)
+        const uint64_t r = f2_sub(m, kr2);
+        float r0, r1;
+        f2_split(r, r0, r1);
+        const uint64_t d = f2_fma(v2, rs2, f2(-r0, -r1));  // v rs - rint(v rs)
+        float m0, m1, d0, d1;
+        f2_split(m, m0, m1);
+        f2_split(d, d0, d1);
+        dmax = max3(dmax, fabsf(d0), fabsf(d1));
+        q[2 * k] = __float_as_uint(m0) - kRoundBits;        // the code, two's complement
+        q[2 * k + 1] = __float_as_uint(m1) - kRoundBits;
+    }
+    if (dmax > 0.5f - 4e-5f) {  // near a tie somewhere in this word: exact divisions
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            q[2 * k] = static_cast<uint32_t>(exact_code(h2f(static_cast<uint16_t>(h[k] & 0xffffu)), s, 127));
+            q[2 * k + 1] = static_cast<uint32_t>(exact_code(h2f(static_cast<uint16_t>(h[k] >> 16)), s, 127));
+        }
+    }
+    // low byte of each code, in order
+    auto bytes4 = [](uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+        uint32_t ab, cd, r;
+        asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(ab) : "r"(a), "r"(b));
+        asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(cd) : "r"(c), "r"(d));
+        asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(ab), "r"(cd));
+        return r;
+    };
+    return make_uint2(bytes4(q[0], q[1], q[2], q[3]), bytes4(q[4], q[5], q[6], q[7]));
 }
 
 // INT8 outlier code (same fast path; |v/s| <= 127(1+u) gives an error bound
@@ -388,7 +430,7 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : GROUPE
             team_sync(bar_id, TT);
             m = 0.0f;
             for (int k = 0; k < (TT >> 5); ++k) m = fmaxf(m, red[team][j & 1][k]);
-            const float sr = div_exact<7, 3>(m), rr = rcp_approx(sr);
+            const float sr = p.bits8 ? div_exact<127, 7>(m) : div_exact<7, 3>(m), rr = rcp_approx(sr);
 #pragma unroll
             for (int i = 0; i < W; ++i) {
                 s[i] = sr;
@@ -397,12 +439,22 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : GROUPE
             if (tl == 0) p.scale[row] = sr;
         }
 
-        // (4) codes, 8 per word, code 2i in the low nibble of byte i
-        uint32_t *qrow = reinterpret_cast<uint32_t *>(p.Q + static_cast<size_t>(row) * (Ki / 2));
+        // (4) codes, 8 per word, code 2i in the low nibble of byte i (or one
+        // byte per code for INT8 activations)
+        if (!GROUPED && p.bits8) {
+            uint2 *qrow8 = reinterpret_cast<uint2 *>(p.Q + static_cast<size_t>(row) * Ki);
 #pragma unroll
-        for (int i = 0; i < W; ++i) {
-            const int w = tl + i * TT;
-            if (w < nwords && QUIK_CHECK(4 * w + 4 <= Ki / 2, 4)) qrow[w] = pack_codes8(v[i], s[i], r[i]);
+            for (int i = 0; i < W; ++i) {
+                const int w = tl + i * TT;
+                if (w < nwords && QUIK_CHECK(8 * w + 8 <= Ki, 4)) qrow8[w] = pack_codes8_i8(v[i], s[i], r[i]);
+            }
+        } else {
+            uint32_t *qrow = reinterpret_cast<uint32_t *>(p.Q + static_cast<size_t>(row) * (Ki / 2));
+#pragma unroll
+            for (int i = 0; i < W; ++i) {
+                const int w = tl + i * TT;
+                if (w < nwords && QUIK_CHECK(4 * w + 4 <= Ki / 2, 4)) qrow[w] = pack_codes8(v[i], s[i], r[i]);
+            }
         }
 
         // (5) the outlier block
@@ -558,7 +610,8 @@ cudaError_t launch_q_w(const QParams &p, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_quantize_rows(const QuantizeArgs &a, cudaStream_t stream) {
-    QParams p{a.X, a.perm, a.rows, a.K, a.k_o, 0, 0, 0, a.Q, a.scale, a.O, a.o_scale};
+    QParams p{a.X, a.perm, a.rows, a.K, a.k_o, 0, 0, 0, a.Q, a.scale, a.O, a.o_scale, a.bits8 ? 1 : 0};
+    if (a.bits8 && a.group > 0) return cudaErrorInvalidValue;  // INT8 codes: per-row scales only
     if (a.group > 0)
         return a.out_int8 ? launch_q_w<true, true>(p, stream) : launch_q_w<true, false>(p, stream);
     return a.out_int8 ? launch_q_w<false, true>(p, stream) : launch_q_w<false, false>(p, stream);

@@ -35,6 +35,7 @@ struct QuantizeArgs {
     const int32_t *perm;
     int rows, K, k_o, group;
     bool out_int8;
+    bool bits8;  // INT8 codes (divisor and clamp 127, one byte each) instead of packed INT4
     uint8_t *Q;
     float *scale;
     void *O;
@@ -50,6 +51,7 @@ unsigned int take_quantize_errors(unsigned int *bad_perm);
 struct GemmArgs {
     int M, N, K, k_o, group;
     bool out_int8;
+    bool a8;  // Xq holds INT8 codes [M, K_i] (W4A8) instead of packed INT4
     const void *Xq;
     const float *sx;
     const void *Xo;

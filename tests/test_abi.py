@@ -37,8 +37,8 @@ def test_status_strings(L):
         assert q.status_string(s) == name
 
 
-def _ws(M, N, K, k_o, group=0, outlier=0):
-    return q.quik_workspace_size(q.make_shape(M, N, K, k_o, group, outlier))
+def _ws(M, N, K, k_o, group=0, outlier=0, act_bits=4):
+    return q.quik_workspace_size(q.make_shape(M, N, K, k_o, group, outlier, act_bits))
 
 
 def test_workspace_size(L):
@@ -50,6 +50,9 @@ def test_workspace_size(L):
     assert _ws(1024, 22016, 8192, 128, 128, 1) == (r(1024 * 8064 // 2) + r(1024 * G * 4)
                                                    + r(1024 * 128) + r(1024 * 4))
     assert _ws(16, 256, 256, 0) == r(16 * 128) + r(16 * 4)
+    # INT8 activations (W4A8): one byte per code; 0 is INT4 as well
+    assert _ws(2048, 4096, 4096, 128, 0, 0, 8) == r(2048 * 3968) + r(2048 * 4) + r(2048 * 128 * 2)
+    assert _ws(2048, 4096, 4096, 128, 0, 0, 0) == _ws(2048, 4096, 4096, 128)
 
 
 @pytest.mark.parametrize("shape", [
@@ -63,6 +66,8 @@ def test_workspace_size(L):
     (16, 16, 256, 0, -1, 0),      # negative group size
     (16, 16, 256, 0, 0, 5),       # unknown outlier kind
     (16, 16, 65536, 0, 0, 0),     # K above the supported maximum
+    (16, 16, 256, 0, 0, 0, 3),    # activation width neither 4 nor 8
+    (16, 16, 256, 0, 0, 0, 16),
 ])
 def test_invalid_shapes_rejected(L, shape):
     assert _ws(*shape) == 0
@@ -73,6 +78,12 @@ def test_invalid_shapes_rejected(L, shape):
 
 def test_unsupported_group_size(L):
     s = q.make_shape(16, 16, 256, 0, 64, 0)
+    assert L.quik_gemm(ctypes.byref(s), *([None] * 11)) == q.QUIK_ERR_UNSUPPORTED
+
+
+def test_grouped_int8_activations_unsupported(L):
+    s = q.make_shape(16, 16, 256, 0, 128, 0, 8)
+    assert _ws(16, 16, 256, 0, 128, 0, 8) == 0
     assert L.quik_gemm(ctypes.byref(s), *([None] * 11)) == q.QUIK_ERR_UNSUPPORTED
 
 

@@ -247,6 +247,7 @@ FULL = [
     ("llama7b_up_2048x11008x4096", None),
     ("llama65b_mlp_grouped_1024x22016x8192", None),
     ("llama7b_down_fused_4096x4096x11008", None),
+    ("llama7b_attn_w4a8_2048x4096x4096", None),
 ]
 
 
@@ -267,11 +268,13 @@ def test_full_size_layer(name):
     perm_d = d["perm"].to(DEV)
     b = d["bias"].to(DEV) if d["bias"] is not None else None
     X = d["X"].to(DEV)
-    layer = q.QuikLinear(d["W"].to(DEV), perm_d, cfg.k_o, cfg.group, cfg.outlier_int8, b)
+    layer = q.QuikLinear(d["W"].to(DEV), perm_d, cfg.k_o, cfg.group, cfg.outlier_int8, b,
+                         act_bits=cfg.act_bits)
     Y = layer(X)
-    gx = q.quantize_reorder(X, perm_d, cfg.k_o, cfg.group, cfg.outlier_int8)
+    gx = q.quantize_reorder(X, perm_d, cfg.k_o, cfg.group, cfg.outlier_int8, act_bits=cfg.act_bits)
     torch.cuda.synchronize()
-    ox = oracle_quant(d["X"], d["perm"], cfg.k_o, cfg.group, cfg.outlier_int8)
+    ox = oracle.quantize_rows(np16(d["X"]), d["perm"].numpy(), cfg.k_o, cfg.group, cfg.outlier_int8,
+                              cfg.act_bits)
     ow = oracle_quant(d["W"], d["perm"], cfg.k_o, cfg.group, cfg.outlier_int8)
     # every code, scale and outlier value, activations and weights
     assert_quant_equal(gpu_tuple_np(gx), ox, f"{name} X")
@@ -295,3 +298,82 @@ def test_full_size_layer(name):
         acc = acc.cpu().numpy()
         full = oracle.int_gemm(ox[0][rows], ow[0][cols], 0)
         np.testing.assert_array_equal(acc, full)
+
+
+# ----------------------------------------------------------------- INT8 activations (W4A8)
+# (M, N, K, k_o, int8 outliers, bias); per-token scales
+SHAPES_A8 = [
+    (16, 256, 256, 32, False, True),      # the tiny layer
+    (200, 300, 640, 64, False, True),     # ragged M, N; K_i = 576 = 4.5 k-blocks
+    (130, 520, 1056, 32, False, False),   # 2 M tiles, 3 N tiles
+    (70, 300, 544, 32, True, True),       # INT8 outliers
+    (64, 100, 256, 0, False, True),       # no outliers; N % 8 != 0
+    (64, 256, 256, 256, True, True),      # everything is outlier
+    (257, 513, 2080, 32, False, True),    # 3 x 3 tiles, long K
+    (130, 260, 8256, 64, False, True),    # 64 k-blocks
+    (33, 72, 20544, 64, True, True),      # the widest rows: sums past 2^24
+    (5, 300, 640, 64, True, True),        # a few tokens
+]
+
+
+def _case_a8(M, N, K, k_o, int8, bias, seed):
+    cfg = wl.custom_config(M, N, K, k_o, 0, int8, bias, outlier_mult=30.0,
+                           student_t=(seed % 2 == 1), act_bits=8)
+    return cfg, wl.make_layer(cfg, seed_offset=seed)
+
+
+@pytest.mark.parametrize("shape", SHAPES_A8, ids=[str(s) for s in SHAPES_A8])
+def test_a8_quantize_bit_exact(shape):
+    M, N, K, k_o, int8, bias = shape
+    cfg, d = _case_a8(*shape, seed=7)
+    gx = q.quantize_reorder(d["X"].to(DEV), d["perm"].to(DEV), k_o, 0, int8, act_bits=8)
+    torch.cuda.synchronize()
+    assert gx[0].dtype == torch.int8 and tuple(gx[0].shape) == (M, K - k_o)
+    ref = oracle.quantize_rows(np16(d["X"]), d["perm"].numpy(), k_o, 0, int8, 8)
+    assert_quant_equal(gpu_tuple_np(gx), ref, "X (INT8 codes)")
+
+
+@pytest.mark.parametrize("shape", SHAPES_A8, ids=[str(s) for s in SHAPES_A8])
+def test_a8_int32_sums_bit_exact(shape):
+    M, N, K, k_o, int8, bias = shape
+    cfg, d = _case_a8(*shape, seed=11)
+    perm_d = d["perm"].to(DEV)
+    gx = q.quantize_reorder(d["X"].to(DEV), perm_d, k_o, 0, int8, act_bits=8)
+    gw = q.pack_weights(d["W"].to(DEV), perm_d, k_o, 0, int8)
+    acc, acc_o = q.gemm_i32(gx[0], gw[0], K, k_o, 0, gx[2], gw[2])
+    torch.cuda.synchronize()
+    ox = oracle.quantize_rows(np16(d["X"]), d["perm"].numpy(), k_o, 0, int8, 8)
+    ow = oracle.quantize_rows(np16(d["W"]), d["perm"].numpy(), k_o, 0, int8, 4)
+    if K - k_o > 0:
+        np.testing.assert_array_equal(acc.cpu().numpy(), oracle.int_gemm(ox[0], ow[0], 0))
+    if int8 and k_o > 0:
+        ref_o = ox[2].astype(np.int64) @ ow[2].astype(np.int64).T
+        np.testing.assert_array_equal(acc_o.cpu().numpy(), ref_o)
+
+
+@pytest.mark.parametrize("shape", SHAPES_A8, ids=[str(s) for s in SHAPES_A8])
+def test_a8_linear_output_within_tolerance(shape):
+    M, N, K, k_o, int8, bias = shape
+    cfg, d = _case_a8(*shape, seed=13)
+    perm_d = d["perm"].to(DEV)
+    b = d["bias"].to(DEV) if d["bias"] is not None else None
+    layer = q.QuikLinear(d["W"].to(DEV), perm_d, k_o, 0, int8, b, act_bits=8)
+    Y = layer(d["X"].to(DEV))
+    gx = q.quantize_reorder(d["X"].to(DEV), perm_d, k_o, 0, int8, act_bits=8)
+    Y2 = q.gemm(gx, (layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale), K, k_o, 0, b)
+    torch.cuda.synchronize()
+    ref = oracle.layer(np16(d["X"]), np16(d["W"]), d["perm"].numpy(),
+                       None if d["bias"] is None else np16(d["bias"]), k_o, 0, int8, act_bits=8)["Y"]
+    assert_y_close(Y.float().cpu().numpy(), ref, f"W4A8 linear {shape}")
+    np.testing.assert_array_equal(Y.cpu().numpy().view(np.uint16), Y2.cpu().numpy().view(np.uint16))
+
+
+def test_a8_grouped_is_unsupported():
+    shape = q.make_shape(16, 256, 512, 0, 128, q.QUIK_OUTLIER_FP16, 8)
+    X = torch.zeros((16, 512), dtype=torch.float16, device=DEV)
+    perm = torch.arange(512, dtype=torch.int32, device=DEV)
+    Xq = torch.empty((16, 512), dtype=torch.int8, device=DEV)
+    sx = torch.empty((16, 4), dtype=torch.float32, device=DEV)
+    with pytest.raises(q.QuikError) as e:
+        q.quik_quantize_reorder(shape, X, perm, Xq, sx, None, None)
+    assert e.value.status == q.QUIK_ERR_UNSUPPORTED
