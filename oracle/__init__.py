@@ -41,10 +41,10 @@ def _load():
         lib = ctypes.CDLL(build())
         _C = ctypes.c_int
         lib.oracle_quantize_rows.argtypes = [_I, _I, _I, _I, _C, _C, _P, _P, _P, _P, _P, _P]
-        lib.oracle_int_gemm.argtypes = [_I, _I, _I, _I, _C, _P, _P, _P]
-        lib.oracle_linear.argtypes = [_I, _I, _I, _I, _I, _C, _C,
+        lib.oracle_int_gemm.argtypes = [_I, _I, _I, _I, _C, _C, _P, _P, _P]
+        lib.oracle_linear.argtypes = [_I, _I, _I, _I, _I, _C, _C, _C,
                                       _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
-        lib.oracle_linear_sampled.argtypes = [_I, _I, _I, _I, _I, _C, _C,
+        lib.oracle_linear_sampled.argtypes = [_I, _I, _I, _I, _I, _C, _C, _C,
                                               _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                               _I, _P, _P, _P, _P]
         lib.oracle_num_threads.argtypes = []
@@ -92,29 +92,30 @@ def quantize_rows(X_f16: np.ndarray, perm: np.ndarray, k_o: int, group: int = 0,
     return Q, scale, O, o_scale
 
 
-def _x_bits(Xq) -> int:
+def _x_bits(Q) -> int:
     """8 for one signed byte per code (int8 array), 4 for packed nibbles."""
-    return 8 if Xq.dtype == np.int8 else 4
+    return 8 if Q.dtype == np.int8 else 4
 
 
 def int_gemm(Xq: np.ndarray, Wq: np.ndarray, group: int = 0) -> np.ndarray:
-    """Exact INT32 sums of the codes (Xq packed INT4 uint8, or int8 codes;
-    Wq packed INT4): [M,N], or [G,M,N] with groups."""
-    xb = _x_bits(Xq)
+    """Exact INT32 sums of the codes (each operand packed INT4 uint8, or int8
+    codes): [M,N], or [G,M,N] with groups."""
+    xb, wb = _x_bits(Xq), _x_bits(Wq)
     Xq = np.ascontiguousarray(Xq.view(np.uint8))
-    Wq = np.ascontiguousarray(Wq, np.uint8)
+    Wq = np.ascontiguousarray(Wq.view(np.uint8))
     M = Xq.shape[0]
     N = Wq.shape[0]
-    Ki = 2 * Wq.shape[1]
+    Ki = Wq.shape[1] if wb == 8 else 2 * Wq.shape[1]
     G = Ki // group if group else 1
     acc = np.zeros((G, M, N), np.int32)
-    _check(_load().oracle_int_gemm(M, N, Ki, group, xb, _ptr(Xq), _ptr(Wq), _ptr(acc)), "int_gemm")
+    _check(_load().oracle_int_gemm(M, N, Ki, group, xb, wb, _ptr(Xq), _ptr(Wq), _ptr(acc)),
+           "int_gemm")
     return acc if group else acc[0]
 
 
 def _linear_args(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias):
     c = np.ascontiguousarray
-    Xq, Wq = c(Xq.view(np.uint8)), c(Wq, np.uint8)
+    Xq, Wq = c(Xq.view(np.uint8)), c(Wq.view(np.uint8))
     sx, sw = c(sx, np.float32), c(sw, np.float32)
     int8 = Xo is not None and Xo.dtype == np.int8
     if Xo is not None:
@@ -128,11 +129,11 @@ def _linear_args(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias):
 
 def linear(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias, K: int, k_o: int, group: int = 0):
     """fp64 Y [M,N] of the layer from quantised operands (no fp16 rounding)."""
-    xb = _x_bits(Xq)
+    xb, wb = _x_bits(Xq), _x_bits(Wq)
     Xq, sx, Xo, sxo, Wq, sw, Wo, swo, b, int8 = _linear_args(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias)
     M, N = Xq.shape[0], Wq.shape[0]
     Y = np.zeros((M, N), np.float64)
-    rc = _load().oracle_linear(M, N, K, k_o, group, int(int8), xb, _ptr(Xq), _ptr(sx), _ptr(Xo),
+    rc = _load().oracle_linear(M, N, K, k_o, group, int(int8), xb, wb, _ptr(Xq), _ptr(sx), _ptr(Xo),
                                _ptr(sxo), _ptr(Wq), _ptr(sw), _ptr(Wo), _ptr(swo), _ptr(b), _ptr(Y))
     _check(rc, "linear")
     return Y
@@ -141,7 +142,7 @@ def linear(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias, K: int, k_o: int, group: int 
 def linear_sampled(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias, K: int, k_o: int, group: int,
                    ms: np.ndarray, ns: np.ndarray):
     """fp64 Y at the (ms[i], ns[i]) positions plus their integer sums [count, G]."""
-    xb = _x_bits(Xq)
+    xb, wb = _x_bits(Xq), _x_bits(Wq)
     Xq, sx, Xo, sxo, Wq, sw, Wo, swo, b, int8 = _linear_args(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias)
     M, N = Xq.shape[0], Wq.shape[0]
     ms = np.ascontiguousarray(ms, np.int64)
@@ -149,7 +150,7 @@ def linear_sampled(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias, K: int, k_o: int, gro
     G = (K - k_o) // group if group else 1
     Y = np.zeros(len(ms), np.float64)
     acc = np.zeros((len(ms), max(G, 1)), np.int32)
-    rc = _load().oracle_linear_sampled(M, N, K, k_o, group, int(int8), xb, _ptr(Xq), _ptr(sx),
+    rc = _load().oracle_linear_sampled(M, N, K, k_o, group, int(int8), xb, wb, _ptr(Xq), _ptr(sx),
                                        _ptr(Xo), _ptr(sxo), _ptr(Wq), _ptr(sw), _ptr(Wo),
                                        _ptr(swo), _ptr(b), len(ms), _ptr(ms), _ptr(ns),
                                        _ptr(Y), _ptr(acc))
@@ -158,15 +159,15 @@ def linear_sampled(Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias, K: int, k_o: int, gro
 
 
 def layer(X_f16, W_f16, perm, bias, k_o: int, group: int = 0, outlier_int8: bool = False,
-          act_bits: int = 4):
-    """The whole layer from fp16 inputs: quantise X (INT4, or INT8 when
-    act_bits == 8) and W (INT4), then the fp64 output.
+          act_bits: int = 4, weight_bits: int = 4):
+    """The whole layer from fp16 inputs: quantise X and W (INT4, or INT8 when
+    act_bits / weight_bits == 8), then the fp64 output.
 
     Returns a dict with every intermediate (codes, scales, outlier blocks, Y).
     """
     K = X_f16.shape[1]
     Xq, sx, Xo, sxo = quantize_rows(X_f16, perm, k_o, group, outlier_int8, act_bits)
-    Wq, sw, Wo, swo = quantize_rows(W_f16, perm, k_o, group, outlier_int8)
+    Wq, sw, Wo, swo = quantize_rows(W_f16, perm, k_o, group, outlier_int8, weight_bits)
     Y = linear(Xq, sx, Xo if k_o else None, sxo, Wq, sw, Wo if k_o else None, swo, bias,
                K, k_o, group)
     return dict(Xq=Xq, sx=sx, Xo=Xo, sxo=sxo, Wq=Wq, sw=sw, Wo=Wo, swo=swo, Y=Y)

@@ -31,6 +31,8 @@
  *    fixes no quantiser.  Reading: the INT8 rule above (divisor and clamp
  *    127) applied per token to the non-outlier positions, one byte per code
  *    in reordered order.
+ *  - 8-bit weights (W8A8, the baseline the same abstracts compare against):
+ *    the same INT8 rule per output channel.
  *  - packing: byte i of a row holds code 2i in the low nibble and code 2i+1
  *    in the high nibble, both 4-bit two's complement.
  *  - integer dot products in int64 (checked to fit int32); dequantisation,
@@ -193,16 +195,17 @@ int oracle_quantize_rows(int64_t R, int64_t K, int64_t k_o, int64_t group, int o
 }
 
 /*
- * oracle_int_gemm -- exact integer product of the quantised codes (W packed
- * INT4; X packed INT4, or one byte per code when x_bits == 8).
+ * oracle_int_gemm -- exact integer product of the quantised codes (each of X
+ * and W packed INT4, or one byte per code when its bits == 8).
  *  acc[m, n]           = sum_{j < Ki} qx[m, j] * qw[n, j]            (group == 0)
  *  acc[g, m, n]        = sum_{j in group g} qx[m, j] * qw[n, j]      (group > 0)
  * Sums are taken in int64 and must fit int32.
  */
-int oracle_int_gemm(int64_t M, int64_t N, int64_t Ki, int64_t group, int x_bits,
+int oracle_int_gemm(int64_t M, int64_t N, int64_t Ki, int64_t group, int x_bits, int w_bits,
                     const uint8_t *Xq, const uint8_t *Wq, int32_t *acc)
 {
     if (M < 0 || N < 0 || Ki < 0 || Ki % 2 || (x_bits != 4 && x_bits != 8)) return ORACLE_EBADARG;
+    if (w_bits != 4 && w_bits != 8) return ORACLE_EBADARG;
     if (group < 0 || (group > 0 && Ki % group)) return ORACLE_EBADARG;
     const int64_t gs = group > 0 ? group : Ki;
     const int64_t G = group > 0 ? Ki / group : 1;
@@ -213,7 +216,7 @@ int oracle_int_gemm(int64_t M, int64_t N, int64_t Ki, int64_t group, int x_bits,
             for (int64_t g = 0; g < G; ++g) {
                 int64_t sum = 0;
                 for (int64_t j = g * gs; j < (g + 1) * gs; ++j)
-                    sum += (int64_t)code_at(Xq, m, j, Ki, x_bits) * (int64_t)code_at(Wq, n, j, Ki, 4);
+                    sum += (int64_t)code_at(Xq, m, j, Ki, x_bits) * (int64_t)code_at(Wq, n, j, Ki, w_bits);
                 if (sum > INT32_MAX || sum < INT32_MIN) {
 #pragma omp atomic write
                     err = ORACLE_EOVERFLOW;
@@ -228,7 +231,7 @@ int oracle_int_gemm(int64_t M, int64_t N, int64_t Ki, int64_t group, int x_bits,
 /* One output element of the layer, in fp64, from quantised operands.
  * Y = sum_g A_g * sx[m,g] * sw[n,g]  +  O  +  bias[n]                  */
 static double linear_element(int64_t m, int64_t n, int64_t M, int64_t N, int64_t K, int64_t k_o,
-                             int64_t group, int outlier_int8, int x_bits,
+                             int64_t group, int outlier_int8, int x_bits, int w_bits,
                              const uint8_t *Xq, const float *sx, const void *Xo, const float *sxo,
                              const uint8_t *Wq, const float *sw, const void *Wo, const float *swo,
                              const uint16_t *bias, int32_t *acc_out, int *overflow)
@@ -243,7 +246,7 @@ static double linear_element(int64_t m, int64_t n, int64_t M, int64_t N, int64_t
     for (int64_t g = 0; g < G; ++g) {
         int64_t sum = 0;
         for (int64_t j = g * gs; j < (g + 1) * gs; ++j)
-            sum += (int64_t)code_at(Xq, m, j, Ki, x_bits) * (int64_t)code_at(Wq, n, j, Ki, 4);
+            sum += (int64_t)code_at(Xq, m, j, Ki, x_bits) * (int64_t)code_at(Wq, n, j, Ki, w_bits);
         if (sum > INT32_MAX || sum < INT32_MIN) *overflow = 1;
         if (acc_out) acc_out[g] = (int32_t)sum;
         if (Ki > 0)
@@ -273,24 +276,24 @@ static double linear_element(int64_t m, int64_t n, int64_t M, int64_t N, int64_t
 
 /*
  * oracle_linear -- the full fp64 output Y [M, N] from quantised operands.
- * Xq holds packed INT4 (x_bits 4) or one byte per code (x_bits 8); Wq packed
- * INT4.  Xo/Wo are fp16 [*, k_o] (outlier_int8 == 0) or int8 [*, k_o] with
+ * Xq and Wq hold packed INT4 (bits 4) or one byte per code (bits 8).  Xo/Wo are fp16 [*, k_o] (outlier_int8 == 0) or int8 [*, k_o] with
  * sxo [M] / swo [N] (outlier_int8 == 1).  bias is fp16 [N] or NULL.
  */
 int oracle_linear(int64_t M, int64_t N, int64_t K, int64_t k_o, int64_t group, int outlier_int8,
-                  int x_bits,
+                  int x_bits, int w_bits,
                   const uint8_t *Xq, const float *sx, const void *Xo, const float *sxo,
                   const uint8_t *Wq, const float *sw, const void *Wo, const float *swo,
                   const uint16_t *bias, double *Y)
 {
     if (M < 0 || N < 0 || K < 0 || k_o < 0 || k_o > K || (K - k_o) % 2) return ORACLE_EBADARG;
     if (group < 0 || (group > 0 && (K - k_o) % group)) return ORACLE_EBADARG;
-    if (x_bits != 4 && x_bits != 8) return ORACLE_EBADARG;
+    if ((x_bits != 4 && x_bits != 8) || (w_bits != 4 && w_bits != 8)) return ORACLE_EBADARG;
     int overflow = 0;
 #pragma omp parallel for schedule(static) reduction(| : overflow)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n)
-            Y[m * N + n] = linear_element(m, n, M, N, K, k_o, group, outlier_int8, x_bits, Xq, sx, Xo,
+            Y[m * N + n] = linear_element(m, n, M, N, K, k_o, group, outlier_int8, x_bits, w_bits,
+                                          Xq, sx, Xo,
                                           sxo, Wq, sw, Wo, swo, bias, NULL, &overflow);
     return overflow ? ORACLE_EOVERFLOW : ORACLE_OK;
 }
@@ -302,7 +305,7 @@ int oracle_linear(int64_t M, int64_t N, int64_t K, int64_t k_o, int64_t group, i
  * ([count, G], G = 1 without groups).
  */
 int oracle_linear_sampled(int64_t M, int64_t N, int64_t K, int64_t k_o, int64_t group,
-                          int outlier_int8, int x_bits,
+                          int outlier_int8, int x_bits, int w_bits,
                           const uint8_t *Xq, const float *sx, const void *Xo, const float *sxo,
                           const uint8_t *Wq, const float *sw, const void *Wo, const float *swo,
                           const uint16_t *bias, int64_t count, const int64_t *ms,
@@ -310,14 +313,15 @@ int oracle_linear_sampled(int64_t M, int64_t N, int64_t K, int64_t k_o, int64_t 
 {
     if (M < 0 || N < 0 || K < 0 || k_o < 0 || k_o > K || (K - k_o) % 2) return ORACLE_EBADARG;
     if (group < 0 || (group > 0 && (K - k_o) % group)) return ORACLE_EBADARG;
-    if (x_bits != 4 && x_bits != 8) return ORACLE_EBADARG;
+    if ((x_bits != 4 && x_bits != 8) || (w_bits != 4 && w_bits != 8)) return ORACLE_EBADARG;
     const int64_t G = group > 0 ? (K - k_o) / group : 1;
     for (int64_t i = 0; i < count; ++i)
         if (ms[i] < 0 || ms[i] >= M || ns[i] < 0 || ns[i] >= N) return ORACLE_EBADARG;
     int overflow = 0;
 #pragma omp parallel for schedule(static) reduction(| : overflow)
     for (int64_t i = 0; i < count; ++i)
-        Y[i] = linear_element(ms[i], ns[i], M, N, K, k_o, group, outlier_int8, x_bits, Xq, sx, Xo, sxo,
+        Y[i] = linear_element(ms[i], ns[i], M, N, K, k_o, group, outlier_int8, x_bits, w_bits,
+                              Xq, sx, Xo, sxo,
                               Wq, sw, Wo, swo, bias, acc ? acc + i * G : NULL, &overflow);
     return overflow ? ORACLE_EOVERFLOW : ORACLE_OK;
 }

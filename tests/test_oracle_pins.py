@@ -431,3 +431,44 @@ def test_a8_int_gemm_equals_int64_matmul(oracle_mod):
     np.testing.assert_array_equal(a[:, 0], acc[ms, ns])
     np.testing.assert_allclose(Y, acc[ms, ns] * sx[ms].astype(np.float64) * sw[ns].astype(np.float64),
                                rtol=1e-15, atol=0)
+
+
+# ----------------------------------------------------------------- 8-bit weights too (W8A8)
+@pytest.mark.parametrize("M,N,K,k_o,int8", [
+    (5, 6, 96, 32, False),
+    (4, 5, 160, 32, True),
+])
+def test_w8a8_lossless_equals_fp64_matmul(oracle_mod, M, N, K, k_o, int8):
+    rng = np.random.default_rng(M * 57 + K)
+    Ki = K - k_o
+    perm = rng.permutation(K).astype(np.int32)
+    cx, sx_true, vx = lossless_rows8(rng, M, Ki)
+    cw, sw_true, vw = lossless_rows8(rng, N, Ki)
+    X = np.zeros((M, K)); W = np.zeros((N, K))
+    X[:, perm[:Ki]] = vx
+    W[:, perm[:Ki]] = vw
+    if int8:
+        _, _, vxo = lossless_rows8(rng, M, k_o)
+        _, _, vwo = lossless_rows8(rng, N, k_o)
+    else:
+        vxo = rng.standard_normal((M, k_o)) * 40
+        vwo = rng.standard_normal((N, k_o)) * 0.05
+    X[:, perm[Ki:]] = vxo
+    W[:, perm[Ki:]] = vwo
+    X16, W16 = X.astype(np.float16), W.astype(np.float16)
+    bias = (rng.standard_normal(N) * 0.01).astype(np.float16)
+    r = oracle_mod.layer(X16, W16, perm, bias, k_o, 0, int8, act_bits=8, weight_bits=8)
+    np.testing.assert_array_equal(r["Xq"].astype(np.int64), cx)
+    np.testing.assert_array_equal(r["Wq"].astype(np.int64), cw)
+    np.testing.assert_array_equal(r["sw"], sw_true[:, 0].astype(np.float32))
+    ref = _fp64_ref(X16, W16, bias)
+    np.testing.assert_allclose(r["Y"], ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_w8a8_int_gemm_equals_int64_matmul(oracle_mod):
+    rng = np.random.default_rng(23)
+    M, N, Ki = 7, 9, 160
+    Xq = rng.integers(-127, 128, size=(M, Ki)).astype(np.int8)
+    Wq = rng.integers(-127, 128, size=(N, Ki)).astype(np.int8)
+    np.testing.assert_array_equal(oracle_mod.int_gemm(Xq, Wq, 0),
+                                  Xq.astype(np.int64) @ Wq.astype(np.int64).T)
