@@ -89,8 +89,9 @@ def gemm_kernel(cfg):
     """The GEMM kernel the library dispatches for this layer, and its profile file."""
     fits = cfg.k_o <= (256 if cfg.outlier_int8 else 128)
     if cfg.act_bits == 8:
-        return ("w4a4_gemm_pair with INT8 activations (W4A8; weights widened from INT4, "
-                "tcgen05 kind::i8 on CTA pairs)", f"w4a4_gemm_{cfg.name}.md")
+        return (("w4a4_gemm_pair with INT8 activations and weights (W8A8)" if cfg.weight_bits == 8 else
+                 "w4a4_gemm_pair with INT8 activations (W4A8; weights widened from INT4)")
+                + ", tcgen05 kind::i8 on CTA pairs", f"w4a4_gemm_{cfg.name}.md")
     if cfg.group == 0 and cfg.M <= 32 and fits:
         return ("w4a4_gemv (decode shapes: W rows as the MMA's M, tokens as N; INT4 codes "
                 "widened to INT8, tcgen05 kind::i8)", f"w4a4_gemv_{cfg.name}.md")
@@ -225,7 +226,7 @@ def prepare_cpu_inputs(cfg, d):
     d["perm_np"] = d["perm"].numpy()
     d["bias_np"] = None if d["bias"] is None else d["bias"].numpy()
     d["w_oracle"] = oracle.quantize_rows(d["W"].numpy(), d["perm_np"], cfg.k_o, cfg.group,
-                                         cfg.outlier_int8)
+                                         cfg.outlier_int8, cfg.weight_bits)
 
 
 def cpu_baseline(cfg, d, budget_s: float = 10.0):
@@ -290,7 +291,7 @@ def run_ours(args, rank, local_rank, world):
     perm = d["perm"].to(dev)
     bias = d["bias"].to(dev) if d["bias"] is not None else None
     layer = q.QuikLinear(d["W"].to(dev), perm, cfg.k_o, cfg.group, cfg.outlier_int8, bias,
-                         act_bits=cfg.act_bits)
+                         act_bits=cfg.act_bits, weight_bits=cfg.weight_bits)
     shape = layer.shape(cfg.M)
     Xq, sx, Xo, sxo = q._binding._quant_outputs(cfg.M, cfg.K, cfg.k_o, cfg.group,
                                                 cfg.outlier_int8, dev, cfg.act_bits)
@@ -426,7 +427,8 @@ def run_ours(args, rank, local_rank, world):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "int4" if cfg.act_bits == 4 else "int4 weights x int8 activations",
+        "dtype": ("int4" if cfg.act_bits == 4 else
+                  "int8" if cfg.weight_bits == 8 else "int4 weights x int8 activations"),
         "data": "synthetic",
         "config": {
             "workload": name, "M": cfg.M, "N": cfg.N, "K": cfg.K, "k_o": cfg.k_o,

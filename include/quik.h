@@ -29,6 +29,10 @@
  * s = max|v| / 127 per token and q = clamp(rint(v / s), -127, 127); Xq is then
  * int8 [M, K_i] row-major, one byte per code in reordered order.  Weights stay
  * packed INT4.  Per-token scales only (group_size 0).
+ *
+ * 8-bit weights (W8A8, the INT8 baseline the same pages compare with),
+ * selected by quik_shape.weight_bits == 8 together with act_bits == 8: the
+ * weights take the same INT8 rule per output channel and Wq is int8 [N, K_i].
 
  *
  * Conventions for every entry point:
@@ -39,9 +43,10 @@
  *   - Every function returns a quik_status; nothing throws across the ABI.
  *   - Arguments are validated before any launch: non-NULL pointers that are
  *     16-byte aligned, M, N >= 1, 0 <= k_o <= K, K_i % 32 == 0, k_o % 16 == 0,
- *     K <= 32768, group_size 0 or 128 (then K_i % 128 == 0), act_bits 0, 4 or
- *     8.  Any violation returns QUIK_ERR_INVALID_ARG with nothing enqueued;
- *     act_bits 8 with group_size 128 returns QUIK_ERR_UNSUPPORTED.  Pointers that are
+ *     K <= 32768, group_size 0 or 128 (then K_i % 128 == 0), act_bits and
+ *     weight_bits 0, 4 or 8.  Any violation returns QUIK_ERR_INVALID_ARG with
+ *     nothing enqueued; act_bits 8 with group_size 128, and weight_bits 8
+ *     without act_bits 8, return QUIK_ERR_UNSUPPORTED.  Pointers that are
  *     unused for the shape (outlier buffers when k_o == 0, INT8 scales in FP16
  *     mode, bias) may be NULL.
  *   - perm must be a permutation of 0..K-1.  Entries outside [0, K) are
@@ -92,6 +97,7 @@ typedef struct {
     int32_t group_size; /* 0: per-token / per-channel scales; 128: per group */
     int32_t outlier;    /* a quik_outlier_t */
     int32_t act_bits;   /* activation codes: 0 or 4 -> INT4 (W4A4); 8 -> INT8 (W4A8) */
+    int32_t weight_bits; /* weight codes: 0 or 4 -> INT4; 8 -> INT8 (W8A8, needs act_bits 8) */
 } quik_shape;
 
 /* Opaque cudaStream_t. */
@@ -125,8 +131,8 @@ QUIK_API quik_status quik_quantize_reorder(const quik_shape *shape, const void *
  * quik_pack_weights -- offline weight preparation (QUIK sample names
  * pack_to_i4 / two_compl; Atom idea I1): the same reorder + symmetric
  * quantiser applied to the rows of W (one scale per output channel, or per
- * channel and group), round-to-nearest codes.  Always INT4, whatever
- * act_bits.
+ * channel and group), round-to-nearest codes.  INT4 (Wq [N, K_i/2]), or INT8
+ * (Wq int8 [N, K_i]) when weight_bits == 8.
  *   W_f16 [N, K] fp16; Wq out [N, K_i/2]; w_scale out [N] or [N, G];
  *   Wo out [N, k_o] fp16 or int8; wo_scale out [N] (INT8 outliers only).
  */

@@ -35,7 +35,8 @@ class QuikError(RuntimeError):
 class quik_shape(ctypes.Structure):
     _fields_ = [("M", ctypes.c_int32), ("N", ctypes.c_int32), ("K", ctypes.c_int32),
                 ("k_o", ctypes.c_int32), ("group_size", ctypes.c_int32),
-                ("outlier", ctypes.c_int32), ("act_bits", ctypes.c_int32)]
+                ("outlier", ctypes.c_int32), ("act_bits", ctypes.c_int32),
+                ("weight_bits", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p
@@ -87,8 +88,9 @@ def _check(status: int, what: str):
 
 
 def make_shape(M: int, N: int, K: int, k_o: int, group_size: int = 0,
-               outlier: int = QUIK_OUTLIER_FP16, act_bits: int = 4) -> quik_shape:
-    return quik_shape(M, N, K, k_o, group_size, outlier, act_bits)
+               outlier: int = QUIK_OUTLIER_FP16, act_bits: int = 4,
+               weight_bits: int = 4) -> quik_shape:
+    return quik_shape(M, N, K, k_o, group_size, outlier, act_bits, weight_bits)
 
 
 def _ptr(t, dtype=None, what="tensor"):
@@ -108,6 +110,11 @@ def _ptr(t, dtype=None, what="tensor"):
 def _xq_dtype(shape: quik_shape):
     """Quantised activations: packed INT4 bytes, or INT8 codes when act_bits == 8."""
     return torch.int8 if shape.act_bits == 8 else torch.uint8
+
+
+def _wq_dtype(shape: quik_shape):
+    """Packed weights: INT4 bytes, or INT8 codes when weight_bits == 8."""
+    return torch.int8 if shape.weight_bits == 8 else torch.uint8
 
 
 def _stream(stream=None) -> int:
@@ -130,7 +137,7 @@ def quik_quantize_reorder(shape, X, perm, Xq, x_scale, Xo, xo_scale, stream=None
 def quik_pack_weights(shape, W, perm, Wq, w_scale, Wo, wo_scale, stream=None):
     _check(lib().quik_pack_weights(
         ctypes.byref(shape), _ptr(W, torch.float16, "W"), _ptr(perm, torch.int32, "perm"),
-        _ptr(Wq, torch.uint8, "Wq"), _ptr(w_scale, torch.float32, "w_scale"), _ptr(Wo, None, "Wo"),
+        _ptr(Wq, _wq_dtype(shape), "Wq"), _ptr(w_scale, torch.float32, "w_scale"), _ptr(Wo, None, "Wo"),
         _ptr(wo_scale, torch.float32, "wo_scale"), _stream(stream)), "quik_pack_weights")
 
 
@@ -138,7 +145,7 @@ def quik_gemm(shape, Xq, x_scale, Xo, xo_scale, Wq, w_scale, Wo, wo_scale, bias,
     _check(lib().quik_gemm(
         ctypes.byref(shape), _ptr(Xq, _xq_dtype(shape), "Xq"), _ptr(x_scale, torch.float32, "x_scale"),
         _ptr(Xo, None, "Xo"), _ptr(xo_scale, torch.float32, "xo_scale"),
-        _ptr(Wq, torch.uint8, "Wq"), _ptr(w_scale, torch.float32, "w_scale"),
+        _ptr(Wq, _wq_dtype(shape), "Wq"), _ptr(w_scale, torch.float32, "w_scale"),
         _ptr(Wo, None, "Wo"), _ptr(wo_scale, torch.float32, "wo_scale"),
         _ptr(bias, torch.float16, "bias"), _ptr(Y, torch.float16, "Y"), _stream(stream)), "quik_gemm")
 
@@ -146,7 +153,7 @@ def quik_gemm(shape, Xq, x_scale, Xo, xo_scale, Wq, w_scale, Wo, wo_scale, bias,
 def quik_linear(shape, X, perm, Wq, w_scale, Wo, wo_scale, bias, Y, workspace, stream=None):
     _check(lib().quik_linear(
         ctypes.byref(shape), _ptr(X, torch.float16, "X"), _ptr(perm, torch.int32, "perm"),
-        _ptr(Wq, torch.uint8, "Wq"), _ptr(w_scale, torch.float32, "w_scale"),
+        _ptr(Wq, _wq_dtype(shape), "Wq"), _ptr(w_scale, torch.float32, "w_scale"),
         _ptr(Wo, None, "Wo"), _ptr(wo_scale, torch.float32, "wo_scale"),
         _ptr(bias, torch.float16, "bias"), _ptr(Y, torch.float16, "Y"),
         _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)), "quik_linear")
@@ -157,7 +164,7 @@ def quik_linear_noalloc(shape, X, perm, Wq, w_scale, Wo, wo_scale, bias, Y, stre
     allocate device memory); see include/quik.h."""
     _check(lib().quik_linear_noalloc(
         ctypes.byref(shape), _ptr(X, torch.float16, "X"), _ptr(perm, torch.int32, "perm"),
-        _ptr(Wq, torch.uint8, "Wq"), _ptr(w_scale, torch.float32, "w_scale"),
+        _ptr(Wq, _wq_dtype(shape), "Wq"), _ptr(w_scale, torch.float32, "w_scale"),
         _ptr(Wo, None, "Wo"), _ptr(wo_scale, torch.float32, "wo_scale"),
         _ptr(bias, torch.float16, "bias"), _ptr(Y, torch.float16, "Y"), _stream(stream)),
         "quik_linear_noalloc")
@@ -165,7 +172,7 @@ def quik_linear_noalloc(shape, X, perm, Wq, w_scale, Wo, wo_scale, bias, Y, stre
 
 def quik_gemm_i32_debug(shape, Xq, Wq, Xo, Wo, acc, acc_outlier, stream=None):
     _check(lib().quik_gemm_i32_debug(
-        ctypes.byref(shape), _ptr(Xq, _xq_dtype(shape), "Xq"), _ptr(Wq, torch.uint8, "Wq"),
+        ctypes.byref(shape), _ptr(Xq, _xq_dtype(shape), "Xq"), _ptr(Wq, _wq_dtype(shape), "Wq"),
         _ptr(Xo, None, "Xo"), _ptr(Wo, None, "Wo"), _ptr(acc, torch.int32, "acc"),
         _ptr(acc_outlier, torch.int32, "acc_outlier"), _stream(stream)), "quik_gemm_i32_debug")
 
@@ -210,11 +217,13 @@ def quantize_reorder(X: torch.Tensor, perm: torch.Tensor, k_o: int, group: int =
 
 
 def pack_weights(W: torch.Tensor, perm: torch.Tensor, k_o: int, group: int = 0,
-                 outlier_int8: bool = False, stream=None):
-    """Weights -> (Wq, w_scale, Wo, wo_scale), allocated on W's device."""
+                 outlier_int8: bool = False, stream=None, weight_bits: int = 4):
+    """Weights -> (Wq, w_scale, Wo, wo_scale), allocated on W's device.
+    Wq is packed INT4 (uint8 [N, K_i/2]), or int8 [N, K_i] when weight_bits == 8."""
     N, K = W.shape
-    shape = make_shape(1, N, K, k_o, group, _outlier_kind(outlier_int8))
-    out = _quant_outputs(N, K, k_o, group, outlier_int8, W.device)
+    shape = make_shape(1, N, K, k_o, group, _outlier_kind(outlier_int8),
+                       8 if weight_bits == 8 else 4, weight_bits)
+    out = _quant_outputs(N, K, k_o, group, outlier_int8, W.device, weight_bits)
     quik_pack_weights(shape, W, perm, *out, stream=stream)
     return out
 
@@ -225,7 +234,8 @@ def gemm(xq, wq, K: int, k_o: int, group: int = 0, bias=None, stream=None):
     Wq, sw, Wo, swo = wq
     M, N = sx.shape[0], sw.shape[0]
     int8 = Xo.dtype == torch.int8
-    shape = make_shape(M, N, K, k_o, group, _outlier_kind(int8), 8 if Xq.dtype == torch.int8 else 4)
+    shape = make_shape(M, N, K, k_o, group, _outlier_kind(int8), 8 if Xq.dtype == torch.int8 else 4,
+                       8 if Wq.dtype == torch.int8 else 4)
     Y = torch.empty((M, N), dtype=torch.float16, device=sx.device)
     quik_gemm(shape, Xq, sx, Xo, sxo, Wq, sw, Wo, swo, bias, Y, stream=stream)
     return Y
@@ -237,7 +247,8 @@ def gemm_i32(Xq, Wq, K: int, k_o: int, group: int = 0, Xo=None, Wo=None, stream=
     Ki = K - k_o
     G = Ki // group if group else 1
     int8 = Xo is not None and Xo.dtype == torch.int8
-    shape = make_shape(M, N, K, k_o, group, _outlier_kind(int8), 8 if Xq.dtype == torch.int8 else 4)
+    shape = make_shape(M, N, K, k_o, group, _outlier_kind(int8), 8 if Xq.dtype == torch.int8 else 4,
+                       8 if Wq.dtype == torch.int8 else 4)
     acc = torch.empty((G, M, N) if group else (M, N), dtype=torch.int32, device=Xq.device)
     acc_o = torch.empty((M, N), dtype=torch.int32, device=Xq.device) if int8 and k_o else None
     quik_gemm_i32_debug(shape, Xq, Wq, Xo if int8 else None, Wo if int8 else None, acc, acc_o,
@@ -246,26 +257,29 @@ def gemm_i32(Xq, Wq, K: int, k_o: int, group: int = 0, Xo=None, Wo=None, stream=
 
 
 class QuikLinear:
-    """A hybrid W4A4 (or W4A8) + outlier linear layer with packed weights resident on the GPU.
+    """A hybrid W4A4 (or W4A8, W8A8) + outlier linear layer with packed weights on the GPU.
 
-    ``QuikLinear(W, perm, k_o, group, outlier_int8, bias, act_bits)`` packs W
-    once (quik_pack_weights); calling it on fp16 activations runs quik_linear
-    into a workspace it keeps.  act_bits 8 quantises the activations to INT8.
+    ``QuikLinear(W, perm, k_o, group, outlier_int8, bias, act_bits, weight_bits)``
+    packs W once (quik_pack_weights); calling it on fp16 activations runs
+    quik_linear into a workspace it keeps.  act_bits / weight_bits 8 quantise
+    the activations / weights to INT8.
     """
 
     def __init__(self, W: torch.Tensor, perm: torch.Tensor, k_o: int, group: int = 0,
-                 outlier_int8: bool = False, bias: torch.Tensor | None = None, act_bits: int = 4):
+                 outlier_int8: bool = False, bias: torch.Tensor | None = None, act_bits: int = 4,
+                 weight_bits: int = 4):
         self.N, self.K = W.shape
         self.k_o, self.group, self.outlier_int8 = k_o, group, outlier_int8
-        self.act_bits = act_bits
+        self.act_bits, self.weight_bits = act_bits, weight_bits
         self.perm = perm
         self.bias = bias
-        self.Wq, self.w_scale, self.Wo, self.wo_scale = pack_weights(W, perm, k_o, group, outlier_int8)
+        self.Wq, self.w_scale, self.Wo, self.wo_scale = pack_weights(W, perm, k_o, group, outlier_int8,
+                                                                     weight_bits=weight_bits)
         self._ws = None
 
     def shape(self, M: int) -> quik_shape:
         return make_shape(M, self.N, self.K, self.k_o, self.group, _outlier_kind(self.outlier_int8),
-                          self.act_bits)
+                          self.act_bits, self.weight_bits)
 
     def workspace(self, M: int, device) -> torch.Tensor:
         need = quik_workspace_size(self.shape(M))

@@ -27,7 +27,9 @@ quik_status check_shape(const quik_shape *s) {
     if (s->outlier != QUIK_OUTLIER_FP16 && s->outlier != QUIK_OUTLIER_INT8)
         return QUIK_ERR_INVALID_ARG;
     if (s->act_bits != 0 && s->act_bits != 4 && s->act_bits != 8) return QUIK_ERR_INVALID_ARG;
+    if (s->weight_bits != 0 && s->weight_bits != 4 && s->weight_bits != 8) return QUIK_ERR_INVALID_ARG;
     if (s->act_bits == 8 && s->group_size != 0) return QUIK_ERR_UNSUPPORTED;
+    if (s->weight_bits == 8 && s->act_bits != 8) return QUIK_ERR_UNSUPPORTED;
     return QUIK_OK;
 }
 
@@ -38,6 +40,7 @@ inline int groups_of(const quik_shape *s) {
 inline bool needs_scale(const quik_shape *s) { return groups_of(s) > 0; }
 inline bool int8_out(const quik_shape *s) { return s->outlier == QUIK_OUTLIER_INT8; }
 inline bool act8(const quik_shape *s) { return s->act_bits == 8; }
+inline bool wt8(const quik_shape *s) { return s->weight_bits == 8; }
 
 // Rows of one operand: packed codes, scales, outlier block (+ INT8 scales).
 quik_status check_quant_ptrs(const quik_shape *s, const void *Q, const float *scale,
@@ -51,7 +54,7 @@ quik_status check_quant_ptrs(const quik_shape *s, const void *Q, const float *sc
     return QUIK_OK;
 }
 
-// bits8: INT8 codes (activations of a W4A8 shape); weights are always INT4.
+// bits8: INT8 codes (activations with act_bits 8, weights with weight_bits 8).
 quik_status quantize(const quik_shape *s, int rows, bool bits8, const void *X, const int32_t *perm,
                      void *Q, float *scale, void *O, float *o_scale, cudaStream_t stream) {
     quik::QuantizeArgs a;
@@ -114,7 +117,7 @@ quik_status quik_pack_weights(const quik_shape *shape, const void *W_f16, const 
     if (st != QUIK_OK) return st;
     if (!ok_ptr(W_f16) || !ok_ptr(perm)) return QUIK_ERR_INVALID_ARG;
     if ((st = check_quant_ptrs(shape, Wq, w_scale, Wo, wo_scale)) != QUIK_OK) return st;
-    return quantize(shape, shape->N, false, W_f16, perm, Wq, w_scale, Wo, wo_scale,
+    return quantize(shape, shape->N, wt8(shape), W_f16, perm, Wq, w_scale, Wo, wo_scale,
                     static_cast<cudaStream_t>(stream));
 }
 
@@ -131,6 +134,7 @@ static quik_status gemm_impl(const quik_shape *shape, const void *Xq, const floa
     a.group = shape->group_size;
     a.out_int8 = int8_out(shape);
     a.a8 = act8(shape);
+    a.w8 = wt8(shape);
     a.Xq = Xq;
     a.sx = x_scale;
     a.Xo = Xo;

@@ -154,17 +154,17 @@ __device__ __forceinline__ float small_int_to_float(int32_t v) {
     return __int_as_float(v + 0x4B400000) - 12582912.0f;
 }
 
-// The INT4-part sum from the tensor-core accumulator.  INT4 activations: both
-// operands carry a factor 16 (sum 256 A, |A| <= 49 K_i < 2^22: exact by the
-// magic-number add).  INT8 activations (W4A8): only the weights do (sum 16 A,
-// |A| <= 889 K_i, which can pass 2^22: a rounding conversion, exact below 2^24).
-template <bool A8>
+// The integer sum A from the tensor-core accumulator.  INT4 codes enter the
+// MMA as 16 c, so the accumulator holds 256 A (W4A4: |A| <= 49 K_i < 2^22,
+// exact by the magic-number add), 16 A (W4A8) or A (W8A8).  With INT8
+// activations |A| can pass 2^22: a rounding conversion, exact below 2^24.
+template <bool A8, bool W8>
 __device__ __forceinline__ int32_t acc_int(uint32_t raw) {
-    return static_cast<int32_t>(raw) >> (A8 ? 4 : 8);
+    return static_cast<int32_t>(raw) >> (W8 ? 0 : A8 ? 4 : 8);
 }
-template <bool A8>
+template <bool A8, bool W8>
 __device__ __forceinline__ float acc_float(uint32_t raw) {
-    return A8 ? __int2float_rn(acc_int<A8>(raw)) : small_int_to_float(acc_int<A8>(raw));
+    return A8 ? __int2float_rn(acc_int<A8, W8>(raw)) : small_int_to_float(acc_int<A8, W8>(raw));
 }
 
 // W4A8: 32 INT8 codes (two 16-byte chunks, codes in order) in the order the
@@ -654,7 +654,7 @@ static_assert(A_COL + 32 * S <= TMEM_COLS, "A stages fit in tensor memory");
 static_assert(SMEM <= 232448, "shared memory budget");
 }  // namespace pair
 
-template <bool OUT_INT8, bool DEBUG, bool A8>
+template <bool OUT_INT8, bool DEBUG, bool A8, bool W8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
     w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_wq,
                           const __grid_constant__ CUtensorMap tm_wo,
@@ -771,9 +771,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
                 if (!wait_bar(&pk_empty[st], ((u / SP) & 1) ^ 1, ab)) break;
                 uint8_t *dst = smem + PK_OFF + st * UNIT;
                 QUIK_TRACE_AT(11, u);
-                if (u < p.nkb_i) {  // this CTA's 128 rows of the packed B tile
-                    mbar_arrive_expect_tx(&pk_full[st], BNH * PK_ROW);
-                    tma_load_2d(dst, &tm_wq, u * PK_ROW, nb0, &pk_full[st]);
+                if (u < p.nkb_i) {  // this CTA's 128 rows of the B tile (packed, or INT8 codes)
+                    constexpr int WB = W8 ? OP_ROW : PK_ROW;
+                    mbar_arrive_expect_tx(&pk_full[st], BNH * WB);
+                    tma_load_2d(dst, &tm_wq, u * WB, nb0, &pk_full[st]);
                 } else {
                     const int v = u - p.nkb_i, ko = v / 2;
                     if (v == 0) grid_dependency_wait();  // Xo comes from the previous kernel
@@ -825,7 +826,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
                     ok = wait_bar(&op_empty[st], ((kb / S) & 1) ^ 1, ab);
                     if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                     uint32_t w[32];
-                    if constexpr (A8) {
+                    if constexpr (A8 && W8) {  // both sides in code order
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            w[4 * c + 0] = buf[j][c].x; w[4 * c + 1] = buf[j][c].y;
+                            w[4 * c + 2] = buf[j][c].z; w[4 * c + 3] = buf[j][c].w;
+                        }
+                    } else if constexpr (A8) {
 #pragma unroll
                         for (int c = 0; c < 4; ++c) order_i8_chunk(buf[j][2 * c], buf[j][2 * c + 1], w + 8 * c);
                     } else {
@@ -874,7 +881,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
                     if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                     if (tb == 0 && part == 0) QUIK_TRACE_AT(8, kb);
                     const uint8_t *pk = smem + PK_OFF + ps * UNIT;
-                    if (kb < p.nkb_i) {
+                    if (kb < p.nkb_i && !W8) {
                         // 128 rows x 4 chunks: unpack each 16-byte chunk into two
                         const int ch = tb & 3;
 #pragma unroll
@@ -888,8 +895,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
                             *reinterpret_cast<uint4 *>(rp + (((2 * ch + 1) ^ (row & 7)) << 4)) = hi;
                         }
                     } else {
-                        // Wo rows (part 0) into the B area, Xo rows (part 1) into the A area:
-                        // 128 rows x 8 chunks each
+                        // INT8 weight rows and Wo rows (part 0) into the B area, Xo rows
+                        // (part 1) into the A area: 128 rows x 8 chunks each
                         const int c = tb & 7;
                         uint8_t *dst = part == 0 ? bst : bst + B_BYTES;
 #pragma unroll
@@ -958,7 +965,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
                             const int n = nb + jj;
                             if (n < p.N) {
                                 if (p.Ki > 0)
-                                    p.acc_dbg[(size_t)grow * p.N + n] = acc_int<A8>(a[jj]);
+                                    p.acc_dbg[(size_t)grow * p.N + n] = acc_int<A8, W8>(a[jj]);
                                 if (OUT_INT8 && p.nkb_o > 0 && p.acc_o_dbg)
                                     p.acc_o_dbg[(size_t)grow * p.N + n] = static_cast<int32_t>(o[jj]);
                             }
@@ -973,7 +980,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int c = cc + jj + h;
-                        float v = acc_float<A8>(a[jj + h]) * sxr * col_sw[c];
+                        float v = acc_float<A8, W8>(a[jj + h]) * sxr * col_sw[c];
                         if (p.Ki == 0) v = 0.0f;
                         if (p.nkb_o > 0) {
                             if (OUT_INT8)
@@ -1460,7 +1467,7 @@ quik_status run(const GemmArgs &a, cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
 }
 
-template <bool OUT_INT8, bool DEBUG, bool A8>
+template <bool OUT_INT8, bool DEBUG, bool A8, bool W8>
 quik_status run_pair(const GemmArgs &a, cudaStream_t stream) {
     const int Ki = a.K - a.k_o;
     const bool outliers = a.k_o > 0 && a.Xo != nullptr;  // debug entry may skip them
@@ -1469,8 +1476,10 @@ quik_status run_pair(const GemmArgs &a, cudaStream_t stream) {
     std::memset(&mwq, 0, sizeof(mwq));
     std::memset(&mwo, 0, sizeof(mwo));
     std::memset(&mxo, 0, sizeof(mxo));
-    if (Ki > 0 && !make_map(&mwq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wq, Ki / 2, a.N, Ki / 2, PK_ROW,
-                            pair::BNH, CU_TENSOR_MAP_SWIZZLE_NONE))
+    // B k-blocks: 128 rows x 64 packed bytes, or x 128 INT8 codes
+    const uint64_t wrow = W8 ? Ki : Ki / 2;
+    if (Ki > 0 && !make_map(&mwq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wq, wrow, a.N, wrow,
+                            W8 ? OP_ROW : PK_ROW, pair::BNH, CU_TENSOR_MAP_SWIZZLE_NONE))
         return QUIK_ERR_CUDA;
     // outlier blocks as plain bytes, 128 rows x 128 bytes per unit
     if (outliers &&
@@ -1502,7 +1511,7 @@ quik_status run_pair(const GemmArgs &a, cudaStream_t stream) {
     p.tma_y = !DEBUG && (a.N % 8 == 0) &&
               make_map(&my, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.Y, a.N, a.M, static_cast<uint64_t>(a.N) * 2,
                        64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
-    auto kern = w4a4_gemm_pair_kernel<OUT_INT8, DEBUG, A8>;
+    auto kern = w4a4_gemm_pair_kernel<OUT_INT8, DEBUG, A8, W8>;
     if (!attribute_set_once(reinterpret_cast<const void *>(kern), pair::SMEM)) return QUIK_ERR_CUDA;
     const dim3 grid(2 * ((a.N + pair::BN - 1) / pair::BN), (a.M + 2 * BM - 1) / (2 * BM));
     if (!a.after_quantize) {
@@ -1599,14 +1608,20 @@ quik_status run_gemv(const GemmArgs &a, cudaStream_t stream) {
 // shared-memory-operand kernel.
 template <bool DEBUG>
 quik_status dispatch(const GemmArgs &a, cudaStream_t stream) {
-    if (a.a8) {  // INT8 activations (W4A8): per-token scales, the pair kernel
+    if (a.a8) {  // INT8 activations (W4A8, W8A8): per-token scales, the pair kernel
         if (a.group != 0) return QUIK_ERR_UNSUPPORTED;
-        return a.out_int8 ? run_pair<true, DEBUG, true>(a, stream) : run_pair<false, DEBUG, true>(a, stream);
+        if (a.w8)
+            return a.out_int8 ? run_pair<true, DEBUG, true, true>(a, stream)
+                              : run_pair<false, DEBUG, true, true>(a, stream);
+        return a.out_int8 ? run_pair<true, DEBUG, true, false>(a, stream)
+                          : run_pair<false, DEBUG, true, false>(a, stream);
     }
+    if (a.w8) return QUIK_ERR_UNSUPPORTED;
     if (a.group == 0 && a.M <= gemv::MT && a.k_o <= (a.out_int8 ? gemv::KO_MAX_I8 : gemv::KO_MAX_F16))
         return a.out_int8 ? run_gemv<true, DEBUG>(a, stream) : run_gemv<false, DEBUG>(a, stream);
     if (a.group == 0)
-        return a.out_int8 ? run_pair<true, DEBUG, false>(a, stream) : run_pair<false, DEBUG, false>(a, stream);
+        return a.out_int8 ? run_pair<true, DEBUG, false, false>(a, stream)
+                          : run_pair<false, DEBUG, false, false>(a, stream);
     return a.out_int8 ? run<CfgGroup<true, DEBUG>>(a, stream) : run<CfgGroup<false, DEBUG>>(a, stream);
 }
 

@@ -52,6 +52,7 @@ struct GemmArgs {
     int M, N, K, k_o, group;
     bool out_int8;
     bool a8;  // Xq holds INT8 codes [M, K_i] (W4A8) instead of packed INT4
+    bool w8;  // Wq holds INT8 codes [N, K_i] (W8A8; with a8)
     const void *Xq;
     const float *sx;
     const void *Xo;

@@ -42,6 +42,7 @@ class LayerConfig:
     w_std: float = 0.02
     bias: bool = False
     act_bits: int = 4           # 4: INT4 activations (W4A4); 8: INT8 activations (W4A8)
+    weight_bits: int = 4        # 4: INT4 weights; 8: INT8 weights (W8A8)
     description: str = field(default="", compare=False)
 
     @property
@@ -59,7 +60,7 @@ class LayerConfig:
         each), the outlier blocks, the fp32 scales, the fp16 output and bias."""
         groups = self.K_i // 128 if self.group else 1
         ob = 1 if self.outlier_int8 else 2
-        b = self.M * self.K_i * self.act_bits // 8 + self.N * self.K_i // 2  # Xq, Wq
+        b = (self.M * self.act_bits + self.N * self.weight_bits) * self.K_i // 8  # Xq, Wq
         b += (self.M + self.N) * self.k_o * ob           # Xo, Wo
         b += (self.M + self.N) * groups * 4              # sx, sw
         if self.outlier_int8 and self.k_o:
@@ -95,6 +96,10 @@ CONFIGS = {
         "llama7b_attn_w4a8_2048x4096x4096", M=2048, N=4096, K=4096, k_o=128, student_t=True,
         act_bits=8,
         description="the attention projection with INT8 activations (W4A8, QQQ), 128 FP16 outliers"),
+    "llama7b_attn_w8a8_2048x4096x4096": LayerConfig(
+        "llama7b_attn_w8a8_2048x4096x4096", M=2048, N=4096, K=4096, k_o=128, student_t=True,
+        act_bits=8, weight_bits=8,
+        description="the attention projection as W8A8 (the INT8 baseline), 128 FP16 outliers"),
     "llama7b_down_fused_4096x4096x11008": LayerConfig(
         "llama7b_down_fused_4096x4096x11008", M=4096, N=4096, K=11008, k_o=256,
         outlier_mult=50.0, bias=True,
@@ -162,9 +167,9 @@ def make_layer(cfg: LayerConfig, M: int | None = None, seed_offset: int = 0):
 
 def custom_config(M: int, N: int, K: int, k_o: int, group: int = 0, outlier_int8: bool = False,
                   bias: bool = True, outlier_mult: float = 30.0, student_t: bool = False,
-                  w_std: float = 0.02, act_bits: int = 4) -> LayerConfig:
+                  w_std: float = 0.02, act_bits: int = 4, weight_bits: int = 4) -> LayerConfig:
     return LayerConfig(f"custom_{M}x{N}x{K}_ko{k_o}_g{group}_{'i8' if outlier_int8 else 'f16'}"
-                       f"_a{act_bits}",
+                       f"_w{weight_bits}a{act_bits}",
                        M=M, N=N, K=K, k_o=k_o, group=group, outlier_int8=outlier_int8,
                        outlier_mult=outlier_mult, student_t=student_t, w_std=w_std, bias=bias,
-                       act_bits=act_bits)
+                       act_bits=act_bits, weight_bits=weight_bits)

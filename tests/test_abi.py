@@ -37,8 +37,8 @@ def test_status_strings(L):
         assert q.status_string(s) == name
 
 
-def _ws(M, N, K, k_o, group=0, outlier=0, act_bits=4):
-    return q.quik_workspace_size(q.make_shape(M, N, K, k_o, group, outlier, act_bits))
+def _ws(M, N, K, k_o, group=0, outlier=0, act_bits=4, weight_bits=4):
+    return q.quik_workspace_size(q.make_shape(M, N, K, k_o, group, outlier, act_bits, weight_bits))
 
 
 def test_workspace_size(L):
@@ -68,6 +68,7 @@ def test_workspace_size(L):
     (16, 16, 65536, 0, 0, 0),     # K above the supported maximum
     (16, 16, 256, 0, 0, 0, 3),    # activation width neither 4 nor 8
     (16, 16, 256, 0, 0, 0, 16),
+    (16, 16, 256, 0, 0, 0, 8, 2),  # weight width neither 4 nor 8
 ])
 def test_invalid_shapes_rejected(L, shape):
     assert _ws(*shape) == 0
@@ -79,6 +80,14 @@ def test_invalid_shapes_rejected(L, shape):
 def test_unsupported_group_size(L):
     s = q.make_shape(16, 16, 256, 0, 64, 0)
     assert L.quik_gemm(ctypes.byref(s), *([None] * 11)) == q.QUIK_ERR_UNSUPPORTED
+
+
+def test_int8_weights_need_int8_activations(L):
+    s = q.make_shape(16, 16, 256, 0, 0, 0, 4, 8)
+    assert q.quik_workspace_size(s) == 0
+    assert L.quik_gemm(ctypes.byref(s), *([None] * 11)) == q.QUIK_ERR_UNSUPPORTED
+    # W8A8: the workspace holds the INT8 activations, as for W4A8
+    assert q.quik_workspace_size(q.make_shape(64, 16, 256, 0, 0, 0, 8, 8)) == 64 * 256 + 256
 
 
 def test_grouped_int8_activations_unsupported(L):

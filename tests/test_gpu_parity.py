@@ -248,6 +248,7 @@ FULL = [
     ("llama65b_mlp_grouped_1024x22016x8192", None),
     ("llama7b_down_fused_4096x4096x11008", None),
     ("llama7b_attn_w4a8_2048x4096x4096", None),
+    ("llama7b_attn_w8a8_2048x4096x4096", None),
 ]
 
 
@@ -269,13 +270,14 @@ def test_full_size_layer(name):
     b = d["bias"].to(DEV) if d["bias"] is not None else None
     X = d["X"].to(DEV)
     layer = q.QuikLinear(d["W"].to(DEV), perm_d, cfg.k_o, cfg.group, cfg.outlier_int8, b,
-                         act_bits=cfg.act_bits)
+                         act_bits=cfg.act_bits, weight_bits=cfg.weight_bits)
     Y = layer(X)
     gx = q.quantize_reorder(X, perm_d, cfg.k_o, cfg.group, cfg.outlier_int8, act_bits=cfg.act_bits)
     torch.cuda.synchronize()
     ox = oracle.quantize_rows(np16(d["X"]), d["perm"].numpy(), cfg.k_o, cfg.group, cfg.outlier_int8,
                               cfg.act_bits)
-    ow = oracle_quant(d["W"], d["perm"], cfg.k_o, cfg.group, cfg.outlier_int8)
+    ow = oracle.quantize_rows(np16(d["W"]), d["perm"].numpy(), cfg.k_o, cfg.group, cfg.outlier_int8,
+                              cfg.weight_bits)
     # every code, scale and outlier value, activations and weights
     assert_quant_equal(gpu_tuple_np(gx), ox, f"{name} X")
     assert_quant_equal(gpu_tuple_np((layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale)), ow,
@@ -316,10 +318,13 @@ SHAPES_A8 = [
 ]
 
 
-def _case_a8(M, N, K, k_o, int8, bias, seed):
+def _case_a8(M, N, K, k_o, int8, bias, seed, wb=4):
     cfg = wl.custom_config(M, N, K, k_o, 0, int8, bias, outlier_mult=30.0,
-                           student_t=(seed % 2 == 1), act_bits=8)
+                           student_t=(seed % 2 == 1), act_bits=8, weight_bits=wb)
     return cfg, wl.make_layer(cfg, seed_offset=seed)
+
+
+WB = [4, 8]  # INT4 weights (W4A8) and INT8 weights (W8A8)
 
 
 @pytest.mark.parametrize("shape", SHAPES_A8, ids=[str(s) for s in SHAPES_A8])
@@ -333,17 +338,20 @@ def test_a8_quantize_bit_exact(shape):
     assert_quant_equal(gpu_tuple_np(gx), ref, "X (INT8 codes)")
 
 
+@pytest.mark.parametrize("wb", WB, ids=["w4a8", "w8a8"])
 @pytest.mark.parametrize("shape", SHAPES_A8, ids=[str(s) for s in SHAPES_A8])
-def test_a8_int32_sums_bit_exact(shape):
+def test_a8_int32_sums_bit_exact(shape, wb):
     M, N, K, k_o, int8, bias = shape
-    cfg, d = _case_a8(*shape, seed=11)
+    cfg, d = _case_a8(*shape, seed=11, wb=wb)
     perm_d = d["perm"].to(DEV)
     gx = q.quantize_reorder(d["X"].to(DEV), perm_d, k_o, 0, int8, act_bits=8)
-    gw = q.pack_weights(d["W"].to(DEV), perm_d, k_o, 0, int8)
+    gw = q.pack_weights(d["W"].to(DEV), perm_d, k_o, 0, int8, weight_bits=wb)
     acc, acc_o = q.gemm_i32(gx[0], gw[0], K, k_o, 0, gx[2], gw[2])
     torch.cuda.synchronize()
     ox = oracle.quantize_rows(np16(d["X"]), d["perm"].numpy(), k_o, 0, int8, 8)
-    ow = oracle.quantize_rows(np16(d["W"]), d["perm"].numpy(), k_o, 0, int8, 4)
+    ow = oracle.quantize_rows(np16(d["W"]), d["perm"].numpy(), k_o, 0, int8, wb)
+    if wb == 8:  # the weights' INT8 codes and scales, bit-exact
+        assert_quant_equal(gpu_tuple_np(gw), ow, "W (INT8 codes)")
     if K - k_o > 0:
         np.testing.assert_array_equal(acc.cpu().numpy(), oracle.int_gemm(ox[0], ow[0], 0))
     if int8 and k_o > 0:
@@ -351,20 +359,22 @@ def test_a8_int32_sums_bit_exact(shape):
         np.testing.assert_array_equal(acc_o.cpu().numpy(), ref_o)
 
 
+@pytest.mark.parametrize("wb", WB, ids=["w4a8", "w8a8"])
 @pytest.mark.parametrize("shape", SHAPES_A8, ids=[str(s) for s in SHAPES_A8])
-def test_a8_linear_output_within_tolerance(shape):
+def test_a8_linear_output_within_tolerance(shape, wb):
     M, N, K, k_o, int8, bias = shape
-    cfg, d = _case_a8(*shape, seed=13)
+    cfg, d = _case_a8(*shape, seed=13, wb=wb)
     perm_d = d["perm"].to(DEV)
     b = d["bias"].to(DEV) if d["bias"] is not None else None
-    layer = q.QuikLinear(d["W"].to(DEV), perm_d, k_o, 0, int8, b, act_bits=8)
+    layer = q.QuikLinear(d["W"].to(DEV), perm_d, k_o, 0, int8, b, act_bits=8, weight_bits=wb)
     Y = layer(d["X"].to(DEV))
     gx = q.quantize_reorder(d["X"].to(DEV), perm_d, k_o, 0, int8, act_bits=8)
     Y2 = q.gemm(gx, (layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale), K, k_o, 0, b)
     torch.cuda.synchronize()
     ref = oracle.layer(np16(d["X"]), np16(d["W"]), d["perm"].numpy(),
-                       None if d["bias"] is None else np16(d["bias"]), k_o, 0, int8, act_bits=8)["Y"]
-    assert_y_close(Y.float().cpu().numpy(), ref, f"W4A8 linear {shape}")
+                       None if d["bias"] is None else np16(d["bias"]), k_o, 0, int8, act_bits=8,
+                       weight_bits=wb)["Y"]
+    assert_y_close(Y.float().cpu().numpy(), ref, f"W{wb}A8 linear {shape}")
     np.testing.assert_array_equal(Y.cpu().numpy().view(np.uint16), Y2.cpu().numpy().view(np.uint16))
 
 
@@ -376,4 +386,15 @@ def test_a8_grouped_is_unsupported():
     sx = torch.empty((16, 4), dtype=torch.float32, device=DEV)
     with pytest.raises(q.QuikError) as e:
         q.quik_quantize_reorder(shape, X, perm, Xq, sx, None, None)
+    assert e.value.status == q.QUIK_ERR_UNSUPPORTED
+
+
+def test_w8_without_a8_is_unsupported():
+    shape = q.make_shape(16, 256, 256, 0, 0, q.QUIK_OUTLIER_FP16, 4, 8)
+    W = torch.zeros((256, 256), dtype=torch.float16, device=DEV)
+    perm = torch.arange(256, dtype=torch.int32, device=DEV)
+    Wq = torch.empty((256, 256), dtype=torch.int8, device=DEV)
+    sw = torch.empty((256,), dtype=torch.float32, device=DEV)
+    with pytest.raises(q.QuikError) as e:
+        q.quik_pack_weights(shape, W, perm, Wq, sw, None, None)
     assert e.value.status == q.QUIK_ERR_UNSUPPORTED
