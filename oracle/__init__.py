@@ -41,6 +41,8 @@ def _load():
         lib = ctypes.CDLL(build())
         _C = ctypes.c_int
         lib.oracle_quantize_rows.argtypes = [_I, _I, _I, _I, _C, _C, _P, _P, _P, _P, _P, _P]
+        lib.oracle_rmsnorm_quantize_rows.argtypes = [_I, _I, _I, _I, _C, _C, _P, _P,
+                                                     ctypes.c_double, _P, _P, _P, _P, _P]
         lib.oracle_int_gemm.argtypes = [_I, _I, _I, _I, _C, _C, _P, _P, _P]
         lib.oracle_linear.argtypes = [_I, _I, _I, _I, _I, _C, _C, _C,
                                       _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
@@ -48,7 +50,8 @@ def _load():
                                               _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                               _I, _P, _P, _P, _P]
         lib.oracle_num_threads.argtypes = []
-        for f in (lib.oracle_quantize_rows, lib.oracle_int_gemm, lib.oracle_linear,
+        for f in (lib.oracle_quantize_rows, lib.oracle_rmsnorm_quantize_rows,
+                  lib.oracle_int_gemm, lib.oracle_linear,
                   lib.oracle_linear_sampled, lib.oracle_num_threads):
             f.restype = ctypes.c_int
         _lib = lib
@@ -89,6 +92,36 @@ def quantize_rows(X_f16: np.ndarray, perm: np.ndarray, k_o: int, group: int = 0,
                                       _ptr(X.view(np.uint16)), _ptr(perm), _ptr(Q),
                                       _ptr(scale), _ptr(O), _ptr(o_scale))
     _check(rc, "quantize_rows")
+    return Q, scale, O, o_scale
+
+
+def rmsnorm_quantize_rows(X_f16: np.ndarray, gamma_f16: np.ndarray, eps: float,
+                          perm: np.ndarray, k_o: int, group: int = 0,
+                          outlier_int8: bool = False, bits: int = 4):
+    """RMS-normalise each row of ``X_f16`` ([R, K] float16) with weight
+    ``gamma_f16`` ([K], source channel order) and ``eps``, then reorder and
+    quantise it ("Atom", idea I2: quantisation fused into the norm).
+
+    Codes and base scales are those of z = X * gamma; the row factor
+    r = 1/sqrt(mean(X^2) + eps) (fp64) multiplies the stored scales, and FP16
+    outliers are fl16(z * r).  Returns the tuple of ``quantize_rows``.
+    """
+    X = np.ascontiguousarray(X_f16, dtype=np.float16)
+    g = np.ascontiguousarray(gamma_f16, dtype=np.float16)
+    R, K = X.shape
+    assert g.shape == (K,)
+    Ki = K - k_o
+    G = Ki // group if group else 1
+    perm = np.ascontiguousarray(perm, dtype=np.int32)
+    Q = np.zeros((R, Ki), np.int8) if bits == 8 else np.zeros((R, Ki // 2), np.uint8)
+    scale = np.zeros((R, G) if group else (R,), np.float32)
+    O = np.zeros((R, k_o), np.int8 if outlier_int8 else np.float16)
+    o_scale = np.zeros((R,), np.float32) if outlier_int8 else None
+    rc = _load().oracle_rmsnorm_quantize_rows(R, K, k_o, group, int(outlier_int8), int(bits),
+                                              _ptr(X.view(np.uint16)), _ptr(g.view(np.uint16)),
+                                              float(eps), _ptr(perm), _ptr(Q), _ptr(scale),
+                                              _ptr(O), _ptr(o_scale))
+    _check(rc, "rmsnorm_quantize_rows")
     return Q, scale, O, o_scale
 
 
@@ -167,6 +200,19 @@ def layer(X_f16, W_f16, perm, bias, k_o: int, group: int = 0, outlier_int8: bool
     """
     K = X_f16.shape[1]
     Xq, sx, Xo, sxo = quantize_rows(X_f16, perm, k_o, group, outlier_int8, act_bits)
+    Wq, sw, Wo, swo = quantize_rows(W_f16, perm, k_o, group, outlier_int8, weight_bits)
+    Y = linear(Xq, sx, Xo if k_o else None, sxo, Wq, sw, Wo if k_o else None, swo, bias,
+               K, k_o, group)
+    return dict(Xq=Xq, sx=sx, Xo=Xo, sxo=sxo, Wq=Wq, sw=sw, Wo=Wo, swo=swo, Y=Y)
+
+
+def rmsnorm_layer(X_f16, gamma_f16, eps, W_f16, perm, bias, k_o: int, group: int = 0,
+                  outlier_int8: bool = False, act_bits: int = 4, weight_bits: int = 4):
+    """The layer behind an RMS norm: ``rmsnorm_quantize_rows`` on the
+    activations, ``quantize_rows`` on the weights, then the fp64 output."""
+    K = X_f16.shape[1]
+    Xq, sx, Xo, sxo = rmsnorm_quantize_rows(X_f16, gamma_f16, eps, perm, k_o, group,
+                                            outlier_int8, act_bits)
     Wq, sw, Wo, swo = quantize_rows(W_f16, perm, k_o, group, outlier_int8, weight_bits)
     Y = linear(Xq, sx, Xo if k_o else None, sxo, Wq, sw, Wo if k_o else None, swo, bias,
                K, k_o, group)

@@ -33,6 +33,11 @@
  *    in reordered order.
  *  - 8-bit weights (W8A8, the baseline the same abstracts compare against):
  *    the same INT8 rule per output channel.
+ *  - RMS norm fused with the activation quantiser (Atom, Summary and idea
+ *    I2: quantisation folded into operators that already run): the norm's
+ *    row factor r = 1/sqrt(mean(h^2) + eps) changes no code, so codes and base
+ *    scales are taken from h * gamma and r multiplies the stored scales (and
+ *    the FP16 outliers, rounded once to fp16).
  *  - packing: byte i of a row holds code 2i in the low nibble and code 2i+1
  *    in the high nibble, both 4-bit two's complement.
  *  - integer dot products in int64 (checked to fit int32); dequantisation,
@@ -189,6 +194,142 @@ int oracle_quantize_rows(int64_t R, int64_t K, int64_t k_o, int64_t group, int o
                 }
             }
         free(xr);
+        free(codes);
+    }
+    return err;
+}
+
+/* IEEE 754 binary64 -> binary16, round to nearest even, from the format's
+ * definition: normal values are m * 2^(e - 10) with m in [1024, 2048) and
+ * e in [-14, 15]; below 2^-14 the step is 2^-24 (subnormals); magnitudes
+ * that round past 65504 become infinity. */
+static uint16_t double_to_half(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (isnan(v)) return 0x7e00;
+    if (a < ldexp(1.0, -14)) {                       /* subnormal (or zero) */
+        double q = nearbyint(a / ldexp(1.0, -24));    /* q <= 1024: 1024 is 2^-14 */
+        return (uint16_t)(sign | (uint16_t)q);
+    }
+    int e2;
+    frexp(a, &e2);                                    /* a = f * 2^e2, f in [0.5, 1) */
+    int e = e2 - 1;                                   /* a in [2^e, 2^(e+1)) */
+    double m = nearbyint(a / ldexp(1.0, e - 10));     /* in [1024, 2048] */
+    if (m == 2048.0) { m = 1024.0; e += 1; }
+    if (e > 15) return (uint16_t)(sign | 0x7c00);
+    return (uint16_t)(sign | (uint16_t)((e + 15) << 10) | (uint16_t)(m - 1024.0));
+}
+
+/*
+ * oracle_rmsnorm_quantize_rows -- the RMS normalisation that precedes a
+ * projection, with the projection's dynamic quantisation and reordering
+ * folded into it ("Atom: Low-bit Quantization for Efficient and Accurate LLM
+ * Serving", Summary and idea I2: quantisation and reordering are fused into
+ * operators that already run).  The normalisation of a row h of K channels
+ * with weight gamma [K] (the norm in front of every Llama projection):
+ *
+ *     r    = 1 / sqrt( (1/K) * sum_{k<K} h[k]^2 + eps )      over ALL K channels
+ *     y[k] = h[k] * r * gamma[k]
+ *
+ * and y is then reordered and quantised by the rule of oracle_quantize_rows.
+ * Reading where the pages are silent: r > 0 multiplies every position of the
+ * row, so it changes no code (y / s_y = z / s_z for z = h * gamma); the codes
+ * and the fp32 base scales are those of z[k] = h[k] * gamma[k] (a product of
+ * two fp16 values, exact in fp32), and r moves onto the stored scales:
+ *
+ *     scale   = fl32(s_z * r),  s_z = fl32(max|z| / 7) per row (or group)
+ *     o_scale = fl32(so_z * r), so_z = fl32(max|z_o| / 127)   (INT8 outliers)
+ *     O       = fl16(z * r)                                    (FP16 outliers)
+ *
+ * r is taken in fp64 here.  The unfused pipeline would round y to fp16
+ * before quantising; fusing the two steps removes that intermediate.
+ *
+ *  X, gamma : [R, K] and [K] fp16 bit patterns (gamma in source channel order)
+ *  other arguments as oracle_quantize_rows
+ */
+int oracle_rmsnorm_quantize_rows(int64_t R, int64_t K, int64_t k_o, int64_t group,
+                                 int outlier_int8, int bits, const uint16_t *X,
+                                 const uint16_t *gamma, double eps, const int32_t *perm,
+                                 uint8_t *Q, float *scale, void *O, float *o_scale)
+{
+    if (R < 0 || K < 1 || k_o < 0 || k_o > K || (bits != 4 && bits != 8)) return ORACLE_EBADARG;
+    if (!(eps >= 0.0)) return ORACLE_EBADARG;
+    const int qmax = bits == 8 ? 127 : 7;
+    const int64_t Ki = K - k_o;
+    if (Ki % 2) return ORACLE_EBADARG;
+    if (group < 0 || (group > 0 && Ki % group)) return ORACLE_EBADARG;
+    const int64_t gs = group > 0 ? group : Ki;
+    const int64_t G = group > 0 ? Ki / group : 1;
+    for (int64_t j = 0; j < K; ++j)
+        if (perm[j] < 0 || perm[j] >= K) return ORACLE_EBADARG;
+
+    int err = ORACLE_OK;
+#pragma omp parallel
+    {
+        float *z = (float *)malloc(sizeof(float) * (size_t)K);
+        int *codes = (int *)malloc(sizeof(int) * (size_t)(Ki > 0 ? Ki : 1));
+        if (!z || !codes) {
+#pragma omp atomic write
+            err = ORACLE_ENOMEM;
+        }
+#pragma omp for schedule(static)
+        for (int64_t r = 0; r < R; ++r) {
+            if (!z || !codes) continue;
+            /* the row's RMS factor, over every channel (order does not matter) */
+            double ss = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double h = half_to_double(X[r * K + k]);
+                ss += h * h;
+            }
+            double rf = 1.0 / sqrt(ss / (double)K + eps);
+
+            /* reorder (Atom I1) the row times its norm weight; exact in fp32 */
+            for (int64_t j = 0; j < K; ++j) {
+                int64_t c = perm[j];
+                z[j] = (float)(half_to_double(X[r * K + c]) * half_to_double(gamma[c]));
+            }
+
+            /* scales and codes of z, the stored scales carry r */
+            for (int64_t g = 0; g < G; ++g) {
+                float amax = 0.0f;
+                for (int64_t j = g * gs; j < (g + 1) * gs; ++j)
+                    if (fabsf(z[j]) > amax) amax = fabsf(z[j]);
+                float s = amax / (float)qmax;
+                scale[r * G + g] = (float)((double)s * rf);
+                for (int64_t j = g * gs; j < (g + 1) * gs; ++j)
+                    codes[j] = quantize_value(z[j], s, qmax);
+            }
+            if (bits == 8) {
+                for (int64_t j = 0; j < Ki; ++j)
+                    Q[r * Ki + j] = (uint8_t)(int8_t)codes[j];
+            } else {
+                for (int64_t i = 0; i < Ki / 2; ++i)
+                    Q[r * (Ki / 2) + i] =
+                        (uint8_t)((codes[2 * i] & 0xF) | ((codes[2 * i + 1] & 0xF) << 4));
+            }
+
+            /* the outlier block: the normalised values in fp16, or INT8 codes of z */
+            if (k_o > 0) {
+                if (!outlier_int8) {
+                    uint16_t *o16 = (uint16_t *)O;
+                    for (int64_t i = 0; i < k_o; ++i)
+                        o16[r * k_o + i] = double_to_half((double)z[Ki + i] * rf);
+                } else {
+                    int8_t *o8 = (int8_t *)O;
+                    float amax = 0.0f;
+                    for (int64_t i = 0; i < k_o; ++i)
+                        if (fabsf(z[Ki + i]) > amax) amax = fabsf(z[Ki + i]);
+                    float s = amax / 127.0f;
+                    o_scale[r] = (float)((double)s * rf);
+                    for (int64_t i = 0; i < k_o; ++i)
+                        o8[r * k_o + i] = (int8_t)quantize_value(z[Ki + i], s, 127);
+                }
+            } else if (outlier_int8 && o_scale) {
+                o_scale[r] = 0.0f;
+            }
+        }
+        free(z);
         free(codes);
     }
     return err;
