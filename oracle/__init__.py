@@ -42,7 +42,7 @@ def _load():
         _C = ctypes.c_int
         lib.oracle_quantize_rows.argtypes = [_I, _I, _I, _I, _C, _C, _P, _P, _P, _P, _P, _P]
         lib.oracle_rmsnorm_quantize_rows.argtypes = [_I, _I, _I, _I, _C, _C, _P, _P,
-                                                     ctypes.c_double, _P, _P, _P, _P, _P]
+                                                     ctypes.c_float, _P, _P, _P, _P, _P]
         lib.oracle_int_gemm.argtypes = [_I, _I, _I, _I, _C, _C, _P, _P, _P]
         lib.oracle_linear.argtypes = [_I, _I, _I, _I, _I, _C, _C, _C,
                                       _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
@@ -103,8 +103,9 @@ def rmsnorm_quantize_rows(X_f16: np.ndarray, gamma_f16: np.ndarray, eps: float,
     quantise it ("Atom", idea I2: quantisation fused into the norm).
 
     Codes and base scales are those of z = X * gamma; the row factor
-    r = 1/sqrt(mean(X^2) + eps) (fp64) multiplies the stored scales, and FP16
-    outliers are fl16(z * r).  Returns the tuple of ``quantize_rows``.
+    r = 1/sqrt(mean(X^2) + eps) (fp64; eps is taken as fp32, the type of the
+    norm's parameter) multiplies the stored scales, and FP16 outliers are
+    fl16(z * r).  Returns the tuple of ``quantize_rows``.
     """
     X = np.ascontiguousarray(X_f16, dtype=np.float16)
     g = np.ascontiguousarray(gamma_f16, dtype=np.float16)

@@ -242,19 +242,21 @@ static uint16_t double_to_half(double v)
  *     o_scale = fl32(so_z * r), so_z = fl32(max|z_o| / 127)   (INT8 outliers)
  *     O       = fl16(z * r)                                    (FP16 outliers)
  *
- * r is taken in fp64 here.  The unfused pipeline would round y to fp16
- * before quantising; fusing the two steps removes that intermediate.
+ * eps is an fp32 value (the norm's parameter as stored); r is taken in
+ * fp64, and the stored scales and outliers are one rounding of an fp64
+ * product.  The unfused pipeline would round y to fp16 before quantising;
+ * fusing the two steps removes that intermediate.
  *
  *  X, gamma : [R, K] and [K] fp16 bit patterns (gamma in source channel order)
  *  other arguments as oracle_quantize_rows
  */
 int oracle_rmsnorm_quantize_rows(int64_t R, int64_t K, int64_t k_o, int64_t group,
                                  int outlier_int8, int bits, const uint16_t *X,
-                                 const uint16_t *gamma, double eps, const int32_t *perm,
+                                 const uint16_t *gamma, float eps, const int32_t *perm,
                                  uint8_t *Q, float *scale, void *O, float *o_scale)
 {
     if (R < 0 || K < 1 || k_o < 0 || k_o > K || (bits != 4 && bits != 8)) return ORACLE_EBADARG;
-    if (!(eps >= 0.0)) return ORACLE_EBADARG;
+    if (!(eps >= 0.0f)) return ORACLE_EBADARG;
     const int qmax = bits == 8 ? 127 : 7;
     const int64_t Ki = K - k_o;
     if (Ki % 2) return ORACLE_EBADARG;
@@ -282,7 +284,7 @@ int oracle_rmsnorm_quantize_rows(int64_t R, int64_t K, int64_t k_o, int64_t grou
                 double h = half_to_double(X[r * K + k]);
                 ss += h * h;
             }
-            double rf = 1.0 / sqrt(ss / (double)K + eps);
+            double rf = 1.0 / sqrt(ss / (double)K + (double)eps);
 
             /* reorder (Atom I1) the row times its norm weight; exact in fp32 */
             for (int64_t j = 0; j < K; ++j) {

@@ -119,7 +119,7 @@ def test_constant_row_closed_form(oracle_mod):
         h = np.full((1, K), c, np.float16)
         g = np.ones(K, np.float16)
         q, s, o, _ = oracle_mod.rmsnorm_quantize_rows(h, g, eps, perm, k_o)
-        r = 1.0 / np.sqrt(float(c) ** 2 + eps)
+        r = 1.0 / np.sqrt(float(c) ** 2 + float(np.float32(eps)))  # eps is an fp32 parameter
         code = 7 if c > 0 else -7
         nib = code & 0xF
         assert np.all(q == (nib | (nib << 4)))
