@@ -211,11 +211,17 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- CPU oracle legs
 def cpu_oracle_step(cfg, d, rows: int):
-    """One bounded CPU pass of the layer: quantise `rows` token rows, then their
-    full output rows (every column) from the pre-packed weights."""
+    """One bounded CPU pass of the layer: quantise `rows` token rows (with the
+    RMS norm folded in, for a norm-fused workload), then their full output rows
+    (every column) from the pre-packed weights."""
     import oracle
     X = d["X"][:rows].numpy()
-    xq = oracle.quantize_rows(X, d["perm_np"], cfg.k_o, cfg.group, cfg.outlier_int8, cfg.act_bits)
+    if cfg.rmsnorm:
+        xq = oracle.rmsnorm_quantize_rows(X, d["gamma"].numpy(), d["eps"], d["perm_np"], cfg.k_o,
+                                          cfg.group, cfg.outlier_int8, cfg.act_bits)
+    else:
+        xq = oracle.quantize_rows(X, d["perm_np"], cfg.k_o, cfg.group, cfg.outlier_int8,
+                                  cfg.act_bits)
     wq = d["w_oracle"]
     oracle.linear(xq[0], xq[1], xq[2] if cfg.k_o else None, xq[3], wq[0], wq[1],
                   wq[2] if cfg.k_o else None, wq[3], d["bias_np"], cfg.K, cfg.k_o, cfg.group)
@@ -290,8 +296,11 @@ def run_ours(args, rank, local_rank, world):
     X = d["X"].to(dev)
     perm = d["perm"].to(dev)
     bias = d["bias"].to(dev) if d["bias"] is not None else None
+    gamma = d["gamma"].to(dev) if cfg.rmsnorm else None
+    eps = d.get("eps", 0.0)
     layer = q.QuikLinear(d["W"].to(dev), perm, cfg.k_o, cfg.group, cfg.outlier_int8, bias,
-                         act_bits=cfg.act_bits, weight_bits=cfg.weight_bits)
+                         act_bits=cfg.act_bits, weight_bits=cfg.weight_bits, norm_weight=gamma,
+                         norm_eps=eps)
     shape = layer.shape(cfg.M)
     Xq, sx, Xo, sxo = q._binding._quant_outputs(cfg.M, cfg.K, cfg.k_o, cfg.group,
                                                 cfg.outlier_int8, dev, cfg.act_bits)
@@ -302,16 +311,25 @@ def run_ours(args, rank, local_rank, world):
     ws = layer.workspace(cfg.M, dev)
 
     def step():
-        # one layer call: quantise + reorder, then the GEMM (which may start
-        # while the quantiser finishes: programmatic dependent launch)
-        q.quik_linear(shape, X, perm, layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale, bias, Y,
-                      ws, stream=stream)
+        # one layer call: quantise + reorder (behind the RMS norm, for a
+        # norm-fused workload), then the GEMM (which may start while the
+        # quantiser finishes: programmatic dependent launch)
+        if cfg.rmsnorm:
+            q.quik_rmsnorm_linear(shape, X, gamma, eps, perm, layer.Wq, layer.w_scale, layer.Wo,
+                                  layer.wo_scale, bias, Y, ws, stream=stream)
+        else:
+            q.quik_linear(shape, X, perm, layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale, bias,
+                          Y, ws, stream=stream)
 
     def split_step(ev):
         # the same two kernels through the two public calls, with an event
         # between them: the per-kernel breakdown
         ev[0].record(stream)
-        q.quik_quantize_reorder(shape, X, perm, Xq, sx, Xo, sxo, stream=stream)
+        if cfg.rmsnorm:
+            q.quik_rmsnorm_quantize_reorder(shape, X, gamma, eps, perm, Xq, sx, Xo, sxo,
+                                            stream=stream)
+        else:
+            q.quik_quantize_reorder(shape, X, perm, Xq, sx, Xo, sxo, stream=stream)
         ev[1].record(stream)
         q.quik_gemm(shape, Xq, sx, Xo, sxo, layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale,
                     bias, Y, stream=stream)
@@ -388,6 +406,26 @@ def run_ours(args, rank, local_rank, world):
     warm_us = float(np.median([a.elapsed_time(b) for a, b in wev])) * 1e3
     context = library_context(cfg, X, d["W"].to(dev), flush)
     context["warm_l2_us_per_call"] = round(warm_us, 2)
+    if cfg.rmsnorm:
+        # the unfused pipeline: torch's RMS norm writes the normalised fp16
+        # rows, then the plain layer call quantises them
+        def unfused():
+            Xn = torch.nn.functional.rms_norm(X, (cfg.K,), gamma, eps)
+            q.quik_linear(shape, Xn, perm, layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale,
+                          bias, Y, ws, stream=stream)
+
+        uev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(20)]
+        for _ in range(3):
+            flush.zero_()
+            unfused()
+        for i in range(20):
+            flush.zero_()
+            uev[i][0].record(stream)
+            unfused()
+            uev[i][1].record(stream)
+        torch.cuda.synchronize()
+        context["unfused_torch_rms_norm_then_layer_us"] = round(
+            float(np.median([a.elapsed_time(b) for a, b in uev])) * 1e3, 2)
     context["layer_speedup_vs_fp16_matmul"] = round(context["fp16_matmul_us"] / (t_step * 1e6), 3)
 
     peaks, peak_kind = measured_peaks()
@@ -435,7 +473,9 @@ def run_ours(args, rank, local_rank, world):
             "group_size": cfg.group, "outliers": "int8" if cfg.outlier_int8 else "fp16",
             "bias": cfg.bias, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": "flushed before every step (256 MiB write, outside the step's events)",
-            "step": "quik_linear: quantise + reorder, then the GEMM (weights packed once, offline)",
+            "step": ("quik_rmsnorm_linear: RMS norm folded into quantise + reorder, then the GEMM"
+                     if cfg.rmsnorm else "quik_linear: quantise + reorder, then the GEMM")
+                    + " (weights packed once, offline)",
         },
         "us_per_call": round(t_step * 1e6, 2),
         "pct_int8_peak": round(100.0 * value / world / int8_peak, 2),
@@ -445,7 +485,8 @@ def run_ours(args, rank, local_rank, world):
         "roofline": roofline,
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
                 "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2,
-                "call": "quik_linear via QuikLinear, pinned host X in, host Y out"},
+                "call": ("quik_rmsnorm_linear" if cfg.rmsnorm else "quik_linear")
+                        + " via QuikLinear, pinned host X in, host Y out"},
         "gpu_launches": 2 * args.steps,
         "clocks": sampler.summary(),
         "context": context,

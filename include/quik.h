@@ -166,6 +166,49 @@ QUIK_API quik_status quik_linear(const quik_shape *shape, const void *X_f16, con
                         void *workspace, size_t workspace_bytes, quik_stream_t stream);
 
 /*
+ * quik_rmsnorm_quantize_reorder -- the RMS norm that precedes a projection,
+ * with the projection's dynamic quantisation and reordering folded into it
+ * (Atom summary and idea I2: quantisation and reordering are fused into
+ * operators that already run).  For each row h of X:
+ *     r = 1 / sqrt(mean_k(h[k]^2) + eps)         (all K channels)
+ *     y[k] = h[k] * r * gamma[k]
+ * and y is quantised as by quik_quantize_reorder, with one reading: r > 0 is
+ * common to the whole row and changes no code, so the codes and the fp32
+ * base scales are those of z = h * gamma (exact in fp32), and r multiplies
+ * what is stored:
+ *     x_scale  = fl32(fl32(max|z| / 7) * r)      (per token, or per group)
+ *     xo_scale = fl32(fl32(max|z_o| / 127) * r)  (INT8 outliers)
+ *     Xo       = fl16(fl32(z * r))               (FP16 outliers)
+ * The normalised fp16 row is never written.  The sum of squares is taken in
+ * fp32 and r with IEEE-rounded steps, so scales and FP16 outliers carry the
+ * rounding of that sum; codes do not depend on it.
+ *   X_f16     [M, K] fp16 (the hidden state before the norm), row-major
+ *   gamma_f16 [K] fp16, the norm's weight in SOURCE channel order
+ *   eps       finite and > 0 (else QUIK_ERR_INVALID_ARG)
+ *   perm, Xq, x_scale, Xo, xo_scale : as quik_quantize_reorder
+ * K up to 24576 (the kernel stages perm and the reordered gamma side by side
+ * in shared memory); a larger K returns QUIK_ERR_UNSUPPORTED.  Other errors,
+ * validation and stream semantics as quik_quantize_reorder.
+ */
+QUIK_API quik_status quik_rmsnorm_quantize_reorder(const quik_shape *shape, const void *X_f16,
+                                                   const void *gamma_f16, float eps,
+                                                   const int32_t *perm, void *Xq, float *x_scale,
+                                                   void *Xo, float *xo_scale, quik_stream_t stream);
+
+/*
+ * quik_rmsnorm_linear -- quik_linear behind an RMS norm:
+ * quik_rmsnorm_quantize_reorder into `workspace` (quik_workspace_size(shape)
+ * bytes, caller-owned) followed by quik_gemm, on `stream`.  Arguments as
+ * quik_linear plus gamma_f16 [K] and eps of quik_rmsnorm_quantize_reorder.
+ */
+QUIK_API quik_status quik_rmsnorm_linear(const quik_shape *shape, const void *X_f16,
+                                         const void *gamma_f16, float eps, const int32_t *perm,
+                                         const void *Wq, const float *w_scale, const void *Wo,
+                                         const float *wo_scale, const void *bias_f16, void *Y_f16,
+                                         void *workspace, size_t workspace_bytes,
+                                         quik_stream_t stream);
+
+/*
  * quik_linear_noalloc -- quik_linear for callers that cannot allocate device
  * memory.  (No counterpart in the papers; an addition of this library.)
  *

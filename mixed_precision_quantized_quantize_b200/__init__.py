@@ -24,12 +24,15 @@ from ._binding import (  # noqa: F401
     make_shape,
     pack_weights,
     quantize_reorder,
+    rmsnorm_quantize_reorder,
     quik_gemm,
     quik_gemm_i32_debug,
     quik_linear,
     quik_linear_noalloc,
     quik_pack_weights,
     quik_quantize_reorder,
+    quik_rmsnorm_linear,
+    quik_rmsnorm_quantize_reorder,
     quik_selftest_timeout,
     quik_shape,
     quik_status_string,

@@ -44,9 +44,13 @@ _S = ctypes.POINTER(quik_shape)
 _SIGS = {
     "quik_workspace_size": (ctypes.c_size_t, [_S]),
     "quik_quantize_reorder": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P]),
+    "quik_rmsnorm_quantize_reorder": (ctypes.c_int, [_S, _P, _P, ctypes.c_float, _P, _P, _P, _P,
+                                                      _P, _P]),
     "quik_pack_weights": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P]),
     "quik_gemm": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "quik_linear": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "quik_rmsnorm_linear": (ctypes.c_int, [_S, _P, _P, ctypes.c_float, _P, _P, _P, _P, _P, _P,
+                                            _P, _P, ctypes.c_size_t, _P]),
     "quik_linear_noalloc": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "quik_gemm_i32_debug": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P]),
     "quik_sync_check": (ctypes.c_int, [_P]),
@@ -134,6 +138,16 @@ def quik_quantize_reorder(shape, X, perm, Xq, x_scale, Xo, xo_scale, stream=None
         _ptr(xo_scale, torch.float32, "xo_scale"), _stream(stream)), "quik_quantize_reorder")
 
 
+def quik_rmsnorm_quantize_reorder(shape, X, gamma, eps, perm, Xq, x_scale, Xo, xo_scale,
+                                  stream=None):
+    _check(lib().quik_rmsnorm_quantize_reorder(
+        ctypes.byref(shape), _ptr(X, torch.float16, "X"), _ptr(gamma, torch.float16, "gamma"),
+        float(eps), _ptr(perm, torch.int32, "perm"), _ptr(Xq, _xq_dtype(shape), "Xq"),
+        _ptr(x_scale, torch.float32, "x_scale"), _ptr(Xo, None, "Xo"),
+        _ptr(xo_scale, torch.float32, "xo_scale"), _stream(stream)),
+        "quik_rmsnorm_quantize_reorder")
+
+
 def quik_pack_weights(shape, W, perm, Wq, w_scale, Wo, wo_scale, stream=None):
     _check(lib().quik_pack_weights(
         ctypes.byref(shape), _ptr(W, torch.float16, "W"), _ptr(perm, torch.int32, "perm"),
@@ -157,6 +171,18 @@ def quik_linear(shape, X, perm, Wq, w_scale, Wo, wo_scale, bias, Y, workspace, s
         _ptr(Wo, None, "Wo"), _ptr(wo_scale, torch.float32, "wo_scale"),
         _ptr(bias, torch.float16, "bias"), _ptr(Y, torch.float16, "Y"),
         _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)), "quik_linear")
+
+
+def quik_rmsnorm_linear(shape, X, gamma, eps, perm, Wq, w_scale, Wo, wo_scale, bias, Y, workspace,
+                        stream=None):
+    _check(lib().quik_rmsnorm_linear(
+        ctypes.byref(shape), _ptr(X, torch.float16, "X"), _ptr(gamma, torch.float16, "gamma"),
+        float(eps), _ptr(perm, torch.int32, "perm"),
+        _ptr(Wq, _wq_dtype(shape), "Wq"), _ptr(w_scale, torch.float32, "w_scale"),
+        _ptr(Wo, None, "Wo"), _ptr(wo_scale, torch.float32, "wo_scale"),
+        _ptr(bias, torch.float16, "bias"), _ptr(Y, torch.float16, "Y"),
+        _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
+        "quik_rmsnorm_linear")
 
 
 def quik_linear_noalloc(shape, X, perm, Wq, w_scale, Wo, wo_scale, bias, Y, stream=None):
@@ -216,6 +242,18 @@ def quantize_reorder(X: torch.Tensor, perm: torch.Tensor, k_o: int, group: int =
     return out
 
 
+def rmsnorm_quantize_reorder(X: torch.Tensor, gamma: torch.Tensor, eps: float, perm: torch.Tensor,
+                             k_o: int, group: int = 0, outlier_int8: bool = False, stream=None,
+                             act_bits: int = 4):
+    """RMS norm (weight gamma [K], eps) fused with quantize_reorder: the hidden
+    state X -> (Xq, x_scale, Xo, xo_scale) of the normalised rows."""
+    M, K = X.shape
+    shape = make_shape(M, 1, K, k_o, group, _outlier_kind(outlier_int8), act_bits)
+    out = _quant_outputs(M, K, k_o, group, outlier_int8, X.device, act_bits)
+    quik_rmsnorm_quantize_reorder(shape, X, gamma, eps, perm, *out, stream=stream)
+    return out
+
+
 def pack_weights(W: torch.Tensor, perm: torch.Tensor, k_o: int, group: int = 0,
                  outlier_int8: bool = False, stream=None, weight_bits: int = 4):
     """Weights -> (Wq, w_scale, Wo, wo_scale), allocated on W's device.
@@ -262,12 +300,17 @@ class QuikLinear:
     ``QuikLinear(W, perm, k_o, group, outlier_int8, bias, act_bits, weight_bits)``
     packs W once (quik_pack_weights); calling it on fp16 activations runs
     quik_linear into a workspace it keeps.  act_bits / weight_bits 8 quantise
-    the activations / weights to INT8.
+    the activations / weights to INT8.  With ``norm_weight`` (fp16 [K]) the
+    layer takes the hidden state before an RMS norm (weight norm_weight,
+    epsilon norm_eps) and runs quik_rmsnorm_linear: the norm is folded into
+    the activation quantiser.
     """
 
     def __init__(self, W: torch.Tensor, perm: torch.Tensor, k_o: int, group: int = 0,
                  outlier_int8: bool = False, bias: torch.Tensor | None = None, act_bits: int = 4,
-                 weight_bits: int = 4):
+                 weight_bits: int = 4, norm_weight: torch.Tensor | None = None,
+                 norm_eps: float = 1e-6):
+        self.norm_weight, self.norm_eps = norm_weight, norm_eps
         self.N, self.K = W.shape
         self.k_o, self.group, self.outlier_int8 = k_o, group, outlier_int8
         self.act_bits, self.weight_bits = act_bits, weight_bits
@@ -292,6 +335,11 @@ class QuikLinear:
     def __call__(self, X: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
         M = X.shape[0]
         Y = out if out is not None else torch.empty((M, self.N), dtype=torch.float16, device=X.device)
-        quik_linear(self.shape(M), X, self.perm, self.Wq, self.w_scale, self.Wo, self.wo_scale,
-                    self.bias, Y, self.workspace(M, X.device), stream=stream)
+        if self.norm_weight is not None:
+            quik_rmsnorm_linear(self.shape(M), X, self.norm_weight, self.norm_eps, self.perm, self.Wq,
+                                self.w_scale, self.Wo, self.wo_scale, self.bias, Y,
+                                self.workspace(M, X.device), stream=stream)
+        else:
+            quik_linear(self.shape(M), X, self.perm, self.Wq, self.w_scale, self.Wo, self.wo_scale,
+                        self.bias, Y, self.workspace(M, X.device), stream=stream)
         return Y

@@ -1,6 +1,7 @@
 // api.cu -- the extern "C" entry points declared in include/quik.h:
 // argument validation, workspace layout and kernel dispatch.  No device
 // memory is allocated here; every buffer belongs to the caller.
+#include <cmath>
 #include <cstdint>
 
 #include "quik_internal.h"
@@ -9,6 +10,7 @@ namespace {
 
 using quik::kGroup;
 using quik::kMaxK;
+using quik::kMaxKNorm;
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool ok_ptr(const void *p) { return p != nullptr && aligned16(p); }
@@ -55,8 +57,10 @@ quik_status check_quant_ptrs(const quik_shape *s, const void *Q, const float *sc
 }
 
 // bits8: INT8 codes (activations with act_bits 8, weights with weight_bits 8).
+// gamma (optional): the rows are RMS-normalised with this weight and eps first.
 quik_status quantize(const quik_shape *s, int rows, bool bits8, const void *X, const int32_t *perm,
-                     void *Q, float *scale, void *O, float *o_scale, cudaStream_t stream) {
+                     void *Q, float *scale, void *O, float *o_scale, cudaStream_t stream,
+                     const void *gamma = nullptr, float eps = 0.0f) {
     quik::QuantizeArgs a;
     a.X = static_cast<const uint16_t *>(X);
     a.perm = perm;
@@ -70,7 +74,14 @@ quik_status quantize(const quik_shape *s, int rows, bool bits8, const void *X, c
     a.scale = scale;
     a.O = O;
     a.o_scale = o_scale;
+    a.gamma = static_cast<const uint16_t *>(gamma);
+    a.eps = eps;
     return quik::launch_quantize_rows(a, stream) == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
+}
+
+// The RMS norm's weight and epsilon: gamma [K] fp16, eps finite and > 0.
+inline bool ok_norm(const void *gamma, float eps) {
+    return ok_ptr(gamma) && std::isfinite(eps) && eps > 0.0f;
 }
 
 struct Workspace {
@@ -108,6 +119,19 @@ quik_status quik_quantize_reorder(const quik_shape *shape, const void *X_f16, co
     if ((st = check_quant_ptrs(shape, Xq, x_scale, Xo, xo_scale)) != QUIK_OK) return st;
     return quantize(shape, shape->M, act8(shape), X_f16, perm, Xq, x_scale, Xo, xo_scale,
                     static_cast<cudaStream_t>(stream));
+}
+
+quik_status quik_rmsnorm_quantize_reorder(const quik_shape *shape, const void *X_f16,
+                                          const void *gamma_f16, float eps, const int32_t *perm,
+                                          void *Xq, float *x_scale, void *Xo, float *xo_scale,
+                                          quik_stream_t stream) {
+    quik_status st = check_shape(shape);
+    if (st != QUIK_OK) return st;
+    if (!ok_ptr(X_f16) || !ok_ptr(perm) || !ok_norm(gamma_f16, eps)) return QUIK_ERR_INVALID_ARG;
+    if ((st = check_quant_ptrs(shape, Xq, x_scale, Xo, xo_scale)) != QUIK_OK) return st;
+    if (shape->K > kMaxKNorm) return QUIK_ERR_UNSUPPORTED;
+    return quantize(shape, shape->M, act8(shape), X_f16, perm, Xq, x_scale, Xo, xo_scale,
+                    static_cast<cudaStream_t>(stream), gamma_f16, eps);
 }
 
 quik_status quik_pack_weights(const quik_shape *shape, const void *W_f16, const int32_t *perm,
@@ -165,14 +189,17 @@ quik_status quik_gemm(const quik_shape *shape, const void *Xq, const float *x_sc
                      false, nullptr, nullptr, static_cast<cudaStream_t>(stream));
 }
 
-quik_status quik_linear(const quik_shape *shape, const void *X_f16, const int32_t *perm,
-                        const void *Wq, const float *w_scale, const void *Wo,
-                        const float *wo_scale, const void *bias_f16, void *Y_f16,
-                        void *workspace, size_t workspace_bytes, quik_stream_t stream) {
+static quik_status linear_impl(const quik_shape *shape, const void *X_f16, const void *gamma,
+                               float eps, const int32_t *perm, const void *Wq,
+                               const float *w_scale, const void *Wo, const float *wo_scale,
+                               const void *bias_f16, void *Y_f16, void *workspace,
+                               size_t workspace_bytes, quik_stream_t stream) {
     quik_status st = check_shape(shape);
     if (st != QUIK_OK) return st;
     if (!ok_ptr(X_f16) || !ok_ptr(perm) || !ok_ptr(Y_f16) || !ok_opt(bias_f16))
         return QUIK_ERR_INVALID_ARG;
+    if (gamma != nullptr && !ok_norm(gamma, eps)) return QUIK_ERR_INVALID_ARG;
+    if (gamma != nullptr && shape->K > kMaxKNorm) return QUIK_ERR_UNSUPPORTED;
     if ((st = check_quant_ptrs(shape, Wq, w_scale, Wo, wo_scale)) != QUIK_OK) return st;
     const Workspace w = layout(shape);
     if (!ok_ptr(workspace) || workspace_bytes < w.total) return QUIK_ERR_INVALID_ARG;
@@ -182,12 +209,31 @@ quik_status quik_linear(const quik_shape *shape, const void *X_f16, const int32_
     void *Xo = ws + w.xo;
     float *sxo = int8_out(shape) ? reinterpret_cast<float *>(ws + w.sxo) : nullptr;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if ((st = quantize(shape, shape->M, act8(shape), X_f16, perm, Xq, sx, Xo, sxo, s)) != QUIK_OK)
+    if ((st = quantize(shape, shape->M, act8(shape), X_f16, perm, Xq, sx, Xo, sxo, s, gamma, eps)) !=
+        QUIK_OK)
         return st;
     // the GEMM follows this quantiser on the same stream: its set-up and weight
     // loads may overlap the quantiser's tail
     return gemm_impl(shape, Xq, sx, Xo, sxo, Wq, w_scale, Wo, wo_scale, bias_f16, Y_f16, false,
                      nullptr, nullptr, s, true);
+}
+
+quik_status quik_linear(const quik_shape *shape, const void *X_f16, const int32_t *perm,
+                        const void *Wq, const float *w_scale, const void *Wo,
+                        const float *wo_scale, const void *bias_f16, void *Y_f16,
+                        void *workspace, size_t workspace_bytes, quik_stream_t stream) {
+    return linear_impl(shape, X_f16, nullptr, 0.0f, perm, Wq, w_scale, Wo, wo_scale, bias_f16,
+                       Y_f16, workspace, workspace_bytes, stream);
+}
+
+quik_status quik_rmsnorm_linear(const quik_shape *shape, const void *X_f16, const void *gamma_f16,
+                                float eps, const int32_t *perm, const void *Wq,
+                                const float *w_scale, const void *Wo, const float *wo_scale,
+                                const void *bias_f16, void *Y_f16, void *workspace,
+                                size_t workspace_bytes, quik_stream_t stream) {
+    if (gamma_f16 == nullptr) return QUIK_ERR_INVALID_ARG;
+    return linear_impl(shape, X_f16, gamma_f16, eps, perm, Wq, w_scale, Wo, wo_scale, bias_f16,
+                       Y_f16, workspace, workspace_bytes, stream);
 }
 
 quik_status quik_gemm_i32_debug(const quik_shape *shape, const void *Xq, const void *Wq,

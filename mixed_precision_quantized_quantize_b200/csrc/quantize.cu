@@ -74,6 +74,8 @@ struct QParams {
     void *O;
     float *o_scale;
     int bits8;  // per-token rows only: INT8 codes (one byte each, divisor 127)
+    const uint16_t *gamma;  // RMS-norm weight [K] in source channel order (NORM kernels only)
+    float eps;              // RMS-norm epsilon (NORM kernels only)
 };
 
 __device__ __forceinline__ float h2f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
@@ -89,9 +91,9 @@ constexpr uint32_t kRoundBits = 0x4B400000u;
 // b_k = 0x4B400000 + q_k the constant term is folded in advance (mod 2^32).
 constexpr uint32_t kPackBias = 0x88888888u - kRoundBits * 0x11111111u;
 
-// fl(m / D) for an odd divisor 2^(L-1) < D < 2^L and m >= 0 an fp16 value
-// widened to fp32 (so m == 0 or m is a normal fp32 with at most 11
-// significant bits).  With m = S 2^(E-150), S the 24-bit significand, the
+// fl(m / D) for an odd divisor 2^(L-1) < D < 2^L and m >= 0 zero or a
+// normal fp32 (an fp16 value widened, or with the fused norm a product of two
+// fp16 values, at least 2^-48).  With m = S 2^(E-150), S the 24-bit significand, the
 // quotient's 24-bit significand is the integer nearest to S 2^sh / D for the
 // shift sh in {L-1, L} that puts it in [2^23, 2^24]; the rounding is exact
 // integer arithmetic and never meets a tie (2 * remainder is even, D odd).
@@ -149,7 +151,24 @@ __device__ __forceinline__ int exact_code(float v, float s, int qmax) {
     return max(-qmax, min(qmax, q));
 }
 
-// Eight codes of one 32-bit output word from four half2 values.
+// The eight values of one word, as fp32: four half2 (widened exactly) or
+// four fp32 pairs (the products h * gamma of the fused norm).
+__device__ __forceinline__ uint64_t pair_f32(const uint32_t (&h)[4], int k) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[k]));
+    return f2(f.x, f.y);
+}
+__device__ __forceinline__ uint64_t pair_f32(const uint64_t (&z)[4], int k) { return z[k]; }
+__device__ __forceinline__ float value_f32(const uint32_t (&h)[4], int k, int hi) {
+    return h2f(static_cast<uint16_t>(hi ? h[k] >> 16 : h[k] & 0xffffu));
+}
+__device__ __forceinline__ float value_f32(const uint64_t (&z)[4], int k, int hi) {
+    float a, b;
+    f2_split(z[k], a, b);
+    return hi ? b : a;
+}
+
+// Eight codes of one 32-bit output word from four half2 values (or four
+// fp32 pairs).
 //   Fast path: r = rint(v * rs) of the exact product (one fused
 //   multiply-add with 1.5 * 2^23), rs the hardware reciprocal of s (relative
 //   error <= 2u, u = 2^-24).  |v rs - fl(v/s)| <= |v/s| 3u <= 1.3e-6 for
@@ -158,14 +177,14 @@ __device__ __forceinline__ int exact_code(float v, float s, int qmax) {
 //   to r as well.  The residual v rs - r comes from a second fused
 //   multiply-add (relative error u), and a word with any near-tie is redone
 //   with IEEE divisions.  No clamp is needed: |r| <= 7.
-__device__ __forceinline__ uint32_t pack_codes8(const uint32_t (&h)[4], float s, float rs) {
+template <typename V>
+__device__ __forceinline__ uint32_t pack_codes8(const V &h, float s, float rs) {
     uint32_t word = kPackBias;
     float dmax = 0.0f;
     const uint64_t rs2 = f2(rs, rs), kr2 = f2(kRound, kRound);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[k]));
-        const uint64_t v2 = f2(f.x, f.y);
+        const uint64_t v2 = pair_f32(h, k);
         const uint64_t m = f2_fma(v2, rs2, kr2);           // 1.5*2^23 + rint(v rs)
         const uint64_t r = f2_sub(m, kr2);                 // rint(v rs), exact
         float r0, r1;
@@ -182,8 +201,8 @@ __device__ __forceinline__ uint32_t pack_codes8(const uint32_t (&h)[4], float s,
         word = 0x88888888u;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const int q0 = exact_code(h2f(static_cast<uint16_t>(h[k] & 0xffffu)), s, 7);
-            const int q1 = exact_code(h2f(static_cast<uint16_t>(h[k] >> 16)), s, 7);
+            const int q0 = exact_code(value_f32(h, k, 0), s, 7);
+            const int q1 = exact_code(value_f32(h, k, 1), s, 7);
             word += static_cast<uint32_t>(q0) << (8 * k);
             word += static_cast<uint32_t>(q1) << (8 * k + 4);
         }
@@ -192,16 +211,16 @@ __device__ __forceinline__ uint32_t pack_codes8(const uint32_t (&h)[4], float s,
 }
 
 // Eight INT8 codes, one byte each in position order, from four half2 values
-// (W4A8 activations): the fast path below for every value, and IEEE
-// divisions for a word with any near-tie.
-__device__ __forceinline__ uint2 pack_codes8_i8(const uint32_t (&h)[4], float s, float rs) {
+// (W4A8 activations; or four fp32 pairs): the fast path below for every
+// value, and IEEE divisions for a word with any near-tie.
+template <typename V>
+__device__ __forceinline__ uint2 pack_codes8_i8(const V &h, float s, float rs) {
     uint32_t q[8];
     float dmax = 0.0f;
     const uint64_t rs2 = f2(rs, rs), kr2 = f2(kRound, kRound);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[k]));
-        const uint64_t v2 = f2(f.x, f.y);
+        const uint64_t v2 = pair_f32(h, k);
         const uint64_t m = f2_fma(v2, rs2, kr2);           // 1.5*2^23 + rint(v rs)
         const uint64_t r = f2_sub(m, kr2);
         float r0, r1;
@@ -217,8 +236,8 @@ __device__ __forceinline__ uint2 pack_codes8_i8(const uint32_t (&h)[4], float s,
     if (dmax > 0.5f - 4e-5f) {  // near a tie somewhere in this word: exact divisions
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            q[2 * k] = static_cast<uint32_t>(exact_code(h2f(static_cast<uint16_t>(h[k] & 0xffffu)), s, 127));
-            q[2 * k + 1] = static_cast<uint32_t>(exact_code(h2f(static_cast<uint16_t>(h[k] >> 16)), s, 127));
+            q[2 * k] = static_cast<uint32_t>(exact_code(value_f32(h, k, 0), s, 127));
+            q[2 * k + 1] = static_cast<uint32_t>(exact_code(value_f32(h, k, 1), s, 127));
         }
     }
     // low byte of each code, in order
@@ -239,6 +258,39 @@ __device__ __forceinline__ int code8(float v, float s, float rs) {
     const float r = __fsub_rn(m, kRound);
     if (fabsf(__fmaf_rn(v, rs, -r)) > 0.5f - 4e-5f) return exact_code(v, s, 127);
     return static_cast<int>(__float_as_uint(m) - kRoundBits);
+}
+
+// z = h * gamma for the eight values of one word (h: four half2 of the row,
+// gamma: the word's eight reordered norm weights).  A product of two fp16
+// values has at most 22 significant bits and lies within fp32's normal
+// range, so every z is exact.
+__device__ __forceinline__ void norm_products(const uint32_t (&h)[4], uint4 g, uint64_t (&z)[4]) {
+    const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float2 gf = __half22float2(*reinterpret_cast<const __half2 *>(&gw[k]));
+        z[k] = ptx::f2_mul(pair_f32(h, k), f2(gf.x, gf.y));
+    }
+}
+
+__device__ __forceinline__ double warp_sum(double t) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    return t;
+}
+
+// The RMS norm's row factor 1 / sqrt(ss / K + eps) in fp64, each step IEEE
+// rounded.  ss is summed in fp64 from exact squares, so r is within a few
+// fp64 ulps of its exact value and the fp32 scales and fp16 outliers that
+// carry it are rounded as from the exact factor (except within ~1e-15 of a
+// rounding boundary).
+__device__ __forceinline__ double rms_factor(double ss, int K, float eps) {
+    return __drcp_rn(__dsqrt_rn(__dadd_rn(__ddiv_rn(ss, static_cast<double>(K)),
+                                          static_cast<double>(eps))));
+}
+// fl32(s * r) and fl16(z * r): one fp64 product, rounded once.
+__device__ __forceinline__ float times_r(float s, double r) {
+    return __double2float_rn(__dmul_rn(static_cast<double>(s), r));
 }
 
 __device__ __forceinline__ float warp_max(float m) {
@@ -271,11 +323,18 @@ __device__ __forceinline__ void team_sync(int id, int nthreads) {
 }
 
 // P32: the perm table holds byte offsets (uint32); else element indices (uint16).
-template <bool GROUPED, bool OUT_INT8, int W, bool P32>
-__global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : GROUPED ? 64 : 56)
+// NORM: the rows are first RMS-normalised with weight p.gamma and p.eps (the
+// norm in front of a projection, with this quantiser folded into it: Atom,
+// idea I2).  The row factor r = 1/sqrt(mean(h^2) + eps) changes no code, so
+// codes and base scales are those of z = h * gamma (exact in fp32) and r
+// multiplies the stored scales and the FP16 outliers.  A second shared table
+// holds gamma in reordered order; the sum of squares is gathered alongside.
+template <bool GROUPED, bool OUT_INT8, int W, bool P32, bool NORM>
+__global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : (GROUPED && NORM) ? 96 : (GROUPED || NORM) ? 64 : 56)
     quantize_rows_kernel(QParams p) {
     extern __shared__ __align__(16) uint8_t qsmem[];
     __shared__ float red[kQMaxTeams][2][kQMaxThreads / 32];  // warp maxima, two slots per team
+    __shared__ double red_ss[kQMaxTeams][2][kQMaxThreads / 32];  // warp sums of squares (NORM)
     __shared__ uint64_t row_full[kQMaxTeams][kQMaxRing];
     const int K = p.K, Ki = K - p.k_o;  // K % 16 == 0
     const int TT = p.team_threads;
@@ -286,10 +345,13 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : GROUPE
     const int G = GROUPED ? Ki / kGroup : 1;
     const uint32_t row_bytes = static_cast<uint32_t>(K) * 2;
     const uint32_t perm_bytes = P32 ? row_bytes * 2 : row_bytes;
+    // the reordered norm weights (fp16 [K]) follow the perm table
+    const uint32_t tab_bytes = perm_bytes + (NORM ? row_bytes : 0u);
+    const uint16_t *gtab = reinterpret_cast<const uint16_t *>(qsmem + perm_bytes);
     const int stride = gridDim.x * p.teams;  // rows between a team's consecutive rows
     const int first = blockIdx.x * p.teams + team;
     const int NR = p.ring;
-    auto slot_off = [&](int t, int j) { return perm_bytes + (t * NR + j % NR) * row_bytes; };
+    auto slot_off = [&](int t, int j) { return tab_bytes + (t * NR + j % NR) * row_bytes; };
     auto issue = [&](int t, int j) {  // bulk-copy team t's j-th row into its slot j % NR
         const int row = blockIdx.x * p.teams + t + j * stride;
         if (row < p.rows) {
@@ -342,6 +404,12 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : GROUPE
                 reinterpret_cast<uint4 *>(qsmem)[i] = make_uint4(2 * e[0], 2 * e[1], 2 * e[2], 2 * e[3]);
             else
                 reinterpret_cast<uint2 *>(qsmem)[i] = make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16));
+            if (NORM) {
+                uint32_t g[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) g[c] = __ldg(p.gamma + e[c]);
+                reinterpret_cast<uint2 *>(qsmem + perm_bytes)[i] = make_uint2(g[0] | (g[1] << 16), g[2] | (g[3] << 16));
+            }
         }
         if (bad && blockIdx.x == 0) atomicAdd(&g_quant_bad_perm, 1u);
     }
@@ -379,8 +447,10 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : GROUPE
         };
 
         // (2) gather 8 reordered values per word (as 4 half2), absmax per word
+        // (of h * gamma with the norm, whose sum of squares of h is gathered too)
         uint32_t v[W][4];
         float wmax[W];
+        double ss = 0.0;  // sum of h^2 (NORM), fp64 from exact fp32 squares
 #pragma unroll
         for (int i = 0; i < W; ++i) {
             const int w = tl + i * TT;
@@ -403,7 +473,42 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : GROUPE
                 }
 #pragma unroll
                 for (int k = 0; k < 4; ++k) v[i][k] = pair16(at(off[2 * k]), at(off[2 * k + 1]));
-                wmax[i] = half2_absmax(absmax2(absmax2(v[i][0], v[i][1]), absmax2(v[i][2], v[i][3])));
+                if (NORM) {
+                    uint64_t z[4];
+                    norm_products(v[i], reinterpret_cast<const uint4 *>(gtab)[w], z);
+                    float a = 0.0f;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t hk = pair_f32(v[i], k);
+                        float q0, q1;
+                        f2_split(ptx::f2_mul(hk, hk), q0, q1);  // exact: 22 significant bits
+                        ss += static_cast<double>(q0);
+                        ss += static_cast<double>(q1);
+                        float z0, z1;
+                        f2_split(z[k], z0, z1);
+                        a = max3(a, fabsf(z0), fabsf(z1));
+                    }
+                    wmax[i] = a;
+                } else {
+                    wmax[i] = half2_absmax(absmax2(absmax2(v[i][0], v[i][1]), absmax2(v[i][2], v[i][3])));
+                }
+            }
+        }
+        // the norm's row factor: the sum of squares runs over every channel,
+        // the outlier block included
+        double rn = 1.0;
+        if (NORM) {
+            for (int i = tl; i < p.k_o; i += TT) {
+                const float h = h2f(static_cast<uint16_t>(at(element(Ki + i))));
+                ss += static_cast<double>(__fmul_rn(h, h));
+            }
+            ss = warp_sum(ss);
+            if (GROUPED) {  // the per-token path below shares the max's barrier
+                if (lane == 0) red_ss[team][j & 1][twarp] = ss;
+                team_sync(bar_id, TT);
+                ss = 0.0;
+                for (int k = 0; k < (TT >> 5); ++k) ss += red_ss[team][j & 1][k];
+                rn = rms_factor(ss, K, p.eps);
             }
         }
 
@@ -419,24 +524,32 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : GROUPE
                 r[i] = rcp_approx(s[i]);
                 const int w = tl + i * TT;
                 if (w < nwords && (lane & 15) == 0 && QUIK_CHECK(w / 16 < G, 3))
-                    p.scale[static_cast<size_t>(row) * G + w / 16] = s[i];
+                    p.scale[static_cast<size_t>(row) * G + w / 16] = NORM ? times_r(s[i], rn) : s[i];
             }
         } else {
             float m = 0.0f;
 #pragma unroll
             for (int i = 0; i < W; ++i) m = fmaxf(m, wmax[i]);
             m = warp_max(m);
-            if (lane == 0) red[team][j & 1][twarp] = m;
+            if (lane == 0) {
+                red[team][j & 1][twarp] = m;
+                if (NORM) red_ss[team][j & 1][twarp] = ss;
+            }
             team_sync(bar_id, TT);
             m = 0.0f;
             for (int k = 0; k < (TT >> 5); ++k) m = fmaxf(m, red[team][j & 1][k]);
+            if (NORM) {
+                ss = 0.0;
+                for (int k = 0; k < (TT >> 5); ++k) ss += red_ss[team][j & 1][k];
+                rn = rms_factor(ss, K, p.eps);
+            }
             const float sr = p.bits8 ? div_exact<127, 7>(m) : div_exact<7, 3>(m), rr = rcp_approx(sr);
 #pragma unroll
             for (int i = 0; i < W; ++i) {
                 s[i] = sr;
                 r[i] = rr;
             }
-            if (tl == 0) p.scale[row] = sr;
+            if (tl == 0) p.scale[row] = NORM ? times_r(sr, rn) : sr;
         }
 
         // (4) codes, 8 per word, code 2i in the low nibble of byte i (or one
@@ -446,14 +559,30 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : GROUPE
 #pragma unroll
             for (int i = 0; i < W; ++i) {
                 const int w = tl + i * TT;
-                if (w < nwords && QUIK_CHECK(8 * w + 8 <= Ki, 4)) qrow8[w] = pack_codes8_i8(v[i], s[i], r[i]);
+                if (w < nwords && QUIK_CHECK(8 * w + 8 <= Ki, 4)) {
+                    if (NORM) {
+                        uint64_t z[4];
+                        norm_products(v[i], reinterpret_cast<const uint4 *>(gtab)[w], z);
+                        qrow8[w] = pack_codes8_i8(z, s[i], r[i]);
+                    } else {
+                        qrow8[w] = pack_codes8_i8(v[i], s[i], r[i]);
+                    }
+                }
             }
         } else {
             uint32_t *qrow = reinterpret_cast<uint32_t *>(p.Q + static_cast<size_t>(row) * (Ki / 2));
 #pragma unroll
             for (int i = 0; i < W; ++i) {
                 const int w = tl + i * TT;
-                if (w < nwords && QUIK_CHECK(4 * w + 4 <= Ki / 2, 4)) qrow[w] = pack_codes8(v[i], s[i], r[i]);
+                if (w < nwords && QUIK_CHECK(4 * w + 4 <= Ki / 2, 4)) {
+                    if (NORM) {
+                        uint64_t z[4];
+                        norm_products(v[i], reinterpret_cast<const uint4 *>(gtab)[w], z);
+                        qrow[w] = pack_codes8(z, s[i], r[i]);
+                    } else {
+                        qrow[w] = pack_codes8(v[i], s[i], r[i]);
+                    }
+                }
             }
         }
 
@@ -461,12 +590,23 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : GROUPE
         if (p.k_o > 0) {
             if (!OUT_INT8) {
                 uint16_t *o = static_cast<uint16_t *>(p.O) + static_cast<size_t>(row) * p.k_o;
-                for (int i = tl; i < p.k_o; i += TT)
-                    o[i] = static_cast<uint16_t>(at(element(Ki + i)));
+                for (int i = tl; i < p.k_o; i += TT) {
+                    if (NORM) {  // fl16(h * gamma * r), the product in fp64
+                        const float z = __fmul_rn(h2f(static_cast<uint16_t>(at(element(Ki + i)))),
+                                                  h2f(gtab[Ki + i]));
+                        o[i] = __half_as_ushort(__double2half(__dmul_rn(static_cast<double>(z), rn)));
+                    } else {
+                        o[i] = static_cast<uint16_t>(at(element(Ki + i)));
+                    }
+                }
             } else {
+                // the outlier values (times gamma with the norm: exact)
+                auto ov = [&](int i) -> float {
+                    const float h = h2f(static_cast<uint16_t>(at(element(Ki + i))));
+                    return NORM ? __fmul_rn(h, h2f(gtab[Ki + i])) : h;
+                };
                 float m = 0.0f;
-                for (int i = tl; i < p.k_o; i += TT)
-                    m = fmaxf(m, fabsf(h2f(static_cast<uint16_t>(at(element(Ki + i))))));
+                for (int i = tl; i < p.k_o; i += TT) m = fmaxf(m, fabsf(ov(i)));
                 m = warp_max(m);
                 // the other reduction slot: this row's slot is read above and
                 // is not written again before the next row's opening barrier
@@ -475,11 +615,9 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : GROUPE
                 m = 0.0f;
                 for (int k = 0; k < (TT >> 5); ++k) m = fmaxf(m, red[team][(j & 1) ^ 1][k]);
                 const float so = div_exact<127, 7>(m), rso = rcp_approx(so);
-                if (tl == 0) p.o_scale[row] = so;
+                if (tl == 0) p.o_scale[row] = NORM ? times_r(so, rn) : so;
                 int8_t *o = static_cast<int8_t *>(p.O) + static_cast<size_t>(row) * p.k_o;
-                for (int i = tl; i < p.k_o; i += TT)
-                    o[i] = static_cast<int8_t>(
-                        code8(h2f(static_cast<uint16_t>(at(element(Ki + i)))), so, rso));
+                for (int i = tl; i < p.k_o; i += TT) o[i] = static_cast<int8_t>(code8(ov(i), so, rso));
             }
         } else if (OUT_INT8 && p.o_scale != nullptr && tl == 0) {
             p.o_scale[row] = 0.0f;
@@ -498,18 +636,23 @@ struct QShape {
     size_t smem;
 };
 
-// Registers per thread of one kernel instance (queried once).
-template <bool GROUPED, bool OUT_INT8, int W, bool P32>
-int q_regs() {
+// Registers per thread of one kernel instance (queried once), and the
+// static shared memory it holds beyond the 1 KB that ctas_per_sm assumes.
+template <bool GROUPED, bool OUT_INT8, int W, bool P32, bool NORM>
+int q_regs(size_t *extra_static = nullptr) {
     static std::atomic<int> regs{0};
+    static std::atomic<int> extra{0};
     int r = regs.load(std::memory_order_relaxed);
     if (r == 0) {
         cudaFuncAttributes fa{};
-        if (cudaFuncGetAttributes(&fa, quantize_rows_kernel<GROUPED, OUT_INT8, W, P32>) != cudaSuccess)
+        if (cudaFuncGetAttributes(&fa, quantize_rows_kernel<GROUPED, OUT_INT8, W, P32, NORM>) != cudaSuccess)
             return 0;
+        extra.store(fa.sharedSizeBytes > 1024 ? static_cast<int>(fa.sharedSizeBytes - 1024) : 0,
+                    std::memory_order_relaxed);
         r = fa.numRegs;
         regs.store(r, std::memory_order_relaxed);
     }
+    if (extra_static != nullptr) *extra_static = static_cast<size_t>(extra.load(std::memory_order_relaxed));
     return r;
 }
 
@@ -533,8 +676,10 @@ int ctas_per_sm(int threads, int regs, size_t smem) {
 // W = 8 (K_i <= 32768).  Then teams per CTA (at most 4 and 512 threads), row
 // slots per team (2 .. 4) and the perm table's width (uint32 byte offsets, or
 // uint16 indices with an extraction per element) are chosen for the most
-// teams per SM; ties go to the uint32 table, then to more slots.
-template <bool GROUPED, bool OUT_INT8>
+// teams per SM; ties go to the uint32 table, then to more slots.  With the
+// fused norm a second table (the reordered norm weights, one row's size)
+// shares the shared memory.
+template <bool GROUPED, bool OUT_INT8, bool NORM>
 QShape q_shape(int rows, int K, int k_o) {
     const int nwords = (K - k_o) / 8;
     int W;
@@ -548,18 +693,19 @@ QShape q_shape(int rows, int K, int k_o) {
     int best_score = -1;
     for (int p32 = 1; p32 >= 0; --p32) {
         int regs = 0;
+        size_t xs = 0;  // static shared memory past 1 KB
         switch (W) {
-            case 1: regs = p32 ? q_regs<GROUPED, OUT_INT8, 1, true>() : q_regs<GROUPED, OUT_INT8, 1, false>(); break;
-            case 2: regs = p32 ? q_regs<GROUPED, OUT_INT8, 2, true>() : q_regs<GROUPED, OUT_INT8, 2, false>(); break;
-            case 4: regs = p32 ? q_regs<GROUPED, OUT_INT8, 4, true>() : q_regs<GROUPED, OUT_INT8, 4, false>(); break;
-            default: regs = p32 ? q_regs<GROUPED, OUT_INT8, 8, true>() : q_regs<GROUPED, OUT_INT8, 8, false>(); break;
+            case 1: regs = p32 ? q_regs<GROUPED, OUT_INT8, 1, true, NORM>(&xs) : q_regs<GROUPED, OUT_INT8, 1, false, NORM>(&xs); break;
+            case 2: regs = p32 ? q_regs<GROUPED, OUT_INT8, 2, true, NORM>(&xs) : q_regs<GROUPED, OUT_INT8, 2, false, NORM>(&xs); break;
+            case 4: regs = p32 ? q_regs<GROUPED, OUT_INT8, 4, true, NORM>(&xs) : q_regs<GROUPED, OUT_INT8, 4, false, NORM>(&xs); break;
+            default: regs = p32 ? q_regs<GROUPED, OUT_INT8, 8, true, NORM>(&xs) : q_regs<GROUPED, OUT_INT8, 8, false, NORM>(&xs); break;
         }
-        const size_t table = p32 ? 2 * row : row;
+        const size_t table = (p32 ? 2 * row : row) + (NORM ? row : 0);
         for (int teams = std::min(kQMaxTeams, kQMaxThreads / TT); teams >= 1; --teams)
             for (int ring = kQMaxRing; ring >= 2; --ring) {
                 const size_t smem = table + static_cast<size_t>(teams) * ring * row;
-                if (smem > (227u << 10) - 1024) continue;
-                const int per_sm = ctas_per_sm(TT * teams, regs, smem);
+                if (smem + xs > (227u << 10) - 1024) continue;
+                const int per_sm = ctas_per_sm(TT * teams, regs, smem + xs);
                 if (per_sm == 0) continue;
                 // teams per SM first; then the wider table; then deeper rings
                 const int score = (per_sm * teams) * 16 + p32 * 8 + ring;
@@ -572,9 +718,9 @@ QShape q_shape(int rows, int K, int k_o) {
     return best;
 }
 
-template <bool GROUPED, bool OUT_INT8, int W, bool P32>
+template <bool GROUPED, bool OUT_INT8, int W, bool P32, bool NORM>
 cudaError_t launch_q(QParams p, const QShape &qs, cudaStream_t stream) {
-    auto kern = quantize_rows_kernel<GROUPED, OUT_INT8, W, P32>;
+    auto kern = quantize_rows_kernel<GROUPED, OUT_INT8, W, P32, NORM>;
     p.team_threads = qs.TT;
     p.teams = qs.teams;
     p.ring = qs.ring;
@@ -584,7 +730,8 @@ cudaError_t launch_q(QParams p, const QShape &qs, cudaStream_t stream) {
         return cudaErrorInvalidConfiguration;
     if (!attribute_set_once(reinterpret_cast<const void *>(kern), static_cast<int>(qs.smem)))
         return cudaErrorInvalidConfiguration;
-    const int per_sm = ctas_per_sm(threads, q_regs<GROUPED, OUT_INT8, W, P32>(), qs.smem);
+    size_t xs = 0;
+    const int per_sm = ctas_per_sm(threads, q_regs<GROUPED, OUT_INT8, W, P32, NORM>(&xs), qs.smem + xs);
     // grid: every CTA that fits at once (persistent), or fewer when the rows run out
     const int need = (p.rows + qs.teams - 1) / qs.teams;
     const int grid = std::max(1, std::min(need, sm_count() * std::max(per_sm, 1)));
@@ -592,29 +739,36 @@ cudaError_t launch_q(QParams p, const QShape &qs, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-template <bool GROUPED, bool OUT_INT8>
+template <bool GROUPED, bool OUT_INT8, bool NORM>
 cudaError_t launch_q_w(const QParams &p, cudaStream_t stream) {
-    const QShape qs = q_shape<GROUPED, OUT_INT8>(p.rows, p.K, p.k_o);
+    const QShape qs = q_shape<GROUPED, OUT_INT8, NORM>(p.rows, p.K, p.k_o);
     switch (qs.W * 2 + (qs.p32 ? 1 : 0)) {
-        case 3: return launch_q<GROUPED, OUT_INT8, 1, true>(p, qs, stream);
-        case 2: return launch_q<GROUPED, OUT_INT8, 1, false>(p, qs, stream);
-        case 5: return launch_q<GROUPED, OUT_INT8, 2, true>(p, qs, stream);
-        case 4: return launch_q<GROUPED, OUT_INT8, 2, false>(p, qs, stream);
-        case 9: return launch_q<GROUPED, OUT_INT8, 4, true>(p, qs, stream);
-        case 8: return launch_q<GROUPED, OUT_INT8, 4, false>(p, qs, stream);
-        case 17: return launch_q<GROUPED, OUT_INT8, 8, true>(p, qs, stream);
-        default: return launch_q<GROUPED, OUT_INT8, 8, false>(p, qs, stream);
+        case 3: return launch_q<GROUPED, OUT_INT8, 1, true, NORM>(p, qs, stream);
+        case 2: return launch_q<GROUPED, OUT_INT8, 1, false, NORM>(p, qs, stream);
+        case 5: return launch_q<GROUPED, OUT_INT8, 2, true, NORM>(p, qs, stream);
+        case 4: return launch_q<GROUPED, OUT_INT8, 2, false, NORM>(p, qs, stream);
+        case 9: return launch_q<GROUPED, OUT_INT8, 4, true, NORM>(p, qs, stream);
+        case 8: return launch_q<GROUPED, OUT_INT8, 4, false, NORM>(p, qs, stream);
+        case 17: return launch_q<GROUPED, OUT_INT8, 8, true, NORM>(p, qs, stream);
+        default: return launch_q<GROUPED, OUT_INT8, 8, false, NORM>(p, qs, stream);
     }
+}
+
+template <bool NORM>
+cudaError_t launch_q_n(const QParams &p, int group, bool out_int8, cudaStream_t stream) {
+    if (group > 0)
+        return out_int8 ? launch_q_w<true, true, NORM>(p, stream) : launch_q_w<true, false, NORM>(p, stream);
+    return out_int8 ? launch_q_w<false, true, NORM>(p, stream) : launch_q_w<false, false, NORM>(p, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_quantize_rows(const QuantizeArgs &a, cudaStream_t stream) {
-    QParams p{a.X, a.perm, a.rows, a.K, a.k_o, 0, 0, 0, a.Q, a.scale, a.O, a.o_scale, a.bits8 ? 1 : 0};
+    QParams p{a.X, a.perm, a.rows, a.K, a.k_o, 0, 0, 0, a.Q, a.scale, a.O, a.o_scale, a.bits8 ? 1 : 0,
+              a.gamma, a.eps};
     if (a.bits8 && a.group > 0) return cudaErrorInvalidValue;  // INT8 codes: per-row scales only
-    if (a.group > 0)
-        return a.out_int8 ? launch_q_w<true, true>(p, stream) : launch_q_w<true, false>(p, stream);
-    return a.out_int8 ? launch_q_w<false, true>(p, stream) : launch_q_w<false, false>(p, stream);
+    if (a.gamma != nullptr) return launch_q_n<true>(p, a.group, a.out_int8, stream);
+    return launch_q_n<false>(p, a.group, a.out_int8, stream);
 }
 
 unsigned int take_quantize_errors(unsigned int *bad_perm) {

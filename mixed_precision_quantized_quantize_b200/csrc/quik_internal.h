@@ -26,6 +26,7 @@
 namespace quik {
 
 constexpr int kMaxK = 32768;       // largest K the quantiser stages in shared memory
+constexpr int kMaxKNorm = 24576;   // with the RMS norm folded in (a second K-wide table)
 constexpr int kGroup = 128;        // the one supported group width
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s bound on every in-kernel wait
 
@@ -40,6 +41,10 @@ struct QuantizeArgs {
     float *scale;
     void *O;
     float *o_scale;
+    // RMS norm folded in (NULL: none): the rows are normalised with weight
+    // gamma [K] (source channel order) and eps before they are quantised
+    const uint16_t *gamma = nullptr;
+    float eps = 0.0f;
 };
 cudaError_t launch_quantize_rows(const QuantizeArgs &a, cudaStream_t stream);
 // Read and clear the quantise kernels' count of expired waits (returned) and

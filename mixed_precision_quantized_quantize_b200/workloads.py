@@ -13,7 +13,11 @@ Llama 7B-65B); their trained weights and datasets are not used.  Values:
   which are multiplied by ``outlier_mult``; with ``student_t`` the outlier
   channels draw from a Student-t with 3 degrees of freedom instead of N(0,1)
   before the multiplication (heavy tails);
-* weights W ~ N(0, w_std^2); bias ~ N(0, 0.01^2) when present.
+* weights W ~ N(0, w_std^2); bias ~ N(0, 0.01^2) when present;
+* with an RMS norm in front of the layer (``rmsnorm``), X is the hidden state
+  before the norm: the activations above with every token row multiplied by
+  2^u, u ~ U(-2, 3) (tokens of different magnitude), and the norm weight is
+  gamma = |1 + 0.25 N(0, 1)| clamped to [0.02, 4]; eps = 1e-5.
 
 Everything is drawn on the CPU in fp32 from ``torch.Generator`` streams with
 fixed seeds and then rounded to fp16.
@@ -25,7 +29,8 @@ from dataclasses import dataclass, field
 import torch
 
 # One seed per independent stream.
-SEED_X, SEED_W, SEED_PERM, SEED_BIAS, SEED_T = 0, 1, 2, 3, 4
+SEED_X, SEED_W, SEED_PERM, SEED_BIAS, SEED_T, SEED_NORM = 0, 1, 2, 3, 4, 5
+NORM_EPS = 1e-5
 
 
 @dataclass(frozen=True)
@@ -43,6 +48,7 @@ class LayerConfig:
     bias: bool = False
     act_bits: int = 4           # 4: INT4 activations (W4A4); 8: INT8 activations (W4A8)
     weight_bits: int = 4        # 4: INT4 weights; 8: INT8 weights (W8A8)
+    rmsnorm: bool = False       # X is the hidden state before an RMS norm folded into the layer
     description: str = field(default="", compare=False)
 
     @property
@@ -100,6 +106,10 @@ CONFIGS = {
         "llama7b_attn_w8a8_2048x4096x4096", M=2048, N=4096, K=4096, k_o=128, student_t=True,
         act_bits=8, weight_bits=8,
         description="the attention projection as W8A8 (the INT8 baseline), 128 FP16 outliers"),
+    "llama7b_attn_rmsnorm_2048x4096x4096": LayerConfig(
+        "llama7b_attn_rmsnorm_2048x4096x4096", M=2048, N=4096, K=4096, k_o=128, student_t=True,
+        rmsnorm=True,
+        description="the attention projection behind its RMS norm (norm folded into the quantiser)"),
     "llama7b_down_fused_4096x4096x11008": LayerConfig(
         "llama7b_down_fused_4096x4096x11008", M=4096, N=4096, K=11008, k_o=256,
         outlier_mult=50.0, bias=True,
@@ -141,6 +151,31 @@ def make_activations(M: int, K: int, perm: torch.Tensor, k_o: int, outlier_mult:
     return x.to(torch.float16)
 
 
+def token_magnitudes(M: int, seed: int = SEED_NORM) -> torch.Tensor:
+    """Per-token factors 2^u, u ~ U(-2, 3), fp32 [M, 1]."""
+    u = torch.rand((M, 1), generator=_gen(seed + 100)) * 5.0 - 2.0
+    return torch.exp2(u)
+
+
+def make_hidden(M: int, K: int, perm: torch.Tensor, k_o: int, outlier_mult: float,
+                student_t: bool = False, seed: int = SEED_X, t_seed: int = SEED_T,
+                norm_seed: int = SEED_NORM) -> torch.Tensor:
+    """The hidden state before an RMS norm, fp16 [M, K]: the activations of
+    make_activations (drawn in fp32) times a per-token magnitude."""
+    x = torch.randn((M, K), generator=_gen(seed))
+    if k_o > 0:
+        cols = perm[K - k_o:].long()
+        base = student_t3((M, k_o), t_seed) if student_t else x[:, cols]
+        x[:, cols] = base * outlier_mult
+    return (x * token_magnitudes(M, norm_seed)).to(torch.float16)
+
+
+def make_norm_weight(K: int, seed: int = SEED_NORM) -> torch.Tensor:
+    """RMS-norm weight gamma fp16 [K]: |1 + 0.25 N(0, 1)| clamped to [0.02, 4]."""
+    g = (1.0 + 0.25 * torch.randn((K,), generator=_gen(seed))).abs().clamp(0.02, 4.0)
+    return g.to(torch.float16)
+
+
 def make_weights(N: int, K: int, w_std: float, seed: int = SEED_W) -> torch.Tensor:
     return (torch.randn((N, K), generator=_gen(seed)) * w_std).to(torch.float16)
 
@@ -150,7 +185,8 @@ def make_bias(N: int, seed: int = SEED_BIAS) -> torch.Tensor:
 
 
 def make_layer(cfg: LayerConfig, M: int | None = None, seed_offset: int = 0):
-    """All inputs of one layer call: dict(X, W, perm, bias) as CPU tensors.
+    """All inputs of one layer call: dict(X, W, perm, bias) as CPU tensors
+    (plus gamma and eps of the RMS norm when ``cfg.rmsnorm``).
 
     ``M`` overrides the token count (same weights); ``seed_offset`` shifts every
     stream so that tests can draw several independent cases of one shape.
@@ -158,18 +194,26 @@ def make_layer(cfg: LayerConfig, M: int | None = None, seed_offset: int = 0):
     M = cfg.M if M is None else M
     so = seed_offset
     perm = make_perm(cfg.K, SEED_PERM + so)
-    X = make_activations(M, cfg.K, perm, cfg.k_o, cfg.outlier_mult, cfg.student_t,
-                         SEED_X + so, SEED_T + so)
+    if cfg.rmsnorm:
+        X = make_hidden(M, cfg.K, perm, cfg.k_o, cfg.outlier_mult, cfg.student_t,
+                        SEED_X + so, SEED_T + so, SEED_NORM + so)
+    else:
+        X = make_activations(M, cfg.K, perm, cfg.k_o, cfg.outlier_mult, cfg.student_t,
+                             SEED_X + so, SEED_T + so)
     W = make_weights(cfg.N, cfg.K, cfg.w_std, SEED_W + so)
     bias = make_bias(cfg.N, SEED_BIAS + so) if cfg.bias else None
-    return dict(X=X, W=W, perm=perm, bias=bias)
+    d = dict(X=X, W=W, perm=perm, bias=bias)
+    if cfg.rmsnorm:
+        d.update(gamma=make_norm_weight(cfg.K, SEED_NORM + so), eps=NORM_EPS)
+    return d
 
 
 def custom_config(M: int, N: int, K: int, k_o: int, group: int = 0, outlier_int8: bool = False,
                   bias: bool = True, outlier_mult: float = 30.0, student_t: bool = False,
-                  w_std: float = 0.02, act_bits: int = 4, weight_bits: int = 4) -> LayerConfig:
+                  w_std: float = 0.02, act_bits: int = 4, weight_bits: int = 4,
+                  rmsnorm: bool = False) -> LayerConfig:
     return LayerConfig(f"custom_{M}x{N}x{K}_ko{k_o}_g{group}_{'i8' if outlier_int8 else 'f16'}"
-                       f"_w{weight_bits}a{act_bits}",
+                       f"_w{weight_bits}a{act_bits}{'_rms' if rmsnorm else ''}",
                        M=M, N=N, K=K, k_o=k_o, group=group, outlier_int8=outlier_int8,
                        outlier_mult=outlier_mult, student_t=student_t, w_std=w_std, bias=bias,
-                       act_bits=act_bits, weight_bits=weight_bits)
+                       act_bits=act_bits, weight_bits=weight_bits, rmsnorm=rmsnorm)

@@ -109,3 +109,30 @@ def test_null_and_misaligned_pointers_rejected(L):
                          1, None) == q.QUIK_ERR_INVALID_ARG  # workspace too small
     assert L.quik_selftest_timeout(0, None) == q.QUIK_ERR_INVALID_ARG
     assert L.quik_selftest_timeout(2000000, None) == q.QUIK_ERR_INVALID_ARG
+
+
+def test_rmsnorm_arguments_rejected(L):
+    """The fused norm needs an aligned gamma and a finite eps > 0; every case
+    below is rejected before anything is launched (fake addresses, never
+    dereferenced)."""
+    s = q.make_shape(16, 16, 256, 32, 0, 0)
+    good = ctypes.c_void_p(0x1000)
+    bad = ctypes.c_void_p(0x1008)
+    f = L.quik_rmsnorm_quantize_reorder
+    for gamma, eps in ((None, 1e-6), (bad, 1e-6), (good, 0.0), (good, -1e-6),
+                       (good, float("nan")), (good, float("inf"))):
+        assert f(ctypes.byref(s), good, gamma, eps, good, good, good, good, None, None) \
+            == q.QUIK_ERR_INVALID_ARG
+        assert L.quik_rmsnorm_linear(ctypes.byref(s), good, gamma, eps, good, good, good, good,
+                                     None, None, good, good, 1 << 30, None) \
+            == q.QUIK_ERR_INVALID_ARG
+
+
+def test_rmsnorm_widest_rows_unsupported(L):
+    """K past 24576 does not fit the fused norm's two shared-memory tables."""
+    s = q.make_shape(16, 16, 24576 + 64, 64, 0, 0)
+    good = ctypes.c_void_p(0x1000)
+    assert L.quik_rmsnorm_quantize_reorder(ctypes.byref(s), good, good, 1e-5, good, good, good,
+                                           good, None, None) == q.QUIK_ERR_UNSUPPORTED
+    assert L.quik_rmsnorm_linear(ctypes.byref(s), good, good, 1e-5, good, good, good, good, None,
+                                 None, good, good, 1 << 30, None) == q.QUIK_ERR_UNSUPPORTED
