@@ -43,6 +43,8 @@ def _load():
         lib.oracle_quantize_rows.argtypes = [_I, _I, _I, _I, _C, _C, _P, _P, _P, _P, _P, _P]
         lib.oracle_rmsnorm_quantize_rows.argtypes = [_I, _I, _I, _I, _C, _C, _P, _P,
                                                      ctypes.c_float, _P, _P, _P, _P, _P]
+        lib.oracle_prune24_quantize_rows.argtypes = [_I, _I, _I, _C, _P, _P, _P, _P, _P, _P, _P]
+        lib.oracle_unpack24.argtypes = [_I, _I, _P, _P, _P]
         lib.oracle_int_gemm.argtypes = [_I, _I, _I, _I, _C, _C, _P, _P, _P]
         lib.oracle_linear.argtypes = [_I, _I, _I, _I, _I, _C, _C, _C,
                                       _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
@@ -51,6 +53,7 @@ def _load():
                                               _I, _P, _P, _P, _P]
         lib.oracle_num_threads.argtypes = []
         for f in (lib.oracle_quantize_rows, lib.oracle_rmsnorm_quantize_rows,
+                  lib.oracle_prune24_quantize_rows, lib.oracle_unpack24,
                   lib.oracle_int_gemm, lib.oracle_linear,
                   lib.oracle_linear_sampled, lib.oracle_num_threads):
             f.restype = ctypes.c_int
@@ -124,6 +127,42 @@ def rmsnorm_quantize_rows(X_f16: np.ndarray, gamma_f16: np.ndarray, eps: float,
                                               _ptr(O), _ptr(o_scale))
     _check(rc, "rmsnorm_quantize_rows")
     return Q, scale, O, o_scale
+
+
+def prune24_quantize_rows(W_f16: np.ndarray, perm: np.ndarray, k_o: int,
+                          outlier_int8: bool = False):
+    """2:4-sparse INT4 rows (QUIK abstract: quantisation plus 2:4 sparsity):
+    each aligned group of four reordered INT4 positions keeps its two values of
+    largest magnitude (lower position on ties), then the usual quantiser.
+
+    Returns (Qs uint8 [R, K_i/4] two kept codes per byte, meta uint8
+    [R, K_i/8] one nibble i0 | i1 << 2 per group, scale float32 [R],
+    O, o_scale as quantize_rows).
+    """
+    X = np.ascontiguousarray(W_f16, dtype=np.float16)
+    R, K = X.shape
+    Ki = K - k_o
+    perm = np.ascontiguousarray(perm, dtype=np.int32)
+    Qs = np.zeros((R, Ki // 4), np.uint8)
+    meta = np.zeros((R, Ki // 8), np.uint8)
+    scale = np.zeros((R,), np.float32)
+    O = np.zeros((R, k_o), np.int8 if outlier_int8 else np.float16)
+    o_scale = np.zeros((R,), np.float32) if outlier_int8 else None
+    rc = _load().oracle_prune24_quantize_rows(R, K, k_o, int(outlier_int8),
+                                              _ptr(X.view(np.uint16)), _ptr(perm), _ptr(Qs),
+                                              _ptr(meta), _ptr(scale), _ptr(O), _ptr(o_scale))
+    _check(rc, "prune24_quantize_rows")
+    return Qs, meta, scale, O, o_scale
+
+
+def unpack24(Qs: np.ndarray, meta: np.ndarray) -> np.ndarray:
+    """Dense packed INT4 rows [R, K_i/2] that 2:4 rows (Qs, meta) stand for."""
+    Qs = np.ascontiguousarray(Qs, np.uint8)
+    meta = np.ascontiguousarray(meta, np.uint8)
+    R, Ki = Qs.shape[0], 4 * Qs.shape[1]
+    Q = np.zeros((R, Ki // 2), np.uint8)
+    _check(_load().oracle_unpack24(R, Ki, _ptr(Qs), _ptr(meta), _ptr(Q)), "unpack24")
+    return Q
 
 
 def _x_bits(Q) -> int:

@@ -38,6 +38,9 @@
  *    row factor r = 1/sqrt(mean(h^2) + eps) changes no code, so codes and base
  *    scales are taken from h * gamma and r multiplies the stored scales (and
  *    the FP16 outliers, rounded once to fp16).
+ *  - 2:4-sparse weights (QUIK abstract: quantisation plus 2:4 sparsity):
+ *    aligned groups of four reordered INT4 positions keep their two values
+ *    of largest magnitude (lower position on ties), then the usual rule.
  *  - packing: byte i of a row holds code 2i in the low nibble and code 2i+1
  *    in the high nibble, both 4-bit two's complement.
  *  - integer dot products in int64 (checked to fit int32); dequantisation,
@@ -335,6 +338,129 @@ int oracle_rmsnorm_quantize_rows(int64_t R, int64_t K, int64_t k_o, int64_t grou
         free(codes);
     }
     return err;
+}
+
+/*
+ * oracle_prune24_quantize_rows -- 2:4-sparse INT4 rows ("QUIK: Towards
+ * End-to-End 4-Bit Inference on Generative Large Language Models", abstract:
+ * quantisation combined with 2:4 sparsity).  Readings where the page is
+ * silent: the pattern applies to the INT4 part of the reordered row, in
+ * aligned groups of four positions 4t .. 4t+3 (t < K_i / 4); each group keeps
+ * the two values of largest magnitude (on equal magnitudes, the lower
+ * position) and the other two become zero; the outlier block stays dense.
+ * The per-row scale and codes then follow oracle_quantize_rows (the largest
+ * value of every group is kept, so pruning leaves the row's absmax as it is).
+ *
+ *  Qs    : [R, K_i / 4]; byte t holds the code at the group's lower kept
+ *          position in bits 0-3 and the higher one in bits 4-7 (two's
+ *          complement nibbles)
+ *  meta  : [R, K_i / 8]; group t's four bits i0 | i1 << 2 (the kept
+ *          positions within the group, i0 < i1) sit in bits 4 (t % 2) ..
+ *          of byte t / 2
+ *  scale : [R]; O, o_scale as oracle_quantize_rows
+ */
+int oracle_prune24_quantize_rows(int64_t R, int64_t K, int64_t k_o, int outlier_int8,
+                                 const uint16_t *X, const int32_t *perm, uint8_t *Qs,
+                                 uint8_t *meta, float *scale, void *O, float *o_scale)
+{
+    if (R < 0 || K < 0 || k_o < 0 || k_o > K) return ORACLE_EBADARG;
+    const int64_t Ki = K - k_o;
+    if (Ki % 8) return ORACLE_EBADARG;
+    for (int64_t j = 0; j < K; ++j)
+        if (perm[j] < 0 || perm[j] >= K) return ORACLE_EBADARG;
+
+    int err = ORACLE_OK;
+#pragma omp parallel
+    {
+        float *xr = (float *)malloc(sizeof(float) * (size_t)(K > 0 ? K : 1));
+        if (!xr) {
+#pragma omp atomic write
+            err = ORACLE_ENOMEM;
+        }
+#pragma omp for schedule(static)
+        for (int64_t r = 0; r < R; ++r) {
+            if (!xr) continue;
+            for (int64_t j = 0; j < K; ++j)
+                xr[j] = half_to_float(X[r * K + perm[j]]);
+
+            /* the scale over the INT4 positions (before pruning: the same value) */
+            float amax = 0.0f;
+            for (int64_t j = 0; j < Ki; ++j)
+                if (fabsf(xr[j]) > amax) amax = fabsf(xr[j]);
+            float s = amax / 7.0f;
+            scale[r] = s;
+
+            for (int64_t t = 0; t < Ki / 4; ++t) {
+                const float *g = xr + 4 * t;
+                /* first kept: the largest magnitude, lowest position among equals */
+                int a = 0;
+                for (int i = 1; i < 4; ++i)
+                    if (fabsf(g[i]) > fabsf(g[a])) a = i;
+                /* second kept: the largest of the other three, lowest position among equals */
+                int b = -1;
+                for (int i = 0; i < 4; ++i)
+                    if (i != a && (b < 0 || fabsf(g[i]) > fabsf(g[b]))) b = i;
+                int i0 = a < b ? a : b, i1 = a < b ? b : a;
+                int q0 = quantize_value(g[i0], s, 7), q1 = quantize_value(g[i1], s, 7);
+                Qs[r * (Ki / 4) + t] = (uint8_t)((q0 & 0xF) | ((q1 & 0xF) << 4));
+                uint8_t nib = (uint8_t)(i0 | (i1 << 2));
+                uint8_t *mb = &meta[r * (Ki / 8) + t / 2];
+                if (t % 2 == 0)
+                    *mb = nib;
+                else
+                    *mb = (uint8_t)(*mb | (nib << 4));
+            }
+
+            if (k_o > 0) {
+                if (!outlier_int8) {
+                    uint16_t *o16 = (uint16_t *)O;
+                    for (int64_t i = 0; i < k_o; ++i)
+                        o16[r * k_o + i] = X[r * K + perm[Ki + i]];
+                } else {
+                    int8_t *o8 = (int8_t *)O;
+                    float om = 0.0f;
+                    for (int64_t i = 0; i < k_o; ++i)
+                        if (fabsf(xr[Ki + i]) > om) om = fabsf(xr[Ki + i]);
+                    float so = om / 127.0f;
+                    o_scale[r] = so;
+                    for (int64_t i = 0; i < k_o; ++i)
+                        o8[r * k_o + i] = (int8_t)quantize_value(xr[Ki + i], so, 127);
+                }
+            } else if (outlier_int8 && o_scale) {
+                o_scale[r] = 0.0f;
+            }
+        }
+        free(xr);
+    }
+    return err;
+}
+
+/*
+ * oracle_unpack24 -- the dense packed INT4 rows [R, K_i / 2] (the layout of
+ * oracle_quantize_rows) that a 2:4 row stands for: the two kept codes at
+ * their positions, zero elsewhere.  A metadata nibble that names no valid
+ * pair (i0 < i1) is an error.
+ */
+int oracle_unpack24(int64_t R, int64_t Ki, const uint8_t *Qs, const uint8_t *meta, uint8_t *Q)
+{
+    if (R < 0 || Ki < 0 || Ki % 8) return ORACLE_EBADARG;
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t i = 0; i < Ki / 2; ++i)
+            Q[r * (Ki / 2) + i] = 0;
+        for (int64_t t = 0; t < Ki / 4; ++t) {
+            unsigned nib = (meta[r * (Ki / 8) + t / 2] >> (4 * (t % 2))) & 0xF;
+            int i0 = nib & 3, i1 = nib >> 2;
+            if (i0 >= i1) return ORACLE_EBADARG;
+            unsigned b = Qs[r * (Ki / 4) + t];
+            int pos[2] = {(int)(4 * t + i0), (int)(4 * t + i1)};
+            unsigned nibs[2] = {b & 0xF, b >> 4};
+            for (int k = 0; k < 2; ++k) {
+                uint8_t *q = &Q[r * (Ki / 2) + pos[k] / 2];
+                *q = (uint8_t)(pos[k] % 2 ? (*q | (nibs[k] << 4)) : (*q | nibs[k]));
+            }
+        }
+    }
+    return ORACLE_OK;
 }
 
 /*
