@@ -88,6 +88,9 @@ def gemm_source_hash() -> str:
 def gemm_kernel(cfg):
     """The GEMM kernel the library dispatches for this layer, and its profile file."""
     fits = cfg.k_o <= (256 if cfg.outlier_int8 else 128)
+    if cfg.sparse24:
+        return ("w4a4_gemv24 (2:4-sparse INT4 weights as the sparse MMA operand, tcgen05.mma.sp "
+                "kind::i8; 128 W rows x 32 tokens per CTA)", f"w4a4_gemv24_{cfg.name}.md")
     if cfg.act_bits == 8:
         return (("w4a4_gemm_pair with INT8 activations and weights (W8A8)" if cfg.weight_bits == 8 else
                  "w4a4_gemm_pair with INT8 activations (W4A8; weights widened from INT4)")
@@ -231,8 +234,13 @@ def prepare_cpu_inputs(cfg, d):
     import oracle
     d["perm_np"] = d["perm"].numpy()
     d["bias_np"] = None if d["bias"] is None else d["bias"].numpy()
-    d["w_oracle"] = oracle.quantize_rows(d["W"].numpy(), d["perm_np"], cfg.k_o, cfg.group,
-                                         cfg.outlier_int8, cfg.weight_bits)
+    if cfg.sparse24:  # the 2:4 weights, expanded to dense codes for the oracle's product
+        Qs, meta, sw, Wo, swo = oracle.prune24_quantize_rows(d["W"].numpy(), d["perm_np"], cfg.k_o,
+                                                             cfg.outlier_int8)
+        d["w_oracle"] = (oracle.unpack24(Qs, meta), sw, Wo, swo)
+    else:
+        d["w_oracle"] = oracle.quantize_rows(d["W"].numpy(), d["perm_np"], cfg.k_o, cfg.group,
+                                             cfg.outlier_int8, cfg.weight_bits)
 
 
 def cpu_baseline(cfg, d, budget_s: float = 10.0):
@@ -298,9 +306,12 @@ def run_ours(args, rank, local_rank, world):
     bias = d["bias"].to(dev) if d["bias"] is not None else None
     gamma = d["gamma"].to(dev) if cfg.rmsnorm else None
     eps = d.get("eps", 0.0)
-    layer = q.QuikLinear(d["W"].to(dev), perm, cfg.k_o, cfg.group, cfg.outlier_int8, bias,
-                         act_bits=cfg.act_bits, weight_bits=cfg.weight_bits, norm_weight=gamma,
-                         norm_eps=eps)
+    if cfg.sparse24:
+        layer = q.QuikLinear24(d["W"].to(dev), perm, cfg.k_o, cfg.outlier_int8, bias)
+    else:
+        layer = q.QuikLinear(d["W"].to(dev), perm, cfg.k_o, cfg.group, cfg.outlier_int8, bias,
+                             act_bits=cfg.act_bits, weight_bits=cfg.weight_bits, norm_weight=gamma,
+                             norm_eps=eps)
     shape = layer.shape(cfg.M)
     Xq, sx, Xo, sxo = q._binding._quant_outputs(cfg.M, cfg.K, cfg.k_o, cfg.group,
                                                 cfg.outlier_int8, dev, cfg.act_bits)
@@ -308,13 +319,16 @@ def run_ours(args, rank, local_rank, world):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    ws = layer.workspace(cfg.M, dev)
+    ws = torch.empty((q.quik_workspace_size(shape),), dtype=torch.uint8, device=dev)
 
     def step():
         # one layer call: quantise + reorder (behind the RMS norm, for a
         # norm-fused workload), then the GEMM (which may start while the
         # quantiser finishes: programmatic dependent launch)
-        if cfg.rmsnorm:
+        if cfg.sparse24:
+            q.quik_linear_24(shape, X, perm, layer.Wq24, layer.Wmeta, layer.w_scale, layer.Wo,
+                             layer.wo_scale, bias, Y, ws, stream=stream)
+        elif cfg.rmsnorm:
             q.quik_rmsnorm_linear(shape, X, gamma, eps, perm, layer.Wq, layer.w_scale, layer.Wo,
                                   layer.wo_scale, bias, Y, ws, stream=stream)
         else:
@@ -331,8 +345,12 @@ def run_ours(args, rank, local_rank, world):
         else:
             q.quik_quantize_reorder(shape, X, perm, Xq, sx, Xo, sxo, stream=stream)
         ev[1].record(stream)
-        q.quik_gemm(shape, Xq, sx, Xo, sxo, layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale,
-                    bias, Y, stream=stream)
+        if cfg.sparse24:
+            q.quik_gemm_24(shape, Xq, sx, Xo, sxo, layer.Wq24, layer.Wmeta, layer.w_scale, layer.Wo,
+                           layer.wo_scale, bias, Y, stream=stream)
+        else:
+            q.quik_gemm(shape, Xq, sx, Xo, sxo, layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale,
+                        bias, Y, stream=stream)
         ev[2].record(stream)
 
     for _ in range(max(3, args.warmup)):
@@ -430,11 +448,15 @@ def run_ours(args, rank, local_rank, world):
 
     peaks, peak_kind = measured_peaks()
     int8_peak = float(peaks["bf16_tflops"]) * INT8_PER_BF16
+    # the 2:4-sparse MMA does half the multiply-adds of the INT4 part: its
+    # dense-equivalent peak is twice the dense one (ops stay 2 M N K)
+    sparse_x = 2.0 if cfg.sparse24 else 1.0
+    tensor_peak = int8_peak * sparse_x
     gemm_tops = cfg.ops / gemm_avg / 1e12
     kernel_name, profile_file = gemm_kernel(cfg)
     hbm_peak = float(peaks["hbm_gbs"])
     # the path's bound: the slower of the tensor work and the bytes it must move
-    if cfg.gemm_bytes / (hbm_peak * 1e9) > cfg.ops / (int8_peak * 1e12):
+    if cfg.gemm_bytes / (hbm_peak * 1e9) > cfg.ops / (tensor_peak * 1e12):
         roofline = {
             "bound": "hbm", "kernel": kernel_name,
             "achieved": round(cfg.gemm_bytes / gemm_avg / 1e9, 1), "peak": hbm_peak,
@@ -446,13 +468,14 @@ def run_ours(args, rank, local_rank, world):
     else:
         roofline = {
             "bound": "tensor", "kernel": kernel_name,
-            "achieved": round(gemm_tops, 2), "peak": round(int8_peak, 1), "unit": "TFLOP/s",
-            "frac": round(gemm_tops / int8_peak, 4),
+            "achieved": round(gemm_tops, 2), "peak": round(tensor_peak, 1), "unit": "TFLOP/s",
+            "frac": round(gemm_tops / tensor_peak, 4),
             "traffic": profiled_traffic(profile_file),
             "algorithmic_bytes_per_launch": cfg.gemm_bytes,
             "peak_source": (f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
-                            f"{INT8_PER_BF16} (nominal INT8:BF16 dense ratio); integer ops "
-                            f"counted 2 per multiply-add"),
+                            f"{INT8_PER_BF16} (nominal INT8:BF16 dense ratio)"
+                            + (" x 2 (2:4-sparse MMA, dense-equivalent)" if cfg.sparse24 else "")
+                            + "; integer ops counted 2 per multiply-add"),
         }
     line = {
         "metric": METRIC,
@@ -473,7 +496,8 @@ def run_ours(args, rank, local_rank, world):
             "group_size": cfg.group, "outliers": "int8" if cfg.outlier_int8 else "fp16",
             "bias": cfg.bias, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": "flushed before every step (256 MiB write, outside the step's events)",
-            "step": ("quik_rmsnorm_linear: RMS norm folded into quantise + reorder, then the GEMM"
+            "step": ("quik_linear_24: quantise + reorder, then the 2:4-sparse GEMM" if cfg.sparse24
+                     else "quik_rmsnorm_linear: RMS norm folded into quantise + reorder, then the GEMM"
                      if cfg.rmsnorm else "quik_linear: quantise + reorder, then the GEMM")
                     + " (weights packed once, offline)",
         },
@@ -485,7 +509,8 @@ def run_ours(args, rank, local_rank, world):
         "roofline": roofline,
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
                 "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2,
-                "call": ("quik_rmsnorm_linear" if cfg.rmsnorm else "quik_linear")
+                "call": ("quik_linear_24" if cfg.sparse24 else "quik_rmsnorm_linear" if cfg.rmsnorm
+                         else "quik_linear")
                         + " via QuikLinear, pinned host X in, host Y out"},
         "gpu_launches": 2 * args.steps,
         "clocks": sampler.summary(),

@@ -209,6 +209,64 @@ QUIK_API quik_status quik_rmsnorm_linear(const quik_shape *shape, const void *X_
                                          quik_stream_t stream);
 
 /*
+ * 2:4-sparse INT4 weights (QUIK abstract: quantisation combined with 2:4
+ * sparsity).  Within the INT4 part of each reordered weight row, every
+ * aligned group of four positions 4t .. 4t+3 keeps its two values of largest
+ * magnitude (on equal magnitudes, the lower position) and the other two are
+ * zero; the row's scale and the kept values' codes follow the dense rule
+ * (s = max|w| / 7 per output channel); the outlier block stays dense.  The
+ * product runs on the sparse tensor-core MMA (W as the 2:4 operand).
+ * Storage:
+ *   Wq24  u8 [N, K_i / 4]: byte t = the group's lower kept code (bits 0-3)
+ *         and higher kept code (bits 4-7), two's complement nibbles;
+ *   Wmeta u8 [N, K_i / 8]: group t's positions i0 | i1 << 2 (i0 < i1) in
+ *         bits 4 (t % 2) .. 4 (t % 2) + 3 of byte t / 2.
+ * Shapes: group_size 0, INT4 activations and weights (act_bits, weight_bits
+ * 0 or 4), K_i % 128 == 0, k_o <= 128 (FP16) or 256 (INT8); anything else
+ * returns QUIK_ERR_UNSUPPORTED.  Activations are dense (quik_quantize_reorder).
+ */
+
+/*
+ * quik_pack_weights_24 -- offline: prune W [N, K] fp16 to 2:4 as above,
+ * quantise and store the kept codes, position pairs, per-channel scales
+ * w_scale [N] and the outlier block Wo / wo_scale (as quik_pack_weights).
+ */
+QUIK_API quik_status quik_pack_weights_24(const quik_shape *shape, const void *W_f16,
+                                          const int32_t *perm, void *Wq24, void *Wmeta,
+                                          float *w_scale, void *Wo, float *wo_scale,
+                                          quik_stream_t stream);
+
+/*
+ * quik_gemm_24 -- quik_gemm with 2:4-sparse weights (Wq24, Wmeta): exact
+ * integer sums over the kept positions, the outlier product and the same
+ * dequantising epilogue.  Tiles of 128 output channels x 32 tokens.
+ */
+QUIK_API quik_status quik_gemm_24(const quik_shape *shape, const void *Xq, const float *x_scale,
+                                  const void *Xo, const float *xo_scale, const void *Wq24,
+                                  const void *Wmeta, const float *w_scale, const void *Wo,
+                                  const float *wo_scale, const void *bias_f16, void *Y_f16,
+                                  quik_stream_t stream);
+
+/*
+ * quik_linear_24 -- quik_quantize_reorder into `workspace`
+ * (quik_workspace_size(shape) bytes) followed by quik_gemm_24.
+ */
+QUIK_API quik_status quik_linear_24(const quik_shape *shape, const void *X_f16, const int32_t *perm,
+                                    const void *Wq24, const void *Wmeta, const float *w_scale,
+                                    const void *Wo, const float *wo_scale, const void *bias_f16,
+                                    void *Y_f16, void *workspace, size_t workspace_bytes,
+                                    quik_stream_t stream);
+
+/*
+ * quik_gemm_24_i32_debug -- test entry: the sparse product's integer sums
+ * acc [M, N] int32 (and the INT8 outlier sums, as quik_gemm_i32_debug).
+ */
+QUIK_API quik_status quik_gemm_24_i32_debug(const quik_shape *shape, const void *Xq,
+                                            const void *Wq24, const void *Wmeta, const void *Xo,
+                                            const void *Wo, int32_t *acc, int32_t *acc_outlier,
+                                            quik_stream_t stream);
+
+/*
  * quik_linear_noalloc -- quik_linear for callers that cannot allocate device
  * memory.  (No counterpart in the papers; an addition of this library.)
  *

@@ -53,6 +53,10 @@ _SIGS = {
                                             _P, _P, ctypes.c_size_t, _P]),
     "quik_linear_noalloc": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "quik_gemm_i32_debug": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P]),
+    "quik_pack_weights_24": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "quik_gemm_24": (ctypes.c_int, [_S] + [_P] * 12),
+    "quik_linear_24": (ctypes.c_int, [_S] + [_P] * 10 + [ctypes.c_size_t, _P]),
+    "quik_gemm_24_i32_debug": (ctypes.c_int, [_S] + [_P] * 8),
     "quik_sync_check": (ctypes.c_int, [_P]),
     "quik_selftest_timeout": (ctypes.c_int, [ctypes.c_uint32, _P]),
     "quik_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -203,6 +207,44 @@ def quik_gemm_i32_debug(shape, Xq, Wq, Xo, Wo, acc, acc_outlier, stream=None):
         _ptr(acc_outlier, torch.int32, "acc_outlier"), _stream(stream)), "quik_gemm_i32_debug")
 
 
+def quik_pack_weights_24(shape, W, perm, Wq24, Wmeta, w_scale, Wo, wo_scale, stream=None):
+    _check(lib().quik_pack_weights_24(
+        ctypes.byref(shape), _ptr(W, torch.float16, "W"), _ptr(perm, torch.int32, "perm"),
+        _ptr(Wq24, torch.uint8, "Wq24"), _ptr(Wmeta, torch.uint8, "Wmeta"),
+        _ptr(w_scale, torch.float32, "w_scale"), _ptr(Wo, None, "Wo"),
+        _ptr(wo_scale, torch.float32, "wo_scale"), _stream(stream)), "quik_pack_weights_24")
+
+
+def quik_gemm_24(shape, Xq, x_scale, Xo, xo_scale, Wq24, Wmeta, w_scale, Wo, wo_scale, bias, Y,
+                 stream=None):
+    _check(lib().quik_gemm_24(
+        ctypes.byref(shape), _ptr(Xq, torch.uint8, "Xq"), _ptr(x_scale, torch.float32, "x_scale"),
+        _ptr(Xo, None, "Xo"), _ptr(xo_scale, torch.float32, "xo_scale"),
+        _ptr(Wq24, torch.uint8, "Wq24"), _ptr(Wmeta, torch.uint8, "Wmeta"),
+        _ptr(w_scale, torch.float32, "w_scale"), _ptr(Wo, None, "Wo"),
+        _ptr(wo_scale, torch.float32, "wo_scale"), _ptr(bias, torch.float16, "bias"),
+        _ptr(Y, torch.float16, "Y"), _stream(stream)), "quik_gemm_24")
+
+
+def quik_linear_24(shape, X, perm, Wq24, Wmeta, w_scale, Wo, wo_scale, bias, Y, workspace,
+                   stream=None):
+    _check(lib().quik_linear_24(
+        ctypes.byref(shape), _ptr(X, torch.float16, "X"), _ptr(perm, torch.int32, "perm"),
+        _ptr(Wq24, torch.uint8, "Wq24"), _ptr(Wmeta, torch.uint8, "Wmeta"),
+        _ptr(w_scale, torch.float32, "w_scale"), _ptr(Wo, None, "Wo"),
+        _ptr(wo_scale, torch.float32, "wo_scale"), _ptr(bias, torch.float16, "bias"),
+        _ptr(Y, torch.float16, "Y"), _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+        _stream(stream)), "quik_linear_24")
+
+
+def quik_gemm_24_i32_debug(shape, Xq, Wq24, Wmeta, Xo, Wo, acc, acc_outlier, stream=None):
+    _check(lib().quik_gemm_24_i32_debug(
+        ctypes.byref(shape), _ptr(Xq, torch.uint8, "Xq"), _ptr(Wq24, torch.uint8, "Wq24"),
+        _ptr(Wmeta, torch.uint8, "Wmeta"), _ptr(Xo, None, "Xo"), _ptr(Wo, None, "Wo"),
+        _ptr(acc, torch.int32, "acc"), _ptr(acc_outlier, torch.int32, "acc_outlier"),
+        _stream(stream)), "quik_gemm_24_i32_debug")
+
+
 def quik_sync_check(stream=None) -> int:
     return int(lib().quik_sync_check(_stream(stream)))
 
@@ -292,6 +334,74 @@ def gemm_i32(Xq, Wq, K: int, k_o: int, group: int = 0, Xo=None, Wo=None, stream=
     quik_gemm_i32_debug(shape, Xq, Wq, Xo if int8 else None, Wo if int8 else None, acc, acc_o,
                         stream=stream)
     return acc, acc_o
+
+
+def pack_weights_24(W: torch.Tensor, perm: torch.Tensor, k_o: int, outlier_int8: bool = False,
+                    stream=None):
+    """Weights -> 2:4-sparse (Wq24 uint8 [N, K_i/4], Wmeta uint8 [N, K_i/8],
+    w_scale [N], Wo, wo_scale), allocated on W's device."""
+    N, K = W.shape
+    Ki = K - k_o
+    shape = make_shape(1, N, K, k_o, 0, _outlier_kind(outlier_int8))
+    dev = W.device
+    Wq24 = torch.empty((N, Ki // 4), dtype=torch.uint8, device=dev)
+    Wmeta = torch.empty((N, Ki // 8), dtype=torch.uint8, device=dev)
+    _, w_scale, Wo, wo_scale = _quant_outputs(N, K, k_o, 0, outlier_int8, dev)
+    quik_pack_weights_24(shape, W, perm, Wq24, Wmeta, w_scale, Wo, wo_scale, stream=stream)
+    return Wq24, Wmeta, w_scale, Wo, wo_scale
+
+
+def gemm_24(xq, w24, K: int, k_o: int, bias=None, stream=None):
+    """Y fp16 [M, N] from quantised activations xq (4-tuple) and 2:4 weights w24 (5-tuple)."""
+    Xq, sx, Xo, sxo = xq
+    Wq24, Wmeta, sw, Wo, swo = w24
+    M, N = sx.shape[0], sw.shape[0]
+    shape = make_shape(M, N, K, k_o, 0, _outlier_kind(Xo.dtype == torch.int8))
+    Y = torch.empty((M, N), dtype=torch.float16, device=sx.device)
+    quik_gemm_24(shape, Xq, sx, Xo, sxo, Wq24, Wmeta, sw, Wo, swo, bias, Y, stream=stream)
+    return Y
+
+
+def gemm24_i32(Xq, Wq24, Wmeta, K: int, k_o: int, Xo=None, Wo=None, stream=None):
+    """Integer sums of the 2:4 product: acc [M, N] and, for INT8 outliers, acc_o."""
+    M, N = Xq.shape[0], Wq24.shape[0]
+    int8 = Xo is not None and Xo.dtype == torch.int8
+    shape = make_shape(M, N, K, k_o, 0, _outlier_kind(int8))
+    acc = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
+    acc_o = torch.empty((M, N), dtype=torch.int32, device=Xq.device) if int8 and k_o else None
+    quik_gemm_24_i32_debug(shape, Xq, Wq24, Wmeta, Xo if int8 else None, Wo if int8 else None, acc,
+                           acc_o, stream=stream)
+    return acc, acc_o
+
+
+class QuikLinear24:
+    """A W4A4 + outlier linear layer with 2:4-sparse INT4 weights.
+
+    ``QuikLinear24(W, perm, k_o, outlier_int8, bias)`` prunes and packs W once
+    (quik_pack_weights_24); calling it on fp16 activations runs quik_linear_24
+    into a workspace it keeps.
+    """
+
+    def __init__(self, W: torch.Tensor, perm: torch.Tensor, k_o: int, outlier_int8: bool = False,
+                 bias: torch.Tensor | None = None):
+        self.N, self.K = W.shape
+        self.k_o, self.outlier_int8, self.perm, self.bias = k_o, outlier_int8, perm, bias
+        (self.Wq24, self.Wmeta, self.w_scale, self.Wo,
+         self.wo_scale) = pack_weights_24(W, perm, k_o, outlier_int8)
+        self._ws = None
+
+    def shape(self, M: int) -> quik_shape:
+        return make_shape(M, self.N, self.K, self.k_o, 0, _outlier_kind(self.outlier_int8))
+
+    def __call__(self, X: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        M = X.shape[0]
+        need = quik_workspace_size(self.shape(M))
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty((need,), dtype=torch.uint8, device=X.device)
+        Y = out if out is not None else torch.empty((M, self.N), dtype=torch.float16, device=X.device)
+        quik_linear_24(self.shape(M), X, self.perm, self.Wq24, self.Wmeta, self.w_scale, self.Wo,
+                       self.wo_scale, self.bias, Y, self._ws, stream=stream)
+        return Y
 
 
 class QuikLinear:

@@ -84,6 +84,30 @@ inline bool ok_norm(const void *gamma, float eps) {
     return ok_ptr(gamma) && std::isfinite(eps) && eps > 0.0f;
 }
 
+// 2:4-sparse weights: INT4 codes with per-channel scales, K_i % 128 == 0 (the
+// rows of position pairs are whole 16-byte units), and an outlier block of at
+// most 128 FP16 or 256 INT8 channels.
+quik_status check_shape24(const quik_shape *s) {
+    quik_status st = check_shape(s);
+    if (st != QUIK_OK) return st;
+    if (s->group_size != 0 || act8(s) || wt8(s) || (s->K - s->k_o) % 128 != 0 ||
+        s->k_o > (int8_out(s) ? 256 : 128))
+        return QUIK_ERR_UNSUPPORTED;
+    return QUIK_OK;
+}
+
+// Kept codes [rows, K_i / 4], position pairs [rows, K_i / 8], per-row scales.
+quik_status check_ptrs24(const quik_shape *s, const void *Qs, const void *meta, const float *scale,
+                         const void *O, const float *o_scale) {
+    const int Ki = s->K - s->k_o;
+    if (Ki > 0 && (!ok_ptr(Qs) || !ok_ptr(meta) || !ok_ptr(scale))) return QUIK_ERR_INVALID_ARG;
+    if (s->k_o > 0 && !ok_ptr(O)) return QUIK_ERR_INVALID_ARG;
+    if (int8_out(s) && s->k_o > 0 && !ok_ptr(o_scale)) return QUIK_ERR_INVALID_ARG;
+    if (!ok_opt(Qs) || !ok_opt(meta) || !ok_opt(scale) || !ok_opt(O) || !ok_opt(o_scale))
+        return QUIK_ERR_INVALID_ARG;
+    return QUIK_OK;
+}
+
 struct Workspace {
     size_t xq, sx, xo, sxo, total;
 };
@@ -234,6 +258,115 @@ quik_status quik_rmsnorm_linear(const quik_shape *shape, const void *X_f16, cons
     if (gamma_f16 == nullptr) return QUIK_ERR_INVALID_ARG;
     return linear_impl(shape, X_f16, gamma_f16, eps, perm, Wq, w_scale, Wo, wo_scale, bias_f16,
                        Y_f16, workspace, workspace_bytes, stream);
+}
+
+quik_status quik_pack_weights_24(const quik_shape *shape, const void *W_f16, const int32_t *perm,
+                                 void *Wq24, void *Wmeta, float *w_scale, void *Wo,
+                                 float *wo_scale, quik_stream_t stream) {
+    quik_status st = check_shape24(shape);
+    if (st != QUIK_OK) return st;
+    if (!ok_ptr(W_f16) || !ok_ptr(perm)) return QUIK_ERR_INVALID_ARG;
+    if ((st = check_ptrs24(shape, Wq24, Wmeta, w_scale, Wo, wo_scale)) != QUIK_OK) return st;
+    quik::Prune24Args a;
+    a.W = static_cast<const uint16_t *>(W_f16);
+    a.perm = perm;
+    a.rows = shape->N;
+    a.K = shape->K;
+    a.k_o = shape->k_o;
+    a.out_int8 = int8_out(shape);
+    a.Qs = static_cast<uint8_t *>(Wq24);
+    a.meta = static_cast<uint8_t *>(Wmeta);
+    a.scale = w_scale;
+    a.O = Wo;
+    a.o_scale = wo_scale;
+    return quik::launch_prune24_rows(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? QUIK_OK
+                                                                                        : QUIK_ERR_CUDA;
+}
+
+static quik_status gemm24_impl(const quik_shape *shape, const void *Xq, const float *x_scale,
+                               const void *Xo, const float *xo_scale, const void *Wq24,
+                               const void *Wmeta, const float *w_scale, const void *Wo,
+                               const float *wo_scale, const void *bias, void *Y, bool debug,
+                               int32_t *acc, int32_t *acc_o, cudaStream_t stream,
+                               bool after_quantize = false) {
+    quik::GemmArgs a;
+    a.M = shape->M;
+    a.N = shape->N;
+    a.K = shape->K;
+    a.k_o = shape->k_o;
+    a.group = 0;
+    a.out_int8 = int8_out(shape);
+    a.a8 = false;
+    a.w8 = false;
+    a.Xq = Xq;
+    a.sx = x_scale;
+    a.Xo = Xo;
+    a.sxo = xo_scale;
+    a.Wq = Wq24;
+    a.Wmeta = static_cast<const uint8_t *>(Wmeta);
+    a.sparse24 = true;
+    a.sw = w_scale;
+    a.Wo = Wo;
+    a.swo = wo_scale;
+    a.bias = static_cast<const uint16_t *>(bias);
+    a.Y = static_cast<uint16_t *>(Y);
+    a.debug = debug;
+    a.after_quantize = after_quantize;
+    a.acc_dbg = acc;
+    a.acc_o_dbg = acc_o;
+    return quik::launch_gemm(a, stream);
+}
+
+quik_status quik_gemm_24(const quik_shape *shape, const void *Xq, const float *x_scale,
+                         const void *Xo, const float *xo_scale, const void *Wq24,
+                         const void *Wmeta, const float *w_scale, const void *Wo,
+                         const float *wo_scale, const void *bias_f16, void *Y_f16,
+                         quik_stream_t stream) {
+    quik_status st = check_shape24(shape);
+    if (st != QUIK_OK) return st;
+    if ((st = check_quant_ptrs(shape, Xq, x_scale, Xo, xo_scale)) != QUIK_OK) return st;
+    if ((st = check_ptrs24(shape, Wq24, Wmeta, w_scale, Wo, wo_scale)) != QUIK_OK) return st;
+    if (!ok_ptr(Y_f16) || !ok_opt(bias_f16)) return QUIK_ERR_INVALID_ARG;
+    return gemm24_impl(shape, Xq, x_scale, Xo, xo_scale, Wq24, Wmeta, w_scale, Wo, wo_scale,
+                       bias_f16, Y_f16, false, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+quik_status quik_linear_24(const quik_shape *shape, const void *X_f16, const int32_t *perm,
+                           const void *Wq24, const void *Wmeta, const float *w_scale,
+                           const void *Wo, const float *wo_scale, const void *bias_f16,
+                           void *Y_f16, void *workspace, size_t workspace_bytes,
+                           quik_stream_t stream) {
+    quik_status st = check_shape24(shape);
+    if (st != QUIK_OK) return st;
+    if (!ok_ptr(X_f16) || !ok_ptr(perm) || !ok_ptr(Y_f16) || !ok_opt(bias_f16))
+        return QUIK_ERR_INVALID_ARG;
+    if ((st = check_ptrs24(shape, Wq24, Wmeta, w_scale, Wo, wo_scale)) != QUIK_OK) return st;
+    const Workspace w = layout(shape);
+    if (!ok_ptr(workspace) || workspace_bytes < w.total) return QUIK_ERR_INVALID_ARG;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    void *Xq = ws + w.xq;
+    float *sx = reinterpret_cast<float *>(ws + w.sx);
+    void *Xo = ws + w.xo;
+    float *sxo = int8_out(shape) ? reinterpret_cast<float *>(ws + w.sxo) : nullptr;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = quantize(shape, shape->M, false, X_f16, perm, Xq, sx, Xo, sxo, s)) != QUIK_OK) return st;
+    return gemm24_impl(shape, Xq, sx, Xo, sxo, Wq24, Wmeta, w_scale, Wo, wo_scale, bias_f16, Y_f16,
+                       false, nullptr, nullptr, s, true);
+}
+
+quik_status quik_gemm_24_i32_debug(const quik_shape *shape, const void *Xq, const void *Wq24,
+                                   const void *Wmeta, const void *Xo, const void *Wo, int32_t *acc,
+                                   int32_t *acc_outlier, quik_stream_t stream) {
+    quik_status st = check_shape24(shape);
+    if (st != QUIK_OK) return st;
+    const int Ki = shape->K - shape->k_o;
+    if (Ki > 0 && (!ok_ptr(Xq) || !ok_ptr(Wq24) || !ok_ptr(Wmeta) || !ok_ptr(acc)))
+        return QUIK_ERR_INVALID_ARG;
+    const bool want_o = int8_out(shape) && shape->k_o > 0;
+    if (want_o && (!ok_ptr(Xo) || !ok_ptr(Wo) || !ok_ptr(acc_outlier))) return QUIK_ERR_INVALID_ARG;
+    return gemm24_impl(shape, Xq, nullptr, want_o ? Xo : nullptr, nullptr, Wq24, Wmeta, nullptr,
+                       want_o ? Wo : nullptr, nullptr, nullptr, nullptr, true, acc,
+                       want_o ? acc_outlier : nullptr, static_cast<cudaStream_t>(stream));
 }
 
 quik_status quik_gemm_i32_debug(const quik_shape *shape, const void *Xq, const void *Wq,

@@ -1380,6 +1380,350 @@ __global__ void __launch_bounds__(gemv::THREADS, 1)
     if (threadIdx.x == 0) QUIK_TRACE_AT(7, 0);
 }
 
+// ============================================================================
+// 2:4-sparse INT4 weights ("QUIK" abstract: quantisation plus 2:4 sparsity) on
+// the sparse tensor-core MMA, for up to 32 tokens per CTA.
+//
+// W is the MMA's A operand, 128 rows per CTA, stored compressed: the two kept
+// INT4 codes of every aligned group of four positions (one byte per group) and
+// the group's position pair (one nibble i0 | i1 << 2).  Per k-block of 256
+// positions the group warps widen the kept codes to INT8 (x16, in order) into
+// a 128-byte-swizzled shared-memory stage (128 rows x 128 bytes) and store the
+// pairs in tensor memory (lane = W row; one sparse MMA reads 64 bits, two
+// columns at a 4-column-aligned address, group g in bits 4g .. 4g+3).  The
+// tokens are the N operand (16 or 32 rows, widened to INT8 x16 in order, two
+// 128-byte-wide tiles per k-block); a second grid dimension covers more tokens.
+// Four sparse MMAs (K = 64 each) per k-block; the accumulator holds 256 A.
+// The outlier block and the epilogue are those of the decode kernel above.
+// ============================================================================
+namespace sp24 {
+constexpr int BW = 128;                      // W rows per CTA = TMEM lanes
+constexpr int MT = 32;                       // tokens per CTA (the MMA's N: 16 or 32)
+constexpr int KBL = 256;                     // positions per k-block
+constexpr int WROW = 64;                     // packed kept codes per row per k-block (bytes)
+constexpr int MROW = 32;                     // position pairs per row per k-block (bytes)
+constexpr int XROW = 128;                    // packed token codes per row per k-block (bytes)
+constexpr int S = 4;                         // operand stages
+constexpr int SPW = 4;                       // staging units
+constexpr int WUNIT = BW * WROW;             // 8 KB
+constexpr int MUNIT = BW * MROW;             // 4 KB
+constexpr int XUNIT = MT * XROW;             // 4 KB
+constexpr int UNIT = WUNIT + MUNIT + XUNIT;  // 16 KB
+constexpr int ASTAGE = BW * 128;             // widened kept codes: 128 rows x 128 bytes
+constexpr int XTILE = MT * 128;              // one 128-byte-wide half of the widened token rows
+constexpr int STAGE = ASTAGE + 2 * XTILE;    // 24 KB
+constexpr int OKB = 2;                       // outlier k-blocks of 128-byte rows
+constexpr int KO_MAX_F16 = 64 * OKB, KO_MAX_I8 = 128 * OKB;
+constexpr int WO_TILE = BW * 128, XO_TILE = MT * 128;
+constexpr int NG = 4, NW = 4 * NG, NI = 2;   // unpack groups (4 warps each), MMA issuers
+constexpr int THREADS = (1 + NW + NI) * 32;
+constexpr int OP_OFF = SPW * UNIT;
+constexpr int WO_OFF = OP_OFF + S * STAGE;
+constexpr int XO_OFF = WO_OFF + OKB * WO_TILE;
+constexpr int SMEM = XO_OFF + OKB * XO_TILE + 1024;  // + alignment
+constexpr int ACC_COL = 0, O_COL = 32 * NI, META_COL = O_COL + 32;
+constexpr int META_STAGE = 16;               // four MMAs x 4 columns (2 used)
+constexpr int TMEM_COLS = 256;
+static_assert(META_COL % 4 == 0 && META_COL + S * META_STAGE <= TMEM_COLS, "metadata in tensor memory");
+static_assert(S % NG == 0 && S % NI == 0, "group g owns stages g, g + NG, ...; one issuer per stage");
+static_assert(WUNIT % 1024 == 0 && (WUNIT + MUNIT) % 1024 == 0 && UNIT % 1024 == 0, "swizzled staging");
+static_assert(OP_OFF % 1024 == 0 && STAGE % 1024 == 0 && ASTAGE % 1024 == 0 && XTILE % 1024 == 0,
+              "128-byte-swizzled operand tiles");
+static_assert(WO_OFF % 1024 == 0 && XO_OFF % 1024 == 0, "128-byte-swizzled outlier tiles");
+static_assert(SMEM <= 232448, "shared memory budget");
+}  // namespace sp24
+
+// 32 packed INT4 codes (16 bytes, code 2i in the low nibble of byte i) ->
+// 32 INT8 values 16 c in order (two 16-byte chunks).
+__device__ __forceinline__ void widen16_ordered(const uint4 v, uint4 &a, uint4 &b) {
+    const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = (x[i] << 4) & 0xF0F0F0F0u;  // codes 0, 2, 4, 6 of the word
+        const uint32_t hi = x[i] & 0xF0F0F0F0u;         // codes 1, 3, 5, 7
+        asm("prmt.b32 %0, %1, %2, 0x5140;" : "=r"(o[2 * i]) : "r"(lo), "r"(hi));
+        asm("prmt.b32 %0, %1, %2, 0x7362;" : "=r"(o[2 * i + 1]) : "r"(lo), "r"(hi));
+    }
+    a = make_uint4(o[0], o[1], o[2], o[3]);
+    b = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+template <bool OUT_INT8, bool DEBUG>
+__global__ void __launch_bounds__(sp24::THREADS, 1)
+    w4a4_gemv24_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_m,
+                       const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wo,
+                       const __grid_constant__ CUtensorMap tm_xo, const GemmParams p) {
+    using namespace sp24;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t w_full[SPW], w_empty[SPW], op_full[S], op_empty[S], o_full, acc_full, mma_done[NI];
+    __shared__ uint32_t tmem_base_s;
+    __shared__ int abort_s;
+    __shared__ unsigned err0_s;
+
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+    const uint32_t smem_base = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BW;
+    const int m0 = blockIdx.y * MT;
+    const int MP = p.M <= 16 ? 16 : 32;  // the MMA's N (token rows past M read as 0)
+    const int nkb = p.nkb_i;
+    const int oke = OUT_INT8 ? 128 : 64;
+    const int nko = (p.k_o + oke - 1) / oke;
+    const uint32_t unit_bytes = WUNIT + MUNIT + MP * XROW;
+
+    const int early = nkb < SPW ? nkb : SPW;  // W units loaded before the CTA barrier
+    if (warp == 1 && lane == 0) {
+        // the producer's barriers and the first W units (kept codes and pairs:
+        // not the previous kernel's output); their token rows follow after
+        // the grid dependency
+        for (int i = 0; i < SPW; ++i) {
+            mbar_init(&w_full[i], 1);
+            mbar_init(&w_empty[i], 4);  // the four warps of the k-block's group
+        }
+        mbar_init(&o_full, 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+        if (nkb > 0) {
+            tma_prefetch_desc(&tm_w);
+            tma_prefetch_desc(&tm_m);
+            tma_prefetch_desc(&tm_x);
+        }
+        for (int u = 0; u < early; ++u) {
+            mbar_arrive_expect_tx(&w_full[u], unit_bytes);
+            tma_load_2d(smem + u * UNIT, &tm_w, u * WROW, n0, &w_full[u]);
+            tma_load_2d(smem + u * UNIT + WUNIT, &tm_m, u * MROW, n0, &w_full[u]);
+        }
+        if (nko > 0) {
+            tma_prefetch_desc(&tm_wo);
+            tma_prefetch_desc(&tm_xo);
+            mbar_arrive_expect_tx(&o_full, nko * (WO_TILE + MP * 128));
+            for (int kb = 0; kb < nko; ++kb)
+                tma_load_2d(smem + WO_OFF + kb * WO_TILE, &tm_wo, kb * oke, n0, &o_full);
+        }
+    }
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&op_full[i], 4);
+            mbar_init(&op_empty[i], 1);
+        }
+        mbar_init(&acc_full, NI);
+        for (int i = 0; i < NI; ++i) mbar_init(&mma_done[i], 1);
+        abort_s = 0;
+        err0_s = *reinterpret_cast<volatile unsigned *>(&g_error_word);
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc(&tmem_base_s, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_s;
+    const AbortState ab{&abort_s, err0_s};
+
+    const int issuer = warp == 0 ? 0 : warp >= 2 + NW ? warp - 1 - NW : -1;
+    if (issuer >= 0) {
+        // ------------------------------------------------------------ MMA issuers
+        if (lane == 0) {
+            bool ok = true;
+            if (issuer == 0 && nko > 0) {  // the dense outlier block
+                ok = wait_bar(&o_full, 0, ab);
+                if (ok) {
+                    tc_fence_after();
+                    const uint32_t id_o = OUT_INT8 ? idesc_s8_s32(BW, MP) : idesc_f16_f32(BW, MP);
+                    for (int kb = 0; kb < nko; ++kb) {
+                        const uint32_t wo = smem_base + WO_OFF + kb * WO_TILE;
+                        const uint32_t xo = smem_base + XO_OFF + kb * XO_TILE;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint64_t ad = sw128_kmajor_desc(wo + 32 * k);
+                            const uint64_t bd = sw128_kmajor_desc(xo + 32 * k);
+                            if (OUT_INT8)
+                                mma_i8(tmem + O_COL, ad, bd, id_o, (kb > 0 || k > 0));
+                            else
+                                mma_f16(tmem + O_COL, ad, bd, id_o, (kb > 0 || k > 0));
+                        }
+                    }
+                }
+            }
+            const uint32_t idesc = idesc_s8_s32_sparse(BW, MP);
+            const uint32_t acc = tmem + ACC_COL + 32 * issuer;
+            for (int kb = issuer; kb < nkb && ok; kb += NI) {
+                const int st = kb % S;
+                if (!(ok = wait_bar(&op_full[st], (kb / S) & 1, ab))) break;
+                tc_fence_after();
+                const uint32_t a0 = smem_base + OP_OFF + st * STAGE;
+                const uint32_t x0 = a0 + ASTAGE;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)  // kept codes 32 bytes apart, tokens 64
+                    mma_sp_i8(acc, sw128_kmajor_desc(a0 + 32 * j),
+                              sw128_kmajor_desc(x0 + (j >> 1) * XTILE + 64 * (j & 1)),
+                              tmem + META_COL + META_STAGE * st + 4 * j, idesc, (kb > issuer || j > 0));
+                mma_commit(&op_empty[st]);
+            }
+            if (ok) mma_commit(&acc_full);
+            mma_commit(&mma_done[issuer]);
+            mbar_wait_bounded(&mma_done[issuer], 0, kWaitLimitNs);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            grid_dependency_wait();  // Xq and Xo come from the previous kernel
+            for (int kb = 0; kb < nko; ++kb)
+                tma_load_2d(smem + XO_OFF + kb * XO_TILE, &tm_xo, kb * oke, m0, &o_full);
+            for (int u = 0; u < early; ++u)
+                tma_load_2d(smem + u * UNIT + WUNIT + MUNIT, &tm_x, u * XROW, m0, &w_full[u]);
+            int filled = early;
+            for (int u = early; u < nkb; ++u, ++filled) {
+                const int st = u % SPW;
+                if (!wait_bar(&w_empty[st], ((u / SPW) & 1) ^ 1, ab)) break;
+                mbar_arrive_expect_tx(&w_full[st], unit_bytes);
+                tma_load_2d(smem + st * UNIT, &tm_w, u * WROW, n0, &w_full[st]);
+                tma_load_2d(smem + st * UNIT + WUNIT, &tm_m, u * MROW, n0, &w_full[st]);
+                tma_load_2d(smem + st * UNIT + WUNIT + MUNIT, &tm_x, u * XROW, m0, &w_full[st]);
+            }
+            // never leave the CTA with a bulk copy still writing its shared memory
+            for (int i = 0; i < early; ++i)
+                mbar_wait_bounded(&w_full[i], ((filled - 1 - i) / SPW) & 1, kWaitLimitNs);
+            if (nko > 0) mbar_wait_bounded(&o_full, 0, kWaitLimitNs);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ kept codes -> A stage,
+        // position pairs -> tensor memory, token rows -> X tiles
+        const int q = warp & 3;           // TMEM lane quadrant
+        const int r = q * 32 + lane;      // W row in the tile = TMEM lane
+        const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
+        const int grp = (warp - 2) >> 2;  // this warp's group: k-blocks grp, grp + NG, ...
+        const int xt = ((warp - 2) & 3) * 32 + lane;  // 0 .. 127 within the group
+        const int n = n0 + r;
+        const bool n_ok = n < p.N;
+        float swn = 0.0f, swon = 0.0f, bn = 0.0f, sxm = 0.0f, sxom = 0.0f;
+        if (grp == 0 && !DEBUG) {
+            if (n_ok && p.Ki > 0) swn = p.sw[n];
+            if (n_ok && OUT_INT8 && nko > 0) swon = p.swo[n];
+            if (n_ok && p.bias != nullptr) bn = __half2float(__ushort_as_half(p.bias[n]));
+        }
+        grid_dependency_wait();  // sx (and sxo) come from the previous kernel
+        if (grp == 0 && !DEBUG && m0 + lane < p.M) {
+            if (p.Ki > 0) sxm = p.sx[m0 + lane];
+            if (OUT_INT8 && nko > 0) sxom = p.sxo[m0 + lane];
+        }
+        bool ok = true;
+        for (int kb = grp; kb < nkb && ok; kb += NG) {
+            const int st = kb % S, ps = kb % SPW;
+            ok = wait_bar(&op_empty[st], ((kb / S) & 1) ^ 1, ab);
+            ok = ok && wait_bar(&w_full[ps], (kb / SPW) & 1, ab);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            const uint8_t *unit = smem + ps * UNIT;
+            // the packed bytes into registers; the staging slot then goes back
+            // to the producer: W row r (4 chunks, 64-byte swizzle), its 32
+            // bytes of pairs, and two of the MP x 8 token chunks (128-byte swizzle)
+            uint4 wv[4], mv[2], xv[2];
+            const uint8_t *wr = unit + r * WROW;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) wv[c] = *reinterpret_cast<const uint4 *>(wr + ((c ^ ((r >> 1) & 3)) << 4));
+            mv[0] = *reinterpret_cast<const uint4 *>(unit + WUNIT + r * MROW);
+            mv[1] = *reinterpret_cast<const uint4 *>(unit + WUNIT + r * MROW + 16);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int task = xt + 128 * i, xr = task >> 3, xc = task & 7;
+                xv[i] = make_uint4(0, 0, 0, 0);
+                if (xr < MP)
+                    xv[i] = *reinterpret_cast<const uint4 *>(unit + WUNIT + MUNIT + xr * XROW + ((xc ^ (xr & 7)) << 4));
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&w_empty[ps]);
+            // kept codes: 64 packed bytes -> 128 widened bytes of row r
+            uint8_t *ar = smem + OP_OFF + st * STAGE + r * 128;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint4 a, b;
+                widen16_ordered(wv[c], a, b);
+                *reinterpret_cast<uint4 *>(ar + (((2 * c) ^ (r & 7)) << 4)) = a;
+                *reinterpret_cast<uint4 *>(ar + (((2 * c + 1) ^ (r & 7)) << 4)) = b;
+            }
+            // token chunk (xr, xc): widened bytes 32 xc .. 32 xc + 31 -> tile xc / 4
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int task = xt + 128 * i, xr = task >> 3, xc = task & 7;
+                if (xr >= MP) continue;
+                uint4 a, b;
+                widen16_ordered(xv[i], a, b);
+                uint8_t *xrow = smem + OP_OFF + st * STAGE + ASTAGE + (xc >> 2) * XTILE + xr * 128;
+                *reinterpret_cast<uint4 *>(xrow + (((2 * (xc & 3)) ^ (xr & 7)) << 4)) = a;
+                *reinterpret_cast<uint4 *>(xrow + (((2 * (xc & 3) + 1) ^ (xr & 7)) << 4)) = b;
+            }
+            // position pairs: 64 bits per MMA at a 4-column-aligned address.
+            // Groups past K_i (read as 0 in a ragged last k-block) get the
+            // valid pair (0, 1); their kept codes and tokens are 0.
+            uint32_t mw[8] = {mv[0].x, mv[0].y, mv[0].z, mv[0].w, mv[1].x, mv[1].y, mv[1].z, mv[1].w};
+            const int valid_words = (p.Ki - kb * KBL) / 32;  // 8 groups per word
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (i >= valid_words) mw[i] = 0x44444444u;
+            const uint32_t mt[16] = {mw[0], mw[1], 0u, 0u, mw[2], mw[3], 0u, 0u,
+                                     mw[4], mw[5], 0u, 0u, mw[6], mw[7], 0u, 0u};
+            tmem_st_32x32b_x16(t_lane + META_COL + META_STAGE * st, mt);
+            tmem_st_wait();
+            fence_proxy_async_smem();  // the stage's stores -> visible to the MMA
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&op_full[st]);
+        }
+        // ------------------------------------------------------------ epilogue (group 0)
+        if (grp == 0) {
+            ok = ok && wait_bar(&acc_full, 0, ab);
+            if (__all_sync(0xffffffffu, ok)) {
+                tc_fence_after();
+                for (int h = 0; h < 32 && m0 + h < p.M; h += 16) {
+                    uint32_t a[16], o[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) a[j] = o[j] = 0;
+                    if (nkb > 0) tmem_ld_32x32b_x16(t_lane + ACC_COL + h, a);
+                    if (nko > 0) tmem_ld_32x32b_x16(t_lane + O_COL + h, o);
+                    tmem_ld_wait();
+                    for (int i = 1; i < NI && i < nkb; ++i) {
+                        uint32_t t[16];
+                        tmem_ld_32x32b_x16(t_lane + ACC_COL + 32 * i + h, t);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) a[j] += t[j];
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int m = m0 + h + j;
+                        const float sx_m = __shfl_sync(0xffffffffu, sxm, h + j);
+                        const float sxo_m = __shfl_sync(0xffffffffu, sxom, h + j);
+                        if (m >= p.M || !n_ok) continue;
+                        const size_t at = (size_t)m * p.N + n;
+                        if (DEBUG) {
+                            if (p.Ki > 0) p.acc_dbg[at] = static_cast<int32_t>(a[j]) >> 8;
+                            if (OUT_INT8 && nko > 0 && p.acc_o_dbg) p.acc_o_dbg[at] = static_cast<int32_t>(o[j]);
+                            continue;
+                        }
+                        float y = p.Ki > 0 ? small_int_to_float(static_cast<int32_t>(a[j]) >> 8) * sx_m * swn : 0.0f;
+                        if (nko > 0)
+                            y += OUT_INT8 ? static_cast<float>(static_cast<int32_t>(o[j])) * sxo_m * swon
+                                          : __uint_as_float(o[j]);
+                        p.Y[at] = __half_as_ushort(__float2half_rn(y + bn));
+                    }
+                }
+                tc_fence_before();
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
 // ----------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -1603,11 +1947,86 @@ quik_status run_gemv(const GemmArgs &a, cudaStream_t stream) {
     return cudaLaunchKernelEx(&cfg, kern, mw, mx, mwo, mxo, p) == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
 }
 
+// 2:4-sparse weights: kept codes [N, K_i / 4] and position pairs
+// [N, K_i / 8]; tiles of 128 W rows x 32 tokens (16 when M <= 16).
+template <bool OUT_INT8, bool DEBUG>
+quik_status run_gemv24(const GemmArgs &a, cudaStream_t stream) {
+    const int Ki = a.K - a.k_o;
+    const bool outliers = a.k_o > 0 && a.Xo != nullptr;  // the debug entry may skip them
+    const uint32_t mp = a.M <= 16 ? 16 : 32;
+    CUtensorMap mw, mm, mx, mwo, mxo;
+    std::memset(&mw, 0, sizeof(mw));
+    std::memset(&mm, 0, sizeof(mm));
+    std::memset(&mx, 0, sizeof(mx));
+    std::memset(&mwo, 0, sizeof(mwo));
+    std::memset(&mxo, 0, sizeof(mxo));
+    if (Ki > 0) {
+        // kept codes: 64 bytes (256 positions) x 128 rows per box, 64-byte
+        // swizzle; pairs: 32 bytes x 128 rows; token rows: 128 bytes x 16 or
+        // 32 rows, 128-byte swizzle (rows past M read as 0)
+        if (!make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wq, Ki / 4, a.N, Ki / 4, sp24::WROW, sp24::BW,
+                      CU_TENSOR_MAP_SWIZZLE_64B) ||
+            !make_map(&mm, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wmeta, Ki / 8, a.N, Ki / 8, sp24::MROW, sp24::BW,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Xq, Ki / 2, a.M, Ki / 2, sp24::XROW, mp,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+            return QUIK_ERR_CUDA;
+    }
+    if (outliers) {
+        const CUtensorMapDataType dt = OUT_INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
+        const uint32_t oke = OUT_INT8 ? 128 : 64;
+        const uint64_t pitch = static_cast<uint64_t>(a.k_o) * (OUT_INT8 ? 1 : 2);
+        if (!make_map(&mwo, dt, a.Wo, a.k_o, a.N, pitch, oke, sp24::BW, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&mxo, dt, a.Xo, a.k_o, a.M, pitch, oke, mp, CU_TENSOR_MAP_SWIZZLE_128B))
+            return QUIK_ERR_CUDA;
+    }
+    GemmParams p{};
+    p.M = a.M;
+    p.N = a.N;
+    p.Ki = Ki;
+    p.k_o = outliers ? a.k_o : 0;
+    p.nkb_i = (Ki + sp24::KBL - 1) / sp24::KBL;
+    p.nkb_o = 0;
+    p.G = 1;
+    p.sx = a.sx;
+    p.sw = a.sw;
+    p.sxo = a.sxo;
+    p.swo = a.swo;
+    p.bias = a.bias;
+    p.Y = a.Y;
+    p.acc_dbg = a.acc_dbg;
+    p.acc_o_dbg = a.acc_o_dbg;
+    auto kern = w4a4_gemv24_kernel<OUT_INT8, DEBUG>;
+    if (!attribute_set_once(reinterpret_cast<const void *>(kern), sp24::SMEM)) return QUIK_ERR_CUDA;
+    const dim3 grid((a.N + sp24::BW - 1) / sp24::BW, (a.M + sp24::MT - 1) / sp24::MT);
+    if (!a.after_quantize) {
+        kern<<<grid, sp24::THREADS, sp24::SMEM, stream>>>(mw, mm, mx, mwo, mxo, p);
+        return cudaGetLastError() == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(sp24::THREADS);
+    cfg.dynamicSmemBytes = sp24::SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, mw, mm, mx, mwo, mxo, p) == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
+}
+
 // Per-channel scales: the CTA-pair kernel (faster than a single-CTA kernel
 // with 128-row tiles at every M measured, 16 to 4096); per-group scales: the
 // shared-memory-operand kernel.
 template <bool DEBUG>
 quik_status dispatch(const GemmArgs &a, cudaStream_t stream) {
+    if (a.sparse24) {  // 2:4-sparse INT4 weights: per-channel scales, INT4 activations
+        if (a.group != 0 || a.a8 || a.w8 || (a.K - a.k_o) % 128 != 0 ||
+            a.k_o > (a.out_int8 ? sp24::KO_MAX_I8 : sp24::KO_MAX_F16))
+            return QUIK_ERR_UNSUPPORTED;
+        return a.out_int8 ? run_gemv24<true, DEBUG>(a, stream) : run_gemv24<false, DEBUG>(a, stream);
+    }
     if (a.a8) {  // INT8 activations (W4A8, W8A8): per-token scales, the pair kernel
         if (a.group != 0) return QUIK_ERR_UNSUPPORTED;
         if (a.w8)

@@ -761,6 +761,82 @@ cudaError_t launch_q_n(const QParams &p, int group, bool out_int8, cudaStream_t 
     return out_int8 ? launch_q_w<false, true, NORM>(p, stream) : launch_q_w<false, false, NORM>(p, stream);
 }
 
+// ----------------------------------------------------------------- 2:4-sparse weight rows
+// The offline pack of 2:4-sparse INT4 weights ("QUIK" abstract: quantisation
+// plus 2:4 sparsity).  One CTA of 256 threads per row, plain code: the
+// reordered row is gathered into shared memory (fp16), the row's absmax over
+// the INT4 positions gives s = fl(m / 7); every aligned group of four keeps
+// its two largest magnitudes (lower position on ties) with codes
+// clamp(rint(v / s), -7, 7) from IEEE divisions; the outlier block is copied
+// (FP16) or quantised with fl(max / 127) (INT8).
+constexpr int kP24Threads = 256;
+
+__device__ __forceinline__ float block_max(float m, float *red) {
+    m = warp_max(m);
+    const int w = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) red[w] = m;
+    __syncthreads();
+    m = 0.0f;
+    for (int i = 0; i < kP24Threads / 32; ++i) m = fmaxf(m, red[i]);
+    __syncthreads();  // red is reused
+    return m;
+}
+
+__global__ void __launch_bounds__(kP24Threads) prune24_rows_kernel(Prune24Args a) {
+    extern __shared__ uint16_t row_s[];  // the reordered row, K fp16 values
+    __shared__ float red[kP24Threads / 32];
+    const int K = a.K, Ki = K - a.k_o, row = blockIdx.x;
+    const uint16_t *x = a.W + static_cast<size_t>(row) * K;
+    bool bad = false;
+    for (int j = threadIdx.x; j < K; j += kP24Threads) {
+        const int c = a.perm[j];
+        bad |= c < 0 || c >= K;
+        row_s[j] = (c >= 0 && c < K) ? x[c] : static_cast<uint16_t>(0);
+    }
+    if (__syncthreads_or(bad) && threadIdx.x == 0 && row == 0) atomicAdd(&g_quant_bad_perm, 1u);
+    float m = 0.0f;
+    for (int j = threadIdx.x; j < Ki; j += kP24Threads) m = fmaxf(m, fabsf(h2f(row_s[j])));
+    const float s = __fdiv_rn(block_max(m, red), 7.0f);
+    if (threadIdx.x == 0 && a.scale != nullptr) a.scale[row] = s;  // may be NULL when K_i == 0
+    // two groups (one metadata byte) per step
+    for (int u = threadIdx.x; u < Ki / 8; u += kP24Threads) {
+        uint32_t nibs = 0;
+        for (int h = 0; h < 2; ++h) {
+            const int t = 2 * u + h;
+            float g[4];
+            for (int i = 0; i < 4; ++i) g[i] = h2f(row_s[4 * t + i]);
+            int ka = 0;
+            for (int i = 1; i < 4; ++i)
+                if (fabsf(g[i]) > fabsf(g[ka])) ka = i;
+            int kb = -1;
+            for (int i = 0; i < 4; ++i)
+                if (i != ka && (kb < 0 || fabsf(g[i]) > fabsf(g[kb]))) kb = i;
+            const int i0 = min(ka, kb), i1 = max(ka, kb);
+            const int q0 = exact_code(g[i0], s, 7), q1 = exact_code(g[i1], s, 7);
+            a.Qs[static_cast<size_t>(row) * (Ki / 4) + t] =
+                static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
+            nibs |= static_cast<uint32_t>(i0 | (i1 << 2)) << (4 * h);
+        }
+        a.meta[static_cast<size_t>(row) * (Ki / 8) + u] = static_cast<uint8_t>(nibs);
+    }
+    if (a.k_o > 0) {
+        if (!a.out_int8) {
+            uint16_t *o = static_cast<uint16_t *>(a.O) + static_cast<size_t>(row) * a.k_o;
+            for (int i = threadIdx.x; i < a.k_o; i += kP24Threads) o[i] = row_s[Ki + i];
+        } else {
+            float om = 0.0f;
+            for (int i = threadIdx.x; i < a.k_o; i += kP24Threads) om = fmaxf(om, fabsf(h2f(row_s[Ki + i])));
+            const float so = __fdiv_rn(block_max(om, red), 127.0f);
+            if (threadIdx.x == 0) a.o_scale[row] = so;
+            int8_t *o = static_cast<int8_t *>(a.O) + static_cast<size_t>(row) * a.k_o;
+            for (int i = threadIdx.x; i < a.k_o; i += kP24Threads)
+                o[i] = static_cast<int8_t>(exact_code(h2f(row_s[Ki + i]), so, 127));
+        }
+    } else if (a.out_int8 && a.o_scale != nullptr && threadIdx.x == 0) {
+        a.o_scale[row] = 0.0f;
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_quantize_rows(const QuantizeArgs &a, cudaStream_t stream) {
@@ -769,6 +845,15 @@ cudaError_t launch_quantize_rows(const QuantizeArgs &a, cudaStream_t stream) {
     if (a.bits8 && a.group > 0) return cudaErrorInvalidValue;  // INT8 codes: per-row scales only
     if (a.gamma != nullptr) return launch_q_n<true>(p, a.group, a.out_int8, stream);
     return launch_q_n<false>(p, a.group, a.out_int8, stream);
+}
+
+cudaError_t launch_prune24_rows(const Prune24Args &a, cudaStream_t stream) {
+    if ((a.K - a.k_o) % 8 != 0) return cudaErrorInvalidValue;
+    const int smem = a.K * 2;
+    if (!attribute_set_once(reinterpret_cast<const void *>(prune24_rows_kernel), smem))
+        return cudaErrorInvalidConfiguration;
+    prune24_rows_kernel<<<a.rows, kP24Threads, smem, stream>>>(a);
+    return cudaGetLastError();
 }
 
 unsigned int take_quantize_errors(unsigned int *bad_perm) {

@@ -47,6 +47,23 @@ struct QuantizeArgs {
     float eps = 0.0f;
 };
 cudaError_t launch_quantize_rows(const QuantizeArgs &a, cudaStream_t stream);
+
+// 2:4-sparse INT4 rows of a [rows, K] fp16 matrix: reorder, keep the two
+// largest magnitudes of every aligned group of four INT4 positions, quantise
+// (per-row scale), write kept codes [rows, K_i / 4] and position pairs
+// [rows, K_i / 8]; the outlier block as launch_quantize_rows.
+struct Prune24Args {
+    const uint16_t *W;
+    const int32_t *perm;
+    int rows, K, k_o;
+    bool out_int8;
+    uint8_t *Qs;
+    uint8_t *meta;
+    float *scale;
+    void *O;
+    float *o_scale;
+};
+cudaError_t launch_prune24_rows(const Prune24Args &a, cudaStream_t stream);
 // Read and clear the quantise kernels' count of expired waits (returned) and
 // of perm entries outside [0, K) (stored in *bad_perm when given); synchronous.
 unsigned int take_quantize_errors(unsigned int *bad_perm);
@@ -62,7 +79,9 @@ struct GemmArgs {
     const float *sx;
     const void *Xo;
     const float *sxo;
-    const void *Wq;
+    const void *Wq;       // packed codes, or the kept codes [N, K_i / 4] of 2:4 weights
+    const uint8_t *Wmeta = nullptr;  // 2:4 weights: position pairs [N, K_i / 8]
+    bool sparse24 = false;           // W is 2:4-sparse (Wq + Wmeta)
     const float *sw;
     const void *Wo;
     const float *swo;

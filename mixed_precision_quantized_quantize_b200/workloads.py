@@ -49,6 +49,7 @@ class LayerConfig:
     act_bits: int = 4           # 4: INT4 activations (W4A4); 8: INT8 activations (W4A8)
     weight_bits: int = 4        # 4: INT4 weights; 8: INT8 weights (W8A8)
     rmsnorm: bool = False       # X is the hidden state before an RMS norm folded into the layer
+    sparse24: bool = False      # W pruned to 2:4 (two kept INT4 codes per group of four)
     description: str = field(default="", compare=False)
 
     @property
@@ -66,7 +67,10 @@ class LayerConfig:
         each), the outlier blocks, the fp32 scales, the fp16 output and bias."""
         groups = self.K_i // 128 if self.group else 1
         ob = 1 if self.outlier_int8 else 2
-        b = (self.M * self.act_bits + self.N * self.weight_bits) * self.K_i // 8  # Xq, Wq
+        if self.sparse24:  # kept codes (K_i / 4 bytes) and position pairs (K_i / 8) per W row
+            b = self.M * self.act_bits * self.K_i // 8 + self.N * (self.K_i // 4 + self.K_i // 8)
+        else:
+            b = (self.M * self.act_bits + self.N * self.weight_bits) * self.K_i // 8  # Xq, Wq
         b += (self.M + self.N) * self.k_o * ob           # Xo, Wo
         b += (self.M + self.N) * groups * 4              # sx, sw
         if self.outlier_int8 and self.k_o:
@@ -110,6 +114,13 @@ CONFIGS = {
         "llama7b_attn_rmsnorm_2048x4096x4096", M=2048, N=4096, K=4096, k_o=128, student_t=True,
         rmsnorm=True,
         description="the attention projection behind its RMS norm (norm folded into the quantiser)"),
+    "llama7b_up_sparse24_16x11008x4096": LayerConfig(
+        "llama7b_up_sparse24_16x11008x4096", M=16, N=11008, K=4096, k_o=128, sparse24=True,
+        description="the MLP up-projection, 16 tokens, with 2:4-sparse INT4 weights"),
+    "llama7b_attn_sparse24_2048x4096x4096": LayerConfig(
+        "llama7b_attn_sparse24_2048x4096x4096", M=2048, N=4096, K=4096, k_o=128, student_t=True,
+        sparse24=True,
+        description="the attention projection with 2:4-sparse INT4 weights"),
     "llama7b_down_fused_4096x4096x11008": LayerConfig(
         "llama7b_down_fused_4096x4096x11008", M=4096, N=4096, K=11008, k_o=256,
         outlier_mult=50.0, bias=True,

@@ -136,3 +136,19 @@ def test_rmsnorm_widest_rows_unsupported(L):
                                            good, None, None) == q.QUIK_ERR_UNSUPPORTED
     assert L.quik_rmsnorm_linear(ctypes.byref(s), good, good, 1e-5, good, good, good, good, None,
                                  None, good, good, 1 << 30, None) == q.QUIK_ERR_UNSUPPORTED
+
+
+def test_sparse24_shape_rules(L):
+    """2:4 weights need per-channel scales, INT4 activations and weights,
+    K_i % 128 == 0 and a small outlier block; anything else is unsupported
+    (rejected before any pointer is looked at)."""
+    good = ctypes.c_void_p(0x1000)
+    for args in ((16, 16, 512, 0, 128, 0, 4, 4),    # groups
+                 (16, 16, 512, 0, 0, 0, 8, 4),      # INT8 activations
+                 (16, 16, 512, 64, 0, 0, 4, 4),     # K_i = 448
+                 (16, 16, 1024, 256, 0, 0, 4, 4),   # 256 FP16 outlier channels
+                 (16, 16, 1024, 384, 0, 1, 4, 4)):  # 384 INT8 outlier channels
+        s = q.make_shape(*args)
+        assert L.quik_pack_weights_24(ctypes.byref(s), good, good, good, good, good, good, good,
+                                      None) == q.QUIK_ERR_UNSUPPORTED
+        assert L.quik_gemm_24(ctypes.byref(s), *([good] * 11), None) == q.QUIK_ERR_UNSUPPORTED
