@@ -91,8 +91,10 @@ struct Cfg {
     static constexpr int PK_OFF = SU * OP_STAGE;
     static constexpr int SMEM = PK_OFF + SP * PK_STAGE + 1024;  // + alignment slack
     // TMEM columns: non-grouped: INT32 sum [0,BN) + outlier sum [BN,2BN);
-    // grouped: two alternating group buffers [0,BN) and [BN,2BN).
-    static constexpr int TMEM_COLS = 2 * BN;
+    // grouped: NACC group buffers [b BN, (b+1) BN) taken in turn, so the MMA
+    // can run NACC - 1 groups ahead of the drain.
+    static constexpr int NACC = GROUPED ? 512 / BN : 2;
+    static constexpr int TMEM_COLS = NACC * BN;
     static constexpr int CHUNKS = (BM + BN) * (PK_ROW / 16);     // 16-byte packed chunks
     static constexpr int CHUNKS_PER_THREAD = CHUNKS / (NT * 32);
     static constexpr int EPI_COLS = BN / (NE / 4);                // columns per epilogue warp
@@ -187,7 +189,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
     constexpr int BN = C::BN, SP = C::SP, SU = C::SU, NT = C::NT, NE = C::NE;
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t pk_full[SP], pk_empty[SP], op_full[SU], op_empty[SU];
-    __shared__ uint64_t acc_full[2], acc_empty[2], mma_done;
+    __shared__ uint64_t acc_full[C::NACC], acc_empty[C::NACC], mma_done;
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     __shared__ unsigned err0_s;
@@ -199,7 +201,9 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
     const uint32_t smem_base = smem_u32(smem);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+    // token tiles vary fastest: the CTAs that share a W tile run in the same
+    // wave, so each W tile leaves DRAM about once (L2 serves the others)
+    const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < SP; ++s) {
@@ -210,7 +214,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
             mbar_init(&op_full[s], NT);
             mbar_init(&op_empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < C::NACC; ++b) {
             mbar_init(&acc_full[b], 1);
             mbar_init(&acc_empty[b], NE);
         }
@@ -264,8 +268,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 const int s = kb % SU;
                 uint32_t d = tmem;
                 if (C::GROUPED) {
-                    const int b = kb & 1;
-                    if (!(ok = wait_bar(&acc_empty[b], ((kb >> 1) & 1) ^ 1, abort_flag))) break;
+                    const int b = kb % C::NACC;
+                    if (!(ok = wait_bar(&acc_empty[b], ((kb / C::NACC) & 1) ^ 1, abort_flag))) break;
                     d = tmem + b * BN;
                 }
                 if (!(ok = wait_bar(&op_full[s], (kb / SU) & 1, abort_flag))) break;
@@ -280,14 +284,14 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                            id_i8, acc);
                 }
                 mma_commit(&op_empty[s]);
-                if (C::GROUPED) mma_commit(&acc_full[kb & 1]);
+                if (C::GROUPED) mma_commit(&acc_full[kb % C::NACC]);
             }
             if (p.nkb_o > 0 && ok) {
                 uint32_t d = tmem + BN;
                 int b = 0;
                 if (C::GROUPED) {
-                    b = p.nkb_i & 1;
-                    ok = wait_bar(&acc_empty[b], ((p.nkb_i >> 1) & 1) ^ 1, abort_flag);
+                    b = p.nkb_i % C::NACC;
+                    ok = wait_bar(&acc_empty[b], ((p.nkb_i / C::NACC) & 1) ^ 1, abort_flag);
                     d = tmem + b * BN;
                 }
                 for (int ko = 0; ko < p.nkb_o && ok; ++ko) {
@@ -479,7 +483,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
             for (int j = 0; j < C::EPI_COLS; ++j) ysum[j] = 0.0f;
             bool ok = true;
             for (int g = 0; g < p.nkb_i && ok; ++g) {
-                const int b = g & 1;
+                const int b = g % C::NACC;
                 // stage this group's weight scales for the warp's columns
 #pragma unroll
                 for (int cc = 0; cc < C::EPI_COLS; cc += 32) {
@@ -491,7 +495,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 const float sxg = (row_ok && QUIK_CHECK(g < p.G, 15))
                                       ? p.sx[(size_t)row * p.G + g] * (1.0f / 256.0f) : 0.0f;
                 __syncwarp();
-                ok = wait_bar(&acc_full[b], (g >> 1) & 1, abort_flag);
+                ok = wait_bar(&acc_full[b], (g / C::NACC) & 1, abort_flag);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
@@ -521,8 +525,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 if (lane == 0) mbar_arrive(&acc_empty[b]);
             }
             if (ok && p.nkb_o > 0) {
-                const int b = p.nkb_i & 1;
-                ok = wait_bar(&acc_full[b], (p.nkb_i >> 1) & 1, abort_flag);
+                const int b = p.nkb_i % C::NACC;
+                ok = wait_bar(&acc_full[b], (p.nkb_i / C::NACC) & 1, abort_flag);
                 if (__all_sync(0xffffffffu, ok)) {
                     tc_fence_after();
                     const float sxo = (row_ok && C::OUT_INT8) ? p.sxo[row] : 0.0f;
@@ -1806,7 +1810,7 @@ quik_status run(const GemmArgs &a, cudaStream_t stream) {
 
     auto kern = w4a4_gemm_kernel<C>;
     if (!attribute_set_once(reinterpret_cast<const void *>(kern), C::SMEM)) return QUIK_ERR_CUDA;
-    const dim3 grid((a.N + C::BN - 1) / C::BN, (a.M + BM - 1) / BM);
+    const dim3 grid((a.M + BM - 1) / BM, (a.N + C::BN - 1) / C::BN);
     kern<<<grid, C::THREADS, C::SMEM, stream>>>(mxq, mwq, mxo, mwo, p);
     return cudaGetLastError() == cudaSuccess ? QUIK_OK : QUIK_ERR_CUDA;
 }
