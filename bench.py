@@ -88,9 +88,12 @@ def gemm_source_hash() -> str:
 def gemm_kernel(cfg):
     """The GEMM kernel the library dispatches for this layer, and its profile file."""
     fits = cfg.k_o <= (256 if cfg.outlier_int8 else 128)
-    if cfg.sparse24:
+    if cfg.sparse24 and cfg.M <= 32:
         return ("w4a4_gemv24 (2:4-sparse INT4 weights as the sparse MMA operand, tcgen05.mma.sp "
                 "kind::i8; 128 W rows x 32 tokens per CTA)", f"w4a4_gemv24_{cfg.name}.md")
+    if cfg.sparse24:
+        return ("w4a4_gemm_pair on the 2:4 weights expanded to dense codes (more than 32 tokens; "
+                "the expansion is timed separately)", f"w4a4_gemm_{cfg.name}.md")
     if cfg.act_bits == 8:
         return (("w4a4_gemm_pair with INT8 activations and weights (W8A8)" if cfg.weight_bits == 8 else
                  "w4a4_gemm_pair with INT8 activations (W4A8; weights widened from INT4)")
@@ -319,7 +322,12 @@ def run_ours(args, rank, local_rank, world):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    ws = torch.empty((q.quik_workspace_size(shape),), dtype=torch.uint8, device=dev)
+    ws_bytes = q.quik_workspace_size_24(shape) if cfg.sparse24 else q.quik_workspace_size(shape)
+    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    # the 2:4 prefill path: the dense copy of the weights its layer call makes
+    prefill24 = cfg.sparse24 and cfg.M > 32
+    Wd = (torch.empty((cfg.N, cfg.K_i // 2), dtype=torch.uint8, device=dev)
+          if prefill24 else None)
 
     def step():
         # one layer call: quantise + reorder (behind the RMS norm, for a
@@ -345,7 +353,12 @@ def run_ours(args, rank, local_rank, world):
         else:
             q.quik_quantize_reorder(shape, X, perm, Xq, sx, Xo, sxo, stream=stream)
         ev[1].record(stream)
-        if cfg.sparse24:
+        if prefill24:
+            q.quik_expand_weights_24(shape, layer.Wq24, layer.Wmeta, Wd, stream=stream)
+            ev[3].record(stream)
+            q.quik_gemm(shape, Xq, sx, Xo, sxo, Wd, layer.w_scale, layer.Wo, layer.wo_scale, bias,
+                        Y, stream=stream)
+        elif cfg.sparse24:
             q.quik_gemm_24(shape, Xq, sx, Xo, sxo, layer.Wq24, layer.Wmeta, layer.w_scale, layer.Wo,
                            layer.wo_scale, bias, Y, stream=stream)
         else:
@@ -378,12 +391,15 @@ def run_ours(args, rank, local_rank, world):
     value, t_step = aggregate(step_s, cfg.ops, world, reduce_max)
     # per-kernel breakdown (separate, untimed-for-value pass)
     n_split = max(10, args.steps // 4)
-    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_split)]
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_split)]
     for i in range(n_split):
         flush.zero_()
         split_step(sev[i])
     torch.cuda.synchronize()
-    gemm_avg = reduce_max(float(np.mean([e[1].elapsed_time(e[2]) / 1e3 for e in sev])))
+    g0 = 3 if prefill24 else 1  # the GEMM starts after the expansion on the 2:4 prefill path
+    gemm_avg = reduce_max(float(np.mean([e[g0].elapsed_time(e[2]) / 1e3 for e in sev])))
+    expand_avg = (reduce_max(float(np.mean([e[1].elapsed_time(e[3]) / 1e3 for e in sev])))
+                  if prefill24 else None)
     quant_avg = reduce_max(float(np.mean([e[0].elapsed_time(e[1]) / 1e3 for e in sev])))
     split_avg = reduce_max(float(np.mean([e[0].elapsed_time(e[2]) / 1e3 for e in sev])))
 
@@ -450,7 +466,7 @@ def run_ours(args, rank, local_rank, world):
     int8_peak = float(peaks["bf16_tflops"]) * INT8_PER_BF16
     # the 2:4-sparse MMA does half the multiply-adds of the INT4 part: its
     # dense-equivalent peak is twice the dense one (ops stay 2 M N K)
-    sparse_x = 2.0 if cfg.sparse24 else 1.0
+    sparse_x = 2.0 if cfg.sparse24 and not prefill24 else 1.0
     tensor_peak = int8_peak * sparse_x
     gemm_tops = cfg.ops / gemm_avg / 1e12
     kernel_name, profile_file = gemm_kernel(cfg)
@@ -474,7 +490,7 @@ def run_ours(args, rank, local_rank, world):
             "algorithmic_bytes_per_launch": cfg.gemm_bytes,
             "peak_source": (f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
                             f"{INT8_PER_BF16} (nominal INT8:BF16 dense ratio)"
-                            + (" x 2 (2:4-sparse MMA, dense-equivalent)" if cfg.sparse24 else "")
+                            + (" x 2 (2:4-sparse MMA, dense-equivalent)" if sparse_x > 1 else "")
                             + "; integer ops counted 2 per multiply-add"),
         }
     line = {
@@ -505,14 +521,15 @@ def run_ours(args, rank, local_rank, world):
         "pct_int8_peak": round(100.0 * value / world / int8_peak, 2),
         "breakdown_us": {"quantize_reorder": round(quant_avg * 1e6, 2),
                          "w4a4_gemm": round(gemm_avg * 1e6, 2),
-                         "two_calls_with_event_between": round(split_avg * 1e6, 2)},
+                         "two_calls_with_event_between": round(split_avg * 1e6, 2),
+                         **({"expand_weights_24": round(expand_avg * 1e6, 2)} if prefill24 else {})},
         "roofline": roofline,
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
                 "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2,
                 "call": ("quik_linear_24" if cfg.sparse24 else "quik_rmsnorm_linear" if cfg.rmsnorm
                          else "quik_linear")
                         + " via QuikLinear, pinned host X in, host Y out"},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (3 if prefill24 else 2) * args.steps,
         "clocks": sampler.summary(),
         "context": context,
     }

@@ -248,8 +248,31 @@ QUIK_API quik_status quik_gemm_24(const quik_shape *shape, const void *Xq, const
                                   quik_stream_t stream);
 
 /*
+ * quik_expand_weights_24 -- the dense packed INT4 weights Wq [N, K_i / 2]
+ * (the layout of quik_pack_weights) that 2:4 weights stand for: the kept
+ * codes at their positions, zero elsewhere.  quik_gemm on them gives the
+ * same integer sums as quik_gemm_24 on (Wq24, Wmeta).  Needs only
+ * K_i % 128 == 0 (else QUIK_ERR_UNSUPPORTED); shape->M is not used.
+ */
+QUIK_API quik_status quik_expand_weights_24(const quik_shape *shape, const void *Wq24,
+                                            const void *Wmeta, void *Wq, quik_stream_t stream);
+
+/*
+ * quik_workspace_size_24 -- bytes of workspace quik_linear_24 needs:
+ * quik_workspace_size(shape), plus room for the expanded weights when
+ * M > 32.  Returns 0 for a shape the 2:4 path does not take.
+ */
+QUIK_API size_t quik_workspace_size_24(const quik_shape *shape);
+
+/*
  * quik_linear_24 -- quik_quantize_reorder into `workspace`
- * (quik_workspace_size(shape) bytes) followed by quik_gemm_24.
+ * (quik_workspace_size_24(shape) bytes) followed by the product.  Up to 32
+ * tokens the product is quik_gemm_24 (the sparse MMA: 3 bits per weight
+ * position cross HBM instead of 4).  With more tokens the weights are
+ * expanded into the workspace (quik_expand_weights_24) and quik_gemm's dense
+ * kernel runs: the sparse MMA's dense operand would take all of an SM's
+ * shared-memory bandwidth at prefill tile widths.  The integer sums are the
+ * same either way.
  */
 QUIK_API quik_status quik_linear_24(const quik_shape *shape, const void *X_f16, const int32_t *perm,
                                     const void *Wq24, const void *Wmeta, const float *w_scale,

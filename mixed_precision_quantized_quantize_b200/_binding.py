@@ -57,6 +57,8 @@ _SIGS = {
     "quik_gemm_24": (ctypes.c_int, [_S] + [_P] * 12),
     "quik_linear_24": (ctypes.c_int, [_S] + [_P] * 10 + [ctypes.c_size_t, _P]),
     "quik_gemm_24_i32_debug": (ctypes.c_int, [_S] + [_P] * 8),
+    "quik_expand_weights_24": (ctypes.c_int, [_S, _P, _P, _P, _P]),
+    "quik_workspace_size_24": (ctypes.c_size_t, [_S]),
     "quik_sync_check": (ctypes.c_int, [_P]),
     "quik_selftest_timeout": (ctypes.c_int, [ctypes.c_uint32, _P]),
     "quik_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -245,6 +247,16 @@ def quik_gemm_24_i32_debug(shape, Xq, Wq24, Wmeta, Xo, Wo, acc, acc_outlier, str
         _stream(stream)), "quik_gemm_24_i32_debug")
 
 
+def quik_expand_weights_24(shape, Wq24, Wmeta, Wq, stream=None):
+    _check(lib().quik_expand_weights_24(
+        ctypes.byref(shape), _ptr(Wq24, torch.uint8, "Wq24"), _ptr(Wmeta, torch.uint8, "Wmeta"),
+        _ptr(Wq, torch.uint8, "Wq"), _stream(stream)), "quik_expand_weights_24")
+
+
+def quik_workspace_size_24(shape: quik_shape) -> int:
+    return int(lib().quik_workspace_size_24(ctypes.byref(shape)))
+
+
 def quik_sync_check(stream=None) -> int:
     return int(lib().quik_sync_check(_stream(stream)))
 
@@ -374,12 +386,22 @@ def gemm24_i32(Xq, Wq24, Wmeta, K: int, k_o: int, Xo=None, Wo=None, stream=None)
     return acc, acc_o
 
 
+def expand_weights_24(Wq24: torch.Tensor, Wmeta: torch.Tensor, K: int, k_o: int, stream=None):
+    """Dense packed INT4 weights uint8 [N, K_i/2] that 2:4 weights stand for."""
+    N = Wq24.shape[0]
+    shape = make_shape(1, N, K, k_o)
+    Wq = torch.empty((N, (K - k_o) // 2), dtype=torch.uint8, device=Wq24.device)
+    quik_expand_weights_24(shape, Wq24, Wmeta, Wq, stream=stream)
+    return Wq
+
+
 class QuikLinear24:
     """A W4A4 + outlier linear layer with 2:4-sparse INT4 weights.
 
     ``QuikLinear24(W, perm, k_o, outlier_int8, bias)`` prunes and packs W once
     (quik_pack_weights_24); calling it on fp16 activations runs quik_linear_24
-    into a workspace it keeps.
+    into a workspace it keeps (above 32 tokens the workspace also holds the
+    weights expanded for the dense kernel).
     """
 
     def __init__(self, W: torch.Tensor, perm: torch.Tensor, k_o: int, outlier_int8: bool = False,
@@ -395,7 +417,9 @@ class QuikLinear24:
 
     def __call__(self, X: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
         M = X.shape[0]
-        need = quik_workspace_size(self.shape(M))
+        need = quik_workspace_size_24(self.shape(M))
+        if need == 0:
+            raise QuikError(QUIK_ERR_UNSUPPORTED, "quik_workspace_size_24")
         if self._ws is None or self._ws.numel() < need:
             self._ws = torch.empty((need,), dtype=torch.uint8, device=X.device)
         Y = out if out is not None else torch.empty((M, self.N), dtype=torch.float16, device=X.device)

@@ -108,6 +108,11 @@ quik_status check_ptrs24(const quik_shape *s, const void *Qs, const void *meta, 
     return QUIK_OK;
 }
 
+// 2:4 layers of more tokens than one sparse tile run the dense kernel on the
+// weights expanded into the workspace (the sparse MMA's B operand would take
+// all of an SM's shared-memory bandwidth at prefill tile widths).
+constexpr int kSparseTokens = 32;
+
 struct Workspace {
     size_t xq, sx, xo, sxo, total;
 };
@@ -331,6 +336,30 @@ quik_status quik_gemm_24(const quik_shape *shape, const void *Xq, const float *x
                        bias_f16, Y_f16, false, nullptr, nullptr, static_cast<cudaStream_t>(stream));
 }
 
+size_t quik_workspace_size_24(const quik_shape *shape) {
+    if (check_shape24(shape) != QUIK_OK) return 0;
+    size_t total = layout(shape).total;
+    if (shape->M > kSparseTokens)
+        total += round256(static_cast<size_t>(shape->N) * static_cast<size_t>(shape->K - shape->k_o) / 2);
+    return total;
+}
+
+quik_status quik_expand_weights_24(const quik_shape *shape, const void *Wq24, const void *Wmeta,
+                                   void *Wq, quik_stream_t stream) {
+    // a change of format only: the 2:4 storage rule (K_i % 128 == 0) is all it needs
+    quik_status st = check_shape(shape);
+    if (st != QUIK_OK) return st;
+    const int Ki = shape->K - shape->k_o;
+    if (Ki % 128 != 0) return QUIK_ERR_UNSUPPORTED;
+    if (Ki == 0) return QUIK_OK;
+    if (!ok_ptr(Wq24) || !ok_ptr(Wmeta) || !ok_ptr(Wq)) return QUIK_ERR_INVALID_ARG;
+    return quik::launch_expand24(static_cast<const uint8_t *>(Wq24), static_cast<const uint8_t *>(Wmeta),
+                                 shape->N, Ki, static_cast<uint8_t *>(Wq),
+                                 static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? QUIK_OK
+               : QUIK_ERR_CUDA;
+}
+
 quik_status quik_linear_24(const quik_shape *shape, const void *X_f16, const int32_t *perm,
                            const void *Wq24, const void *Wmeta, const float *w_scale,
                            const void *Wo, const float *wo_scale, const void *bias_f16,
@@ -342,13 +371,22 @@ quik_status quik_linear_24(const quik_shape *shape, const void *X_f16, const int
         return QUIK_ERR_INVALID_ARG;
     if ((st = check_ptrs24(shape, Wq24, Wmeta, w_scale, Wo, wo_scale)) != QUIK_OK) return st;
     const Workspace w = layout(shape);
-    if (!ok_ptr(workspace) || workspace_bytes < w.total) return QUIK_ERR_INVALID_ARG;
+    if (!ok_ptr(workspace) || workspace_bytes < quik_workspace_size_24(shape)) return QUIK_ERR_INVALID_ARG;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     void *Xq = ws + w.xq;
     float *sx = reinterpret_cast<float *>(ws + w.sx);
     void *Xo = ws + w.xo;
     float *sxo = int8_out(shape) ? reinterpret_cast<float *>(ws + w.sxo) : nullptr;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (shape->M > kSparseTokens) {
+        // prefill: expand the weights, quantise, then the dense kernel (the
+        // GEMM directly follows the quantiser, as quik_linear's does)
+        void *Wd = ws + w.total;
+        if ((st = quik_expand_weights_24(shape, Wq24, Wmeta, Wd, stream)) != QUIK_OK) return st;
+        if ((st = quantize(shape, shape->M, false, X_f16, perm, Xq, sx, Xo, sxo, s)) != QUIK_OK) return st;
+        return gemm_impl(shape, Xq, sx, Xo, sxo, Wd, w_scale, Wo, wo_scale, bias_f16, Y_f16, false,
+                         nullptr, nullptr, s, true);
+    }
     if ((st = quantize(shape, shape->M, false, X_f16, perm, Xq, sx, Xo, sxo, s)) != QUIK_OK) return st;
     return gemm24_impl(shape, Xq, sx, Xo, sxo, Wq24, Wmeta, w_scale, Wo, wo_scale, bias_f16, Y_f16,
                        false, nullptr, nullptr, s, true);

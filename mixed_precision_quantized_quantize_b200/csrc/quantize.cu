@@ -837,6 +837,31 @@ __global__ void __launch_bounds__(kP24Threads) prune24_rows_kernel(Prune24Args a
     }
 }
 
+// The dense packed INT4 rows [rows, K_i / 2] that 2:4 rows stand for: the
+// two kept codes of every group at their positions, zero elsewhere.  One
+// thread per metadata byte (two groups = eight positions = one 32-bit word of
+// the dense row).
+__global__ void expand24_kernel(const uint8_t *__restrict__ Qs, const uint8_t *__restrict__ meta,
+                                long long total, int Ki, uint32_t *__restrict__ Q) {
+    const int per_row = Ki / 8;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long row = i / per_row;
+        const int u = static_cast<int>(i - row * per_row);
+        const uint32_t m = meta[i];
+        const uint8_t *q = Qs + row * (Ki / 4) + 2 * u;
+        uint32_t word = 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t nib = (m >> (4 * h)) & 0xFu, codes = q[h];
+            const int p0 = 4 * h + static_cast<int>(nib & 3u), p1 = 4 * h + static_cast<int>(nib >> 2);
+            word |= (codes & 0xFu) << (4 * p0);
+            word |= (codes >> 4) << (4 * p1);
+        }
+        Q[row * (Ki / 8) + u] = word;
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_quantize_rows(const QuantizeArgs &a, cudaStream_t stream) {
@@ -853,6 +878,18 @@ cudaError_t launch_prune24_rows(const Prune24Args &a, cudaStream_t stream) {
     if (!attribute_set_once(reinterpret_cast<const void *>(prune24_rows_kernel), smem))
         return cudaErrorInvalidConfiguration;
     prune24_rows_kernel<<<a.rows, kP24Threads, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_expand24(const uint8_t *Qs, const uint8_t *meta, int rows, int Ki, uint8_t *Q,
+                            cudaStream_t stream) {
+    if (Ki % 128 != 0) return cudaErrorInvalidValue;
+    const long long total = static_cast<long long>(rows) * (Ki / 8);
+    if (total == 0) return cudaSuccess;
+    const int threads = 256;
+    const long long want = (total + threads - 1) / threads;
+    const int grid = static_cast<int>(want < 8LL * sm_count() ? want : 8LL * sm_count());
+    expand24_kernel<<<grid, threads, 0, stream>>>(Qs, meta, total, Ki, reinterpret_cast<uint32_t *>(Q));
     return cudaGetLastError();
 }
 

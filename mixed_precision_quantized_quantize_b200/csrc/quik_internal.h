@@ -64,6 +64,9 @@ struct Prune24Args {
     float *o_scale;
 };
 cudaError_t launch_prune24_rows(const Prune24Args &a, cudaStream_t stream);
+// The dense packed INT4 rows [rows, K_i / 2] of 2:4 rows (K_i % 128 == 0).
+cudaError_t launch_expand24(const uint8_t *Qs, const uint8_t *meta, int rows, int Ki, uint8_t *Q,
+                            cudaStream_t stream);
 // Read and clear the quantise kernels' count of expired waits (returned) and
 // of perm entries outside [0, K) (stored in *bad_perm when given); synchronous.
 unsigned int take_quantize_errors(unsigned int *bad_perm);

@@ -152,3 +152,14 @@ def test_sparse24_shape_rules(L):
         assert L.quik_pack_weights_24(ctypes.byref(s), good, good, good, good, good, good, good,
                                       None) == q.QUIK_ERR_UNSUPPORTED
         assert L.quik_gemm_24(ctypes.byref(s), *([good] * 11), None) == q.QUIK_ERR_UNSUPPORTED
+
+
+def test_sparse24_workspace_size(L):
+    """Up to 32 tokens the 2:4 layer needs the dense layer's workspace; with
+    more it also holds the expanded weights (N x K_i / 2 bytes, 256-aligned)."""
+    for M in (1, 16, 32, 33, 2048):
+        s = q.make_shape(M, 4096, 4096, 128)
+        base = L.quik_workspace_size(ctypes.byref(s))
+        extra = 0 if M <= 32 else -(-(4096 * 3968 // 2) // 256) * 256
+        assert L.quik_workspace_size_24(ctypes.byref(s)) == base + extra
+    assert L.quik_workspace_size_24(ctypes.byref(q.make_shape(16, 16, 512, 64))) == 0  # K_i = 448

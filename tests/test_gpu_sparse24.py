@@ -77,6 +77,20 @@ def test_pack24_bit_exact(shape):
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=[str(s) for s in SHAPES])
+def test_expand24_bit_exact(shape):
+    """The dense packed codes the 2:4 weights stand for (the prefill path)."""
+    M, N, K, k_o, int8, bias = shape
+    if K == k_o:
+        pytest.skip("no INT4 part")
+    cfg, d = _case(*shape, seed=24)
+    g = q.pack_weights_24(d["W"].to(DEV), d["perm"].to(DEV), k_o, int8)
+    Wd = q.expand_weights_24(g[0], g[1], K, k_o)
+    torch.cuda.synchronize()
+    ow = _oracle_w24(d, k_o, int8)
+    np.testing.assert_array_equal(Wd.cpu().numpy(), oracle.unpack24(ow[0], ow[1]))
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=[str(s) for s in SHAPES])
 def test_sums24_bit_exact(shape):
     M, N, K, k_o, int8, bias = shape
     cfg, d = _case(*shape, seed=22)
@@ -115,10 +129,19 @@ def test_linear24_within_tolerance(shape):
     X = d["X"].to(DEV)
     Y = layer(X)
     gx = q.quantize_reorder(X, perm_d, k_o, 0, int8)
-    Y2 = q.gemm_24(gx, (layer.Wq24, layer.Wmeta, layer.w_scale, layer.Wo, layer.wo_scale), K, k_o, b)
+    if M <= 32:  # the layer runs the sparse kernel
+        Y2 = q.gemm_24(gx, (layer.Wq24, layer.Wmeta, layer.w_scale, layer.Wo, layer.wo_scale), K, k_o, b)
+    else:        # the dense kernel on the expanded weights
+        Wd = q.expand_weights_24(layer.Wq24, layer.Wmeta, K, k_o) if K > k_o else \
+            torch.empty((N, 0), dtype=torch.uint8, device=DEV)
+        Y2 = q.gemm(gx, (Wd, layer.w_scale, layer.Wo, layer.wo_scale), K, k_o, 0, b)
     torch.cuda.synchronize()
     assert_y_close(Y.float().cpu().numpy(), _oracle_y24(d, k_o, int8), f"linear24 {shape}")
     np.testing.assert_array_equal(Y.cpu().numpy().view(np.uint16), Y2.cpu().numpy().view(np.uint16))
+    if M > 32 and K > k_o:  # the sparse kernel on the same inputs, within the criterion
+        Y3 = q.gemm_24(gx, (layer.Wq24, layer.Wmeta, layer.w_scale, layer.Wo, layer.wo_scale), K, k_o, b)
+        torch.cuda.synchronize()
+        assert_y_close(Y3.float().cpu().numpy(), _oracle_y24(d, k_o, int8), f"gemm24 {shape}")
 
 
 def _samples(M, N, count, seed):
