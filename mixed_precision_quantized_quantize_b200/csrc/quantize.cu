@@ -839,26 +839,34 @@ __global__ void __launch_bounds__(kP24Threads) prune24_rows_kernel(Prune24Args a
 
 // The dense packed INT4 rows [rows, K_i / 2] that 2:4 rows stand for: the
 // two kept codes of every group at their positions, zero elsewhere.  One
-// thread per metadata byte (two groups = eight positions = one 32-bit word of
-// the dense row).
+// thread per four metadata bytes: eight groups, 32 positions, 16 bytes of the
+// dense row (every row pitch is a multiple of 16 bytes for K_i % 128 == 0).
 __global__ void expand24_kernel(const uint8_t *__restrict__ Qs, const uint8_t *__restrict__ meta,
-                                long long total, int Ki, uint32_t *__restrict__ Q) {
-    const int per_row = Ki / 8;
+                                long long total, int Ki, uint4 *__restrict__ Q) {
+    const int per_row = Ki / 32;
     for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
          i += static_cast<long long>(gridDim.x) * blockDim.x) {
         const long long row = i / per_row;
         const int u = static_cast<int>(i - row * per_row);
-        const uint32_t m = meta[i];
-        const uint8_t *q = Qs + row * (Ki / 4) + 2 * u;
-        uint32_t word = 0;
+        const uint32_t m4 = *reinterpret_cast<const uint32_t *>(meta + row * (Ki / 8) + 4 * u);
+        const uint2 q8 = *reinterpret_cast<const uint2 *>(Qs + row * (Ki / 4) + 8 * u);
+        uint32_t out[4];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const uint32_t nib = (m >> (4 * h)) & 0xFu, codes = q[h];
-            const int p0 = 4 * h + static_cast<int>(nib & 3u), p1 = 4 * h + static_cast<int>(nib >> 2);
-            word |= (codes & 0xFu) << (4 * p0);
-            word |= (codes >> 4) << (4 * p1);
+        for (int w = 0; w < 4; ++w) {  // metadata byte w: groups 2w and 2w + 1
+            const uint32_t m = (m4 >> (8 * w)) & 0xFFu;
+            const uint32_t qw = w < 2 ? q8.x : q8.y;  // their kept-code bytes
+            uint32_t word = 0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t nib = (m >> (4 * h)) & 0xFu;
+                const uint32_t codes = (qw >> (8 * (2 * (w & 1) + h))) & 0xFFu;
+                const int p0 = 4 * h + static_cast<int>(nib & 3u), p1 = 4 * h + static_cast<int>(nib >> 2);
+                word |= (codes & 0xFu) << (4 * p0);
+                word |= (codes >> 4) << (4 * p1);
+            }
+            out[w] = word;
         }
-        Q[row * (Ki / 8) + u] = word;
+        Q[row * (Ki / 32) + u] = make_uint4(out[0], out[1], out[2], out[3]);
     }
 }
 
@@ -884,12 +892,12 @@ cudaError_t launch_prune24_rows(const Prune24Args &a, cudaStream_t stream) {
 cudaError_t launch_expand24(const uint8_t *Qs, const uint8_t *meta, int rows, int Ki, uint8_t *Q,
                             cudaStream_t stream) {
     if (Ki % 128 != 0) return cudaErrorInvalidValue;
-    const long long total = static_cast<long long>(rows) * (Ki / 8);
+    const long long total = static_cast<long long>(rows) * (Ki / 32);
     if (total == 0) return cudaSuccess;
     const int threads = 256;
     const long long want = (total + threads - 1) / threads;
     const int grid = static_cast<int>(want < 8LL * sm_count() ? want : 8LL * sm_count());
-    expand24_kernel<<<grid, threads, 0, stream>>>(Qs, meta, total, Ki, reinterpret_cast<uint32_t *>(Q));
+    expand24_kernel<<<grid, threads, 0, stream>>>(Qs, meta, total, Ki, reinterpret_cast<uint4 *>(Q));
     return cudaGetLastError();
 }
 
