@@ -163,3 +163,32 @@ def test_sparse24_workspace_size(L):
         extra = 0 if M <= 32 else -(-(4096 * 3968 // 2) // 256) * 256
         assert L.quik_workspace_size_24(ctypes.byref(s)) == base + extra
     assert L.quik_workspace_size_24(ctypes.byref(q.make_shape(16, 16, 512, 64))) == 0  # K_i = 448
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/quik.h compiles as C99 and a C program links against the
+    library and calls it (size queries need no GPU)."""
+    import os
+    import shutil
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    libdir = os.path.dirname(q.LIB_PATH)
+    src = tmp_path / "abi.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "quik.h"\n'
+        "int main(void) {\n"
+        "    quik_shape s = {2048, 4096, 4096, 128, 0, QUIK_OUTLIER_FP16, 4, 4};\n"
+        '    printf("%zu %zu %s\\n", quik_workspace_size(&s), quik_workspace_size_24(&s),\n'
+        "           quik_status_string(QUIK_ERR_UNSUPPORTED));\n"
+        "    return 0;\n}\n")
+    exe = tmp_path / "abi"
+    subprocess.check_call([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", inc,
+                           str(src), "-o", str(exe), "-L", libdir, "-lquik_b200",
+                           f"-Wl,-rpath,{libdir}"])
+    out = subprocess.check_output([str(exe)], text=True).split()
+    s = q.make_shape(2048, 4096, 4096, 128)
+    assert int(out[0]) == q.quik_workspace_size(s)
+    assert int(out[1]) == q.quik_workspace_size_24(s)
+    assert out[2] == "QUIK_ERR_UNSUPPORTED"
