@@ -265,6 +265,28 @@ def cpu_baseline(cfg, d, budget_s: float = 10.0):
                       f"(quantise + fp64 layer output), {dt:.1f} s"}
 
 
+# ----------------------------------------------------------------- path roofline
+def path_roofline(cfg, peaks: dict, t_step_s: float) -> dict:
+    """The layer call's floor, serial: the quantiser's bytes at HBM speed,
+    then the GEMM's slower of its tensor work and its bytes.  The INT4 part
+    runs at the INT8 rate (twice that on the 2:4 sparse kernel), an FP16
+    outlier block at the FP16 rate (the bf16 figure), an INT8 one at the INT8
+    rate."""
+    bw = float(peaks["hbm_gbs"]) * 1e9
+    p_f16 = float(peaks["bf16_tflops"]) * 1e12
+    p_i8 = p_f16 * INT8_PER_BF16
+    p_int4 = p_i8 * (2.0 if cfg.sparse24 and cfg.M <= 32 else 1.0)
+    p_out = p_i8 if cfg.outlier_int8 else p_f16
+    t_tensor = 2.0 * cfg.M * cfg.N * cfg.K_i / p_int4 + 2.0 * cfg.M * cfg.N * cfg.k_o / p_out
+    t_gemm = max(t_tensor, cfg.gemm_bytes / bw)
+    t_quant = cfg.quant_bytes / bw
+    t_roof = t_gemm + t_quant
+    return {"t_roof_us": round(t_roof * 1e6, 4), "t_us": round(t_step_s * 1e6, 2),
+            "frac": round(t_roof / t_step_s, 4) if t_step_s > 0 else None,
+            "gemm_roof_us": round(t_gemm * 1e6, 4), "quantise_roof_us": round(t_quant * 1e6, 4),
+            "gemm_bound": "tensor" if t_tensor >= cfg.gemm_bytes / bw else "hbm"}
+
+
 # ----------------------------------------------------------------- aggregation
 def aggregate(step_times_s, ops_per_rank: float, world: int, reduce_max):
     """Whole-job throughput from this rank's per-step times (weak scaling:
@@ -524,6 +546,7 @@ def run_ours(args, rank, local_rank, world):
                          "two_calls_with_event_between": round(split_avg * 1e6, 2),
                          **({"expand_weights_24": round(expand_avg * 1e6, 2)} if prefill24 else {})},
         "roofline": roofline,
+        "path_roofline": path_roofline(cfg, peaks, t_step),
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
                 "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2,
                 "call": ("quik_linear_24" if cfg.sparse24 else "quik_rmsnorm_linear" if cfg.rmsnorm

@@ -81,6 +81,20 @@ class LayerConfig:
         return b
 
 
+    @property
+    def quant_bytes(self) -> int:
+        """Bytes the activation quantiser must move: the fp16 row read once,
+        the codes, outlier block and scales written."""
+        groups = self.K_i // 128 if self.group else 1
+        b = self.M * self.K * 2                                      # X
+        b += self.M * self.act_bits * self.K_i // 8                  # Xq
+        b += self.M * self.k_o * (1 if self.outlier_int8 else 2)     # Xo
+        b += self.M * groups * 4                                     # sx
+        if self.outlier_int8 and self.k_o:
+            b += self.M * 4                                          # sxo
+        return b
+
+
 # The five layer workloads (the third has three token counts).
 CONFIGS = {
     "tiny_16x256x256": LayerConfig(
