@@ -1,17 +1,27 @@
-"""The mbarrier protocols of the 2:4 decode kernel and the grouped-scale
-kernel, run on the CPU under random schedules (no GPU).
+"""The mbarrier protocols of the GEMM kernels (the CTA-pair kernel, the dense
+and 2:4 decode kernels, the grouped-scale kernel), run on the CPU under
+random schedules (no GPU).
 
 An mbarrier completes a phase when its expected arrivals have come; a wait
 on parity P passes while the barrier's current phase parity differs from P.
 That wait is exact only if the phase the waiter wants is the one in progress
 or the one just completed: a waiter two phases behind would block on a phase
-that already passed, one two phases ahead would pass early.  Each kernel
-role below is the sequence of waits and arrivals its code makes (with the
-same stage counts), the waits written as the phase they want; completions
-of TMA copies and tensor-core commits arrive at random later steps.  The
-simulation asserts the exactness condition at every step a waiter is
-blocked, that no barrier gets more arrivals than a phase takes, and that no
-schedule deadlocks.
+that already passed, one two phases ahead would pass early.
+
+Each kernel role below is the sequence of waits, arrivals and buffer
+accesses its code makes (with the kernel's stage counts), the waits written
+as the phase they want.  Completions of TMA copies and tensor-core commits
+arrive at random later steps.  Buffers are owned while in use: an operand
+stage by the MMA from its full-wait until its commit lands, a staging slot
+by its readers from their full-wait until their empty-arrival, an
+accumulator by the drain while it reads it.  The simulation asserts:
+
+* the exactness condition, at every step a waiter is blocked;
+* that no barrier gets more arrivals than a phase takes;
+* that nothing writes a buffer while another role still owns it (a TMA copy
+  into a staging slot, unpacked operands into a stage, an MMA into an
+  accumulator);
+* that no schedule deadlocks.
 """
 import random
 
@@ -30,11 +40,20 @@ class Bar:
             self.pending = self.count
 
 
-def run(roles, seed, max_steps=200000):
-    """roles: generators of ('wait', bar, phase), ('arrive', bar), ('async', bar)."""
+class Buf:
+    """A buffer and how many roles own it right now."""
+
+    def __init__(self, name):
+        self.name, self.owners = name, 0
+
+
+def run(roles, seed, max_steps=400000):
+    """roles: generators of ('wait', bar, phase), ('arrive', bar),
+    ('async', bar[, buf released when it lands]), ('own', buf),
+    ('free', buf), ('write', buf)."""
     rng = random.Random(seed)
     live = [[r, next(r, None)] for r in roles]
-    asyncs = []  # arrivals still in flight (copies, commits)
+    asyncs = []  # (barrier, buffer released when the arrival lands) still in flight
     for _ in range(max_steps):
         live = [x for x in live if x[1] is not None]
         for _, act in live:  # every blocked waiter: the exactness condition
@@ -47,35 +66,50 @@ def run(roles, seed, max_steps=200000):
             assert not live, "deadlock"
             return
         if asyncs and (not ready or rng.random() < 0.3):
-            asyncs.pop(rng.randrange(len(asyncs))).arrive()
+            bar, buf = asyncs.pop(rng.randrange(len(asyncs)))
+            if buf is not None:
+                buf.owners -= 1
+            bar.arrive()
             continue
         x = rng.choice(ready)
         act = x[1]
         if act[0] == "arrive":
             act[1].arrive()
         elif act[0] == "async":
-            asyncs.append(act[1])
+            asyncs.append((act[1], act[2] if len(act) > 2 else None))
+        elif act[0] == "own":
+            act[1].owners += 1
+        elif act[0] == "free":
+            act[1].owners -= 1
+        elif act[0] == "write":
+            assert act[1].owners == 0, f"{act[1].name} written while in use"
         x[1] = next(x[0], None)
     raise AssertionError("schedule did not finish")
 
 
-# ----------------------------------------------------------------- 2:4 decode kernel
-def gemv24_roles(nkb, nko, S=4, SPW=4, NG=4, NI=2):
+# ----------------------------------------------------------------- decode kernels (dense and 2:4)
+def decode_roles(nkb, nko, S=4, SPW=4, NG=4, NI=2):
+    """Producer, NG groups of four unpack warps (group g: k-blocks g, g + NG,
+    ...), NI MMA issuers (issuer i: k-blocks i, i + NI, ...)."""
     w_full = [Bar(1) for _ in range(SPW)]
     w_empty = [Bar(4) for _ in range(SPW)]  # the four warps of a group
     op_full = [Bar(4) for _ in range(S)]
     op_empty = [Bar(1) for _ in range(S)]
     o_full, acc_full = Bar(1), Bar(NI)
+    slot = [Buf(f"staging slot {i}") for i in range(SPW)]
+    stage = [Buf(f"operand stage {i}") for i in range(S)]
     early = min(nkb, SPW)
 
     def producer():
         for u in range(early):          # the first units, expected before the CTA barrier
+            yield ("write", slot[u])
             yield ("async", w_full[u])
         if nko:
             yield ("async", o_full)
         for u in range(early, nkb):
             st = u % SPW
             yield ("wait", w_empty[st], u // SPW - 1)
+            yield ("write", slot[st])
             yield ("async", w_full[st])
 
     def group_warp(g):
@@ -84,7 +118,10 @@ def gemv24_roles(nkb, nko, S=4, SPW=4, NG=4, NI=2):
             if kb >= S:                 # a fresh barrier passes the first wait
                 yield ("wait", op_empty[st], kb // S - 1)
             yield ("wait", w_full[ps], kb // SPW)
+            yield ("own", slot[ps])     # the packed bytes into registers
+            yield ("free", slot[ps])
             yield ("arrive", w_empty[ps])
+            yield ("write", stage[st])  # unpacked operands (and pairs) into the stage
             yield ("arrive", op_full[st])
         if g == 0:                      # the epilogue
             yield ("wait", acc_full, 0)
@@ -95,7 +132,8 @@ def gemv24_roles(nkb, nko, S=4, SPW=4, NG=4, NI=2):
         for kb in range(i, nkb, NI):
             st = kb % S
             yield ("wait", op_full[st], kb // S)
-            yield ("async", op_empty[st])   # tcgen05.commit
+            yield ("own", stage[st])
+            yield ("async", op_empty[st], stage[st])   # tcgen05.commit
         yield ("async", acc_full)
 
     return ([producer()] + [group_warp(g) for g in range(NG) for _ in range(4)] +
@@ -104,25 +142,120 @@ def gemv24_roles(nkb, nko, S=4, SPW=4, NG=4, NI=2):
 
 @pytest.mark.parametrize("nkb", [0, 1, 2, 3, 4, 5, 7, 8, 16, 31, 33])
 @pytest.mark.parametrize("nko", [0, 1])
-def test_gemv24_protocol(nkb, nko):
+def test_sparse_decode_protocol(nkb, nko):
+    """The 2:4 decode kernel: 4 operand stages, 4 staging units."""
     for seed in range(40):
-        run(gemv24_roles(nkb, nko), seed)
+        run(decode_roles(nkb, nko), seed)
+
+
+@pytest.mark.parametrize("nkb", [1, 4, 8, 9, 10, 11, 31, 64])
+@pytest.mark.parametrize("nko", [0, 1])
+def test_dense_decode_protocol(nkb, nko):
+    """The dense decode kernel: 8 operand stages, 10 staging units."""
+    for seed in range(30):
+        run(decode_roles(nkb, nko, S=8, SPW=10), seed)
+
+
+# ----------------------------------------------------------------- CTA-pair kernel
+def pair_roles(nkb_i, nkb_o, S=4, SP=4, NA=4, NB=8, b_waits_outliers=True):
+    """Two CTAs; the leader's operand-full barriers take the arrivals of
+    every A and B warp of both CTAs (remote arrivals); each commit arrives on
+    both CTAs' operand-empty barriers; each CTA has its own staging ring.
+    Outlier k-blocks take two staging units (Wo rows, then Xo rows)."""
+    nkb = nkb_i + nkb_o
+    nunits = nkb_i + 2 * nkb_o
+    op_full = [Bar(2 * (NA + NB)) for _ in range(S)]            # the leader's
+    op_empty = [[Bar(1) for _ in range(S)] for _ in range(2)]   # per CTA
+    pk_full = [[Bar(1) for _ in range(SP)] for _ in range(2)]
+    pk_empty = [[Bar(NB) for _ in range(SP)] for _ in range(2)]
+    acc_full = [Bar(1), Bar(1)]
+    drain = Bar(1)
+    slot = [[Buf(f"CTA {c} staging slot {i}") for i in range(SP)] for c in range(2)]
+    stage = [[Buf(f"CTA {c} operand stage {i}") for i in range(S)] for c in range(2)]
+
+    def issuer():
+        for kb in range(nkb):
+            if kb == nkb_i and nkb_i:   # the outlier sums reuse the A-stage columns
+                yield ("async", drain)
+                yield ("wait", drain, 0)
+            st = kb % S
+            yield ("wait", op_full[st], kb // S)
+            for c in range(2):
+                yield ("own", stage[c][st])
+            for c in range(2):          # commit, multicast to both CTAs
+                yield ("async", op_empty[c][st], stage[c][st])
+        yield ("async", acc_full[0])
+        yield ("async", acc_full[1])
+
+    def producer(c):
+        for u in range(nunits):
+            st = u % SP
+            if u >= SP:
+                yield ("wait", pk_empty[c][st], u // SP - 1)
+            yield ("write", slot[c][st])
+            yield ("async", pk_full[c][st])
+
+    def a_warp(c):
+        for kb in range(nkb):
+            st = kb % S
+            if kb >= S:
+                yield ("wait", op_empty[c][st], kb // S - 1)
+            if kb < nkb_i:
+                yield ("write", stage[c][st])   # its rows into the tensor-memory stage
+            yield ("arrive", op_full[st])
+        yield ("wait", acc_full[c], 0)
+
+    def b_warp(c):
+        u = 0
+        for kb in range(nkb):
+            st = kb % S
+            if kb >= S and (b_waits_outliers or kb < nkb_i):
+                yield ("wait", op_empty[c][st], kb // S - 1)
+            for _ in range(1 if kb < nkb_i else 2):
+                ps = u % SP
+                yield ("wait", pk_full[c][ps], u // SP)
+                yield ("own", slot[c][ps])
+                yield ("write", stage[c][st])
+                yield ("free", slot[c][ps])
+                yield ("arrive", pk_empty[c][ps])
+                u += 1
+            yield ("arrive", op_full[st])
+        yield ("wait", acc_full[c], 0)
+
+    roles = [issuer()]
+    for c in range(2):
+        roles += [producer(c)] + [a_warp(c) for _ in range(NA)] + [b_warp(c) for _ in range(NB)]
+    return roles
+
+
+@pytest.mark.parametrize("nkb_i", [0, 1, 3, 4, 5, 8, 31, 64])
+@pytest.mark.parametrize("nkb_o", [0, 1, 2])
+def test_pair_protocol(nkb_i, nkb_o):
+    if nkb_i + nkb_o == 0:
+        pytest.skip("no k-blocks")
+    for seed in range(15):
+        run(pair_roles(nkb_i, nkb_o), seed)
 
 
 # ----------------------------------------------------------------- grouped-scale kernel
-def grouped_roles(nkb_i, nkb_o, SP=4, SU=4, NT=4, NE=8, NACC=4):
+def grouped_roles(nkb_i, nkb_o, SP=4, SU=4, NT=4, NE=8, NACC=4, drain_phase_div=None):
     pk_full = [Bar(1) for _ in range(SP)]
     pk_empty = [Bar(NT) for _ in range(SP)]
     op_full = [Bar(NT) for _ in range(SU)]
     op_empty = [Bar(1) for _ in range(SU)]
     acc_full = [Bar(1) for _ in range(NACC)]
     acc_empty = [Bar(NE) for _ in range(NACC)]
+    slot = [Buf(f"staging slot {i}") for i in range(SP)]
+    stage = [Buf(f"operand stage {i}") for i in range(SU)]
+    acc = [Buf(f"accumulator {i}") for i in range(NACC)]
+    div = drain_phase_div or NACC
 
     def producer():
         for kb in range(nkb_i):
             s = kb % SP
             if kb >= SP:
                 yield ("wait", pk_empty[s], kb // SP - 1)
+            yield ("write", slot[s])
             yield ("async", pk_full[s])
 
     def unpack_warp(t):
@@ -131,11 +264,16 @@ def grouped_roles(nkb_i, nkb_o, SP=4, SU=4, NT=4, NE=8, NACC=4):
             if kb >= nkb_i:             # outlier k-block: by TMA, one warp's copy
                 if kb >= SU:
                     yield ("wait", op_empty[su], kb // SU - 1)
+                if t == 0:
+                    yield ("write", stage[su])
                 yield ("async" if t == 0 else "arrive", op_full[su])
                 continue
             yield ("wait", pk_full[sp], kb // SP)
             if kb >= SU:
                 yield ("wait", op_empty[su], kb // SU - 1)
+            yield ("own", slot[sp])
+            yield ("write", stage[su])
+            yield ("free", slot[sp])
             yield ("arrive", pk_empty[sp])
             yield ("arrive", op_full[su])
 
@@ -145,23 +283,29 @@ def grouped_roles(nkb_i, nkb_o, SP=4, SU=4, NT=4, NE=8, NACC=4):
             if kb >= NACC:
                 yield ("wait", acc_empty[b], kb // NACC - 1)
             yield ("wait", op_full[s], kb // SU)
-            yield ("async", op_empty[s])
+            yield ("write", acc[b])     # this group's sums overwrite the buffer
+            yield ("own", stage[s])
+            yield ("async", op_empty[s], stage[s])
             yield ("async", acc_full[b])
         if nkb_o:
             b = nkb_i % NACC
             if nkb_i >= NACC:
                 yield ("wait", acc_empty[b], nkb_i // NACC - 1)
+            yield ("write", acc[b])
             for ko in range(nkb_o):
                 kb = nkb_i + ko
                 s = kb % SU
                 yield ("wait", op_full[s], kb // SU)
-                yield ("async", op_empty[s])
+                yield ("own", stage[s])
+                yield ("async", op_empty[s], stage[s])
             yield ("async", acc_full[b])
 
     def drain_warp():
         for g in range(nkb_i):
             b = g % NACC
-            yield ("wait", acc_full[b], g // NACC)
+            yield ("wait", acc_full[b], g // div)
+            yield ("own", acc[b])
+            yield ("free", acc[b])
             yield ("arrive", acc_empty[b])
         if nkb_o:
             yield ("wait", acc_full[nkb_i % NACC], nkb_i // NACC)
@@ -177,13 +321,22 @@ def test_grouped_protocol(nkb_i, nkb_o):
         run(grouped_roles(nkb_i, nkb_o), seed)
 
 
+# ----------------------------------------------------------------- the checker itself
+def _caught(make, seeds=60):
+    for seed in range(seeds):
+        try:
+            run(make(), seed)
+        except AssertionError:
+            return True
+    return False
+
+
 def test_checker_catches_a_ring_filled_out_of_order():
-    """The checker itself: a producer that runs two phases ahead (no wait on
-    the empty barrier) trips the exactness assertion."""
+    """A producer that never waits on the empty barrier runs phases ahead."""
     full, empty = Bar(1), Bar(1)
 
     def producer():
-        for u in range(6):
+        for _ in range(6):
             yield ("arrive", full)
 
     def consumer():
@@ -191,6 +344,15 @@ def test_checker_catches_a_ring_filled_out_of_order():
             yield ("wait", full, u)
             yield ("arrive", empty)
 
-    with pytest.raises(AssertionError):
-        for seed in range(20):
-            run([producer(), consumer()], seed)
+    assert _caught(lambda: [producer(), consumer()])
+
+
+def test_checker_catches_a_stage_overwritten_under_the_mma():
+    """B warps that skip the empty wait on the outlier k-blocks (the phases
+    still add up) overwrite a stage the MMA still reads."""
+    assert _caught(lambda: pair_roles(9, 4, b_waits_outliers=False))
+
+
+def test_checker_catches_a_wrong_accumulator_phase():
+    """A drain that waits with the two-buffer phase on four buffers."""
+    assert _caught(lambda: grouped_roles(9, 0, drain_phase_div=2))
