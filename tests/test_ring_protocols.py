@@ -1,6 +1,6 @@
-"""The mbarrier protocols of the GEMM kernels (the CTA-pair kernel, the dense
-and 2:4 decode kernels, the grouped-scale kernel), run on the CPU under
-random schedules (no GPU).
+"""The mbarrier and named-barrier protocols of the kernels (the CTA-pair
+kernel, the dense and 2:4 decode kernels, the grouped-scale kernel, the
+quantiser's team ring), run on the CPU under random schedules (no GPU).
 
 An mbarrier completes a phase when its expected arrivals have come; a wait
 on parity P passes while the barrier's current phase parity differs from P.
@@ -40,6 +40,21 @@ class Bar:
             self.pending = self.count
 
 
+class Sync:
+    """A named barrier (bar.sync) over n roles: each waits until all n have
+    arrived at the same generation."""
+
+    def __init__(self, n):
+        self.n, self.arrived, self.gen = n, 0, 0
+
+    def arrive(self):
+        self.arrived += 1
+        my = self.gen
+        if self.arrived == self.n:
+            self.arrived, self.gen = 0, self.gen + 1
+        return my
+
+
 class Buf:
     """A buffer and how many roles own it right now."""
 
@@ -50,9 +65,12 @@ class Buf:
 def run(roles, seed, max_steps=400000):
     """roles: generators of ('wait', bar, phase), ('arrive', bar),
     ('async', bar[, buf released when it lands]), ('own', buf),
-    ('free', buf), ('write', buf)."""
+    ('free', buf), ('write', buf), ('sync', named barrier)."""
     rng = random.Random(seed)
     live = [[r, next(r, None)] for r in roles]
+    for x in live:  # a role at a named barrier has arrived there
+        if x[1] is not None and x[1][0] == "sync":
+            x[1] = ("synced", x[1][1], x[1][1].arrive())
     asyncs = []  # (barrier, buffer released when the arrival lands) still in flight
     for _ in range(max_steps):
         live = [x for x in live if x[1] is not None]
@@ -61,7 +79,9 @@ def run(roles, seed, max_steps=400000):
                 bar, phase = act[1], act[2]
                 assert phase <= bar.done <= phase + 1, (
                     f"a wait for phase {phase} sees {bar.done} completed phases")
-        ready = [x for x in live if x[1][0] != "wait" or x[1][1].done >= x[1][2] + 1]
+        ready = [x for x in live
+                 if (x[1][0] != "wait" or x[1][1].done >= x[1][2] + 1) and
+                 (x[1][0] != "synced" or x[1][1].gen > x[1][2])]
         if not ready and not asyncs:
             assert not live, "deadlock"
             return
@@ -84,6 +104,8 @@ def run(roles, seed, max_steps=400000):
         elif act[0] == "write":
             assert act[1].owners == 0, f"{act[1].name} written while in use"
         x[1] = next(x[0], None)
+        if x[1] is not None and x[1][0] == "sync":
+            x[1] = ("synced", x[1][1], x[1][1].arrive())
     raise AssertionError("schedule did not finish")
 
 
@@ -321,6 +343,71 @@ def test_grouped_protocol(nkb_i, nkb_o):
         run(grouped_roles(nkb_i, nkb_o), seed)
 
 
+# ----------------------------------------------------------------- quantiser team
+def quantizer_roles(rows, NR, W=4, per_token=True, int8_out=False, norm=False):
+    """One team of W warps (warp 0's lane 0 leads) over `rows` rows, with NR
+    row slots: the leader waits for a row's copy, a named barrier hands the
+    row to the team (and ends every warp's use of the previous row's slot,
+    which the leader then refills with the row a ring ahead); the reductions
+    go through shared slots written by each warp's lane 0 before a named
+    barrier and read by all after it: per token, the absmax (and, with the
+    norm, the sum of squares) in slot j & 1, the INT8 outliers' absmax in
+    slot (j & 1) ^ 1; per group with the norm, the sum of squares in slot
+    j & 1 behind its own barrier."""
+    row_full = [Bar(1) for _ in range(NR)]
+    slot = [Buf(f"row slot {i}") for i in range(NR)]
+    red = [Buf(f"reduction slot {i}") for i in range(2)]
+    red_ss = [Buf(f"sum-of-squares slot {i}") for i in range(2)]
+    team = Sync(W)
+
+    def warp(w):
+        if w == 0:
+            for j in range(min(NR, rows)):   # the first rows, one per slot
+                yield ("write", slot[j])
+                yield ("async", row_full[j])
+        for j in range(rows):
+            if w == 0:
+                yield ("wait", row_full[j % NR], j // NR)
+            yield ("sync", team)             # the row is the team's; row j-1's slot is free
+            if w == 0 and j > 0 and j - 1 + NR < rows:
+                yield ("write", slot[(j - 1) % NR])
+                yield ("async", row_full[(j - 1) % NR])
+            yield ("own", slot[j % NR])      # gather (and sum of squares)
+            if norm and not per_token:       # grouped: the sum of squares' own barrier
+                yield ("write", red_ss[j & 1])
+                yield ("sync", team)
+                yield ("own", red_ss[j & 1])
+                yield ("free", red_ss[j & 1])
+            if per_token:
+                yield ("write", red[j & 1])
+                if norm:
+                    yield ("write", red_ss[j & 1])
+                yield ("sync", team)
+                yield ("own", red[j & 1])
+                yield ("free", red[j & 1])
+                if norm:
+                    yield ("own", red_ss[j & 1])
+                    yield ("free", red_ss[j & 1])
+            if int8_out:                     # the outlier block's absmax, the other slot
+                yield ("write", red[(j & 1) ^ 1])
+                yield ("sync", team)
+                yield ("own", red[(j & 1) ^ 1])
+                yield ("free", red[(j & 1) ^ 1])
+            yield ("free", slot[j % NR])     # codes and outliers written from registers
+
+    return [warp(w) for w in range(W)]
+
+
+@pytest.mark.parametrize("NR", [2, 3, 4])
+@pytest.mark.parametrize("mode", ["token", "token-int8", "group", "token-norm",
+                                  "token-norm-int8", "group-norm", "group-norm-int8"])
+def test_quantizer_team_protocol(NR, mode):
+    for rows in (1, 2, 3, 5, 9):
+        for seed in range(20):
+            run(quantizer_roles(rows, NR, per_token=mode.startswith("token"),
+                                int8_out=mode.endswith("int8"), norm="norm" in mode), seed)
+
+
 # ----------------------------------------------------------------- the checker itself
 def _caught(make, seeds=60):
     for seed in range(seeds):
@@ -351,6 +438,38 @@ def test_checker_catches_a_stage_overwritten_under_the_mma():
     """B warps that skip the empty wait on the outlier k-blocks (the phases
     still add up) overwrite a stage the MMA still reads."""
     assert _caught(lambda: pair_roles(9, 4, b_waits_outliers=False))
+
+
+def test_checker_catches_a_single_reduction_slot():
+    """The per-token reduction and the INT8 outliers' reduction in the same
+    slot (the quantiser's team with the two slots aliased): a fast warp's
+    next write races a slower warp's read."""
+    def single_slot_roles(rows=6, NR=2, W=4):
+        row_full = [Bar(1) for _ in range(NR)]
+        red = Buf("reduction slot")
+        team = Sync(W)
+
+        def warp(w):
+            if w == 0:
+                for j in range(min(NR, rows)):
+                    yield ("async", row_full[j])
+            for j in range(rows):
+                if w == 0:
+                    yield ("wait", row_full[j % NR], j // NR)
+                yield ("sync", team)
+                if w == 0 and j > 0 and j - 1 + NR < rows:
+                    yield ("async", row_full[(j - 1) % NR])
+                yield ("write", red)
+                yield ("sync", team)
+                yield ("own", red)
+                yield ("free", red)
+                yield ("write", red)
+                yield ("sync", team)
+                yield ("own", red)
+                yield ("free", red)
+        return [warp(w) for w in range(W)]
+
+    assert _caught(single_slot_roles)
 
 
 def test_checker_catches_a_wrong_accumulator_phase():
