@@ -36,8 +36,10 @@
 
  *
  * Conventions for every entry point:
- *   - All tensor pointers are DEVICE memory owned by the caller; the library
- *     never allocates device memory and keeps no pointer after returning.
+ *   - All tensor pointers are DEVICE memory owned by the caller; no call
+ *     allocates device memory and none keeps a pointer after returning.  The
+ *     one device buffer the library owns is quik_linear_noalloc's static
+ *     workspace (below), part of the library's device module.
  *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
  *     the legacy default stream) and is asynchronous: nothing synchronises.
  *   - Every function returns a quik_status; nothing throws across the ABI.
@@ -300,7 +302,8 @@ QUIK_API quik_status quik_gemm_24_i32_debug(const quik_shape *shape, const void 
  * takes the same arguments as quik_linear minus the workspace and uses a
  * workspace of QUIK_NOALLOC_SCRATCH_BYTES that the library keeps in its own
  * device data segment: every GPU that loads the library holds it until the
- * process exits.  No call allocates or frees anything.
+ * process exits.  Calls allocate and free nothing (but see the first call,
+ * below).
  *   - Shapes whose quik_workspace_size exceeds QUIK_NOALLOC_SCRATCH_BYTES
  *     return QUIK_ERR_UNSUPPORTED (use quik_linear with your own workspace).
  *   - All calls on a device share that one workspace: two calls whose work
@@ -310,7 +313,16 @@ QUIK_API quik_status quik_gemm_24_i32_debug(const quik_shape *shape, const void 
  *     byte it reads, so no clearing is needed.
  *   - The first call on each device looks up the workspace's device address
  *     (with that device current) and caches it; make that first call before
- *     any stream capture.
+ *     any stream capture.  Under CUDA's default lazy module loading, that
+ *     first call is also when the runtime loads the library's device module
+ *     on the device and commits the workspace's memory, which can allocate
+ *     and synchronise.  A caller that may not allocate at all should make
+ *     one warm-up call (or run with CUDA_MODULE_LOADING=EAGER, which commits
+ *     the workspace when the library's module loads) before entering the
+ *     region where allocation is forbidden; later calls allocate nothing.
+ *   - The cached address belongs to the device's current context: after
+ *     cudaDeviceReset on a device, do not call this entry point on that
+ *     device again in the same process.
  * Errors and argument rules are those of quik_linear.
  */
 #define QUIK_NOALLOC_SCRATCH_BYTES (32u << 20)
@@ -331,10 +343,14 @@ QUIK_API quik_status quik_gemm_i32_debug(const quik_shape *shape, const void *Xq
                                 int32_t *acc_outlier, quik_stream_t stream);
 
 /*
- * quik_sync_check -- synchronise `stream`, then report (and clear) the
- * device error words: QUIK_ERR_TIMEOUT if a bounded wait ran out in any
- * kernel since the last check, else QUIK_ERR_INVALID_ARG if a quantiser met
- * a perm entry outside [0, K), QUIK_ERR_CUDA on a CUDA error, else QUIK_OK.
+ * quik_sync_check -- synchronise `stream`, then report the device error
+ * counters of the current device: QUIK_ERR_TIMEOUT if a bounded wait ran out
+ * in any kernel since the previous check, else QUIK_ERR_INVALID_ARG if a
+ * quantiser met a perm entry outside [0, K) since then, QUIK_ERR_CUDA on a
+ * CUDA error, else QUIK_OK.  The counters are never reset on the device (a
+ * kernel running on another stream meanwhile is not disturbed); each check
+ * reports what was added since the previous one, whichever stream it came
+ * from.
  */
 QUIK_API quik_status quik_sync_check(quik_stream_t stream);
 

@@ -1729,40 +1729,6 @@ __global__ void __launch_bounds__(sp24::THREADS, 1)
 }
 
 // ----------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = []() -> EncodeTiledFn {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q{};
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        return reinterpret_cast<EncodeTiledFn>(ptr);
-    }();
-    return fn;
-}
-
-// 2-D row-major map: `inner` elements per row (contiguous), `rows` rows,
-// `stride` bytes between rows; box of box_inner x box_rows.
-bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
-              uint64_t rows, uint64_t stride, uint32_t box_inner, uint32_t box_rows,
-              CUtensorMapSwizzle sw) {
-    EncodeTiledFn fn = encode_fn();
-    if (fn == nullptr) return false;
-    const cuuint64_t dims[2] = {inner, rows};
-    const cuuint64_t strides[1] = {stride};
-    const cuuint32_t box[2] = {box_inner, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <class C>
 quik_status run(const GemmArgs &a, cudaStream_t stream) {
     static_assert(sizeof(C) > 0, "");
@@ -2094,13 +2060,11 @@ quik_status sync_check(cudaStream_t stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return QUIK_ERR_CUDA;
     unsigned int word = 0, bad_perm = 0;
     if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return QUIK_ERR_CUDA;
-    const unsigned int qword = take_quantize_errors(&bad_perm);
-    if (word != 0) {
-        const unsigned int zero = 0;
-        if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess)
-            return QUIK_ERR_CUDA;
-    }
-    if (word != 0 || qword != 0) return QUIK_ERR_TIMEOUT;
+    // the counters are never reset on the device: a kernel running on another
+    // stream keeps its start-time snapshot valid, and no increase is lost
+    const unsigned int waits = counter_increase(kCounterGemmWaits, word);
+    const unsigned int qwaits = take_quantize_errors(&bad_perm);
+    if (waits != 0 || qwaits != 0) return QUIK_ERR_TIMEOUT;
     if (bad_perm != 0) return QUIK_ERR_INVALID_ARG;
     return QUIK_OK;
 }

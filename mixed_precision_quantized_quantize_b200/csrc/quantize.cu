@@ -45,8 +45,8 @@ namespace quik {
 QUIK_CHECK_DECL
 
 // Count of bounded waits that ran out in this file's kernels, and of perm
-// entries outside [0, K) (both read and cleared by quik_sync_check through
-// take_quantize_errors).
+// entries outside [0, K).  Both only grow; quik_sync_check reports their
+// increase since its previous call (take_quantize_errors).
 __device__ unsigned int g_quant_error;
 __device__ unsigned int g_quant_bad_perm;
 
@@ -905,11 +905,8 @@ unsigned int take_quantize_errors(unsigned int *bad_perm) {
     unsigned int word = 0, bad = 0;
     if (cudaMemcpyFromSymbol(&word, g_quant_error, sizeof(word)) != cudaSuccess) return 0;
     if (cudaMemcpyFromSymbol(&bad, g_quant_bad_perm, sizeof(bad)) != cudaSuccess) return 0;
-    const unsigned int zero = 0;
-    if (word != 0) cudaMemcpyToSymbol(g_quant_error, &zero, sizeof(zero));
-    if (bad != 0) cudaMemcpyToSymbol(g_quant_bad_perm, &zero, sizeof(zero));
-    if (bad_perm != nullptr) *bad_perm = bad;
-    return word;
+    if (bad_perm != nullptr) *bad_perm = counter_increase(kCounterBadPerm, bad);
+    return counter_increase(kCounterQuantWaits, word);
 }
 
 }  // namespace quik

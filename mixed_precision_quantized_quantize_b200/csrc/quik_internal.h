@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/quik.h"
@@ -67,8 +68,15 @@ cudaError_t launch_prune24_rows(const Prune24Args &a, cudaStream_t stream);
 // The dense packed INT4 rows [rows, K_i / 2] of 2:4 rows (K_i % 128 == 0).
 cudaError_t launch_expand24(const uint8_t *Qs, const uint8_t *meta, int rows, int Ki, uint8_t *Q,
                             cudaStream_t stream);
-// Read and clear the quantise kernels' count of expired waits (returned) and
-// of perm entries outside [0, K) (stored in *bad_perm when given); synchronous.
+// The device error counters only ever grow: kernels add to them and nothing
+// resets them, so a kernel that compares the counter with the value it saw at
+// its start learns of every error recorded since.  A check reports the
+// increase since the previous check of the same counter on the current device.
+enum { kCounterGemmWaits = 0, kCounterQuantWaits = 1, kCounterBadPerm = 2, kCounters = 3 };
+unsigned counter_increase(int counter, unsigned value);
+// Expired waits in the quantise kernels since the last check (returned), and
+// perm entries outside [0, K) met since the last check (in *bad_perm when
+// given); synchronous.
 unsigned int take_quantize_errors(unsigned int *bad_perm);
 
 // INT4 x INT4 (+ outlier) product with the dequantising epilogue, or the raw
@@ -104,6 +112,12 @@ int sm_count();
 // cannot fit or a CUDA call fails.
 bool attribute_set_once(const void *kernel, int dyn_smem_bytes);
 quik_status launch_gemm(const GemmArgs &a, cudaStream_t stream);
+// 2-D row-major TMA map: `inner` elements per row (contiguous), `rows` rows,
+// `stride` bytes between rows; box of box_inner x box_rows; elements outside
+// the tensor read as zero.
+bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
+              uint64_t rows, uint64_t stride, uint32_t box_inner, uint32_t box_rows,
+              CUtensorMapSwizzle sw);
 
 quik_status sync_check(cudaStream_t stream);
 quik_status launch_timeout_selftest(uint32_t limit_us, cudaStream_t stream);
