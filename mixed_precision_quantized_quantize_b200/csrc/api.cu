@@ -43,6 +43,14 @@ inline bool needs_scale(const quik_shape *s) { return groups_of(s) > 0; }
 inline bool int8_out(const quik_shape *s) { return s->outlier == QUIK_OUTLIER_INT8; }
 inline bool act8(const quik_shape *s) { return s->act_bits == 8; }
 inline bool wt8(const quik_shape *s) { return s->weight_bits == 8; }
+// quik_linear's quantiser writes the wide INT4 form (the bytes 16 c, read by
+// the persistent GEMM without unpacking) exactly when that kernel takes the
+// product: per-channel scales, INT4 activations and weights, FP16 or no
+// outliers, K_i > 0 and more than kDecodeTokens tokens.
+inline bool wide_acts(const quik_shape *s) {
+    return s->group_size == 0 && !act8(s) && !wt8(s) && s->K - s->k_o > 0 &&
+           (s->k_o == 0 || !int8_out(s)) && s->M > quik::kDecodeTokens;
+}
 
 // Rows of one operand: packed codes, scales, outlier block (+ INT8 scales).
 quik_status check_quant_ptrs(const quik_shape *s, const void *Q, const float *scale,
@@ -60,7 +68,7 @@ quik_status check_quant_ptrs(const quik_shape *s, const void *Q, const float *sc
 // gamma (optional): the rows are RMS-normalised with this weight and eps first.
 quik_status quantize(const quik_shape *s, int rows, bool bits8, const void *X, const int32_t *perm,
                      void *Q, float *scale, void *O, float *o_scale, cudaStream_t stream,
-                     const void *gamma = nullptr, float eps = 0.0f) {
+                     const void *gamma = nullptr, float eps = 0.0f, bool wide = false) {
     quik::QuantizeArgs a;
     a.X = static_cast<const uint16_t *>(X);
     a.perm = perm;
@@ -70,6 +78,7 @@ quik_status quantize(const quik_shape *s, int rows, bool bits8, const void *X, c
     a.group = s->group_size;
     a.out_int8 = int8_out(s);
     a.bits8 = bits8;
+    a.wide = wide;
     a.Q = static_cast<uint8_t *>(Q);
     a.scale = scale;
     a.O = O;
@@ -123,7 +132,7 @@ Workspace layout(const quik_shape *s) {
     const size_t G = static_cast<size_t>(groups_of(s));
     Workspace w;
     w.xq = 0;
-    w.sx = w.xq + round256(act8(s) ? M * Ki : M * Ki / 2);
+    w.sx = w.xq + round256(act8(s) || wide_acts(s) ? M * Ki : M * Ki / 2);
     w.xo = w.sx + round256(M * G * sizeof(float));
     w.sxo = w.xo + round256(M * s->k_o * (int8_out(s) ? 1 : 2));
     w.total = w.sxo + round256(int8_out(s) ? M * sizeof(float) : 0);
@@ -178,7 +187,8 @@ static quik_status gemm_impl(const quik_shape *shape, const void *Xq, const floa
                              const void *Xo, const float *xo_scale, const void *Wq,
                              const float *w_scale, const void *Wo, const float *wo_scale,
                              const void *bias, void *Y, bool debug, int32_t *acc,
-                             int32_t *acc_o, cudaStream_t stream, bool after_quantize = false) {
+                             int32_t *acc_o, cudaStream_t stream, bool after_quantize = false,
+                             bool x_wide = false) {
     quik::GemmArgs a;
     a.M = shape->M;
     a.N = shape->N;
@@ -188,6 +198,7 @@ static quik_status gemm_impl(const quik_shape *shape, const void *Xq, const floa
     a.out_int8 = int8_out(shape);
     a.a8 = act8(shape);
     a.w8 = wt8(shape);
+    a.x_wide = x_wide;
     a.Xq = Xq;
     a.sx = x_scale;
     a.Xo = Xo;
@@ -238,13 +249,14 @@ static quik_status linear_impl(const quik_shape *shape, const void *X_f16, const
     void *Xo = ws + w.xo;
     float *sxo = int8_out(shape) ? reinterpret_cast<float *>(ws + w.sxo) : nullptr;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if ((st = quantize(shape, shape->M, act8(shape), X_f16, perm, Xq, sx, Xo, sxo, s, gamma, eps)) !=
-        QUIK_OK)
+    const bool wide = wide_acts(shape);
+    if ((st = quantize(shape, shape->M, act8(shape), X_f16, perm, Xq, sx, Xo, sxo, s, gamma, eps,
+                       wide)) != QUIK_OK)
         return st;
     // the GEMM follows this quantiser on the same stream: its set-up and weight
     // loads may overlap the quantiser's tail
     return gemm_impl(shape, Xq, sx, Xo, sxo, Wq, w_scale, Wo, wo_scale, bias_f16, Y_f16, false,
-                     nullptr, nullptr, s, true);
+                     nullptr, nullptr, s, true, wide);
 }
 
 quik_status quik_linear(const quik_shape *shape, const void *X_f16, const int32_t *perm,
@@ -382,10 +394,13 @@ quik_status quik_linear_24(const quik_shape *shape, const void *X_f16, const int
         // prefill: expand the weights, quantise, then the dense kernel (the
         // GEMM directly follows the quantiser, as quik_linear's does)
         void *Wd = ws + w.total;
+        const bool wide = wide_acts(shape);
         if ((st = quik_expand_weights_24(shape, Wq24, Wmeta, Wd, stream)) != QUIK_OK) return st;
-        if ((st = quantize(shape, shape->M, false, X_f16, perm, Xq, sx, Xo, sxo, s)) != QUIK_OK) return st;
+        if ((st = quantize(shape, shape->M, false, X_f16, perm, Xq, sx, Xo, sxo, s, nullptr, 0.0f,
+                           wide)) != QUIK_OK)
+            return st;
         return gemm_impl(shape, Xq, sx, Xo, sxo, Wd, w_scale, Wo, wo_scale, bias_f16, Y_f16, false,
-                         nullptr, nullptr, s, true);
+                         nullptr, nullptr, s, true, wide);
     }
     if ((st = quantize(shape, shape->M, false, X_f16, perm, Xq, sx, Xo, sxo, s)) != QUIK_OK) return st;
     return gemm24_impl(shape, Xq, sx, Xo, sxo, Wq24, Wmeta, w_scale, Wo, wo_scale, bias_f16, Y_f16,

@@ -1071,7 +1071,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
 //                (coalesced).
 namespace gemv {
 constexpr int BW = 128;                      // W rows per CTA = TMEM lanes
-constexpr int MT = 32;                       // most tokens (the MMA's N: 16 or 32)
+constexpr int MT = kDecodeTokens;            // most tokens (the MMA's N: 16 or 32)
 #ifndef QUIK_GEMV_S
 #define QUIK_GEMV_S 8
 #endif
@@ -2008,6 +2008,7 @@ quik_status dispatch(const GemmArgs &a, cudaStream_t stream) {
     if (a.w8) return QUIK_ERR_UNSUPPORTED;
     if (a.group == 0 && a.M <= gemv::MT && a.k_o <= (a.out_int8 ? gemv::KO_MAX_I8 : gemv::KO_MAX_F16))
         return a.out_int8 ? run_gemv<true, DEBUG>(a, stream) : run_gemv<false, DEBUG>(a, stream);
+    if (persistent_gemm_takes(a)) return launch_gemm_persistent(a, stream);
     if (a.group == 0)
         return a.out_int8 ? run_pair<true, DEBUG, false, false>(a, stream)
                           : run_pair<false, DEBUG, false, false>(a, stream);
@@ -2062,7 +2063,7 @@ quik_status sync_check(cudaStream_t stream) {
     if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return QUIK_ERR_CUDA;
     // the counters are never reset on the device: a kernel running on another
     // stream keeps its start-time snapshot valid, and no increase is lost
-    const unsigned int waits = counter_increase(kCounterGemmWaits, word);
+    const unsigned int waits = counter_increase(kCounterGemmWaits, word) + persistent_gemm_errors();
     const unsigned int qwaits = take_quantize_errors(&bad_perm);
     if (waits != 0 || qwaits != 0) return QUIK_ERR_TIMEOUT;
     if (bad_perm != 0) return QUIK_ERR_INVALID_ARG;

@@ -74,6 +74,7 @@ struct QParams {
     void *O;
     float *o_scale;
     int bits8;  // per-token rows only: INT8 codes (one byte each, divisor 127)
+    int wide;   // per-token rows only: INT4 codes as the bytes 16 c in the persistent GEMM's operand order
     const uint16_t *gamma;  // RMS-norm weight [K] in source channel order (NORM kernels only)
     float eps;              // RMS-norm epsilon (NORM kernels only)
 };
@@ -569,6 +570,28 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : (GROUP
                     }
                 }
             }
+        } else if (!GROUPED && p.wide) {
+            // one signed byte 16 c per code; per 32 positions, the 16 even ones
+            // then the 16 odd ones (the order in which the GEMM widens packed
+            // weights, so both operands share one K order)
+            uint8_t *qrow = p.Q + static_cast<size_t>(row) * Ki;
+#pragma unroll
+            for (int i = 0; i < W; ++i) {
+                const int w = tl + i * TT;
+                if (w < nwords && QUIK_CHECK(8 * w + 8 <= Ki, 4)) {
+                    uint32_t word;
+                    if (NORM) {
+                        uint64_t z[4];
+                        norm_products(v[i], reinterpret_cast<const uint4 *>(gtab)[w], z);
+                        word = pack_codes8(z, s[i], r[i]);
+                    } else {
+                        word = pack_codes8(v[i], s[i], r[i]);
+                    }
+                    uint32_t *g = reinterpret_cast<uint32_t *>(qrow + 32 * (w >> 2)) + (w & 3);
+                    g[0] = (word << 4) & 0xF0F0F0F0u;  // codes 8w, 8w+2, 8w+4, 8w+6
+                    g[4] = word & 0xF0F0F0F0u;         // codes 8w+1, 8w+3, 8w+5, 8w+7
+                }
+            }
         } else {
             uint32_t *qrow = reinterpret_cast<uint32_t *>(p.Q + static_cast<size_t>(row) * (Ki / 2));
 #pragma unroll
@@ -874,8 +897,10 @@ __global__ void expand24_kernel(const uint8_t *__restrict__ Qs, const uint8_t *_
 
 cudaError_t launch_quantize_rows(const QuantizeArgs &a, cudaStream_t stream) {
     QParams p{a.X, a.perm, a.rows, a.K, a.k_o, 0, 0, 0, a.Q, a.scale, a.O, a.o_scale, a.bits8 ? 1 : 0,
-              a.gamma, a.eps};
-    if (a.bits8 && a.group > 0) return cudaErrorInvalidValue;  // INT8 codes: per-row scales only
+              a.wide ? 1 : 0, a.gamma, a.eps};
+    // INT8 codes and the wide INT4 form: per-row scales only
+    if ((a.bits8 || a.wide) && a.group > 0) return cudaErrorInvalidValue;
+    if (a.bits8 && a.wide) return cudaErrorInvalidValue;
     if (a.gamma != nullptr) return launch_q_n<true>(p, a.group, a.out_int8, stream);
     return launch_q_n<false>(p, a.group, a.out_int8, stream);
 }

@@ -30,6 +30,7 @@ constexpr int kMaxK = 32768;       // largest K the quantiser stages in shared m
 constexpr int kMaxKNorm = 24576;   // with the RMS norm folded in (a second K-wide table)
 constexpr int kGroup = 128;        // the one supported group width
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s bound on every in-kernel wait
+constexpr int kDecodeTokens = 32;  // up to this many tokens the product is decode-shaped
 
 // Reorder + quantise + pack `rows` rows of a [rows, K] fp16 matrix.
 struct QuantizeArgs {
@@ -38,6 +39,10 @@ struct QuantizeArgs {
     int rows, K, k_o, group;
     bool out_int8;
     bool bits8;  // INT8 codes (divisor and clamp 127, one byte each) instead of packed INT4
+    // INT4 codes written wide, as the signed bytes 16 c [rows, K_i] in the
+    // persistent GEMM's operand order (per 32 positions: the 16 even ones,
+    // then the 16 odd ones); per-row scales only
+    bool wide = false;
     uint8_t *Q;
     float *scale;
     void *O;
@@ -72,7 +77,7 @@ cudaError_t launch_expand24(const uint8_t *Qs, const uint8_t *meta, int rows, in
 // resets them, so a kernel that compares the counter with the value it saw at
 // its start learns of every error recorded since.  A check reports the
 // increase since the previous check of the same counter on the current device.
-enum { kCounterGemmWaits = 0, kCounterQuantWaits = 1, kCounterBadPerm = 2, kCounters = 3 };
+enum { kCounterGemmWaits = 0, kCounterQuantWaits = 1, kCounterBadPerm = 2, kCounterPGemmWaits = 3, kCounters = 4 };
 unsigned counter_increase(int counter, unsigned value);
 // Expired waits in the quantise kernels since the last check (returned), and
 // perm entries outside [0, K) met since the last check (in *bad_perm when
@@ -86,6 +91,7 @@ struct GemmArgs {
     bool out_int8;
     bool a8;  // Xq holds INT8 codes [M, K_i] (W4A8) instead of packed INT4
     bool w8;  // Wq holds INT8 codes [N, K_i] (W8A8; with a8)
+    bool x_wide = false;  // Xq holds the bytes 16 c [M, K_i] in operand order (quantiser's wide output)
     const void *Xq;
     const float *sx;
     const void *Xo;
@@ -112,6 +118,12 @@ int sm_count();
 // cannot fit or a CUDA call fails.
 bool attribute_set_once(const void *kernel, int dyn_smem_bytes);
 quik_status launch_gemm(const GemmArgs &a, cudaStream_t stream);
+// The persistent CTA-pair kernel (per-channel scales, INT4 activations and
+// weights, FP16 or no outliers, more than kDecodeTokens tokens, K_i > 0).
+bool persistent_gemm_takes(const GemmArgs &a);
+quik_status launch_gemm_persistent(const GemmArgs &a, cudaStream_t stream);
+// Expired waits in the persistent kernel since the last check.
+unsigned int persistent_gemm_errors();
 // 2-D row-major TMA map: `inner` elements per row (contiguous), `rows` rows,
 // `stride` bytes between rows; box of box_inner x box_rows; elements outside
 // the tensor read as zero.
