@@ -43,8 +43,12 @@ def _ws(M, N, K, k_o, group=0, outlier=0, act_bits=4, weight_bits=4):
 
 def test_workspace_size(L):
     r = lambda b: (b + 255) // 256 * 256
-    # FP16 outliers: codes, per-token scales, fp16 outlier block
-    assert _ws(2048, 4096, 4096, 128) == r(2048 * 3968 // 2) + r(2048 * 4) + r(2048 * 128 * 2)
+    # FP16 outliers above 32 tokens: the codes widened to one byte each (the
+    # persistent GEMM's operand), per-token scales, fp16 outlier block
+    assert _ws(2048, 4096, 4096, 128) == r(2048 * 3968) + r(2048 * 4) + r(2048 * 128 * 2)
+    # up to 32 tokens (the decode kernel) and with INT8 outliers: packed codes
+    assert _ws(32, 4096, 4096, 128) == r(32 * 3968 // 2) + r(32 * 4) + r(32 * 128 * 2)
+    assert _ws(64, 4096, 4096, 128, 0, 1) == r(64 * 3968 // 2) + r(64 * 4) + r(64 * 128) + r(64 * 4)
     # grouped + INT8 outliers: G scales per token, int8 block, one INT8 scale per token
     G = (8192 - 128) // 128
     assert _ws(1024, 22016, 8192, 128, 128, 1) == (r(1024 * 8064 // 2) + r(1024 * G * 4)
