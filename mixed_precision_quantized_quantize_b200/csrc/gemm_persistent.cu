@@ -209,6 +209,24 @@ __device__ __forceinline__ float int_to_float_exact(int32_t v) {
     return __int_as_float(v + 0x4B400000) - 12582912.0f;
 }
 
+// y = A sx[m] sw + bias for one 32-column chunk, A = acc >> 8 (the INT4 codes
+// enter the MMA as 16 c): pairs of columns in paired fp32 arithmetic, the
+// scaling and the bias in one fused multiply-add per pair.
+__device__ __forceinline__ void dequant32(uint32_t (&a)[32], const float *sx, float sw, float bias) {
+    const uint64_t sw2 = f2(sw, sw), b2 = f2(bias, bias);
+#pragma unroll
+    for (int jj = 0; jj < 32; jj += 2) {
+        const float2 s = *reinterpret_cast<const float2 *>(sx + jj);
+        const uint64_t v = f2_mul(f2(int_to_float_exact(static_cast<int32_t>(a[jj]) >> 8),
+                                     int_to_float_exact(static_cast<int32_t>(a[jj + 1]) >> 8)),
+                                  f2(s.x, s.y));
+        float y0, y1;
+        f2_split(f2_fma(v, sw2, b2), y0, y1);
+        a[jj] = __float_as_uint(y0);
+        a[jj + 1] = __float_as_uint(y1);
+    }
+}
+
 // 32 packed codes (16 bytes) -> the signed bytes 16 c: even positions in the
 // first 16 bytes, odd positions in the next 16 (the same order on both
 // operands, so every dot product is unchanged).
@@ -319,7 +337,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     __shared__ unsigned err0_s;
-    __shared__ float sx_s[2][BT];
+    __shared__ __align__(16) float sx_s[2][BT];
 
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -578,11 +596,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
                     uint32_t a[32];
                     tmem_ld_32x32b_x32(acc + 32 * c, a);
                     tmem_ld_wait();
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const float y = int_to_float_exact(static_cast<int32_t>(a[jj]) >> 8) * sxr[32 * c + jj] * swn + bn;
-                        a[jj] = __float_as_uint(y);
-                    }
+                    dequant32(a, sxr + 32 * c, swn, bn);
                     tmem_st_32x32b_x32(acc + 32 * c, a);
                 }
                 tmem_st_wait();
@@ -604,6 +618,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
                 uint32_t a[32];
                 tmem_ld_32x32b_x32(acc + 32 * c, a);
                 tmem_ld_wait();
+                if (!DEBUG && p.nkb_o == 0) dequant32(a, sxr + 32 * c, swn, bn);  // else rescaled already
                 const int m0 = tok0 + 32 * c;
                 if (DEBUG) {
                     if (n_ok) {
@@ -621,12 +636,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
                     if (lane == 0) bulk_wait_group_read0();
                     __syncwarp();
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const float y = p.nkb_o > 0
-                                            ? __uint_as_float(a[jj])
-                                            : int_to_float_exact(static_cast<int32_t>(a[jj]) >> 8) * sxr[32 * c + jj] * swn + bn;
-                        ystage[jj * 32 + lane] = __half_as_ushort(__float2half_rn(y));
-                    }
+                    for (int jj = 0; jj < 32; ++jj)
+                        ystage[jj * 32 + lane] = __half_as_ushort(__float2half_rn(__uint_as_float(a[jj])));
                     fence_proxy_async_smem();  // generic stores -> visible to the TMA store
                     __syncwarp();
                     if (lane == 0) {
@@ -635,13 +646,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
                     }
                 } else {
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const float y = p.nkb_o > 0
-                                            ? __uint_as_float(a[jj])
-                                            : int_to_float_exact(static_cast<int32_t>(a[jj]) >> 8) * sxr[32 * c + jj] * swn + bn;
+                    for (int jj = 0; jj < 32; ++jj)
                         if (n_ok && m0 + jj < p.M)
-                            p.Y[static_cast<size_t>(m0 + jj) * p.N + gn] = __half_as_ushort(__float2half_rn(y));
-                    }
+                            p.Y[static_cast<size_t>(m0 + jj) * p.N + gn] =
+                                __half_as_ushort(__float2half_rn(__uint_as_float(a[jj])));
                 }
             }
             tc_fence_before();
