@@ -168,6 +168,23 @@ QUIK_API quik_status quik_linear(const quik_shape *shape, const void *X_f16, con
                         void *workspace, size_t workspace_bytes, quik_stream_t stream);
 
 /*
+ * quik_linear_timed -- quik_linear with the CUDA event `between` (a
+ * cudaEvent_t passed as void *, created by the caller) recorded on `stream`
+ * after the quantiser's launch and before the GEMM's.  A measurement aid of
+ * this library (no counterpart in the papers): with the event between them
+ * the GEMM waits for the quantiser to finish instead of starting during its
+ * tail, so events recorded before the call, `between`, and after the call
+ * time the layer's two kernels one by one.  Y is bit-identical to
+ * quik_linear's.  `between` NULL: QUIK_ERR_INVALID_ARG; a failed record:
+ * QUIK_ERR_CUDA; otherwise as quik_linear.
+ */
+QUIK_API quik_status quik_linear_timed(const quik_shape *shape, const void *X_f16,
+                                       const int32_t *perm, const void *Wq, const float *w_scale,
+                                       const void *Wo, const float *wo_scale, const void *bias_f16,
+                                       void *Y_f16, void *workspace, size_t workspace_bytes,
+                                       void *between, quik_stream_t stream);
+
+/*
  * quik_rmsnorm_quantize_reorder -- the RMS norm that precedes a projection,
  * with the projection's dynamic quantisation and reordering folded into it
  * (Atom summary and idea I2: quantisation and reordering are fused into
@@ -325,7 +342,7 @@ QUIK_API quik_status quik_gemm_24_i32_debug(const quik_shape *shape, const void 
  *     device again in the same process.
  * Errors and argument rules are those of quik_linear.
  */
-#define QUIK_NOALLOC_SCRATCH_BYTES (32u << 20)
+#define QUIK_NOALLOC_SCRATCH_BYTES (64u << 20)
 QUIK_API quik_status quik_linear_noalloc(const quik_shape *shape, const void *X_f16,
                                          const int32_t *perm, const void *Wq,
                                          const float *w_scale, const void *Wo,

@@ -52,6 +52,8 @@ _SIGS = {
     "quik_rmsnorm_linear": (ctypes.c_int, [_S, _P, _P, ctypes.c_float, _P, _P, _P, _P, _P, _P,
                                             _P, _P, ctypes.c_size_t, _P]),
     "quik_linear_noalloc": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "quik_linear_timed": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
+                                         _P, _P]),
     "quik_gemm_i32_debug": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P]),
     "quik_pack_weights_24": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P, _P]),
     "quik_gemm_24": (ctypes.c_int, [_S] + [_P] * 12),
@@ -177,6 +179,21 @@ def quik_linear(shape, X, perm, Wq, w_scale, Wo, wo_scale, bias, Y, workspace, s
         _ptr(Wo, None, "Wo"), _ptr(wo_scale, torch.float32, "wo_scale"),
         _ptr(bias, torch.float16, "bias"), _ptr(Y, torch.float16, "Y"),
         _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)), "quik_linear")
+
+
+def quik_linear_timed(shape, X, perm, Wq, w_scale, Wo, wo_scale, bias, Y, workspace, between,
+                      stream=None):
+    """quik_linear with the torch.cuda.Event `between` recorded between its two
+    kernels (the GEMM then waits for the quantiser to finish)."""
+    if between.cuda_event == 0:
+        between.record(stream)  # torch creates the CUDA event on its first record
+    _check(lib().quik_linear_timed(
+        ctypes.byref(shape), _ptr(X, torch.float16, "X"), _ptr(perm, torch.int32, "perm"),
+        _ptr(Wq, _wq_dtype(shape), "Wq"), _ptr(w_scale, torch.float32, "w_scale"),
+        _ptr(Wo, None, "Wo"), _ptr(wo_scale, torch.float32, "wo_scale"),
+        _ptr(bias, torch.float16, "bias"), _ptr(Y, torch.float16, "Y"),
+        _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), between.cuda_event,
+        _stream(stream)), "quik_linear_timed")
 
 
 def quik_rmsnorm_linear(shape, X, gamma, eps, perm, Wq, w_scale, Wo, wo_scale, bias, Y, workspace,

@@ -233,7 +233,8 @@ static quik_status linear_impl(const quik_shape *shape, const void *X_f16, const
                                float eps, const int32_t *perm, const void *Wq,
                                const float *w_scale, const void *Wo, const float *wo_scale,
                                const void *bias_f16, void *Y_f16, void *workspace,
-                               size_t workspace_bytes, quik_stream_t stream) {
+                               size_t workspace_bytes, quik_stream_t stream,
+                               cudaEvent_t between = nullptr) {
     quik_status st = check_shape(shape);
     if (st != QUIK_OK) return st;
     if (!ok_ptr(X_f16) || !ok_ptr(perm) || !ok_ptr(Y_f16) || !ok_opt(bias_f16))
@@ -254,9 +255,10 @@ static quik_status linear_impl(const quik_shape *shape, const void *X_f16, const
                        wide)) != QUIK_OK)
         return st;
     // the GEMM follows this quantiser on the same stream: its set-up and weight
-    // loads may overlap the quantiser's tail
+    // loads may overlap the quantiser's tail (not with an event between them)
+    if (between != nullptr && cudaEventRecord(between, s) != cudaSuccess) return QUIK_ERR_CUDA;
     return gemm_impl(shape, Xq, sx, Xo, sxo, Wq, w_scale, Wo, wo_scale, bias_f16, Y_f16, false,
-                     nullptr, nullptr, s, true, wide);
+                     nullptr, nullptr, s, between == nullptr, wide);
 }
 
 quik_status quik_linear(const quik_shape *shape, const void *X_f16, const int32_t *perm,
@@ -265,6 +267,16 @@ quik_status quik_linear(const quik_shape *shape, const void *X_f16, const int32_
                         void *workspace, size_t workspace_bytes, quik_stream_t stream) {
     return linear_impl(shape, X_f16, nullptr, 0.0f, perm, Wq, w_scale, Wo, wo_scale, bias_f16,
                        Y_f16, workspace, workspace_bytes, stream);
+}
+
+quik_status quik_linear_timed(const quik_shape *shape, const void *X_f16, const int32_t *perm,
+                              const void *Wq, const float *w_scale, const void *Wo,
+                              const float *wo_scale, const void *bias_f16, void *Y_f16,
+                              void *workspace, size_t workspace_bytes, void *between,
+                              quik_stream_t stream) {
+    if (between == nullptr) return QUIK_ERR_INVALID_ARG;
+    return linear_impl(shape, X_f16, nullptr, 0.0f, perm, Wq, w_scale, Wo, wo_scale, bias_f16,
+                       Y_f16, workspace, workspace_bytes, stream, static_cast<cudaEvent_t>(between));
 }
 
 quik_status quik_rmsnorm_linear(const quik_shape *shape, const void *X_f16, const void *gamma_f16,

@@ -274,17 +274,61 @@ __device__ __forceinline__ void norm_products(const uint32_t (&h)[4], uint4 g, u
     }
 }
 
-__device__ __forceinline__ double warp_sum(double t) {
+// The norm's sum of squares, exact.  Every finite fp16 value is an integer
+// multiple of 2^-24, so its square is an integer multiple of 2^-48 below
+// 2^80, and at most 2^15 of them (K <= 24576) sum below 2^95: a 96-bit
+// integer (lo, hi) in units of 2^-48 holds the sum exactly, whatever the
+// order of the additions.  (Non-finite inputs give an unspecified sum.)
+struct SumSq {
+    uint64_t lo;
+    uint32_t hi;
+};
+
+__device__ __forceinline__ void sumsq_add(SumSq &s, uint64_t lo, uint32_t hi) {
+    s.lo += lo;
+    s.hi += hi + (s.lo < lo ? 1u : 0u);
+}
+
+// h^2 of the fp16 bit pattern h16 (low 16 bits): h = m 2^(max(e,1) - 25)
+// with m = f (e = 0) or 1024 + f, so h^2 = m^2 2^(sh - 48), sh = 2e - 2 (0
+// for e = 0) <= 58.
+__device__ __forceinline__ void sumsq_add_half(SumSq &s, uint32_t h16) {
+    const uint32_t e = (h16 >> 10) & 31u, f = h16 & 1023u;
+    const uint64_t m = e ? (f | 1024u) : f;
+    const uint32_t sh = e ? 2u * e - 2u : 0u;
+    const uint64_t m2 = m * m;  // < 2^22
+    sumsq_add(s, m2 << sh, sh > 42u ? static_cast<uint32_t>(m2 >> (64u - sh)) : 0u);
+}
+
+__device__ __forceinline__ SumSq sumsq_warp(SumSq s) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-    return t;
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t lo = __shfl_xor_sync(0xffffffffu, s.lo, o);
+        const uint32_t hi = __shfl_xor_sync(0xffffffffu, s.hi, o);
+        sumsq_add(s, lo, hi);
+    }
+    return s;
+}
+
+// The exact sum rounded once to fp64 (to nearest, ties to even).  Above 64
+// bits the value is shifted right by n bits into 64, the bits shifted out
+// folded into bit 0 (a sticky bit: the rounding position of a 64-bit
+// significand is bit 11, so only a remainder's zero-or-not reaches it),
+// converted by the correctly rounded 64-bit conversion, and scaled back by
+// 2^n; both scalings by powers of two are exact.
+__device__ __forceinline__ double sumsq_to_double(SumSq s) {
+    if (s.hi == 0) return __dmul_rn(__ull2double_rn(s.lo), 0x1p-48);
+    const int n = 32 - __clz(s.hi);  // 1 .. 31
+    const uint64_t v = (static_cast<uint64_t>(s.hi) << (64 - n)) | (s.lo >> n) |
+                       ((s.lo & ((1ull << n) - 1)) != 0 ? 1ull : 0ull);
+    const double two_n48 = __longlong_as_double(static_cast<long long>(1023 + n - 48) << 52);
+    return __dmul_rn(__ull2double_rn(v), two_n48);
 }
 
 // The RMS norm's row factor 1 / sqrt(ss / K + eps) in fp64, each step IEEE
-// rounded.  ss is summed in fp64 from exact squares, so r is within a few
-// fp64 ulps of its exact value and the fp32 scales and fp16 outliers that
-// carry it are rounded as from the exact factor (except within ~1e-15 of a
-// rounding boundary).
+// rounded, from ss = the exact sum of squares rounded once to fp64: the
+// factor, and so the fp32 scales and fp16 outliers that carry it, do not
+// depend on the order in which the row's values were summed.
 __device__ __forceinline__ double rms_factor(double ss, int K, float eps) {
     return __drcp_rn(__dsqrt_rn(__dadd_rn(__ddiv_rn(ss, static_cast<double>(K)),
                                           static_cast<double>(eps))));
@@ -335,7 +379,7 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : (GROUP
     quantize_rows_kernel(QParams p) {
     extern __shared__ __align__(16) uint8_t qsmem[];
     __shared__ float red[kQMaxTeams][2][kQMaxThreads / 32];  // warp maxima, two slots per team
-    __shared__ double red_ss[kQMaxTeams][2][kQMaxThreads / 32];  // warp sums of squares (NORM)
+    __shared__ SumSq red_ss[kQMaxTeams][2][kQMaxThreads / 32];  // warp sums of squares (NORM)
     __shared__ uint64_t row_full[kQMaxTeams][kQMaxRing];
     const int K = p.K, Ki = K - p.k_o;  // K % 16 == 0
     const int TT = p.team_threads;
@@ -451,7 +495,7 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : (GROUP
         // (of h * gamma with the norm, whose sum of squares of h is gathered too)
         uint32_t v[W][4];
         float wmax[W];
-        double ss = 0.0;  // sum of h^2 (NORM), fp64 from exact fp32 squares
+        SumSq ss = {0ull, 0u};  // exact sum of h^2 (NORM)
 #pragma unroll
         for (int i = 0; i < W; ++i) {
             const int w = tl + i * TT;
@@ -480,11 +524,8 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : (GROUP
                     float a = 0.0f;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const uint64_t hk = pair_f32(v[i], k);
-                        float q0, q1;
-                        f2_split(ptx::f2_mul(hk, hk), q0, q1);  // exact: 22 significant bits
-                        ss += static_cast<double>(q0);
-                        ss += static_cast<double>(q1);
+                        sumsq_add_half(ss, v[i][k] & 0xffffu);
+                        sumsq_add_half(ss, v[i][k] >> 16);
                         float z0, z1;
                         f2_split(z[k], z0, z1);
                         a = max3(a, fabsf(z0), fabsf(z1));
@@ -499,17 +540,14 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : (GROUP
         // the outlier block included
         double rn = 1.0;
         if (NORM) {
-            for (int i = tl; i < p.k_o; i += TT) {
-                const float h = h2f(static_cast<uint16_t>(at(element(Ki + i))));
-                ss += static_cast<double>(__fmul_rn(h, h));
-            }
-            ss = warp_sum(ss);
+            for (int i = tl; i < p.k_o; i += TT) sumsq_add_half(ss, at(element(Ki + i)));
+            ss = sumsq_warp(ss);
             if (GROUPED) {  // the per-token path below shares the max's barrier
                 if (lane == 0) red_ss[team][j & 1][twarp] = ss;
                 team_sync(bar_id, TT);
-                ss = 0.0;
-                for (int k = 0; k < (TT >> 5); ++k) ss += red_ss[team][j & 1][k];
-                rn = rms_factor(ss, K, p.eps);
+                ss = SumSq{0ull, 0u};
+                for (int k = 0; k < (TT >> 5); ++k) sumsq_add(ss, red_ss[team][j & 1][k].lo, red_ss[team][j & 1][k].hi);
+                rn = rms_factor(sumsq_to_double(ss), K, p.eps);
             }
         }
 
@@ -540,9 +578,9 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : (GROUP
             m = 0.0f;
             for (int k = 0; k < (TT >> 5); ++k) m = fmaxf(m, red[team][j & 1][k]);
             if (NORM) {
-                ss = 0.0;
-                for (int k = 0; k < (TT >> 5); ++k) ss += red_ss[team][j & 1][k];
-                rn = rms_factor(ss, K, p.eps);
+                ss = SumSq{0ull, 0u};
+                for (int k = 0; k < (TT >> 5); ++k) sumsq_add(ss, red_ss[team][j & 1][k].lo, red_ss[team][j & 1][k].hi);
+                rn = rms_factor(sumsq_to_double(ss), K, p.eps);
             }
             const float sr = p.bits8 ? div_exact<127, 7>(m) : div_exact<7, 3>(m), rr = rcp_approx(sr);
 #pragma unroll

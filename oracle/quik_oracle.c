@@ -245,9 +245,12 @@ static uint16_t double_to_half(double v)
  *     o_scale = fl32(so_z * r), so_z = fl32(max|z_o| / 127)   (INT8 outliers)
  *     O       = fl16(z * r)                                    (FP16 outliers)
  *
- * eps is an fp32 value (the norm's parameter as stored); r is taken in
- * fp64, and the stored scales and outliers are one rounding of an fp64
- * product.  The unfused pipeline would round y to fp16 before quantising;
+ * eps is an fp32 value (the norm's parameter as stored); the sum of
+ * squares is taken exactly and rounded once to fp64 (reading: the pages fix
+ * no precision; an exact sum makes r independent of summation order), r is
+ * taken in fp64, and the stored scales and outliers are one rounding of an
+ * fp64 product.  A row with a non-finite value has no norm: the call
+ * returns ORACLE_EBADARG.  The unfused pipeline would round y to fp16 before quantising;
  * fusing the two steps removes that intermediate.
  *
  *  X, gamma : [R, K] and [K] fp16 bit patterns (gamma in source channel order)
@@ -281,12 +284,23 @@ int oracle_rmsnorm_quantize_rows(int64_t R, int64_t K, int64_t k_o, int64_t grou
 #pragma omp for schedule(static)
         for (int64_t r = 0; r < R; ++r) {
             if (!z || !codes) continue;
-            /* the row's RMS factor, over every channel (order does not matter) */
-            double ss = 0.0;
+            /* the row's RMS factor, over every channel.  The sum of squares
+             * is exact: each fp16 h is a multiple of 2^-24, so h^2 * 2^48 is
+             * an integer (below 2^80), summed in 128 bits and rounded once to
+             * fp64; the order of the terms cannot matter. */
+            unsigned __int128 S = 0;
+            int finite = 1;
             for (int64_t k = 0; k < K; ++k) {
                 double h = half_to_double(X[r * K + k]);
-                ss += h * h;
+                if (!isfinite(h)) finite = 0;
+                else S += (unsigned __int128)ldexp(h * h, 48);
             }
+            if (!finite) {
+#pragma omp atomic write
+                err = ORACLE_EBADARG;
+                continue;
+            }
+            double ss = ldexp((double)S, -48);
             double rf = 1.0 / sqrt(ss / (double)K + (double)eps);
 
             /* reorder (Atom I1) the row times its norm weight; exact in fp32 */

@@ -290,16 +290,56 @@ def test_full_size_layer(name):
                                          cfg.K, cfg.k_o, cfg.group, ms, ns)
     y = Y.float().cpu().numpy()[ms, ns]
     assert_y_close(y, ref, name)
-    # integer sums at sampled positions, from a row/column slice of the same kernel
-    if not cfg.group:
-        rows = np.unique(ms)[:256]
-        cols = np.unique(ns)[:512]
-        r_t = torch.from_numpy(rows).to(DEV)
-        c_t = torch.from_numpy(cols).to(DEV)
-        acc, _ = q.gemm_i32(gx[0][r_t].contiguous(), layer.Wq[c_t].contiguous(), cfg.K, cfg.k_o, 0)
-        acc = acc.cpu().numpy()
-        full = oracle.int_gemm(ox[0][rows], ow[0][cols], 0)
-        np.testing.assert_array_equal(acc, full)
+    # integer sums at sampled positions (one per group with groups), from a
+    # row/column slice of the same kernel
+    rows = np.unique(ms)[:256]
+    cols = np.unique(ns)[:512]
+    r_t = torch.from_numpy(rows).to(DEV)
+    c_t = torch.from_numpy(cols).to(DEV)
+    acc, _ = q.gemm_i32(gx[0][r_t].contiguous(), layer.Wq[c_t].contiguous(), cfg.K, cfg.k_o,
+                        cfg.group)
+    acc = acc.cpu().numpy()
+    full = oracle.int_gemm(ox[0][rows], ow[0][cols], cfg.group)
+    np.testing.assert_array_equal(acc, full)
+
+
+# the layers small enough for the oracle to compute every output: c1, c2 and
+# the two smaller token counts of the up projection
+EVERY_ELEMENT = ["tiny_16x256x256", "llama7b_attn_2048x4096x4096", "llama7b_up_16x11008x4096",
+                 "llama7b_up_256x11008x4096"]
+
+
+@pytest.mark.parametrize("name", EVERY_ELEMENT)
+def test_full_size_every_element(name):
+    """At the full size, every output of the layer call (the kernels the bench
+    times: the widened-operand persistent GEMM above 32 tokens, the decode
+    kernel up to 32) against the oracle's fp64 layer; every INT32 sum of the
+    same GEMM (its debug instantiation, fed the packed codes, writes all M x N
+    sums) against the oracle's exact sums; and the two-call path
+    (quik_quantize_reorder + quik_gemm) bit-identical to the layer call."""
+    cfg = wl.CONFIGS[name]
+    d = wl.make_layer(cfg, seed_offset=5)
+    perm_d = d["perm"].to(DEV)
+    b = d["bias"].to(DEV) if d["bias"] is not None else None
+    X = d["X"].to(DEV)
+    layer = q.QuikLinear(d["W"].to(DEV), perm_d, cfg.k_o, cfg.group, cfg.outlier_int8, b)
+    Y = layer(X)
+    gx = q.quantize_reorder(X, perm_d, cfg.k_o, cfg.group, cfg.outlier_int8)
+    Y2 = q.gemm(gx, (layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale), cfg.K, cfg.k_o,
+                cfg.group, b)
+    acc, _ = q.gemm_i32(gx[0], layer.Wq, cfg.K, cfg.k_o, 0)
+    torch.cuda.synchronize()
+    ox = oracle.quantize_rows(np16(d["X"]), d["perm"].numpy(), cfg.k_o, 0, cfg.outlier_int8)
+    ow = oracle.quantize_rows(np16(d["W"]), d["perm"].numpy(), cfg.k_o, 0, cfg.outlier_int8)
+    assert_quant_equal(gpu_tuple_np(gx), ox, f"{name} X")
+    assert_quant_equal(gpu_tuple_np((layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale)), ow,
+                       f"{name} W")
+    np.testing.assert_array_equal(acc.cpu().numpy(), oracle.int_gemm(ox[0], ow[0], 0))
+    bias_np = None if d["bias"] is None else np16(d["bias"])
+    ref = oracle.linear(ox[0], ox[1], ox[2] if cfg.k_o else None, ox[3], ow[0], ow[1],
+                        ow[2] if cfg.k_o else None, ow[3], bias_np, cfg.K, cfg.k_o, 0)
+    assert_y_close(Y.float().cpu().numpy(), ref, name)
+    np.testing.assert_array_equal(Y.cpu().numpy().view(np.uint16), Y2.cpu().numpy().view(np.uint16))
 
 
 # ----------------------------------------------------------------- INT8 activations (W4A8)
@@ -398,3 +438,29 @@ def test_w8_without_a8_is_unsupported():
     with pytest.raises(q.QuikError) as e:
         q.quik_pack_weights(shape, W, perm, Wq, sw, None, None)
     assert e.value.status == q.QUIK_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("shape", [(257, 513, 2080, 32, 0, False, True),
+                                   (16, 256, 256, 32, 0, False, True)])
+def test_linear_timed_is_linear(shape):
+    """quik_linear_timed (an event between the layer's two kernels) writes
+    the same Y as quik_linear, bit for bit, and its event falls between the
+    events around the call."""
+    M, N, K, k_o, group, int8, bias = shape
+    cfg, d = _case(*shape, seed=17)
+    perm_d = d["perm"].to(DEV)
+    b = d["bias"].to(DEV) if d["bias"] is not None else None
+    X = d["X"].to(DEV)
+    layer = q.QuikLinear(d["W"].to(DEV), perm_d, k_o, group, int8, b)
+    Y = layer(X)
+    shape_s = layer.shape(M)
+    ws = torch.empty(q.quik_workspace_size(shape_s), dtype=torch.uint8, device=DEV)
+    Y2 = torch.full_like(Y, float("nan"))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record()
+    q.quik_linear_timed(shape_s, X, perm_d, layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale, b,
+                        Y2, ws, ev[1])
+    ev[2].record()
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(Y.cpu().numpy().view(np.uint16), Y2.cpu().numpy().view(np.uint16))
+    assert ev[0].elapsed_time(ev[1]) > 0 and ev[1].elapsed_time(ev[2]) > 0

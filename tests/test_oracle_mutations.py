@@ -17,6 +17,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "quik_oracle.c")
 
 DENSE, NORM, SPARSE = "test_oracle_pins.py", "test_oracle_rmsnorm_pins.py", "test_oracle_sparse24_pins.py"
+EXACT = "test_oracle_rmsnorm_exact_sum.py"
 
 # (name, function whose body is changed, or None for a unique line anywhere,
 #  old text, new text, pin file)
@@ -66,6 +67,18 @@ MUTATIONS = [
      "double_to_half((double)z[Ki + i] * rf)", "double_to_half((double)z[Ki + i])", NORM),
     ("norm: INT8 outlier scale without the row factor", "oracle_rmsnorm_quantize_rows",
      "o_scale[r] = (float)((double)s * rf);", "o_scale[r] = s;", NORM),
+    ("norm: squares summed in fp64, in order", "oracle_rmsnorm_quantize_rows",
+     "double ss = ldexp((double)S, -48);",
+     "double ss = 0.0;\n            for (int64_t k2 = 0; k2 < K; ++k2) {\n"
+     "                double h2 = half_to_double(X[r * K + k2]);\n                ss += h2 * h2;\n"
+     "            }", EXACT),
+    ("norm: squares summed in fp64, reversed", "oracle_rmsnorm_quantize_rows",
+     "double ss = ldexp((double)S, -48);",
+     "double ss = 0.0;\n            for (int64_t k2 = K - 1; k2 >= 0; --k2) {\n"
+     "                double h2 = half_to_double(X[r * K + k2]);\n                ss += h2 * h2;\n"
+     "            }", EXACT),
+    ("norm: exact sum truncated to 64 bits", "oracle_rmsnorm_quantize_rows",
+     "double ss = ldexp((double)S, -48);", "double ss = ldexp((double)(uint64_t)S, -48);", EXACT),
     # 2:4-sparse weights
     ("2:4: ties to the higher position", "oracle_prune24_quantize_rows",
      "if (fabsf(g[i]) > fabsf(g[a])) a = i;", "if (fabsf(g[i]) >= fabsf(g[a])) a = i;", SPARSE),
@@ -120,6 +133,6 @@ def test_unmutated_copy_passes(tmp_path):
                     ignore=shutil.ignore_patterns("__pycache__", ".pytest_cache"))
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider",
                         os.path.join("tests", DENSE), os.path.join("tests", NORM),
-                        os.path.join("tests", SPARSE)], cwd=work, capture_output=True, text=True,
+                        os.path.join("tests", SPARSE), os.path.join("tests", EXACT)], cwd=work, capture_output=True, text=True,
                        timeout=600)
     assert r.returncode == 0, r.stdout[-2000:]

@@ -61,16 +61,18 @@ def _run_both(cfg, seed):
 
 
 @pytest.mark.parametrize("name", ["tiny_16x256x256", "llama7b_attn_2048x4096x4096",
-                                  "llama65b_mlp_grouped_1024x22016x8192"])
+                                  "llama65b_mlp_grouped_1024x22016x8192",
+                                  "llama7b_down_fused_4096x4096x11008"])
 def test_noalloc_matches_linear_twice(name):
     _run_both(wl.CONFIGS[name], seed=0)
 
 
 def test_noalloc_rejects_shapes_beyond_its_workspace():
     L = q.lib()
-    # M x K_i / 2 alone exceeds the fixed workspace: refused before any launch
+    # the widened codes alone (M x K_i bytes) exceed the fixed workspace:
+    # refused before any launch
     s = q.make_shape(32768, 256, 4096, 0)
-    assert q.quik_workspace_size(s) > (32 << 20)
+    assert q.quik_workspace_size(s) > (64 << 20)
     st = L.quik_linear_noalloc(ctypes.byref(s), None, None, None, None, None, None, None, None,
                                None)
     assert st == q.QUIK_ERR_UNSUPPORTED
