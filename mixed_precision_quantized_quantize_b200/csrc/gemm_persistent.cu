@@ -333,7 +333,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
     constexpr int S = C::S, SP = C::SP;
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t op_full[S], op_empty[S], x_full[S], pk_full[SP], pk_empty[SP];
-    __shared__ uint64_t acc_empty[2], rescaled[2], int_done[2], acc_full[2], mma_done;
+    __shared__ uint64_t acc_empty[2], rescaled[2], int_done[2], acc_full[2], mma_done, rescaled_last;
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     __shared__ unsigned err0_s;
@@ -366,6 +366,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
             mbar_init(&acc_full[b], 1);
         }
         mbar_init(&mma_done, 1);
+        mbar_init(&rescaled_last, 2 * 16);  // every warp of both CTAs (leader only)
         abort_s = 0;
         err0_s = *reinterpret_cast<volatile unsigned *>(&g_pgemm_error);
         fence_barrier_init();
@@ -398,6 +399,90 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
     const uint32_t tmem = tmem_base_s;
     const Abort ab{&abort_s, err0_s};
 
+    // A warp's view of tile j in the epilogue: TMEM lane quadrant warp % 4
+    // (the lanes this warp may access), its output channel, scales and bias.
+    struct TileLane {
+        uint32_t acc;
+        int gn, tok0;
+        bool n_ok;
+        float swn, bn;
+        const float *sxr;
+    };
+    auto tile_lane = [&](int j) {
+        TileLane t;
+        const int qd = warp & 3;
+        t.acc = tmem + (static_cast<uint32_t>(qd * 32) << 16) + 256u * (j & 1);
+        t.gn = w_row0(j) + qd * 32 + lane;
+        t.n_ok = t.gn < p.N;
+        t.tok0 = ((pair + j * npairs) % p.n_tt) * BT;
+        t.swn = (!DEBUG && t.n_ok) ? p.sw[t.gn] : 0.0f;
+        t.bn = (!DEBUG && t.n_ok && p.bias != nullptr) ? __half2float(__ushort_as_half(p.bias[t.gn])) : 0.0f;
+        t.sxr = &sx_s[j & 1][0];
+        return t;
+    };
+    // y = A sx sw + bias in place, 32-column chunks c0, c0 + cstep, ...
+    auto rescale_chunks = [&](const TileLane &t, uint32_t acc, int c0, int cstep) {
+#pragma unroll 1
+        for (int c = c0; c < BT / 32; c += cstep) {
+            uint32_t a[32];
+            tmem_ld_32x32b_x32(acc + 32 * c, a);
+            tmem_ld_wait();
+            dequant32(a, t.sxr + 32 * c, t.swn, t.bn);
+            tmem_st_32x32b_x32(acc + 32 * c, a);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+    };
+    // fp16 Y for chunks c0, c0 + cstep, ... (the integer sums with DEBUG),
+    // through the warp's 32 x 32 staging tile and TMA stores when tma_y
+    auto final_chunks = [&](int j, const TileLane &t, uint32_t acc, uint16_t *ystage, int c0, int cstep) {
+#pragma unroll 1
+        for (int c = c0; c < BT / 32; c += cstep) {
+            uint32_t a[32];
+            tmem_ld_32x32b_x32(acc + 32 * c, a);
+            tmem_ld_wait();
+            if (!DEBUG && p.nkb_o == 0) dequant32(a, t.sxr + 32 * c, t.swn, t.bn);  // else rescaled already
+            const int m0 = t.tok0 + 32 * c;
+            if (DEBUG) {
+                if (t.n_ok) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj)
+                        if (m0 + jj < p.M)
+                            p.acc_dbg[static_cast<size_t>(m0 + jj) * p.N + t.gn] = static_cast<int32_t>(a[jj]) >> 8;
+                }
+                continue;
+            }
+            if (p.tma_y) {
+                // transpose through the staging tile ([token][channel], a warp's
+                // stores of one token are 64 contiguous bytes), then one TMA
+                // store; the tile's previous store must have read it first
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj)
+                    ystage[jj * 32 + lane] = __half_as_ushort(__float2half_rn(__uint_as_float(a[jj])));
+                fence_proxy_async_smem();  // generic stores -> visible to the TMA store
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tm_y, ystage, w_row0(j) + 32 * (warp & 3), m0);  // clipped at N and M
+                    bulk_commit_group();
+                }
+            } else {
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj)
+                    if (t.n_ok && m0 + jj < p.M)
+                        p.Y[static_cast<size_t>(m0 + jj) * p.N + t.gn] =
+                            __half_as_ushort(__float2half_rn(__uint_as_float(a[jj])));
+            }
+        }
+    };
+    // the issuer's state, kept for the last tile's outlier units (issued from
+    // the all-warps pass below)
+    const uint32_t id_f16 = idesc_f16_f32(2 * BW, BT);
+    const uint64_t d0 = sw128_kmajor_desc(smem_base);  // + (byte offset >> 4) per stage and k-step
+    Ring ring{0, 0u, 0};
+    bool issue_ok = true;
     if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer (leader)
         // Straight-line issue code: the tensor core queues about one MMA ahead
@@ -409,9 +494,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
         // of for_each_unit.
         if (rank == 0 && lane == 0) {
             const uint32_t id_i8 = idesc_s8_s32(2 * BW, BT);
-            const uint32_t id_f16 = idesc_f16_f32(2 * BW, BT);
-            const uint64_t d0 = sw128_kmajor_desc(smem_base);  // + (byte offset >> 4) per stage and k-step
-            Ring ring{0, 0u, 0};
             bool ok = true;
             for (int j = 0; j < ntp && ok; ++j) {
                 const int b = j & 1;
@@ -432,16 +514,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
                     ok = issue_unit<false, S>(ring, op_full, op_empty, d0, acc, id_i8, 1u, ab);
                 if (ok) mma2_commit_both(p.nkb_o > 0 ? &int_done[b] : &acc_full[b]);
             }
-            if (ok && ntp > 0 && p.nkb_o > 0) {
-                const int bo = (ntp - 1) & 1;
-                ok = wait_bar(&rescaled[bo], ((ntp - 1) >> 1) & 1, ab);
-                for (int o = 0; o < p.nkb_o && ok; ++o)
-                    ok = issue_unit<true, S>(ring, op_full, op_empty, d0, tmem + 256u * bo, id_f16, 1u, ab);
-                if (ok) mma2_commit_both(&acc_full[bo]);
-            }
-            // TMEM and the stages stay allocated until every issued MMA is done
-            mma2_commit_local(&mma_done);
-            mbar_wait_bounded(&mma_done, 0, kWaitLimitNs);
+            issue_ok = ok;
         }
         __syncwarp();
     } else if (warp == W_XPROD) {
@@ -559,11 +632,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int e = warp - W_EPI;  // 0 .. 3
-        const int qd = warp & 3;     // TMEM lane quadrant this warp may access
         const int et = threadIdx.x - 32 * W_EPI;  // 0 .. 127
-        const int r = qd * 32 + lane;             // TMEM lane = output channel in the CTA
-        const uint32_t t_lane = tmem + ((uint32_t)(qd * 32) << 16);
-
         uint16_t *ystage = reinterpret_cast<uint16_t *>(smem + C::EPI_OFF + e * C::EPI_TILE);
         if (!DEBUG) grid_dependency_wait();  // sx comes from the previous kernel
         // After a failed wait a warp skips the work of the remaining tiles but
@@ -571,8 +640,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
         bool ok = true;
         for (int j = 0; j < ntp; ++j) {
             const int b = j & 1, uj = j >> 1;
-            const int gn = w_row0(j) + r;
-            const bool n_ok = gn < p.N;
             const int tok0 = ((pair + j * npairs) % p.n_tt) * BT;
             if (!DEBUG) {
                 for (int c = et; c < BT; c += 32 * NE) {
@@ -580,28 +647,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
                     sx_s[b][c] = m < p.M ? p.sx[m] : 0.0f;
                 }
             }
+            if (j == ntp - 1) break;  // the last tile: every warp of the CTA, below
             named_barrier_sync(1, 32 * NE);  // sx_s[b] filled (and tile j-2 done with it)
             if (!ok) continue;
-            const float swn = (!DEBUG && n_ok) ? p.sw[gn] : 0.0f;
-            const float bn = (!DEBUG && n_ok && p.bias != nullptr) ? __half2float(__ushort_as_half(p.bias[gn])) : 0.0f;
-            const uint32_t acc = t_lane + 256u * b;
-            const float *sxr = &sx_s[b][0];
+            const TileLane t = tile_lane(j);
+            const uint32_t acc = t.acc;
             if (p.nkb_o > 0) {
                 if (!(ok = warp_wait_lazy(&int_done[b], uj & 1, ab, lane))) continue;
                 tc_fence_after();
                 if (et == 0) PTRACE(7, 4 * j);
                 // y = A sx sw + bias in place; the outlier MMAs accumulate onto it
-#pragma unroll 1
-                for (int c = 0; c < BT / 32; ++c) {
-                    uint32_t a[32];
-                    tmem_ld_32x32b_x32(acc + 32 * c, a);
-                    tmem_ld_wait();
-                    dequant32(a, sxr + 32 * c, swn, bn);
-                    tmem_st_32x32b_x32(acc + 32 * c, a);
-                }
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
+                rescale_chunks(t, acc, 0, 1);
                 if (et == 0) PTRACE(7, 4 * j + 1);
                 if (lane == 0) {
                     if (rank == 0)
@@ -613,45 +669,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
             if (!(ok = warp_wait_lazy(&acc_full[b], uj & 1, ab, lane))) continue;
             tc_fence_after();
             if (et == 0) PTRACE(7, 4 * j + 2);
-#pragma unroll 1
-            for (int c = 0; c < BT / 32; ++c) {
-                uint32_t a[32];
-                tmem_ld_32x32b_x32(acc + 32 * c, a);
-                tmem_ld_wait();
-                if (!DEBUG && p.nkb_o == 0) dequant32(a, sxr + 32 * c, swn, bn);  // else rescaled already
-                const int m0 = tok0 + 32 * c;
-                if (DEBUG) {
-                    if (n_ok) {
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj)
-                            if (m0 + jj < p.M)
-                                p.acc_dbg[static_cast<size_t>(m0 + jj) * p.N + gn] = static_cast<int32_t>(a[jj]) >> 8;
-                    }
-                    continue;
-                }
-                if (p.tma_y) {
-                    // transpose through this warp's 32 x 32 staging tile ([token][channel],
-                    // a warp's stores of one token are 64 contiguous bytes), then one
-                    // TMA store; the tile's previous store must have read it first
-                    if (lane == 0) bulk_wait_group_read0();
-                    __syncwarp();
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj)
-                        ystage[jj * 32 + lane] = __half_as_ushort(__float2half_rn(__uint_as_float(a[jj])));
-                    fence_proxy_async_smem();  // generic stores -> visible to the TMA store
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tm_y, ystage, w_row0(j) + 32 * qd, m0);  // clipped at N and M
-                        bulk_commit_group();
-                    }
-                } else {
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj)
-                        if (n_ok && m0 + jj < p.M)
-                            p.Y[static_cast<size_t>(m0 + jj) * p.N + gn] =
-                                __half_as_ushort(__float2half_rn(__uint_as_float(a[jj])));
-                }
-            }
+            final_chunks(j, t, acc, ystage, 0, 1);
             tc_fence_before();
             __syncwarp();
             if (et == 0) PTRACE(7, 4 * j + 3);
@@ -662,7 +680,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
                     mbar_arrive_remote(mapa_shared(smem_u32(&acc_empty[b]), 0));
             }
         }
-        if (lane == 0 && p.tma_y) bulk_wait_group0();  // the stores complete before the CTA leaves
+        if (lane == 0 && p.tma_y) bulk_wait_group_read0();  // tile ntp-2's stores have read their tiles
+    }
+
+    // ------------------------------------------------------------ the last tile, every warp
+    // Its two epilogue passes are the exposed tail of the kernel: all 16 warps
+    // of each CTA share them (warp w: TMEM lane quadrant w % 4, column chunks
+    // w / 4 and w / 4 + 4), and the last tile's outlier units are issued in
+    // between.  Each warp stages its 32 x 32 output tiles in the operand
+    // ring, which every MMA has finished reading by then.
+    named_barrier_sync(2, THREADS);  // every role done with its loop; the last tile's sx_s filled
+    if (ntp > 0) {
+        const int j = ntp - 1, b = j & 1, uj = j >> 1;
+        bool ok = abort_s == 0;
+        const TileLane t = tile_lane(j);
+        const uint32_t acc = t.acc;
+        const int c0 = warp >> 2;
+        if (p.nkb_o > 0) {
+            if (ok && (ok = warp_wait_lazy(&int_done[b], uj & 1, ab, lane))) {
+                tc_fence_after();
+                rescale_chunks(t, acc, c0, 4);
+            }
+            if (lane == 0) {  // also after a failed wait: the issuer's wait below then ends at once
+                if (rank == 0)
+                    mbar_arrive(&rescaled_last);
+                else
+                    mbar_arrive_remote(mapa_shared(smem_u32(&rescaled_last), 0));
+            }
+            if (warp == W_MMA && rank == 0 && lane == 0 && issue_ok) {
+                bool iok = wait_bar(&rescaled_last, 0, ab);
+                for (int o = 0; o < p.nkb_o && iok; ++o)
+                    iok = issue_unit<true, S>(ring, op_full, op_empty, d0, tmem + 256u * b, id_f16, 1u, ab);
+                if (iok) mma2_commit_both(&acc_full[b]);
+            }
+            __syncwarp();
+        }
+        if (ok && (ok = warp_wait_lazy(&acc_full[b], uj & 1, ab, lane))) {
+            tc_fence_after();
+            final_chunks(j, t, acc, reinterpret_cast<uint16_t *>(smem + warp * C::EPI_TILE), c0, 4);
+            // the stores have read their staging tiles before the CTA leaves (the
+            // global writes complete with the grid)
+            if (lane == 0 && p.tma_y) bulk_wait_group_read0();
+        }
+        if (warp == W_MMA && rank == 0 && lane == 0) {
+            // TMEM and the stages stay allocated until every issued MMA is done
+            mma2_commit_local(&mma_done);
+            mbar_wait_bounded(&mma_done, 0, kWaitLimitNs);
+        }
+        __syncwarp();
     }
 
     // ---------------------------------------------------------------- teardown
