@@ -1,6 +1,7 @@
 """The mbarrier and named-barrier protocols of the kernels (the CTA-pair
-kernel, the dense and 2:4 decode kernels, the grouped-scale kernel, the
-quantiser's team ring), run on the CPU under random schedules (no GPU).
+kernel, the persistent warp-specialised CTA-pair kernel, the dense and 2:4
+decode kernels, the grouped-scale kernel, the quantiser's team ring), run on
+the CPU under random schedules (no GPU).
 
 An mbarrier completes a phase when its expected arrivals have come; a wait
 on parity P passes while the barrier's current phase parity differs from P.
@@ -409,6 +410,202 @@ def test_quantizer_team_protocol(NR, mode):
 
 
 # ----------------------------------------------------------------- the checker itself
+# ----------------------------------------------------------------- persistent CTA-pair kernel
+def unit_order(ntp, nkb_i, nkb_o, out_delay):
+    """The persistent kernel's work units in issue order: (tile, outlier, k).
+    Tile j's INT4 k-blocks, tile j-1's outlier units after the first
+    out_delay of them, the last tile's outlier units at the end."""
+    units = []
+    for j in range(ntp):
+        for k in range(nkb_i):
+            if j > 0 and k == out_delay:
+                units += [(j - 1, True, o) for o in range(nkb_o)]
+            units.append((j, False, k))
+        if j > 0 and nkb_i <= out_delay:
+            units += [(j - 1, True, o) for o in range(nkb_o)]
+    if ntp > 0:
+        units += [(ntp - 1, True, o) for o in range(nkb_o)]
+    return units
+
+
+def persistent_roles(ntp, nkb_i, nkb_o, x4=False, S=5, SP=6, NG=3, GW=3, NE=4, out_delay=6,
+                     last_rescale_count=None):
+    """Two CTAs of 16 warps: the leader's MMA issuer, per CTA one operand
+    TMA producer, one packed-staging producer, NG unpack groups of GW warps
+    (group g takes units g, g + NG, ...) and NE epilogue warps.  The leader's
+    operand-full barriers take the arrivals of the unit's group in both CTAs;
+    commits reach both CTAs.  Tiles alternate between two accumulators; the
+    epilogue rescales tile j-1 (FP16 outliers) while tile j's k-blocks run;
+    the last tile's two epilogue passes are shared by every warp after a
+    CTA-wide barrier, with its own arrival count on the rescale barrier."""
+    units = unit_order(ntp, nkb_i, nkb_o, out_delay)
+    op_full = [Bar(2 * GW) for _ in range(S)]
+    op_empty = [[Bar(1) for _ in range(S)] for _ in range(2)]
+    x_full = [[Bar(1) for _ in range(S)] for _ in range(2)]
+    pk_full = [[Bar(1) for _ in range(SP)] for _ in range(2)]
+    pk_empty = [[Bar(GW) for _ in range(SP)] for _ in range(2)]
+    acc_empty = [Bar(2 * NE) for _ in range(2)]
+    rescaled = [Bar(2 * NE) for _ in range(2)]
+    int_done = [[Bar(1) for _ in range(2)] for _ in range(2)]
+    acc_full = [[Bar(1) for _ in range(2)] for _ in range(2)]
+    rescaled_last = Bar(last_rescale_count or 2 * 16)
+    mma_done = Bar(1)
+    epi = [Sync(NE) for _ in range(2)]
+    everyone = [Sync(16) for _ in range(2)]
+    stage = [[Buf(f"CTA {c} operand stage {i}") for i in range(S)] for c in range(2)]
+    slot = [[Buf(f"CTA {c} staging slot {i}") for i in range(SP)] for c in range(2)]
+    acc = [[Buf(f"CTA {c} accumulator {b}") for b in range(2)] for c in range(2)]
+    last, bl = ntp - 1, (ntp - 1) & 1
+    ring = {"u": 0}
+
+    def issue(u, b):
+        st = u % S
+        yield ("wait", op_full[st], u // S)
+        for c in range(2):
+            yield ("own", stage[c][st])
+        for c in range(2):
+            yield ("write", acc[c][b])
+        for c in range(2):
+            yield ("async", op_empty[c][st], stage[c][st])
+
+    def issuer():
+        u = 0
+        for j in range(ntp):
+            b = j & 1
+            if j >= 2:
+                yield ("wait", acc_empty[b], (j >> 1) - 1)
+            k1 = min(out_delay, nkb_i) if j > 0 else nkb_i
+            for _ in range(k1):
+                yield from issue(u, b)
+                u += 1
+            if j > 0 and nkb_o > 0:
+                bo = (j - 1) & 1
+                yield ("wait", rescaled[bo], (j - 1) >> 1)
+                for _ in range(nkb_o):
+                    yield from issue(u, bo)
+                    u += 1
+                for c in range(2):
+                    yield ("async", acc_full[c][bo])
+            for _ in range(nkb_i - k1):
+                yield from issue(u, b)
+                u += 1
+            for c in range(2):
+                yield ("async", (int_done if nkb_o > 0 else acc_full)[c][b])
+        ring["u"] = u
+
+    def last_tile(c, w):
+        """Every warp's share of the last tile (warp w of CTA c)."""
+        yield ("sync", everyone[c])
+        if nkb_o > 0:
+            yield ("wait", int_done[c][bl], last >> 1)
+            yield ("own", acc[c][bl])
+            yield ("free", acc[c][bl])
+            yield ("arrive", rescaled_last)
+            if c == 0 and w == 0:
+                yield ("wait", rescaled_last, 0)
+                u = ring["u"]
+                for _ in range(nkb_o):
+                    yield from issue(u, bl)
+                    u += 1
+                for cc in range(2):
+                    yield ("async", acc_full[cc][bl])
+        yield ("wait", acc_full[c][bl], last >> 1)
+        yield ("own", acc[c][bl])
+        yield ("free", acc[c][bl])
+        if c == 0 and w == 0:
+            yield ("async", mma_done)
+            yield ("wait", mma_done, 0)
+
+    def mma_warp(c):
+        if c == 0:
+            yield from issuer()
+        yield from last_tile(c, 0)
+
+    def xprod(c):
+        for u, (j, outl, k) in enumerate(units):
+            st = u % S
+            if u >= S:
+                yield ("wait", op_empty[c][st], u // S - 1)
+            if outl or not x4:
+                yield ("write", stage[c][st])
+                yield ("async", x_full[c][st])
+            else:
+                yield ("arrive", x_full[c][st])
+        yield from last_tile(c, 4)
+
+    def pprod(c):
+        q = 0
+        for (j, outl, k) in units:
+            if outl:
+                continue
+            ps = q % SP
+            if q >= SP:
+                yield ("wait", pk_empty[c][ps], q // SP - 1)
+            yield ("write", slot[c][ps])
+            yield ("async", pk_full[c][ps])
+            q += 1
+        yield from last_tile(c, 8)
+
+    def unpack(c, g, w):
+        q = 0
+        for u, (j, outl, k) in enumerate(units):
+            if u % NG != g:
+                q += 0 if outl else 1
+                continue
+            st = u % S
+            if u >= S:
+                yield ("wait", op_empty[c][st], u // S - 1)
+            if not outl:
+                ps = q % SP
+                yield ("wait", pk_full[c][ps], q // SP)
+                yield ("own", slot[c][ps])
+                yield ("write", stage[c][st])
+                yield ("free", slot[c][ps])
+                yield ("arrive", pk_empty[c][ps])
+                q += 1
+            if outl or not x4:
+                yield ("wait", x_full[c][st], u // S)
+            yield ("arrive", op_full[st])
+        yield from last_tile(c, 1 + 4 * g + w)
+
+    def epilogue(c, e):
+        for j in range(ntp - 1):
+            b, uj = j & 1, j >> 1
+            yield ("sync", epi[c])
+            if nkb_o > 0:
+                yield ("wait", int_done[c][b], uj)
+                yield ("own", acc[c][b])
+                yield ("free", acc[c][b])
+                yield ("arrive", rescaled[b])
+            yield ("wait", acc_full[c][b], uj)
+            yield ("own", acc[c][b])
+            yield ("free", acc[c][b])
+            yield ("arrive", acc_empty[b])
+        yield from last_tile(c, 12 + e)
+
+    roles = []
+    for c in range(2):
+        roles += [mma_warp(c), xprod(c), pprod(c)]
+        roles += [unpack(c, g, w) for g in range(NG) for w in range(GW)]
+        roles += [epilogue(c, e) for e in range(NE)]
+    return roles
+
+
+@pytest.mark.parametrize("ntp", [1, 2, 3, 5])
+@pytest.mark.parametrize("nkb_i,nkb_o", [(1, 0), (4, 1), (7, 2), (31, 2), (31, 0), (6, 2)])
+@pytest.mark.parametrize("x4", [False, True])
+def test_persistent_protocol(ntp, nkb_i, nkb_o, x4):
+    for seed in range(4):
+        run(persistent_roles(ntp, nkb_i, nkb_o, x4=x4), seed)
+
+
+def test_checker_catches_a_short_last_rescale_count():
+    """The last tile's rescale barrier counting only the epilogue warps (the
+    count of the other tiles' barrier): its phase completes before every
+    warp has rescaled, and the later arrivals overflow it."""
+    assert _caught(lambda: persistent_roles(2, 7, 2, last_rescale_count=2 * 4))
+
+
 def _caught(make, seeds=60):
     for seed in range(seeds):
         try:
