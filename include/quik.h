@@ -379,6 +379,22 @@ QUIK_API quik_status quik_sync_check(quik_stream_t stream);
  */
 QUIK_API quik_status quik_selftest_timeout(uint32_t limit_us, quik_stream_t stream);
 
+/*
+ * quik_test_stall -- test entry: makes a production kernel take its timeout
+ * path without a fault.  site 1: each team leader of the quantiser
+ * (quik_quantize_reorder and the layer calls' quantiser) first waits on a
+ * barrier that nothing completes; site 2: the persistent GEMM's MMA issuer
+ * (more than 32 tokens, per-channel scales, FP16 or no outliers) does.  The
+ * wait runs out after the kernels' limit (2 s), the kernel records the error
+ * and exits through its abort path (its other waits give up at once), and
+ * quik_sync_check reports QUIK_ERR_TIMEOUT; that call's outputs are
+ * unspecified.  site 0 restores normal operation.  The switch is global to
+ * the library and the device that is current; it is copied synchronously.
+ * Returns QUIK_ERR_INVALID_ARG for another site, QUIK_ERR_CUDA if the copy
+ * fails.
+ */
+QUIK_API quik_status quik_test_stall(int site);
+
 /* Static string for a status code. */
 QUIK_API const char *quik_status_string(quik_status status);
 

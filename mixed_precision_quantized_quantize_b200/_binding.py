@@ -63,6 +63,7 @@ _SIGS = {
     "quik_workspace_size_24": (ctypes.c_size_t, [_S]),
     "quik_sync_check": (ctypes.c_int, [_P]),
     "quik_selftest_timeout": (ctypes.c_int, [ctypes.c_uint32, _P]),
+    "quik_test_stall": (ctypes.c_int, [ctypes.c_int]),
     "quik_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 _lib = None
@@ -276,6 +277,13 @@ def quik_workspace_size_24(shape: quik_shape) -> int:
 
 def quik_sync_check(stream=None) -> int:
     return int(lib().quik_sync_check(_stream(stream)))
+
+
+def quik_test_stall(site: int):
+    """Test entry: 1 stalls the quantiser's first row wait, 2 the persistent
+    GEMM's MMA issuer (each then times out and reports QUIK_ERR_TIMEOUT);
+    0 restores normal operation."""
+    _check(lib().quik_test_stall(int(site)), "quik_test_stall")
 
 
 def quik_selftest_timeout(limit_us: int, stream=None):

@@ -458,6 +458,13 @@ quik_status quik_selftest_timeout(uint32_t limit_us, quik_stream_t stream) {
     return quik::launch_timeout_selftest(limit_us, static_cast<cudaStream_t>(stream));
 }
 
+quik_status quik_test_stall(int site) {
+    if (site < 0 || site > 2) return QUIK_ERR_INVALID_ARG;
+    if (quik::set_quantize_stall(site == 1) != cudaSuccess) return QUIK_ERR_CUDA;
+    if (quik::set_persistent_gemm_stall(site == 2) != cudaSuccess) return QUIK_ERR_CUDA;
+    return QUIK_OK;
+}
+
 const char *quik_status_string(quik_status status) {
     switch (status) {
         case QUIK_OK: return "QUIK_OK";

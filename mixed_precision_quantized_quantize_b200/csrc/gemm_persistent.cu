@@ -53,6 +53,10 @@ namespace quik {
 // Expired waits in this file's kernel.  It only grows; quik_sync_check
 // reports its increase.
 __device__ unsigned int g_pgemm_error;
+// Test entry (quik_test_stall): nonzero makes the MMA issuer wait first on a
+// barrier that nothing completes, so its bounded wait runs out and every role
+// of every CTA takes the abort path.
+__device__ int g_pgemm_stall;
 
 // Optional pipeline timeline (build with -DQUIK_TRACE): SM clock stamps of
 // each role's events per work unit, for the first pair of a launch.
@@ -334,6 +338,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t op_full[S], op_empty[S], x_full[S], pk_full[SP], pk_empty[SP];
     __shared__ uint64_t acc_empty[2], rescaled[2], int_done[2], acc_full[2], mma_done, rescaled_last;
+    __shared__ uint64_t stall_bar;  // never completed (quik_test_stall)
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     __shared__ unsigned err0_s;
@@ -367,6 +372,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
         }
         mbar_init(&mma_done, 1);
         mbar_init(&rescaled_last, 2 * 16);  // every warp of both CTAs (leader only)
+        mbar_init(&stall_bar, 1);
         abort_s = 0;
         err0_s = *reinterpret_cast<volatile unsigned *>(&g_pgemm_error);
         fence_barrier_init();
@@ -494,7 +500,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
         // of for_each_unit.
         if (rank == 0 && lane == 0) {
             const uint32_t id_i8 = idesc_s8_s32(2 * BW, BT);
-            bool ok = true;
+            bool ok = *reinterpret_cast<volatile int *>(&g_pgemm_stall) == 0 || wait_bar(&stall_bar, 0, ab);
             for (int j = 0; j < ntp && ok; ++j) {
                 const int b = j & 1;
                 const uint32_t acc = tmem + 256u * b;
@@ -826,6 +832,10 @@ extern "C" __attribute__((visibility("default"))) int ptrace_read(unsigned long 
     return cudaMemcpyFromSymbol(dst, g_ptrace, sizeof(g_ptrace)) == cudaSuccess ? 0 : -1;
 }
 #endif
+
+cudaError_t set_persistent_gemm_stall(int on) {
+    return cudaMemcpyToSymbol(g_pgemm_stall, &on, sizeof(on));
+}
 
 unsigned int persistent_gemm_errors() {
     unsigned int word = 0;

@@ -49,6 +49,10 @@ QUIK_CHECK_DECL
 // increase since its previous call (take_quantize_errors).
 __device__ unsigned int g_quant_error;
 __device__ unsigned int g_quant_bad_perm;
+// Test entry (quik_test_stall): nonzero makes each team leader's first row
+// wait on a barrier that nothing completes, so the bounded wait runs out and
+// the kernel takes its error path.
+__device__ int g_quant_stall;
 
 namespace {
 
@@ -381,6 +385,7 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : (GROUP
     __shared__ float red[kQMaxTeams][2][kQMaxThreads / 32];  // warp maxima, two slots per team
     __shared__ SumSq red_ss[kQMaxTeams][2][kQMaxThreads / 32];  // warp sums of squares (NORM)
     __shared__ uint64_t row_full[kQMaxTeams][kQMaxRing];
+    __shared__ uint64_t stall_bar;  // never completed (quik_test_stall)
     const int K = p.K, Ki = K - p.k_o;  // K % 16 == 0
     const int TT = p.team_threads;
     const int team = threadIdx.x / TT, tl = threadIdx.x - team * TT;  // team-local thread
@@ -413,6 +418,7 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : (GROUP
         for (int t = 0; t < p.teams; ++t)
             for (int r = 0; r < NR; ++r) ptx::mbar_init(&row_full[t][r], 1);
         ptx::mbar_init(&perm_full, 1);
+        ptx::mbar_init(&stall_bar, 1);
         ptx::fence_barrier_init();
         if (P32) {  // the int32 perm lands in the table area and is converted in place
             ptx::mbar_arrive_expect_tx(&perm_full, perm_bytes);
@@ -475,7 +481,10 @@ __global__ void __launch_bounds__(kQMaxThreads) __maxnreg__(W > 4 ? 128 : (GROUP
         // (1) the leader waits for this row (bounded); the barrier hands it to
         // the team and ends every thread's use of the previous slot
         bool ok = true;
-        if (tl == 0) ok = ptx::mbar_wait_bounded_sleep(&row_full[team][j % NR], (j / NR) & 1, kWaitLimitNs);
+        if (tl == 0)
+            ok = (j == 0 && *reinterpret_cast<volatile int *>(&g_quant_stall) != 0)
+                     ? ptx::mbar_wait_bounded_sleep(&stall_bar, 0, kWaitLimitNs)
+                     : ptx::mbar_wait_bounded_sleep(&row_full[team][j % NR], (j / NR) & 1, kWaitLimitNs);
         if (team_sync_or(bar_id, TT, !ok)) {
             if (tl == 0) atomicAdd(&g_quant_error, 1u);
             break;
@@ -962,6 +971,10 @@ cudaError_t launch_expand24(const uint8_t *Qs, const uint8_t *meta, int rows, in
     const int grid = static_cast<int>(want < 8LL * sm_count() ? want : 8LL * sm_count());
     expand24_kernel<<<grid, threads, 0, stream>>>(Qs, meta, total, Ki, reinterpret_cast<uint4 *>(Q));
     return cudaGetLastError();
+}
+
+cudaError_t set_quantize_stall(int on) {
+    return cudaMemcpyToSymbol(g_quant_stall, &on, sizeof(on));
 }
 
 unsigned int take_quantize_errors(unsigned int *bad_perm) {

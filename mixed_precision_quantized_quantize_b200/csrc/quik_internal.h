@@ -124,6 +124,9 @@ bool persistent_gemm_takes(const GemmArgs &a);
 quik_status launch_gemm_persistent(const GemmArgs &a, cudaStream_t stream);
 // Expired waits in the persistent kernel since the last check.
 unsigned int persistent_gemm_errors();
+// quik_test_stall's switches (test entry)
+cudaError_t set_quantize_stall(int on);
+cudaError_t set_persistent_gemm_stall(int on);
 // 2-D row-major TMA map: `inner` elements per row (contiguous), `rows` rows,
 // `stride` bytes between rows; box of box_inner x box_rows; elements outside
 // the tensor read as zero.

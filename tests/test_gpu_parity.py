@@ -464,3 +464,144 @@ def test_linear_timed_is_linear(shape):
     torch.cuda.synchronize()
     np.testing.assert_array_equal(Y.cpu().numpy().view(np.uint16), Y2.cpu().numpy().view(np.uint16))
     assert ev[0].elapsed_time(ev[1]) > 0 and ev[1].elapsed_time(ev[2]) > 0
+
+
+@pytest.mark.parametrize("site,shape", [(1, (64, 256, 512, 64)), (2, (257, 513, 2080, 32))],
+                         ids=["quantiser", "persistent-gemm"])
+def test_production_kernel_timeout_path(site, shape):
+    """quik_test_stall: a production kernel (1: the quantiser's row wait, 2:
+    the persistent GEMM's MMA issuer) first waits on a barrier that nothing
+    completes.  The bounded wait runs out (2 s), the kernel leaves through
+    its abort path without a fault, quik_sync_check reports
+    QUIK_ERR_TIMEOUT once, and the next layer call is correct (bit-identical
+    to the one before the stall)."""
+    M, N, K, k_o = shape
+    cfg, d = _case(M, N, K, k_o, 0, False, True, seed=21)
+    perm_d = d["perm"].to(DEV)
+    layer = q.QuikLinear(d["W"].to(DEV), perm_d, k_o, 0, False, d["bias"].to(DEV))
+    X = d["X"].to(DEV)
+    Y_ref = layer(X)
+    torch.cuda.synchronize()
+    assert q.quik_sync_check() == q.QUIK_OK
+    q.quik_test_stall(site)
+    try:
+        layer(X)
+        torch.cuda.synchronize()
+    finally:
+        q.quik_test_stall(0)
+    assert q.quik_sync_check() == q.QUIK_ERR_TIMEOUT
+    assert q.quik_sync_check() == q.QUIK_OK
+    Y = layer(X)
+    torch.cuda.synchronize()
+    assert q.quik_sync_check() == q.QUIK_OK
+    np.testing.assert_array_equal(Y.cpu().numpy().view(np.uint16), Y_ref.cpu().numpy().view(np.uint16))
+
+
+# the layer calls the canary and self-checking tests run: (M, N, K, k_o, group, int8 outliers, act bits)
+GUARDED = [
+    (130, 300, 640, 64, 0, False, 4),     # persistent GEMM (packed X through quik_gemm; widened in the layer)
+    (16, 520, 1056, 32, 0, False, 4),     # decode kernel
+    (70, 300, 544, 32, 0, True, 4),       # pair kernel with INT8 outliers
+    (150, 260, 1152, 128, 128, True, 4),  # grouped scales
+    (200, 300, 640, 64, 0, False, 8),     # W4A8
+]
+
+
+@pytest.mark.parametrize("shape", GUARDED, ids=[str(s) for s in GUARDED])
+def test_canary_guards_untouched_every_kernel(shape):
+    """Guard bytes around the workspace and Y of a layer call, and around
+    the outputs of the two-call path, stay untouched on every GEMM kernel
+    (persistent, decode, pair, grouped, W4A8) and the quantiser."""
+    M, N, K, k_o, group, int8, ab = shape
+    cfg = wl.custom_config(M, N, K, k_o, group, int8, True, outlier_mult=30.0, act_bits=ab)
+    d = wl.make_layer(cfg, seed_offset=3)
+    G, pat = 4096, 0xA5
+
+    def guarded(nbytes):
+        buf = torch.full((G + nbytes + G,), pat, dtype=torch.uint8, device=DEV)
+        return buf, buf[G:G + nbytes]
+
+    perm_d = d["perm"].to(DEV)
+    layer = q.QuikLinear(d["W"].to(DEV), perm_d, k_o, group, int8, d["bias"].to(DEV), act_bits=ab)
+    s = layer.shape(M)
+    bw, ws = guarded(q.quik_workspace_size(s))
+    by, Yb = guarded(M * N * 2)
+    q.quik_linear(s, d["X"].to(DEV), perm_d, layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale,
+                  d["bias"].to(DEV), Yb.view(torch.float16).view(M, N), ws)
+    torch.cuda.synchronize()
+    assert q.quik_sync_check() == q.QUIK_OK
+    for buf in (bw, by):
+        h = buf.cpu().numpy()
+        assert (h[:G] == pat).all() and (h[-G:] == pat).all()
+
+
+def test_sparse24_canary_guards_untouched():
+    """The same for the 2:4 layer, at decode (sparse kernel) and prefill
+    (expanded weights) token counts."""
+    for M in (16, 130):
+        cfg = wl.custom_config(M, 264, 1088, 64, 0, False, True, outlier_mult=30.0)
+        d = wl.make_layer(cfg, seed_offset=4)
+        G, pat = 4096, 0xA5
+        perm_d = d["perm"].to(DEV)
+        layer = q.QuikLinear24(d["W"].to(DEV), perm_d, 64, False, d["bias"].to(DEV))
+        s = layer.shape(M)
+        buf_w = torch.full((G + q.quik_workspace_size_24(s) + G,), pat, dtype=torch.uint8, device=DEV)
+        buf_y = torch.full((G + M * 264 * 2 + G,), pat, dtype=torch.uint8, device=DEV)
+        ws = buf_w[G:G + q.quik_workspace_size_24(s)]
+        Yb = buf_y[G:G + M * 264 * 2].view(torch.float16).view(M, 264)
+        q.quik_linear_24(s, d["X"].to(DEV), perm_d, layer.Wq24, layer.Wmeta, layer.w_scale, layer.Wo,
+                         layer.wo_scale, d["bias"].to(DEV), Yb, ws)
+        torch.cuda.synchronize()
+        assert q.quik_sync_check() == q.QUIK_OK
+        for b in (buf_w, buf_y):
+            h = b.cpu().numpy()
+            assert (h[:G] == pat).all() and (h[-G:] == pat).all(), M
+
+
+_CHECKED_CHILD = r'''
+import ctypes, sys
+import numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+import mixed_precision_quantized_quantize_b200._binding as B
+B.LIB_PATH = sys.argv[2]
+import mixed_precision_quantized_quantize_b200 as q
+from mixed_precision_quantized_quantize_b200 import workloads as wl
+out = {}
+for i, (M, N, K, k_o, group, int8, ab) in enumerate(eval(sys.argv[3])):
+    cfg = wl.custom_config(M, N, K, k_o, group, int8, True, outlier_mult=30.0, act_bits=ab)
+    d = wl.make_layer(cfg, seed_offset=9)
+    layer = q.QuikLinear(d["W"].cuda(), d["perm"].cuda(), k_o, group, int8, d["bias"].cuda(), act_bits=ab)
+    out[f"y{i}"] = layer(d["X"].cuda()).cpu().numpy().view(np.uint16)
+torch.cuda.synchronize()
+L = q.lib()
+for f in ("qchk_quantize_word", "qchk_gemm_word"):
+    getattr(L, f).restype = ctypes.c_ulonglong
+out["words"] = np.array([L.qchk_quantize_word(), L.qchk_gemm_word(), L.quik_sync_check(None)], np.uint64)
+np.savez(sys.argv[4], **out)
+'''
+
+
+def test_self_checking_build_matches(tmp_path):
+    """The self-checking build (-DQUIK_CHECKS: computed indices and
+    alignments checked, the first violation recorded and the access
+    skipped) runs the layer on every GEMM kernel with no violation and the
+    same outputs, bit for bit, as the normal build (in a child process: one
+    copy of the library per process)."""
+    import os
+    import subprocess
+    import sys
+    from mixed_precision_quantized_quantize_b200 import build as qbuild
+    checked = qbuild.build(checks=True)
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    npz = str(tmp_path / "checked.npz")
+    subprocess.run([sys.executable, "-c", _CHECKED_CHILD, root, checked, repr(GUARDED), npz],
+                   check=True, timeout=600)
+    got = np.load(npz)
+    assert got["words"].tolist() == [0, 0, q.QUIK_OK], got["words"]
+    for i, (M, N, K, k_o, group, int8, ab) in enumerate(GUARDED):
+        cfg = wl.custom_config(M, N, K, k_o, group, int8, True, outlier_mult=30.0, act_bits=ab)
+        d = wl.make_layer(cfg, seed_offset=9)
+        layer = q.QuikLinear(d["W"].to(DEV), d["perm"].to(DEV), k_o, group, int8, d["bias"].to(DEV),
+                             act_bits=ab)
+        y = layer(d["X"].to(DEV)).cpu().numpy().view(np.uint16)
+        np.testing.assert_array_equal(y, got[f"y{i}"], err_msg=str(GUARDED[i]))
