@@ -431,25 +431,32 @@ def run_ours(args, rank, local_rank, world):
     # per-kernel breakdown (separate, untimed-for-value pass)
     n_split = max(10, args.steps // 4)
     sev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_split)]
+    for _ in range(3):  # warm-up: the first launches of the split path's kernels
+        split_step([torch.cuda.Event(enable_timing=True) for _ in range(4)])
+    torch.cuda.synchronize()
     for i in range(n_split):
         flush.zero_()
         split_step(sev[i])
     torch.cuda.synchronize()
     g0 = 3 if prefill24 else 1  # the GEMM starts after the expansion on the 2:4 prefill path
-    gemm_avg = reduce_max(float(np.mean([e[g0].elapsed_time(e[2]) / 1e3 for e in sev])))
-    expand_avg = (reduce_max(float(np.mean([e[1].elapsed_time(e[3]) / 1e3 for e in sev])))
+    # per-kernel breakdown: medians over the split steps
+    gemm_avg = reduce_max(float(np.median([e[g0].elapsed_time(e[2]) / 1e3 for e in sev])))
+    expand_avg = (reduce_max(float(np.median([e[1].elapsed_time(e[3]) / 1e3 for e in sev])))
                   if prefill24 else None)
-    quant_avg = reduce_max(float(np.mean([e[0].elapsed_time(e[1]) / 1e3 for e in sev])))
-    split_avg = reduce_max(float(np.mean([e[0].elapsed_time(e[2]) / 1e3 for e in sev])))
+    quant_avg = reduce_max(float(np.median([e[0].elapsed_time(e[1]) / 1e3 for e in sev])))
+    split_avg = reduce_max(float(np.median([e[0].elapsed_time(e[2]) / 1e3 for e in sev])))
     layer_quant = layer_gemm = None
     if timed_layer:
         mev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_split)]
+        for _ in range(3):
+            marked_step([torch.cuda.Event(enable_timing=True) for _ in range(3)])
+        torch.cuda.synchronize()
         for i in range(n_split):
             flush.zero_()
             marked_step(mev[i])
         torch.cuda.synchronize()
-        layer_quant = reduce_max(float(np.mean([e[0].elapsed_time(e[1]) / 1e3 for e in mev])))
-        layer_gemm = reduce_max(float(np.mean([e[1].elapsed_time(e[2]) / 1e3 for e in mev])))
+        layer_quant = reduce_max(float(np.median([e[0].elapsed_time(e[1]) / 1e3 for e in mev])))
+        layer_gemm = reduce_max(float(np.median([e[1].elapsed_time(e[2]) / 1e3 for e in mev])))
     # the dominant kernel: the layer call's own GEMM where it can be timed
     # apart, else quik_gemm's
     dom_avg = layer_gemm if layer_gemm is not None else gemm_avg
