@@ -296,15 +296,20 @@ def test_full_size_layer(name):
     cols = np.unique(ns)[:512]
     r_t = torch.from_numpy(rows).to(DEV)
     c_t = torch.from_numpy(cols).to(DEV)
-    acc, _ = q.gemm_i32(gx[0][r_t].contiguous(), layer.Wq[c_t].contiguous(), cfg.K, cfg.k_o,
-                        cfg.group)
-    acc = acc.cpu().numpy()
+    int8_o = cfg.outlier_int8 and cfg.k_o > 0
+    acc, acc_o = q.gemm_i32(gx[0][r_t].contiguous(), layer.Wq[c_t].contiguous(), cfg.K, cfg.k_o,
+                            cfg.group, gx[2][r_t].contiguous() if int8_o else None,
+                            layer.Wo[c_t].contiguous() if int8_o else None)
     full = oracle.int_gemm(ox[0][rows], ow[0][cols], cfg.group)
-    np.testing.assert_array_equal(acc, full)
+    np.testing.assert_array_equal(acc.cpu().numpy(), full)
+    if int8_o:  # the INT8 outlier block's sums, exact
+        ref_o = ox[2][rows].astype(np.int64) @ ow[2][cols].astype(np.int64).T
+        np.testing.assert_array_equal(acc_o.cpu().numpy(), ref_o)
 
 
-# the layers small enough for the oracle to compute every output: c1, c2 and
-# the two smaller token counts of the up projection
+# the layers small enough for the oracle to compute every output: the tiny
+# layer, the Llama-7B attention projection at 2048 tokens and the up
+# projection at 16 and 256 tokens
 EVERY_ELEMENT = ["tiny_16x256x256", "llama7b_attn_2048x4096x4096", "llama7b_up_16x11008x4096",
                  "llama7b_up_256x11008x4096"]
 
