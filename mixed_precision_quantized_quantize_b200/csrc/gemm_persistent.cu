@@ -746,6 +746,354 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
     }
 }
 
+// ---------------------------------------------------------------- two token halves per weight unit
+// The same pipeline with tiles of 256 weight rows x 512 tokens, for widened
+// activations: every widened weight unit feeds the MMAs of two 256-token
+// halves, each into its own 256-column accumulator (all of tensor memory), so
+// the weight unpack and its shared-memory traffic are paid once per 512
+// tokens.  With both accumulators in one tile there is no next tile for the
+// epilogue to hide under: after each tile's k-blocks every warp of both CTAs
+// takes a share of its passes (rescale, the outlier MMAs, the output), as in
+// the last tile of the kernel above.  The operand ring is idle meanwhile and
+// holds the output staging tiles.
+namespace pk2 {
+constexpr int NT = 2;                                  // 256-token halves per tile
+constexpr int BT = NT * pk::BT;                        // 512 tokens per tile
+constexpr int STAGE = pk::A_BYTES + NT * pk::B_BYTES;  // 48 KB
+constexpr int S = 3;                                   // operand stages
+constexpr int SP = 6;                                  // packed weight staging units
+constexpr int UNIT = pk::BW * pk::PKROW;               // 8 KB
+constexpr int PK_OFF = S * STAGE;
+constexpr int EPI_TILE = 32 * 32 * 2;                  // a warp's 32 x 32 fp16 output tile
+constexpr int SMEM = PK_OFF + SP * UNIT + 1024;        // + alignment slack
+static_assert(SMEM + 4096 <= 232448, "shared memory budget (dynamic + static)");
+static_assert(16 * EPI_TILE <= S * STAGE, "the output staging tiles fit in the operand ring");
+static_assert(STAGE % 1024 == 0, "128-byte-swizzled operand tiles");
+}  // namespace pk2
+
+// One work unit on the pair MMA for both token halves: wait for its stage,
+// four MMAs per half (K = 32 bytes each) into that half's accumulator,
+// release the stage.
+template <bool F16>
+__device__ __forceinline__ bool issue_unit2(Ring &r, uint64_t *op_full, uint64_t *op_empty, uint64_t d0,
+                                            uint32_t tmem, uint32_t idesc, uint32_t acc_in, const Abort &ab) {
+    if (!wait_bar(&op_full[r.st], r.ph, ab)) return false;
+    tc_fence_after();
+    const uint64_t da = d0 + static_cast<uint64_t>((r.st * pk2::STAGE) >> 4);
+    const uint64_t db0 = da + (pk::A_BYTES >> 4), db1 = db0 + (pk::B_BYTES >> 4);
+    if (F16) {
+        mma2_f16(tmem, da, db0, idesc, 1u);
+        mma2_f16(tmem, da + 2, db0 + 2, idesc, 1u);
+        mma2_f16(tmem, da + 4, db0 + 4, idesc, 1u);
+        mma2_f16(tmem, da + 6, db0 + 6, idesc, 1u);
+        mma2_f16(tmem + 256u, da, db1, idesc, 1u);
+        mma2_f16(tmem + 256u, da + 2, db1 + 2, idesc, 1u);
+        mma2_f16(tmem + 256u, da + 4, db1 + 4, idesc, 1u);
+        mma2_f16(tmem + 256u, da + 6, db1 + 6, idesc, 1u);
+    } else {
+        mma2_i8(tmem, da, db0, idesc, acc_in);
+        mma2_i8(tmem, da + 2, db0 + 2, idesc, 1u);
+        mma2_i8(tmem, da + 4, db0 + 4, idesc, 1u);
+        mma2_i8(tmem, da + 6, db0 + 6, idesc, 1u);
+        mma2_i8(tmem + 256u, da, db1, idesc, acc_in);
+        mma2_i8(tmem + 256u, da + 2, db1 + 2, idesc, 1u);
+        mma2_i8(tmem + 256u, da + 4, db1 + 4, idesc, 1u);
+        mma2_i8(tmem + 256u, da + 6, db1 + 6, idesc, 1u);
+    }
+    mma2_commit_both(&op_empty[r.st]);
+    ++r.u;
+    if (++r.st == pk2::S) {
+        r.st = 0;
+        r.ph ^= 1u;
+    }
+    return true;
+}
+
+// DEBUG: write the integer sums instead of Y (no outliers, no scales).
+template <bool DEBUG>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
+    w4a4_gemm_persistent2_kernel(const __grid_constant__ CUtensorMap tm_w,
+                                 const __grid_constant__ CUtensorMap tm_x,
+                                 const __grid_constant__ CUtensorMap tm_wo,
+                                 const __grid_constant__ CUtensorMap tm_xo,
+                                 const __grid_constant__ CUtensorMap tm_y, const PParams p) {
+    using namespace pk;
+    constexpr int S = pk2::S, SP = pk2::SP;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t op_full[S], op_empty[S], x_full[S], pk_full[SP], pk_empty[SP];
+    __shared__ uint64_t int_done, acc_full, rescaled, epi_done, mma_done;
+    __shared__ uint64_t stall_bar;  // never completed (quik_test_stall)
+    __shared__ uint32_t tmem_base_s;
+    __shared__ int abort_s;
+    __shared__ unsigned err0_s;
+    __shared__ __align__(16) float sx_s[pk2::BT];
+
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+    const uint32_t smem_base = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();  // 0 = leader
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int ntp = pair < p.ntiles ? (p.ntiles - pair + npairs - 1) / npairs : 0;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&op_full[i], 2 * GW);  // the unit's unpack group in both CTAs (leader only)
+            mbar_init(&op_empty[i], 1);
+            mbar_init(&x_full[i], 1);
+        }
+        mbar_init(&int_done, 1);
+        mbar_init(&acc_full, 1);
+        mbar_init(&rescaled, 2 * 16);  // every warp of both CTAs (leader only)
+        mbar_init(&epi_done, 2 * 16);  // every warp of both CTAs (leader only)
+        mbar_init(&mma_done, 1);
+        mbar_init(&stall_bar, 1);
+        abort_s = 0;
+        err0_s = *reinterpret_cast<volatile unsigned *>(&g_pgemm_error);
+        fence_barrier_init();
+    }
+    // this CTA's rows of W and tokens of token half h for the pair's j-th tile
+    auto w_row0 = [&](int j) { return ((pair + j * npairs) / p.n_tt) * 256 + static_cast<int>(rank) * BW; };
+    auto tok0 = [&](int j) { return ((pair + j * npairs) % p.n_tt) * pk2::BT; };
+    auto t_row0 = [&](int j, int h) { return tok0(j) + h * pk::BT + static_cast<int>(rank) * BTH; };
+    const int early = min(SP, ntp * p.nkb_i);
+    if (warp == W_PPROD && lane == 0) {
+        for (int i = 0; i < SP; ++i) {
+            mbar_init(&pk_full[i], 1);
+            mbar_init(&pk_empty[i], GW);
+        }
+        fence_barrier_init();
+        if (early > 0) tma_prefetch_desc(&tm_w);
+        for (int q = 0; q < early; ++q) {
+            mbar_arrive_expect_tx(&pk_full[q], pk2::UNIT);
+            tma_load_2d(smem + pk2::PK_OFF + q * pk2::UNIT, &tm_w, PKROW * (q % p.nkb_i), w_row0(q / p.nkb_i),
+                        &pk_full[q]);
+        }
+    }
+    if (warp == W_MMA) tmem_alloc_pair(&tmem_base_s, TMEM_COLS);
+    tc_fence_before();
+    cluster_sync();  // barriers and TMEM allocation visible to both CTAs
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_s;
+    const Abort ab{&abort_s, err0_s};
+    const uint32_t id_i8 = idesc_s8_s32(2 * BW, pk::BT);
+    const uint32_t id_f16 = idesc_f16_f32(2 * BW, pk::BT);
+    const uint64_t d0 = sw128_kmajor_desc(smem_base);
+    Ring ring{0, 0u, 0};
+    bool issue_ok = rank != 0 || warp != W_MMA || lane != 0 ||
+                    *reinterpret_cast<volatile int *>(&g_pgemm_stall) == 0 || wait_bar(&stall_bar, 0, ab);
+    int u_x = 0, q_p = 0;     // the producers' unit counters (all tiles)
+    int u_g = 0, q_g = 0;     // the unpack warps' unit and staging counters (all tiles)
+    bool ok = true;           // this warp's waits have all succeeded
+    const int qd = warp & 3;  // TMEM lane quadrant this warp may access
+    if (warp == W_XPROD && lane == 0) {
+        tma_prefetch_desc(&tm_x);
+        if (p.nkb_o > 0) {
+            tma_prefetch_desc(&tm_wo);
+            tma_prefetch_desc(&tm_xo);
+        }
+    }
+    if (warp == W_PPROD && lane == 0) tma_prefetch_desc(&tm_w);
+
+    for (int j = 0; j < ntp; ++j) {
+        // ------------------------------------------------------------ tile j's k-blocks
+        if (warp == W_MMA) {
+            if (rank == 0 && lane == 0 && issue_ok) {
+                // both CTAs have read tile j-1's accumulators
+                if (j > 0) issue_ok = wait_bar(&epi_done, (j - 1) & 1, ab);
+                for (int k = 0; k < p.nkb_i && issue_ok; ++k)
+                    issue_ok = issue_unit2<false>(ring, op_full, op_empty, d0, tmem, id_i8, k > 0 ? 1u : 0u, ab);
+                if (issue_ok) mma2_commit_both(p.nkb_o > 0 ? &int_done : &acc_full);
+            }
+            __syncwarp();
+        } else if (warp == W_XPROD) {
+            if (lane == 0) {
+                if (j == 0) grid_dependency_wait();  // the activations come from the previous kernel
+                for (int v = 0; v < p.nkb_i + p.nkb_o && ok; ++v, ++u_x) {
+                    const int st = u_x % S;
+                    if (!(ok = wait_bar_lazy(&op_empty[st], ((u_x / S) & 1) ^ 1, ab))) break;
+                    uint8_t *a_st = smem + st * pk2::STAGE;
+                    if (v < p.nkb_i) {
+                        mbar_arrive_expect_tx(&x_full[st], pk2::NT * B_BYTES);
+                        for (int h = 0; h < pk2::NT; ++h)
+                            tma_load_2d(a_st + A_BYTES + h * B_BYTES, &tm_x, KB * v, t_row0(j, h), &x_full[st]);
+                    } else {
+                        const int o = v - p.nkb_i;
+                        mbar_arrive_expect_tx(&x_full[st], A_BYTES + pk2::NT * B_BYTES);
+                        tma_load_2d(a_st, &tm_wo, OKB * o, w_row0(j), &x_full[st]);
+                        for (int h = 0; h < pk2::NT; ++h)
+                            tma_load_2d(a_st + A_BYTES + h * B_BYTES, &tm_xo, OKB * o, t_row0(j, h), &x_full[st]);
+                    }
+                }
+            }
+            __syncwarp();
+        } else if (warp == W_PPROD) {
+            if (lane == 0) {
+                for (int k = 0; k < p.nkb_i && ok; ++k, ++q_p) {
+                    if (q_p < early) continue;  // requested before the set-up barrier
+                    const int ps = q_p % SP;
+                    if (!(ok = wait_bar_lazy(&pk_empty[ps], ((q_p / SP) & 1) ^ 1, ab))) break;
+                    mbar_arrive_expect_tx(&pk_full[ps], pk2::UNIT);
+                    tma_load_2d(smem + pk2::PK_OFF + ps * pk2::UNIT, &tm_w, PKROW * k, w_row0(j), &pk_full[ps]);
+                }
+            }
+            __syncwarp();
+        } else if (is_unpack_warp(warp)) {
+            const int g = unpack_group(warp);
+            const int tb = unpack_lane0(warp) + lane;  // thread in the group: 0 .. GT - 1
+            for (int v = 0; v < p.nkb_i + p.nkb_o && ok; ++v, ++u_g) {
+                const bool outl = v >= p.nkb_i;
+                if (u_g % NG != g) {  // another group's unit
+                    if (!outl) ++q_g;
+                    continue;
+                }
+                const int st = u_g % S;
+                if (!(ok = warp_wait(&op_empty[st], ((u_g / S) & 1) ^ 1, ab))) break;
+                if (!outl) {
+                    const int ps = q_g % SP;
+                    if (!(ok = warp_wait(&pk_full[ps], (q_g / SP) & 1, ab))) break;
+                    unpack_rows(smem + pk2::PK_OFF + ps * pk2::UNIT, smem + st * pk2::STAGE, tb);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pk_empty[ps]);
+                    fence_proxy_async_smem();  // generic-proxy stores -> visible to the pair's MMA
+                    ++q_g;
+                }
+                if (!(ok = warp_wait(&x_full[st], (u_g / S) & 1, ab))) break;
+                __syncwarp();
+                if (lane == 0) {
+                    if (rank == 0)
+                        mbar_arrive(&op_full[st]);
+                    else
+                        mbar_arrive_remote(mapa_shared(smem_u32(&op_full[st]), 0));
+                }
+            }
+            // keep the counters in step after an early stop (the remaining
+            // tiles' work is skipped, but the loops' counts stay consistent)
+        }
+
+        // ------------------------------------------------------------ tile j's epilogue, every warp
+        named_barrier_sync(2, THREADS);  // tile j-1's passes and every role's part of tile j are done
+        if (!DEBUG) {
+            grid_dependency_wait();  // sx comes from the previous kernel
+            const int m = tok0(j) + threadIdx.x;
+            sx_s[threadIdx.x] = m < p.M ? p.sx[m] : 0.0f;
+        }
+        named_barrier_sync(2, THREADS);  // sx_s filled
+        bool eok = abort_s == 0;
+        const int gn = w_row0(j) + qd * 32 + lane;  // this lane's output channel (TMEM lane)
+        const bool n_ok = gn < p.N;
+        const float swn = (!DEBUG && n_ok) ? p.sw[gn] : 0.0f;
+        const float bn = (!DEBUG && n_ok && p.bias != nullptr) ? __half2float(__ushort_as_half(p.bias[gn])) : 0.0f;
+        const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+        const int c0 = warp >> 2;  // chunks c0, c0 + 4, c0 + 8, c0 + 12 of the 16 (two halves x 8)
+        if (p.nkb_o > 0) {
+            if (eok && (eok = warp_wait_lazy(&int_done, j & 1, ab, lane))) {
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = c0; c < 16; c += 4) {
+                    const int col = 256 * (c >> 3) + 32 * (c & 7);
+                    uint32_t a[32];
+                    tmem_ld_32x32b_x32(t_lane + col, a);
+                    tmem_ld_wait();
+                    dequant32(a, sx_s + col, swn, bn);
+                    tmem_st_32x32b_x32(t_lane + col, a);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+            }
+            __syncwarp();
+            if (lane == 0) {  // also after a failed wait: the issuer's wait below then ends at once
+                if (rank == 0)
+                    mbar_arrive(&rescaled);
+                else
+                    mbar_arrive_remote(mapa_shared(smem_u32(&rescaled), 0));
+            }
+            if (warp == W_MMA && rank == 0 && lane == 0 && issue_ok) {
+                issue_ok = wait_bar(&rescaled, j & 1, ab);
+                for (int o = 0; o < p.nkb_o && issue_ok; ++o)
+                    issue_ok = issue_unit2<true>(ring, op_full, op_empty, d0, tmem, id_f16, 1u, ab);
+                if (issue_ok) mma2_commit_both(&acc_full);
+            }
+            __syncwarp();
+        }
+        if (eok && (eok = warp_wait_lazy(&acc_full, j & 1, ab, lane))) {
+            tc_fence_after();
+            uint16_t *ystage = reinterpret_cast<uint16_t *>(smem + warp * pk2::EPI_TILE);
+#pragma unroll 1
+            for (int c = c0; c < 16; c += 4) {
+                const int col = 256 * (c >> 3) + 32 * (c & 7);
+                uint32_t a[32];
+                tmem_ld_32x32b_x32(t_lane + col, a);
+                tmem_ld_wait();
+                if (!DEBUG && p.nkb_o == 0) dequant32(a, sx_s + col, swn, bn);  // else rescaled already
+                const int m0 = tok0(j) + col;
+                if (DEBUG) {
+                    if (n_ok) {
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj)
+                            if (m0 + jj < p.M)
+                                p.acc_dbg[static_cast<size_t>(m0 + jj) * p.N + gn] = static_cast<int32_t>(a[jj]) >> 8;
+                    }
+                    continue;
+                }
+                if (p.tma_y) {
+                    // transpose through the warp's staging tile, then one TMA store
+                    if (lane == 0) bulk_wait_group_read0();
+                    __syncwarp();
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj)
+                        ystage[jj * 32 + lane] = __half_as_ushort(__float2half_rn(__uint_as_float(a[jj])));
+                    fence_proxy_async_smem();  // generic stores -> visible to the TMA store
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tm_y, ystage, w_row0(j) + 32 * qd, m0);  // clipped at N and M
+                        bulk_commit_group();
+                    }
+                } else {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj)
+                        if (n_ok && m0 + jj < p.M)
+                            p.Y[static_cast<size_t>(m0 + jj) * p.N + gn] =
+                                __half_as_ushort(__float2half_rn(__uint_as_float(a[jj])));
+                }
+            }
+            // the staging tiles are read before the ring takes the next tile's operands
+            if (lane == 0 && p.tma_y) bulk_wait_group_read0();
+            tc_fence_before();
+        }
+        __syncwarp();
+        if (lane == 0) {  // this warp is done with the accumulators
+            if (rank == 0)
+                mbar_arrive(&epi_done);
+            else
+                mbar_arrive_remote(mapa_shared(smem_u32(&epi_done), 0));
+        }
+        named_barrier_sync(2, THREADS);  // the ring may take tile j+1's operands
+    }
+
+    // ---------------------------------------------------------------- teardown
+    if (warp == W_XPROD && lane == 0)  // no bulk copy may still write the ring
+        for (int v = u_x - 1; v >= 0 && v >= u_x - S; --v) mbar_wait_bounded(&x_full[v % S], (v / S) & 1, kWaitLimitNs);
+    if (warp == W_PPROD && lane == 0) {
+        const int issued = max(q_p, early);
+        for (int v = issued - 1; v >= 0 && v >= issued - SP; --v)
+            mbar_wait_bounded(&pk_full[v % SP], (v / SP) & 1, kWaitLimitNs);
+    }
+    if (warp == W_MMA && rank == 0 && lane == 0) {
+        // TMEM and the stages stay allocated until every issued MMA is done
+        mma2_commit_local(&mma_done);
+        mbar_wait_bounded(&mma_done, 0, kWaitLimitNs);
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // neither CTA leaves while the pair's MMAs or remote arrivals may touch it
+    if (warp == W_MMA) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, TMEM_COLS);
+    }
+}
+
 template <bool X4, bool DEBUG>
 quik_status run_persistent(const GemmArgs &a, cudaStream_t stream) {
     using C = PkCfg<X4>;
@@ -790,20 +1138,32 @@ quik_status run_persistent(const GemmArgs &a, cudaStream_t stream) {
     p.tma_y = tma_y ? 1 : 0;
     p.nkb_i = (Ki + pk::KB - 1) / pk::KB;
     p.nkb_o = outliers ? (a.k_o + pk::OKB - 1) / pk::OKB : 0;
-    p.n_tt = (a.M + pk::BT - 1) / pk::BT;
-    p.ntiles = p.n_tt * ((a.N + 2 * pk::BW - 1) / (2 * pk::BW));
+    const int n_wt = (a.N + 2 * pk::BW - 1) / (2 * pk::BW);
     p.sx = a.sx;
     p.sw = a.sw;
     p.bias = a.bias;
     p.Y = a.Y;
     p.acc_dbg = a.acc_dbg;
-    auto kern = w4a4_gemm_persistent_kernel<X4, DEBUG>;
-    if (!attribute_set_once(reinterpret_cast<const void *>(kern), C::SMEM)) return QUIK_ERR_CUDA;
-    const int npairs = std::max(1, std::min(p.ntiles, sm_count() / 2));
+    const int np_max = std::max(1, sm_count() / 2);
+    // 512-token tiles (widened activations, at most S outlier units) when
+    // they fit in one wave where 256-token tiles need two or more: measured,
+    // the main loop runs at the same rate per k-block and token either way,
+    // but a 512-token tile's epilogue does not overlap a next tile, so the
+    // larger tiles pay only where they remove a wave (the attention
+    // projection at 2048 tokens: GEMM 42.8 -> 37.9 us; at 2048 x 11008, three
+    // waves against five, they were slower: 92.1 against 83.2 us)
+    const int tiles1 = ((a.M + pk::BT - 1) / pk::BT) * n_wt, tiles2 = ((a.M + pk2::BT - 1) / pk2::BT) * n_wt;
+    const bool two = !X4 && !DEBUG && p.nkb_o <= pk2::S && tiles2 <= np_max && tiles1 > np_max;
+    p.n_tt = two ? (a.M + pk2::BT - 1) / pk2::BT : (a.M + pk::BT - 1) / pk::BT;
+    p.ntiles = p.n_tt * n_wt;
+    auto kern = two ? w4a4_gemm_persistent2_kernel<false> : w4a4_gemm_persistent_kernel<X4, DEBUG>;
+    const int smem_bytes = two ? pk2::SMEM : C::SMEM;
+    if (!attribute_set_once(reinterpret_cast<const void *>(kern), smem_bytes)) return QUIK_ERR_CUDA;
+    const int npairs = std::max(1, std::min(p.ntiles, np_max));
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(2 * npairs);
     cfg.blockDim = dim3(pk::THREADS);
-    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.dynamicSmemBytes = smem_bytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -610,3 +610,36 @@ def test_self_checking_build_matches(tmp_path):
                              act_bits=ab)
         y = layer(d["X"].to(DEV)).cpu().numpy().view(np.uint16)
         np.testing.assert_array_equal(y, got[f"y{i}"], err_msg=str(GUARDED[i]))
+
+
+# shapes whose layer call takes the 512-token tiles (two 256-token halves per
+# widened weight unit): ragged tokens and channels, FP16 outliers or none,
+# TMA or plain output stores
+TWO_HALVES = [
+    (1100, 4000, 1056, 32, True),   # 3 token tiles of 512 (the last one ragged), 16 weight tiles
+    (1100, 4100, 1088, 0, False),   # no outliers; N % 8 != 0 (plain stores), a ragged weight tile
+    (1536, 4096, 2176, 192, True),  # three outlier units (the most this form takes)
+]
+
+
+@pytest.mark.parametrize("shape", TWO_HALVES, ids=[str(s) for s in TWO_HALVES])
+def test_two_halves_layer(shape):
+    """The layer call on shapes that take the 512-token persistent tiles:
+    every output against the oracle's fp64 layer, and bit-identical to the
+    two-call path (quik_quantize_reorder + quik_gemm, 256-token tiles on the
+    packed codes)."""
+    M, N, K, k_o, bias = shape
+    cfg, d = _case(M, N, K, k_o, 0, False, bias, seed=31)
+    perm_d = d["perm"].to(DEV)
+    b = d["bias"].to(DEV) if d["bias"] is not None else None
+    X = d["X"].to(DEV)
+    layer = q.QuikLinear(d["W"].to(DEV), perm_d, k_o, 0, False, b)
+    Y = layer(X)
+    gx = q.quantize_reorder(X, perm_d, k_o, 0, False)
+    Y2 = q.gemm(gx, (layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale), K, k_o, 0, b)
+    torch.cuda.synchronize()
+    assert q.quik_sync_check() == q.QUIK_OK
+    np.testing.assert_array_equal(Y.cpu().numpy().view(np.uint16), Y2.cpu().numpy().view(np.uint16))
+    ref = oracle.layer(np16(d["X"]), np16(d["W"]), d["perm"].numpy(),
+                       None if d["bias"] is None else np16(d["bias"]), k_o, 0, False)["Y"]
+    assert_y_close(Y.float().cpu().numpy(), ref, f"two halves {shape}")
