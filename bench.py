@@ -106,6 +106,16 @@ def gemm_kernel(cfg):
         return ("w4a4_gemv (decode shapes: W rows as the MMA's M, tokens as N; INT4 codes "
                 "widened to INT8, tcgen05 kind::i8)", f"w4a4_gemv_{cfg.name}.md")
     if cfg.group == 0 and (cfg.k_o == 0 or not cfg.outlier_int8):
+        # the library's rule for 512-token tiles (one wave of them where
+        # 256-token tiles need two; at most three FP16 outlier units)
+        n_wt = -(-cfg.N // 256)
+        tiles1, tiles2 = -(-cfg.M // 256) * n_wt, -(-cfg.M // 512) * n_wt
+        if -(-cfg.k_o // 64) <= 3 and tiles2 <= 74 and tiles1 > 74 and not cfg.rmsnorm:
+            return ("w4a4_gemm_persistent2 (the persistent kernel with 256 weight rows x 512 tokens per "
+                    "tile: each widened weight k-block feeds two 256-token halves, two TMEM "
+                    "accumulators, all-warps epilogue per tile; tcgen05 kind::i8, FP16 outliers as "
+                    "kind::f16 MMAs onto the dequantised tile)",
+                    f"w4a4_gemm_persistent2_{cfg.name}.md")
         return persistent, f"w4a4_gemm_persistent_{cfg.name}.md"
     if cfg.group == 0:
         return ("w4a4_gemm_pair (INT4 codes widened to INT8, tcgen05 kind::i8 on CTA pairs)",
