@@ -606,6 +606,154 @@ def test_checker_catches_a_short_last_rescale_count():
     assert _caught(lambda: persistent_roles(2, 7, 2, last_rescale_count=2 * 4))
 
 
+def persistent2_roles(ntp, nkb_i, nkb_o, S=3, SP=6, NG=3, GW=3, skip_epi_done=False, rescale_count=None):
+    """The persistent kernel's 512-token form: tiles one after another, each
+    tile's k-blocks feeding both accumulators, then every warp of both CTAs
+    in the tile's epilogue between CTA-wide named barriers; the next tile's
+    MMAs wait until every warp of both CTAs has read the accumulators.  (That
+    wait is also implied: the next tile's first operand-full phase needs the
+    peer CTA's unpack group, which passes its CTA's closing barrier only after
+    all of that CTA's warps have read; skip_epi_done models the kernel
+    without it and stays correct.)"""
+    op_full = [Bar(2 * GW) for _ in range(S)]
+    op_empty = [[Bar(1) for _ in range(S)] for _ in range(2)]
+    x_full = [[Bar(1) for _ in range(S)] for _ in range(2)]
+    pk_full = [[Bar(1) for _ in range(SP)] for _ in range(2)]
+    pk_empty = [[Bar(GW) for _ in range(SP)] for _ in range(2)]
+    int_done = [Bar(1) for _ in range(2)]
+    acc_full = [Bar(1) for _ in range(2)]
+    rescaled, epi_done, mma_done = Bar(rescale_count or 2 * 16), Bar(2 * 16), Bar(1)
+    cta = [Sync(16) for _ in range(2)]
+    stage = [[Buf(f"CTA {c} operand stage {i}") for i in range(S)] for c in range(2)]
+    slot = [[Buf(f"CTA {c} staging slot {i}") for i in range(SP)] for c in range(2)]
+    acc = [Buf(f"CTA {c} accumulators") for c in range(2)]
+    early = min(SP, ntp * nkb_i)
+    ring = {"u": 0}
+
+    def issue(u):
+        st = u % S
+        yield ("wait", op_full[st], u // S)
+        for c in range(2):
+            yield ("own", stage[c][st])
+        for c in range(2):
+            yield ("write", acc[c])
+        for c in range(2):
+            yield ("async", op_empty[c][st], stage[c][st])
+
+    def epilogue(c, w, j):
+        yield ("sync", cta[c])  # every role done with tile j's k-blocks
+        yield ("sync", cta[c])  # the token scales staged
+        if nkb_o > 0:
+            yield ("wait", int_done[c], j)
+            yield ("own", acc[c])
+            yield ("free", acc[c])
+            yield ("arrive", rescaled)
+            if c == 0 and w == 0:
+                yield ("wait", rescaled, j)
+                for _ in range(nkb_o):
+                    yield from issue(ring["u"])
+                    ring["u"] += 1
+                for cc in range(2):
+                    yield ("async", acc_full[cc])
+        yield ("wait", acc_full[c], j)
+        yield ("own", acc[c])
+        yield ("free", acc[c])
+        yield ("arrive", epi_done)
+        yield ("sync", cta[c])  # the ring may take the next tile's operands
+
+    def mma_warp(c):
+        for j in range(ntp):
+            if c == 0:
+                if j > 0 and not skip_epi_done:
+                    yield ("wait", epi_done, j - 1)
+                for _ in range(nkb_i):
+                    yield from issue(ring["u"])
+                    ring["u"] += 1
+                for cc in range(2):
+                    yield ("async", (int_done if nkb_o > 0 else acc_full)[cc])
+            yield from epilogue(c, 0, j)
+        if c == 0:
+            yield ("async", mma_done)
+            yield ("wait", mma_done, 0)
+
+    def xprod(c):
+        u = 0
+        for j in range(ntp):
+            for v in range(nkb_i + nkb_o):
+                st = u % S
+                if u >= S:
+                    yield ("wait", op_empty[c][st], u // S - 1)
+                yield ("write", stage[c][st])
+                yield ("async", x_full[c][st])
+                u += 1
+            yield from epilogue(c, 4, j)
+
+    def pprod(c):
+        q = 0
+        for j in range(ntp):
+            for k in range(nkb_i):
+                if q >= early:
+                    ps = q % SP
+                    if q >= SP:
+                        yield ("wait", pk_empty[c][ps], q // SP - 1)
+                    yield ("write", slot[c][ps])
+                    yield ("async", pk_full[c][ps])
+                q += 1
+            yield from epilogue(c, 8, j)
+
+    def prologue(c):
+        for q in range(early):  # requested before the set-up barrier
+            yield ("write", slot[c][q])
+            yield ("async", pk_full[c][q])
+
+    def unpack(c, g, w):
+        u = q = 0
+        for j in range(ntp):
+            for v in range(nkb_i + nkb_o):
+                outl = v >= nkb_i
+                if u % NG == g:
+                    st = u % S
+                    if u >= S:
+                        yield ("wait", op_empty[c][st], u // S - 1)
+                    if not outl:
+                        ps = q % SP
+                        yield ("wait", pk_full[c][ps], q // SP)
+                        yield ("own", slot[c][ps])
+                        yield ("write", stage[c][st])
+                        yield ("free", slot[c][ps])
+                        yield ("arrive", pk_empty[c][ps])
+                    yield ("wait", x_full[c][st], u // S)
+                    yield ("arrive", op_full[st])
+                u += 1
+                q += 0 if outl else 1
+            yield from epilogue(c, 1 + 4 * g + w, j)
+
+    def epi_warp(c, e):
+        for j in range(ntp):
+            yield from epilogue(c, 12 + e, j)
+
+    roles = []
+    for c in range(2):
+        roles += [prologue(c), mma_warp(c), xprod(c), pprod(c)]
+        roles += [unpack(c, g, w) for g in range(NG) for w in range(GW)]
+        roles += [epi_warp(c, e) for e in range(4)]
+    return roles
+
+
+@pytest.mark.parametrize("ntp", [1, 2, 3])
+@pytest.mark.parametrize("nkb_i,nkb_o", [(1, 0), (2, 1), (7, 3), (31, 2), (16, 0)])
+@pytest.mark.parametrize("skip", [False, True])
+def test_persistent2_protocol(ntp, nkb_i, nkb_o, skip):
+    for seed in range(4):
+        run(persistent2_roles(ntp, nkb_i, nkb_o, skip_epi_done=skip), seed)
+
+
+def test_checker_catches_a_short_tile_rescale_count():
+    """The 512-token form's rescale barrier counting only four warps per CTA:
+    the later arrivals overflow its phase."""
+    assert _caught(lambda: persistent2_roles(2, 7, 2, rescale_count=2 * 4))
+
+
 def _caught(make, seeds=60):
     for seed in range(seeds):
         try:
