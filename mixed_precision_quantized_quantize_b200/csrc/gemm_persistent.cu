@@ -760,8 +760,8 @@ namespace pk2 {
 constexpr int NT = 2;                                  // 256-token halves per tile
 constexpr int BT = NT * pk::BT;                        // 512 tokens per tile
 constexpr int STAGE = pk::A_BYTES + NT * pk::B_BYTES;  // 48 KB
-constexpr int S = 3;                                   // operand stages
-constexpr int SP = 6;                                  // packed weight staging units
+constexpr int S = 4;                                   // operand stages
+constexpr int SP = 3;                                  // packed weight staging units
 constexpr int UNIT = pk::BW * pk::PKROW;               // 8 KB
 constexpr int PK_OFF = S * STAGE;
 constexpr int EPI_TILE = 32 * 32 * 2;                  // a warp's 32 x 32 fp16 output tile
