@@ -748,6 +748,14 @@ def test_persistent2_protocol(ntp, nkb_i, nkb_o, skip):
         run(persistent2_roles(ntp, nkb_i, nkb_o, skip_epi_done=skip), seed)
 
 
+def test_checker_catches_a_staging_ring_smaller_than_the_groups():
+    """Six operand stages with two staging slots for three unpack groups: a
+    group can reach a slot's phase before its previous phase has landed (a
+    parity wait then passes early).  This configuration was built once and
+    produced wrong outputs and timeouts on the GPU; the simulation flags it."""
+    assert _caught(lambda: persistent_roles(2, 8, 1, S=6, SP=2))
+
+
 def test_checker_catches_a_short_tile_rescale_count():
     """The 512-token form's rescale barrier counting only four warps per CTA:
     the later arrivals overflow its phase."""
