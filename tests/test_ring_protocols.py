@@ -606,7 +606,7 @@ def test_checker_catches_a_short_last_rescale_count():
     assert _caught(lambda: persistent_roles(2, 7, 2, last_rescale_count=2 * 4))
 
 
-def persistent2_roles(ntp, nkb_i, nkb_o, S=3, SP=6, NG=3, GW=3, skip_epi_done=False, rescale_count=None):
+def persistent2_roles(ntp, nkb_i, nkb_o, S=4, SP=3, NG=3, GW=3, skip_epi_done=False, rescale_count=None):
     """The persistent kernel's 512-token form: tiles one after another, each
     tile's k-blocks feeding both accumulators, then every warp of both CTAs
     in the tile's epilogue between CTA-wide named barriers; the next tile's
@@ -741,7 +741,7 @@ def persistent2_roles(ntp, nkb_i, nkb_o, S=3, SP=6, NG=3, GW=3, skip_epi_done=Fa
 
 
 @pytest.mark.parametrize("ntp", [1, 2, 3])
-@pytest.mark.parametrize("nkb_i,nkb_o", [(1, 0), (2, 1), (7, 3), (31, 2), (16, 0)])
+@pytest.mark.parametrize("nkb_i,nkb_o", [(1, 0), (2, 1), (7, 3), (31, 2), (16, 0), (10, 4)])
 @pytest.mark.parametrize("skip", [False, True])
 def test_persistent2_protocol(ntp, nkb_i, nkb_o, skip):
     for seed in range(4):
