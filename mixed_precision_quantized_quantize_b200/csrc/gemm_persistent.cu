@@ -747,11 +747,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
 }
 
 // ---------------------------------------------------------------- two token halves per weight unit
-// The same pipeline with tiles of 256 weight rows x 512 tokens, for widened
-// activations: every widened weight unit feeds the MMAs of two 256-token
-// halves, each into its own 256-column accumulator (all of tensor memory), so
-// the weight unpack and its shared-memory traffic are paid once per 512
-// tokens.  With both accumulators in one tile there is no next tile for the
+// The same pipeline with tiles of 256 weight rows x 512 tokens: every widened
+// weight unit feeds the MMAs of two 256-token halves, each into its own
+// 256-column accumulator (all of tensor memory), so the weight unpack and its
+// shared-memory traffic are paid once per 512 tokens.  X4: the activations
+// come packed through the staging ring with the weights and are widened too
+// (half the bytes each SM must pull in by TMA per MMA, whose rate the loads
+// otherwise bound); else they come widened straight into the operand stage.  With both accumulators in one tile there is no next tile for the
 // epilogue to hide under: after each tile's k-blocks every warp of both CTAs
 // takes a share of its passes (rescale, the outlier MMAs, the output), as in
 // the last tile of the kernel above.  The operand ring is idle meanwhile and
@@ -760,21 +762,26 @@ namespace pk2 {
 constexpr int NT = 2;                                  // 256-token halves per tile
 constexpr int BT = NT * pk::BT;                        // 512 tokens per tile
 constexpr int STAGE = pk::A_BYTES + NT * pk::B_BYTES;  // 48 KB
-constexpr int S = 4;                                   // operand stages
-constexpr int SP = 3;                                  // packed weight staging units
-constexpr int UNIT = pk::BW * pk::PKROW;               // 8 KB
-constexpr int PK_OFF = S * STAGE;
 constexpr int EPI_TILE = 32 * 32 * 2;                  // a warp's 32 x 32 fp16 output tile
-constexpr int SMEM = PK_OFF + SP * UNIT + 1024;        // + alignment slack
-static_assert(SMEM + 4096 <= 232448, "shared memory budget (dynamic + static)");
-static_assert(16 * EPI_TILE <= S * STAGE, "the output staging tiles fit in the operand ring");
+constexpr int SP = 3;                                  // packed staging units
 static_assert(STAGE % 1024 == 0, "128-byte-swizzled operand tiles");
 }  // namespace pk2
+
+template <bool X4>
+struct Pk2Cfg {
+    static constexpr int S = X4 ? 3 : 4;  // operand stages (48 KB each)
+    // packed k-block: W, and with X4 the two token halves
+    static constexpr int UNIT = pk::BW * pk::PKROW + (X4 ? pk2::NT * pk::BTH * pk::PKROW : 0);
+    static constexpr int PK_OFF = S * pk2::STAGE;
+    static constexpr int SMEM = PK_OFF + pk2::SP * UNIT + 1024;  // + alignment slack
+    static_assert(SMEM + 4096 <= 232448, "shared memory budget (dynamic + static)");
+    static_assert(16 * pk2::EPI_TILE <= S * pk2::STAGE, "the output staging tiles fit in the operand ring");
+};
 
 // One work unit on the pair MMA for both token halves: wait for its stage,
 // four MMAs per half (K = 32 bytes each) into that half's accumulator,
 // release the stage.
-template <bool F16>
+template <bool F16, int S_ISSUE>
 __device__ __forceinline__ bool issue_unit2(Ring &r, uint64_t *op_full, uint64_t *op_empty, uint64_t d0,
                                             uint32_t tmem, uint32_t idesc, uint32_t acc_in, const Abort &ab) {
     if (!wait_bar(&op_full[r.st], r.ph, ab)) return false;
@@ -802,7 +809,7 @@ __device__ __forceinline__ bool issue_unit2(Ring &r, uint64_t *op_full, uint64_t
     }
     mma2_commit_both(&op_empty[r.st]);
     ++r.u;
-    if (++r.st == pk2::S) {
+    if (++r.st == S_ISSUE) {
         r.st = 0;
         r.ph ^= 1u;
     }
@@ -810,7 +817,7 @@ __device__ __forceinline__ bool issue_unit2(Ring &r, uint64_t *op_full, uint64_t
 }
 
 // DEBUG: write the integer sums instead of Y (no outliers, no scales).
-template <bool DEBUG>
+template <bool X4, bool DEBUG>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
     w4a4_gemm_persistent2_kernel(const __grid_constant__ CUtensorMap tm_w,
                                  const __grid_constant__ CUtensorMap tm_x,
@@ -818,7 +825,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
                                  const __grid_constant__ CUtensorMap tm_xo,
                                  const __grid_constant__ CUtensorMap tm_y, const PParams p) {
     using namespace pk;
-    constexpr int S = pk2::S, SP = pk2::SP;
+    using C2 = Pk2Cfg<X4>;
+    constexpr int S = C2::S, SP = pk2::SP;
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t op_full[S], op_empty[S], x_full[S], pk_full[SP], pk_empty[SP];
     __shared__ uint64_t int_done, acc_full, rescaled, epi_done, mma_done;
@@ -856,7 +864,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
     auto w_row0 = [&](int j) { return ((pair + j * npairs) / p.n_tt) * 256 + static_cast<int>(rank) * BW; };
     auto tok0 = [&](int j) { return ((pair + j * npairs) % p.n_tt) * pk2::BT; };
     auto t_row0 = [&](int j, int h) { return tok0(j) + h * pk::BT + static_cast<int>(rank) * BTH; };
-    const int early = min(SP, ntp * p.nkb_i);
+    // W units requested before the set-up barrier (W is not the previous
+    // kernel's output; with X4 the units also hold X, which must wait)
+    const int early = X4 ? 0 : min(SP, ntp * p.nkb_i);
     if (warp == W_PPROD && lane == 0) {
         for (int i = 0; i < SP; ++i) {
             mbar_init(&pk_full[i], 1);
@@ -865,8 +875,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
         fence_barrier_init();
         if (early > 0) tma_prefetch_desc(&tm_w);
         for (int q = 0; q < early; ++q) {
-            mbar_arrive_expect_tx(&pk_full[q], pk2::UNIT);
-            tma_load_2d(smem + pk2::PK_OFF + q * pk2::UNIT, &tm_w, PKROW * (q % p.nkb_i), w_row0(q / p.nkb_i),
+            mbar_arrive_expect_tx(&pk_full[q], C2::UNIT);
+            tma_load_2d(smem + C2::PK_OFF + q * C2::UNIT, &tm_w, PKROW * (q % p.nkb_i), w_row0(q / p.nkb_i),
                         &pk_full[q]);
         }
     }
@@ -902,7 +912,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
                 // both CTAs have read tile j-1's accumulators
                 if (j > 0) issue_ok = wait_bar(&epi_done, (j - 1) & 1, ab);
                 for (int k = 0; k < p.nkb_i && issue_ok; ++k)
-                    issue_ok = issue_unit2<false>(ring, op_full, op_empty, d0, tmem, id_i8, k > 0 ? 1u : 0u, ab);
+                    issue_ok = issue_unit2<false, S>(ring, op_full, op_empty, d0, tmem, id_i8, k > 0 ? 1u : 0u, ab);
                 if (issue_ok) mma2_commit_both(p.nkb_o > 0 ? &int_done : &acc_full);
             }
             __syncwarp();
@@ -913,7 +923,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
                     const int st = u_x % S;
                     if (!(ok = wait_bar_lazy(&op_empty[st], ((u_x / S) & 1) ^ 1, ab))) break;
                     uint8_t *a_st = smem + st * pk2::STAGE;
-                    if (v < p.nkb_i) {
+                    if (v < p.nkb_i && X4) {
+                        mbar_arrive(&x_full[st]);  // one phase per unit on every stage
+                    } else if (v < p.nkb_i) {
                         mbar_arrive_expect_tx(&x_full[st], pk2::NT * B_BYTES);
                         for (int h = 0; h < pk2::NT; ++h)
                             tma_load_2d(a_st + A_BYTES + h * B_BYTES, &tm_x, KB * v, t_row0(j, h), &x_full[st]);
@@ -929,12 +941,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
             __syncwarp();
         } else if (warp == W_PPROD) {
             if (lane == 0) {
+                if (X4 && j == 0) grid_dependency_wait();  // packed X comes from the previous kernel
                 for (int k = 0; k < p.nkb_i && ok; ++k, ++q_p) {
                     if (q_p < early) continue;  // requested before the set-up barrier
                     const int ps = q_p % SP;
                     if (!(ok = wait_bar_lazy(&pk_empty[ps], ((q_p / SP) & 1) ^ 1, ab))) break;
-                    mbar_arrive_expect_tx(&pk_full[ps], pk2::UNIT);
-                    tma_load_2d(smem + pk2::PK_OFF + ps * pk2::UNIT, &tm_w, PKROW * k, w_row0(j), &pk_full[ps]);
+                    uint8_t *dst = smem + C2::PK_OFF + ps * C2::UNIT;
+                    mbar_arrive_expect_tx(&pk_full[ps], C2::UNIT);
+                    tma_load_2d(dst, &tm_w, PKROW * k, w_row0(j), &pk_full[ps]);
+                    if (X4)
+                        for (int h = 0; h < pk2::NT; ++h)
+                            tma_load_2d(dst + BW * PKROW + h * BTH * PKROW, &tm_x, PKROW * k, t_row0(j, h), &pk_full[ps]);
                 }
             }
             __syncwarp();
@@ -952,7 +969,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
                 if (!outl) {
                     const int ps = q_g % SP;
                     if (!(ok = warp_wait(&pk_full[ps], (q_g / SP) & 1, ab))) break;
-                    unpack_rows(smem + pk2::PK_OFF + ps * pk2::UNIT, smem + st * pk2::STAGE, tb);
+                    const uint8_t *src = smem + C2::PK_OFF + ps * C2::UNIT;
+                    uint8_t *a_st = smem + st * pk2::STAGE;
+                    unpack_rows(src, a_st, tb);
+                    if (X4)
+                        for (int h = 0; h < pk2::NT; ++h)
+                            unpack_rows(src + BW * PKROW + h * BTH * PKROW, a_st + A_BYTES + h * B_BYTES, tb);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pk_empty[ps]);
                     fence_proxy_async_smem();  // generic-proxy stores -> visible to the pair's MMA
@@ -1011,7 +1033,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pk::THREADS, 1)
             if (warp == W_MMA && rank == 0 && lane == 0 && issue_ok) {
                 issue_ok = wait_bar(&rescaled, j & 1, ab);
                 for (int o = 0; o < p.nkb_o && issue_ok; ++o)
-                    issue_ok = issue_unit2<true>(ring, op_full, op_empty, d0, tmem, id_f16, 1u, ab);
+                    issue_ok = issue_unit2<true, S>(ring, op_full, op_empty, d0, tmem, id_f16, 1u, ab);
                 if (issue_ok) mma2_commit_both(&acc_full);
             }
             __syncwarp();
@@ -1153,11 +1175,11 @@ quik_status run_persistent(const GemmArgs &a, cudaStream_t stream) {
     // projection at 2048 tokens: GEMM 42.8 -> 37.9 us; at 2048 x 11008, three
     // waves against five, they were slower: 92.1 against 83.2 us)
     const int tiles1 = ((a.M + pk::BT - 1) / pk::BT) * n_wt, tiles2 = ((a.M + pk2::BT - 1) / pk2::BT) * n_wt;
-    const bool two = !X4 && !DEBUG && p.nkb_o <= pk2::S && tiles2 <= np_max && tiles1 > np_max;
+    const bool two = !DEBUG && p.nkb_o <= Pk2Cfg<X4>::S && tiles2 <= np_max && tiles1 > np_max;
     p.n_tt = two ? (a.M + pk2::BT - 1) / pk2::BT : (a.M + pk::BT - 1) / pk::BT;
     p.ntiles = p.n_tt * n_wt;
-    auto kern = two ? w4a4_gemm_persistent2_kernel<false> : w4a4_gemm_persistent_kernel<X4, DEBUG>;
-    const int smem_bytes = two ? pk2::SMEM : C::SMEM;
+    auto kern = two ? w4a4_gemm_persistent2_kernel<X4, false> : w4a4_gemm_persistent_kernel<X4, DEBUG>;
+    const int smem_bytes = two ? Pk2Cfg<X4>::SMEM : C::SMEM;
     if (!attribute_set_once(reinterpret_cast<const void *>(kern), smem_bytes)) return QUIK_ERR_CUDA;
     const int npairs = std::max(1, std::min(p.ntiles, np_max));
     cudaLaunchConfig_t cfg{};
