@@ -117,6 +117,90 @@ def test_linear_output_within_tolerance(shape):
     np.testing.assert_array_equal(Y.cpu().numpy().view(np.uint16), Y2.cpu().numpy().view(np.uint16))
 
 
+def _wide_expected(Q, Ki):
+    """The oracle's packed codes (code 2i in the low nibble of byte i) as the
+    layer call's widened operand: per 32 positions the 16 even ones, then the
+    16 odd ones, each as the signed byte 16 c."""
+    lo = (Q & 0xF).astype(np.int16)
+    hi = (Q >> 4).astype(np.int16)
+    codes = np.empty((Q.shape[0], Ki), np.int16)
+    codes[:, 0::2] = np.where(lo > 7, lo - 16, lo)
+    codes[:, 1::2] = np.where(hi > 7, hi - 16, hi)
+    blocks = codes.reshape(Q.shape[0], Ki // 32, 16, 2)     # [row, block, j, parity]
+    wide = blocks.transpose(0, 1, 3, 2).reshape(Q.shape[0], Ki)  # [row, block, parity, j]
+    return (wide * 16).astype(np.int8)
+
+
+def _r256(n):
+    return (n + 255) // 256 * 256
+
+
+# (M, K, k_o): layer calls above 32 tokens with FP16 or no outliers, whose
+# quantiser writes the widened codes: one to eight words per thread (K_i from
+# 448 to 20480), a few rows per SM up to more than 16 (4101 rows), the
+# attention projection's rows, no outliers
+WIDE = [(64, 512, 64), (200, 640, 64), (2048, 4096, 128), (4101, 1024, 0), (300, 8256, 64),
+        (130, 11008, 0), (40, 20544, 64)]
+
+
+@pytest.mark.parametrize("shape", WIDE, ids=[str(s) for s in WIDE])
+def test_wide_codes_bit_exact(shape):
+    """The layer call's widened codes, scales and FP16 outliers (read from
+    its workspace) against the oracle's, bit for bit."""
+    M, K, k_o = shape
+    Ki = K - k_o
+    cfg, d = _case(M, 64, K, k_o, 0, False, False, seed=17)
+    perm_d = d["perm"].to(DEV)
+    layer = q.QuikLinear(d["W"].to(DEV), perm_d, k_o, 0, False, None)
+    shape_s = layer.shape(M)
+    ws = torch.full((q.quik_workspace_size(shape_s),), 0x5A, dtype=torch.uint8, device=DEV)
+    Y = torch.empty((M, 64), dtype=torch.float16, device=DEV)
+    q.quik_linear(shape_s, d["X"].to(DEV), perm_d, layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale,
+                  None, Y, ws)
+    torch.cuda.synchronize()
+    w = ws.cpu().numpy()
+    Q, sx, O, _ = oracle_quant(d["X"], d["perm"], k_o, 0, False)
+    np.testing.assert_array_equal(w[:M * Ki].view(np.int8).reshape(M, Ki), _wide_expected(Q, Ki))
+    o_sx = _r256(M * Ki)
+    np.testing.assert_array_equal(w[o_sx:o_sx + 4 * M].view(np.uint32), sx.view(np.uint32))
+    if k_o:
+        o_xo = o_sx + _r256(4 * M)
+        np.testing.assert_array_equal(w[o_xo:o_xo + 2 * M * k_o].view(np.uint16).reshape(M, k_o),
+                                      O.view(np.uint16))
+
+
+def test_wide_codes_bad_perm_reported():
+    """Entries of perm outside [0, K) read channel 0 and are reported, in the
+    widened quantiser too; its codes then equal the oracle's on that perm
+    (channel 0 twice: a repeated channel)."""
+    M, K, k_o = 100, 512, 64
+    cfg, d = _case(M, 64, K, k_o, 0, False, False, seed=19)
+    perm = d["perm"].clone()
+    perm[7] = K + 5
+    perm[K - 3] = -2
+    perm_d = perm.to(DEV)
+    layer = q.QuikLinear(d["W"].to(DEV), d["perm"].to(DEV), k_o, 0, False, None)
+    shape_s = layer.shape(M)
+    ws = torch.zeros((q.quik_workspace_size(shape_s),), dtype=torch.uint8, device=DEV)
+    Y = torch.empty((M, 64), dtype=torch.float16, device=DEV)
+    assert q.quik_sync_check() == q.QUIK_OK
+    q.quik_linear(shape_s, d["X"].to(DEV), perm_d, layer.Wq, layer.w_scale, layer.Wo, layer.wo_scale,
+                  None, Y, ws)
+    torch.cuda.synchronize()
+    assert q.quik_sync_check() == q.QUIK_ERR_INVALID_ARG
+    assert q.quik_sync_check() == q.QUIK_OK
+    p0 = perm.numpy().copy()
+    p0[(p0 < 0) | (p0 >= K)] = 0
+    Q, sx, O, _ = oracle.quantize_rows(np16(d["X"]), p0, k_o, 0, False)
+    w = ws.cpu().numpy()
+    Ki = K - k_o
+    np.testing.assert_array_equal(w[:M * Ki].view(np.int8).reshape(M, Ki), _wide_expected(Q, Ki))
+    o_sx = _r256(M * Ki)
+    np.testing.assert_array_equal(w[o_sx:o_sx + 4 * M].view(np.uint32), sx.view(np.uint32))
+    o_xo = o_sx + _r256(4 * M)
+    np.testing.assert_array_equal(w[o_xo:o_xo + 2 * M * k_o].view(np.uint16).reshape(M, k_o), O.view(np.uint16))
+
+
 def test_zero_rows_and_ties():
     """All-zero rows give zero scales and codes; exact half-way values round to even."""
     M, N, K, k_o = 40, 64, 256, 32
