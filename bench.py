@@ -95,9 +95,26 @@ def gemm_kernel(cfg):
                   "x 256 tokens per tile, double-buffered TMEM accumulators; INT4 codes widened "
                   "to INT8, tcgen05 kind::i8; FP16 outliers as kind::f16 MMAs onto the "
                   "dequantised tile)")
+    persistent2 = ("w4a4_gemm_persistent2 (the persistent kernel with 256 weight rows x 512 tokens per "
+                   "tile: each widened weight k-block feeds two 256-token halves, two TMEM "
+                   "accumulators, all-warps epilogue per tile; tcgen05 kind::i8, FP16 outliers as "
+                   "kind::f16 MMAs onto the dequantised tile)")
+
+    def tiles512(packed):
+        # the library's rule for 512-token tiles: one wave of them where
+        # 256-token tiles need two or more, with at most as many FP16
+        # outlier units as operand stages (three with packed activations,
+        # four with the layer call's widened ones)
+        n_wt = -(-cfg.N // 256)
+        tiles1, tiles2 = -(-cfg.M // 256) * n_wt, -(-cfg.M // 512) * n_wt
+        return -(-cfg.k_o // 64) <= (3 if packed else 4) and tiles2 <= 74 and tiles1 > 74
+
     if cfg.sparse24:
-        return (persistent + " on the 2:4 weights expanded to dense codes (more than 32 tokens; "
-                "the expansion is timed separately)", f"w4a4_gemm_persistent_{cfg.name}.md")
+        # the timed GEMM is quik_gemm on packed codes and the expanded weights
+        two = tiles512(True)
+        return ((persistent2 if two else persistent) + " on the 2:4 weights expanded to dense codes "
+                "(more than 32 tokens; the expansion is timed separately)",
+                f"w4a4_gemm_persistent{'2' if two else ''}_{cfg.name}.md")
     if cfg.act_bits == 8:
         return (("w4a4_gemm_pair with INT8 activations and weights (W8A8)" if cfg.weight_bits == 8 else
                  "w4a4_gemm_pair with INT8 activations (W4A8; weights widened from INT4)")
@@ -106,16 +123,10 @@ def gemm_kernel(cfg):
         return ("w4a4_gemv (decode shapes: W rows as the MMA's M, tokens as N; INT4 codes "
                 "widened to INT8, tcgen05 kind::i8)", f"w4a4_gemv_{cfg.name}.md")
     if cfg.group == 0 and (cfg.k_o == 0 or not cfg.outlier_int8):
-        # the library's rule for 512-token tiles (one wave of them where
-        # 256-token tiles need two; at most three FP16 outlier units)
-        n_wt = -(-cfg.N // 256)
-        tiles1, tiles2 = -(-cfg.M // 256) * n_wt, -(-cfg.M // 512) * n_wt
-        if -(-cfg.k_o // 64) <= 3 and tiles2 <= 74 and tiles1 > 74 and not cfg.rmsnorm:
-            return ("w4a4_gemm_persistent2 (the persistent kernel with 256 weight rows x 512 tokens per "
-                    "tile: each widened weight k-block feeds two 256-token halves, two TMEM "
-                    "accumulators, all-warps epilogue per tile; tcgen05 kind::i8, FP16 outliers as "
-                    "kind::f16 MMAs onto the dequantised tile)",
-                    f"w4a4_gemm_persistent2_{cfg.name}.md")
+        # the norm-fused workload's GEMM is timed through quik_gemm on packed
+        # codes; the others' inside the layer call, on widened codes
+        if tiles512(cfg.rmsnorm):
+            return persistent2, f"w4a4_gemm_persistent2_{cfg.name}.md"
         return persistent, f"w4a4_gemm_persistent_{cfg.name}.md"
     if cfg.group == 0:
         return ("w4a4_gemm_pair (INT4 codes widened to INT8, tcgen05 kind::i8 on CTA pairs)",

@@ -40,3 +40,28 @@ def test_path_roofline_decode_is_byte_bound():
     r = bench.path_roofline(cfg, PEAKS, 19.5e-6)
     assert r["gemm_bound"] == "hbm"
     assert r["gemm_roof_us"] == pytest.approx(cfg.gemm_bytes / 6.5e12 * 1e6, abs=0.01)
+
+
+@pytest.mark.parametrize("M,N,K,k_o,rmsnorm,kernel", [
+    # the attention projection: 128 tiles of 256 x 256 (two waves on 74
+    # pairs), 64 of 256 x 512 (one wave) -> 512-token tiles, widened or
+    # packed (the norm-fused workload's GEMM is timed on packed codes)
+    (2048, 4096, 4096, 128, False, "w4a4_gemm_persistent2"),
+    (2048, 4096, 4096, 128, True, "w4a4_gemm_persistent2"),
+    # four FP16 outlier units: four operand stages with widened codes, three
+    # with packed ones
+    (2048, 4096, 4352, 256, False, "w4a4_gemm_persistent2"),
+    (2048, 4096, 4352, 256, True, "w4a4_gemm_persistent "),
+    # 172 tiles of 512 tokens: more than one wave either way
+    (2048, 11008, 4096, 128, False, "w4a4_gemm_persistent "),
+    # 43 tiles of 256: already one wave
+    (256, 11008, 4096, 128, False, "w4a4_gemm_persistent "),
+])
+def test_gemm_kernel_names_the_tile_form(M, N, K, k_o, rmsnorm, kernel):
+    """bench.py names the persistent GEMM's tile form by the library's
+    dispatch rule (one wave of 512-token tiles where 256-token tiles need
+    more, at most three or four outlier units)."""
+    cfg = wl.custom_config(M, N, K, k_o, 0, False, False, rmsnorm=rmsnorm)
+    name, profile = bench.gemm_kernel(cfg)
+    assert name.startswith(kernel)
+    assert profile.startswith(kernel.strip() + "_")
